@@ -1,0 +1,262 @@
+"""Seeded synthetic inputs for the verify workloads.
+
+This module feeds both the CPU oracle and the GPU library with the same
+bytes.  It holds none of the verifier's arithmetic: it draws logits from
+normal distributions (numpy's Philox bit generator), rounds them to bf16,
+and draws draft tokens the way a draft model's sampler would (inverse CDF
+over the draft softmax, or "argmax with probability p, else uniform" for the
+greedy and lookahead workloads).
+
+Logit arrays are numpy arrays: float32 for "f32", uint16 bf16 bit patterns
+for "bf16".  ``as_torch`` turns one into a torch tensor of the right dtype.
+
+The five named workloads (sizes, distributions, temperatures and seeds of the
+verify step they stand for):
+
+  stoch_b1_k4_v32000_f32   stochastic, B=1 k=4 V=32000, target fp32 ~ N(0, 2^2),
+                           draft fp32 = target + N(0, 1), T=1.0, seed 0
+  greedy_b64_k4_v128256    greedy, B=64 k=4 V=128256, bf16 ~ N(0, 3^2), draft token
+                           = argmax w.p. 0.7 else uniform, seed 2
+  stoch_b64_k4_v128256     stochastic, B=64 k=4 V=128256, target bf16 ~ N(0, 3^2),
+                           draft fp32 = target + N(0, 1.5^2), T=0.7, seed 1
+  stoch_b256_k8_v128256    stochastic, B=256 k=8 V=128256, target bf16 ~ N(0, 3^2),
+                           draft bf16 = RNE(target + N(0, 1)), T=1.0, seed 3
+  multi_b16_g8_k4_v32000   multi-candidate, B=16 G=8 k=4 V=32000, bf16 ~ N(0, 3^2);
+                           half the sequences share a random-length (1..3) prefix
+                           of candidate 0 across branches; each other token is the
+                           row argmax w.p. 0.6 else uniform, seed 4
+"""
+from __future__ import annotations
+
+import concurrent.futures as _fut
+import os
+
+import numpy as np
+
+# ----------------------------------------------------------- named workloads
+
+WORKLOADS = {
+    "stoch_b1_k4_v32000_f32": dict(mode="stochastic", B=1, k=4, V=32000, t_dtype="f32",
+                                   d_dtype="f32", t_std=2.0, d_noise=1.0, temperature=1.0,
+                                   seed=0),
+    "greedy_b64_k4_v128256": dict(mode="greedy", B=64, k=4, V=128256, t_dtype="bf16",
+                                  t_std=3.0, p_match=0.7, seed=2),
+    "stoch_b64_k4_v128256": dict(mode="stochastic", B=64, k=4, V=128256, t_dtype="bf16",
+                                 d_dtype="f32", t_std=3.0, d_noise=1.5, temperature=0.7,
+                                 seed=1),
+    "stoch_b256_k8_v128256": dict(mode="stochastic", B=256, k=8, V=128256, t_dtype="bf16",
+                                  d_dtype="bf16", t_std=3.0, d_noise=1.0, temperature=1.0,
+                                  seed=3),
+    "multi_b16_g8_k4_v32000": dict(mode="multi", B=16, G=8, k=4, V=32000, t_dtype="bf16",
+                                   t_std=3.0, p_match=0.6, p_shared=0.5, seed=4),
+}
+
+ELEM_BYTES = {"f32": 4, "bf16": 2}
+
+
+def _threads(threads: int | None) -> int:
+    return max(1, threads if threads else min(32, os.cpu_count() or 1))
+
+
+def _rng(seed: int, *stream: int) -> np.random.Generator:
+    """Independent Philox stream for (seed, *stream)."""
+    return np.random.Generator(np.random.Philox(np.random.SeedSequence([seed, *stream])))
+
+
+def _pmap(fn, n: int, threads: int | None):
+    t = _threads(threads)
+    if t == 1 or n < 2:
+        return [fn(j) for j in range(n)]
+    with _fut.ThreadPoolExecutor(t) as ex:
+        return list(ex.map(fn, range(n)))
+
+
+# ------------------------------------------------------------------- bf16
+
+def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round float32 to bf16 (round to nearest, ties to even); uint16 bits."""
+    b = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    bias = ((b >> np.uint32(16)) & np.uint32(1)) + np.uint32(0x7FFF)
+    return ((b + bias) >> np.uint32(16)).astype(np.uint16)
+
+
+def bf16_bits_to_f32(h: np.ndarray) -> np.ndarray:
+    """Exact widening of bf16 bit patterns to float32."""
+    return (np.asarray(h).astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+def to_f32(arr: np.ndarray, dtype: str) -> np.ndarray:
+    return bf16_bits_to_f32(arr) if dtype == "bf16" else np.asarray(arr, np.float32)
+
+
+def as_torch(arr: np.ndarray, dtype: str):
+    """numpy logits (f32 or bf16 bits) -> CPU torch tensor of that dtype."""
+    import torch
+
+    if dtype == "bf16":
+        return torch.from_numpy(np.ascontiguousarray(arr).view(np.int16)).view(torch.bfloat16)
+    return torch.from_numpy(np.ascontiguousarray(arr, dtype=np.float32))
+
+
+def from_torch(t) -> tuple[np.ndarray, str]:
+    """CPU torch tensor (bf16 or f32) -> (numpy array, dtype)."""
+    import torch
+
+    t = t.detach().cpu().contiguous()
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).numpy().view(np.uint16), "bf16"
+    if t.dtype == torch.float32:
+        return t.numpy(), "f32"
+    raise TypeError(f"unsupported logit dtype {t.dtype}")
+
+
+# -------------------------------------------------------------- primitives
+
+def normal_rows(seed: int, stream: int, rows: int, V: int, std: float,
+                threads: int | None = None) -> np.ndarray:
+    """[rows, V] float32, row r drawn from its own Philox stream (seed, stream, r)."""
+    out = np.empty((rows, V), np.float32)
+
+    def fill(r):
+        g = _rng(seed, stream, r)
+        g.standard_normal(V, dtype=np.float32, out=out[r])
+        out[r] *= np.float32(std)
+
+    _pmap(fill, rows, threads)
+    return out
+
+
+def sample_from_softmax(logits_f32: np.ndarray, temperature: float, seed: int, stream: int,
+                        threads: int | None = None) -> np.ndarray:
+    """One token per row from softmax(row / T), by inverse CDF (draft-model sampler)."""
+    rows, V = logits_f32.shape
+    T = float(np.float32(temperature))
+    out = np.empty(rows, np.int32)
+
+    def draw(r):
+        z = logits_f32[r].astype(np.float64) / T
+        w = np.exp(z - z.max())
+        c = np.cumsum(w)
+        u = _rng(seed, stream, r).random() * c[-1]
+        out[r] = min(int(np.searchsorted(c, u, side="right")), V - 1)
+
+    _pmap(draw, rows, threads)
+    return out
+
+
+def argmax_or_uniform(logits_f32: np.ndarray, p_match: float, seed: int, stream: int,
+                      threads: int | None = None) -> np.ndarray:
+    """Per row: the row's argmax with probability p_match, else a uniform token."""
+    rows, V = logits_f32.shape
+    am = np.empty(rows, np.int64)
+
+    def f(r):
+        am[r] = int(np.argmax(logits_f32[r]))
+
+    _pmap(f, rows, threads)
+    g = _rng(seed, stream)
+    hit = g.random(rows) < p_match
+    uni = g.integers(0, V, rows)
+    return np.where(hit, am, uni).astype(np.int32)
+
+
+# ------------------------------------------------------------- generators
+
+# stream ids inside one seed
+_S_TARGET, _S_DRAFT, _S_TOKENS, _S_SHARE = 1, 2, 3, 4
+
+
+def make_stochastic(B: int, k: int, V: int, t_dtype: str = "bf16", d_dtype: str = "bf16",
+                    t_std: float = 3.0, d_noise: float = 1.0, temperature: float = 1.0,
+                    seed: int = 0, threads: int | None = None) -> dict:
+    """Target [B,k+1,V] ~ N(0, t_std^2); draft [B,k,V] = target + N(0, d_noise^2);
+    draft tokens [B,k] drawn from softmax(draft / T)."""
+    t32 = normal_rows(seed, _S_TARGET, B * (k + 1), V, t_std, threads)
+    if t_dtype == "bf16":
+        target = f32_to_bf16_bits(t32)
+        t32 = bf16_bits_to_f32(target)
+    else:
+        target = t32
+    target = target.reshape(B, k + 1, V)
+    tv = t32.reshape(B, k + 1, V)[:, :k, :].reshape(B * k, V)
+    noise = normal_rows(seed, _S_DRAFT, B * k, V, d_noise, threads)
+    d32 = tv + noise
+    if d_dtype == "bf16":
+        draft = f32_to_bf16_bits(d32)
+        d32 = bf16_bits_to_f32(draft)
+    else:
+        draft = d32
+    draft = draft.reshape(B, k, V)
+    tokens = (sample_from_softmax(d32, temperature, seed, _S_TOKENS, threads).reshape(B, k)
+              if B * k else np.zeros((B, k), np.int32))
+    return dict(mode="stochastic", target=target, t_dtype=t_dtype, draft=draft,
+                d_dtype=d_dtype, tokens=tokens, temperature=float(np.float32(temperature)),
+                seed=seed, B=B, k=k, V=V)
+
+
+def make_greedy(B: int, k: int, V: int, t_dtype: str = "bf16", t_std: float = 3.0,
+                p_match: float = 0.7, seed: int = 0, threads: int | None = None) -> dict:
+    """Target [B,k+1,V] ~ N(0, t_std^2); draft token = row argmax w.p. p_match."""
+    t32 = normal_rows(seed, _S_TARGET, B * (k + 1), V, t_std, threads)
+    if t_dtype == "bf16":
+        target = f32_to_bf16_bits(t32)
+        t32 = bf16_bits_to_f32(target)
+    else:
+        target = t32
+    rows = t32.reshape(B, k + 1, V)[:, :k, :].reshape(B * k, V)
+    tokens = (argmax_or_uniform(rows, p_match, seed, _S_TOKENS, threads).reshape(B, k)
+              if B * k else np.zeros((B, k), np.int32))
+    return dict(mode="greedy", target=target.reshape(B, k + 1, V), t_dtype=t_dtype,
+                tokens=tokens, seed=seed, B=B, k=k, V=V)
+
+
+def make_multi(B: int, G: int, k: int, V: int, t_dtype: str = "bf16", t_std: float = 3.0,
+               p_match: float = 0.6, p_shared: float = 0.5, seed: int = 0,
+               threads: int | None = None) -> dict:
+    """Target [B,G,k+1,V] ~ N(0, t_std^2), i.i.d. rows; candidates [B,G,k].
+
+    With probability p_shared a sequence picks s in {1,2,3} and branches
+    1..G-1 copy branch 0's first s tokens; every other token is its own row's
+    argmax with probability p_match, else uniform.
+    """
+    t32 = normal_rows(seed, _S_TARGET, B * G * (k + 1), V, t_std, threads)
+    if t_dtype == "bf16":
+        target = f32_to_bf16_bits(t32)
+        t32 = bf16_bits_to_f32(target)
+    else:
+        target = t32
+    rows = t32.reshape(B, G, k + 1, V)[:, :, :k, :].reshape(B * G * k, V)
+    cand = (argmax_or_uniform(rows, p_match, seed, _S_TOKENS, threads).reshape(B, G, k)
+            if B * G * k else np.zeros((B, G, k), np.int32))
+    g = _rng(seed, _S_SHARE)
+    shared = g.random(B) < p_shared
+    s = g.integers(1, 4, B)
+    for b in range(B):
+        if shared[b] and k > 0:
+            m = min(int(s[b]), k)
+            cand[b, 1:, :m] = cand[b, 0, :m]
+    return dict(mode="multi", target=target.reshape(B, G, k + 1, V), t_dtype=t_dtype,
+                tokens=cand, seed=seed, B=B, G=G, k=k, V=V)
+
+
+def make(name: str, threads: int | None = None, **overrides) -> dict:
+    """Inputs of a named workload (``WORKLOADS``), with optional overrides
+    (e.g. ``B=4`` for a bounded sample of the same workload)."""
+    cfg = dict(WORKLOADS[name])
+    cfg.update(overrides)
+    mode = cfg.pop("mode")
+    if mode == "stochastic":
+        return make_stochastic(threads=threads, **cfg)
+    if mode == "greedy":
+        return make_greedy(threads=threads, **cfg)
+    if mode == "multi":
+        return make_multi(threads=threads, **cfg)
+    raise ValueError(mode)
+
+
+def logit_bytes(w: dict) -> int:
+    """Bytes of logits a verify call over workload ``w`` streams (all rows)."""
+    n = w["target"].size * ELEM_BYTES[w["t_dtype"]]
+    if "draft" in w:
+        n += w["draft"].size * ELEM_BYTES[w["d_dtype"]]
+    return n
