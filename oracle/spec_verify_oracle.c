@@ -45,7 +45,7 @@
  *  (c0, position, sequence, tag).  The acceptance draw of position i uses
  *  c0 = 0, word 0.  A per-vocabulary draw for entry x uses c0 = x >> 2 and
  *  output word x & 3.  Uniforms: u = (w >> 8) * 2^-24 in [0,1) for
- *  acceptance; u' = ((w >> 8) + 0.5) * 2^-24 in (0,1) and
+ *  acceptance; u' = ((w >> 9) + 0.5) * 2^-23 in (0,1) and
  *  g = -ln(-ln u') for Gumbel noise.  The pages fix none of this; it is the
  *  layout chosen so that the oracle and the GPU library draw the same
  *  numbers.
@@ -136,7 +136,9 @@ static double accept_uniform(uint32_t w)
 
 static double gumbel_noise(uint32_t w)
 {
-    double u = ((double)(w >> 8) + 0.5) * 0x1p-24; /* (0, 1) */
+    /* 23 random bits: ((w >> 9) + 0.5) * 2^-23 has at most 24 significant
+     * bits, so it is exact in fp32 as well as fp64 */
+    double u = ((double)(w >> 9) + 0.5) * 0x1p-23; /* (0, 1) */
     return -log(-log(u));
 }
 
