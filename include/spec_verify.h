@@ -1,0 +1,179 @@
+/*
+ * spec_verify.h -- C ABI of libspecverify.so, the B200 (sm_100a) library for
+ * the verify-and-accept step of speculative decoding.
+ *
+ * The step turns the target model's logits over a block of k drafted tokens
+ * (plus one more position) into an accepted length and the tokens to commit.
+ * "Accelerating Sonar through speculation" (Perplexity), section
+ * "Speculative decoding", stages "Acceptance" and "Target generation": the
+ * target runs over the draft, the longest acceptable prefix is found, and
+ * the target logits at the first mismatch, or after the last draft, give one
+ * more token, so n drafted tokens commit up to n + 1.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every pointer argument except those named "host" is a DEVICE pointer
+ *    owned by the caller.  The library allocates nothing and frees nothing.
+ *  - `stream` is a cudaStream_t passed as void*; NULL means the legacy
+ *    default stream.  Calls only enqueue work on it and never synchronise,
+ *    except spec_verify_read_device_status, which says so.
+ *  - Logit tensors are row-major with the vocabulary axis contiguous; the
+ *    other axes take strides in ELEMENTS (>= 0; 0 broadcasts one row).
+ *    Row starts that are all 16-byte aligned take the bulk-copy (TMA) path;
+ *    any other alignment takes a plain-load path with the same results.
+ *  - Token and output tensors are contiguous int32.
+ *  - Limits: 0 <= k <= 32, 1 <= V < 2^31, 1 <= G <= 64, B >= 0 (B = 0 is a
+ *    no-op).  Every row must hold at least one finite logit; -inf is allowed,
+ *    +inf and NaN are not valid logits.
+ *  - The return value reports host-side validation and launch errors only
+ *    (sv_status).  Errors seen on the device are recorded in the workspace
+ *    and read with spec_verify_read_device_status.
+ *  - Workspace: a caller-owned device buffer of at least
+ *    spec_verify_workspace_size(B, G, k, V) bytes, 16-byte aligned, zeroed
+ *    once (spec_verify_workspace_init) before its first use.  Each call
+ *    leaves it zeroed again except for the sticky device status word.  One
+ *    workspace must not be used by two calls that may run at the same time.
+ *    After SV_FLAG_TIMEOUT has been reported, re-initialise it.
+ */
+#ifndef SPEC_VERIFY_H
+#define SPEC_VERIFY_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Logit element types. */
+typedef enum { SV_F32 = 0, SV_BF16 = 1 } sv_dtype;
+
+/* Host-side return codes. */
+typedef enum {
+    SV_OK = 0,
+    SV_ERR_INVALID_ARG = 1,    /* null pointer, size out of range, bad dtype or temperature */
+    SV_ERR_MISALIGNED = 2,     /* pointer not aligned to its element size / workspace not 16-B */
+    SV_ERR_WORKSPACE = 3,      /* workspace_bytes smaller than spec_verify_workspace_size */
+    SV_ERR_CUDA = 4,           /* a CUDA runtime call or kernel launch failed */
+    SV_ERR_DEVICE_TIMEOUT = 5  /* reported through the device status word only */
+} sv_status;
+
+/* Bits of the sticky device status word. */
+#define SV_FLAG_INVALID_TOKEN 1u     /* a draft token was outside [0, V); it was rejected */
+#define SV_FLAG_RESIDUAL_FALLBACK 2u /* no positive residual mass; correction drawn from p_n */
+#define SV_FLAG_TIMEOUT 4u           /* a bounded device wait gave up; outputs are invalid */
+
+/*
+ * Bytes of workspace that calls with these sizes need (any mode, any dtype).
+ * Returns 0 for sizes outside the limits above.
+ */
+size_t spec_verify_workspace_size(int B, int G, int k, int V);
+
+/* Static, human-readable name of an sv_status value. */
+const char *spec_verify_status_string(int status);
+
+/*
+ * Zero a workspace (cudaMemsetAsync on `stream`).  Needed once after the
+ * buffer is allocated and again after a device timeout.
+ */
+int spec_verify_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Copy the sticky device status word (SV_FLAG_* bits) into *flags_host and,
+ * if `clear` is nonzero, reset it.  SYNCHRONISES `stream`.
+ */
+int spec_verify_read_device_status(void *workspace, uint32_t *flags_host, int clear,
+                                   void *stream);
+
+/*
+ * Stochastic verify (speculative rejection sampling).
+ *
+ * "Accelerating Sonar through speculation", section "Draft-Target":
+ * acceptance compares the full draft and target probability distributions,
+ * and the one logits set that the target emits after the accepted prefix is
+ * sampled for the next token.  The pages give no formula; the library
+ * implements the rejection-sampling rule of speculative sampling
+ * (Leviathan et al. 2023; Chen et al. 2023), which keeps the output law equal
+ * to the target's:
+ *   p_i = softmax(target[b,i,:] / T), q_i = softmax(draft[b,i,:] / T)
+ *   accept draft token x_i while u_i * q_i(x_i) < p_i(x_i)  (u_i < min(1, p/q))
+ *   n = first rejected position (or k)
+ *   n < k: token ~ normalize(max(0, p_n - q_n)); n = k: token ~ p_k
+ * Both draws are Gumbel-max over Philox4x32-10 noise (Salmon et al., SC'11)
+ * keyed by key = (seed lo, seed hi) and counter = (x >> 2, position,
+ * b + seq_offset, tag), word x & 3; tags ACCEPT = 0 (c0 = 0, word 0),
+ * CORRECTION = 1, BONUS = 2.  u_i = (w >> 8) 2^-24; Gumbel noise
+ * g = -ln(-ln(((w >> 9) + 0.5) 2^-23)).
+ *
+ * target_logits  [B, k+1, V], element (b,i,x) at b*t_stride_b + i*t_stride_pos + x
+ * draft_logits   [B, k, V],   element (b,i,x) at b*d_stride_b + i*d_stride_pos + x
+ * draft_tokens   [B, k] int32 (a token outside [0,V) is rejected and flagged)
+ * temperature    T > 0 and finite, applied to both target and draft
+ * seq_offset     added to b in the Philox counter (lets a sharded batch
+ *                reproduce the unsharded draws)
+ * accepted_len   [B] out: n in [0, k]
+ * out_tokens     [B, k+1] out: drafts 0..n-1, the sampled token at n, -1 after
+ * probs_out      [B, k, 2] out, may be NULL: p_i(x_i), q_i(x_i) (0 for an
+ *                invalid token)
+ */
+int spec_verify_stochastic(const void *target_logits, int t_dtype, int64_t t_stride_b,
+                           int64_t t_stride_pos, const void *draft_logits, int d_dtype,
+                           int64_t d_stride_b, int64_t d_stride_pos,
+                           const int32_t *draft_tokens, int B, int k, int V,
+                           float temperature, uint64_t seed, uint32_t seq_offset,
+                           int32_t *accepted_len, int32_t *out_tokens, float *probs_out,
+                           void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Greedy verify.
+ *
+ * "Accelerating Sonar through speculation", section "Speculative decoding":
+ * the longest acceptable prefix of the draft is kept and the target gives the
+ * next token for free.  Greedy acceptance: draft token i is accepted while it
+ * equals argmax_x target[b,i,x] (first maximum; -0 == +0).
+ *
+ * target_logits [B, k+1, V] (strides as above), draft_tokens [B, k];
+ * accepted_len [B] out; out_tokens [B, k+1] out: drafts 0..n-1, the argmax
+ * of row n at n, -1 after.
+ */
+int spec_verify_greedy(const void *target_logits, int t_dtype, int64_t t_stride_b,
+                       int64_t t_stride_pos, const int32_t *draft_tokens, int B, int k, int V,
+                       int32_t *accepted_len, int32_t *out_tokens, void *workspace,
+                       size_t workspace_bytes, void *stream);
+
+/*
+ * Multi-candidate (lookahead / Jacobi n-gram) greedy verify.
+ *
+ * "Lookahead decoding" news piece, section "Lookahead decoding breaks the
+ * order dependency" and steps 3-4: captured n-grams are validated against
+ * the target and the longest accepted one is appended.  Branch g of sequence
+ * b has its own rows target[b,g,0..k,:]; its accepted length n_g is its
+ * longest prefix equal to the row argmaxes; the chosen branch is the longest
+ * (lowest g on a tie; branch 0 when all are empty).
+ *
+ * target_logits [B, G, k+1, V], element (b,g,i,x) at
+ *   b*t_stride_b + g*t_stride_g + i*t_stride_pos + x
+ * cand_tokens [B, G, k]; best_candidate [B], accepted_len [B],
+ * out_tokens [B, k+1] out (candidate g*'s first n tokens, then the argmax of
+ * its row n, then -1).
+ */
+int spec_verify_multi_candidate(const void *target_logits, int t_dtype, int64_t t_stride_b,
+                                int64_t t_stride_g, int64_t t_stride_pos,
+                                const int32_t *cand_tokens, int B, int G, int k, int V,
+                                int32_t *best_candidate, int32_t *accepted_len,
+                                int32_t *out_tokens, void *workspace, size_t workspace_bytes,
+                                void *stream);
+
+/*
+ * Philox4x32-10 (Salmon et al., SC'11) on the device, as the verify kernels
+ * draw it: out[j] = Philox(counters[j], key = (seed lo, seed hi)).
+ * counters and out are device arrays of n uint32x4 (16-byte aligned).
+ */
+int spec_verify_philox4x32_10(const uint32_t *counters, int64_t n, uint64_t seed,
+                              uint32_t *out, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPEC_VERIFY_H */

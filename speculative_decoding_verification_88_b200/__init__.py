@@ -1,0 +1,289 @@
+"""speculative_decoding_verification_88_b200 -- verify-and-accept for
+speculative decoding on B200 (sm_100a).
+
+A thin ctypes binding over ``libspecverify.so`` (C ABI in
+``include/spec_verify.h``).  PyTorch is used only for device memory and
+streams: every step of the verify path runs in the library's CUDA kernels.
+There is no CPU fallback; calls raise if the library or a CUDA device is
+missing.
+
+    import speculative_decoding_verification_88_b200 as sv
+    r = sv.stochastic(target, draft, draft_tokens, temperature=0.7, seed=1)
+    r["accepted_len"], r["out_tokens"]
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+from .build import LIB_PATH
+
+SV_F32, SV_BF16 = 0, 1
+SV_FLAG_INVALID_TOKEN, SV_FLAG_RESIDUAL_FALLBACK, SV_FLAG_TIMEOUT = 1, 2, 4
+
+# Entry points declared in include/spec_verify.h.
+EXPORTS = (
+    "spec_verify_workspace_size", "spec_verify_status_string", "spec_verify_workspace_init",
+    "spec_verify_read_device_status", "spec_verify_stochastic", "spec_verify_greedy",
+    "spec_verify_multi_candidate", "spec_verify_philox4x32_10",
+)
+
+_lib = None
+_lock = threading.Lock()
+_launches = 0
+
+
+class SpecVerifyError(RuntimeError):
+    pass
+
+
+def library_path() -> str:
+    return LIB_PATH
+
+
+def load_library():
+    """Load libspecverify.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(LIB_PATH):
+            raise SpecVerifyError(
+                f"{LIB_PATH} is missing: build it with "
+                "`python -m speculative_decoding_verification_88_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        P, I, I64, U32, U64, SZ, F = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64,
+                                      ctypes.c_uint32, ctypes.c_uint64, ctypes.c_size_t,
+                                      ctypes.c_float)
+        lib.spec_verify_workspace_size.argtypes = [I, I, I, I]
+        lib.spec_verify_workspace_size.restype = SZ
+        lib.spec_verify_status_string.argtypes = [I]
+        lib.spec_verify_status_string.restype = ctypes.c_char_p
+        lib.spec_verify_workspace_init.argtypes = [P, SZ, P]
+        lib.spec_verify_workspace_init.restype = I
+        lib.spec_verify_read_device_status.argtypes = [P, ctypes.POINTER(U32), I, P]
+        lib.spec_verify_read_device_status.restype = I
+        lib.spec_verify_stochastic.argtypes = [
+            P, I, I64, I64, P, I, I64, I64, P, I, I, I, F, U64, U32, P, P, P, P, SZ, P]
+        lib.spec_verify_stochastic.restype = I
+        lib.spec_verify_greedy.argtypes = [P, I, I64, I64, P, I, I, I, P, P, P, SZ, P]
+        lib.spec_verify_greedy.restype = I
+        lib.spec_verify_multi_candidate.argtypes = [
+            P, I, I64, I64, I64, P, I, I, I, I, P, P, P, P, SZ, P]
+        lib.spec_verify_multi_candidate.restype = I
+        lib.spec_verify_philox4x32_10.argtypes = [P, I64, U64, P, P]
+        lib.spec_verify_philox4x32_10.restype = I
+        _lib = lib
+        return lib
+
+
+def status_string(code: int) -> str:
+    return load_library().spec_verify_status_string(int(code)).decode()
+
+
+def _check(code: int, what: str):
+    if code != 0:
+        raise SpecVerifyError(f"{what}: {status_string(code)}")
+
+
+def launch_count() -> int:
+    """Number of verify/philox calls (one kernel launch each) so far."""
+    return _launches
+
+
+def _count():
+    global _launches
+    _launches += 1
+
+
+def workspace_size(B: int, G: int, k: int, V: int) -> int:
+    return int(load_library().spec_verify_workspace_size(B, G, k, V))
+
+
+class Workspace:
+    """A zero-initialised device workspace, grown on demand (one per stream)."""
+
+    def __init__(self, device=None, nbytes: int = 0):
+        self.device = torch.device(device if device is not None else "cuda")
+        self.buf = None
+        self.ensure(nbytes)
+
+    @property
+    def nbytes(self) -> int:
+        return 0 if self.buf is None else self.buf.numel()
+
+    def ensure(self, nbytes: int, stream=None):
+        if nbytes <= self.nbytes:
+            return self
+        self.buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=self.device)
+        _check(load_library().spec_verify_workspace_init(
+            self.buf.data_ptr(), self.buf.numel(), _stream_ptr(stream, self.device)),
+            "spec_verify_workspace_init")
+        return self
+
+    def reset(self, stream=None):
+        if self.buf is not None:
+            _check(load_library().spec_verify_workspace_init(
+                self.buf.data_ptr(), self.buf.numel(), _stream_ptr(stream, self.device)),
+                "spec_verify_workspace_init")
+
+    def device_status(self, clear: bool = True, stream=None) -> int:
+        """Sticky SV_FLAG_* bits of the device (synchronises the stream)."""
+        v = ctypes.c_uint32(0)
+        _check(load_library().spec_verify_read_device_status(
+            self.buf.data_ptr(), ctypes.byref(v), int(clear), _stream_ptr(stream, self.device)),
+            "spec_verify_read_device_status")
+        return int(v.value)
+
+
+_default_ws: dict = {}
+
+
+def default_workspace(device) -> Workspace:
+    key = (torch.device(device), torch.cuda.current_stream(device).cuda_stream)
+    ws = _default_ws.get(key)
+    if ws is None:
+        ws = _default_ws[key] = Workspace(device)
+    return ws
+
+
+def _stream_ptr(stream, device):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return SV_F32
+    if t.dtype == torch.bfloat16:
+        return SV_BF16
+    raise TypeError(f"logits must be float32 or bfloat16, got {t.dtype}")
+
+
+def _logits(t: torch.Tensor, ndim: int, name: str):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must be {ndim}-d, got shape {tuple(t.shape)}")
+    if t.shape[-1] > 1 and t.stride(-1) != 1:
+        raise ValueError(f"{name}: the vocabulary axis must be contiguous")
+    return _dtype_code(t), t.stride()
+
+
+def _tokens(t: torch.Tensor, shape, device, name: str) -> torch.Tensor:
+    if not isinstance(t, torch.Tensor) or t.device != device or t.dtype != torch.int32:
+        raise TypeError(f"{name} must be an int32 tensor on {device}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t.contiguous()
+
+
+def _out(out, key, shape, dtype, device):
+    if out is not None and key in out:
+        t = out[key]
+        if tuple(t.shape) != tuple(shape) or t.dtype != dtype or not t.is_contiguous():
+            raise ValueError(f"out[{key!r}] must be a contiguous {dtype} tensor {tuple(shape)}")
+        return t
+    return torch.empty(shape, dtype=dtype, device=device)
+
+
+def stochastic(target: torch.Tensor, draft: torch.Tensor, draft_tokens: torch.Tensor,
+               temperature: float, seed: int, seq_offset: int = 0, *, probs: bool = False,
+               out: dict | None = None, workspace: Workspace | None = None,
+               stream=None) -> dict:
+    """Stochastic verify: target [B,k+1,V], draft [B,k,V], draft_tokens [B,k].
+
+    Returns accepted_len [B], out_tokens [B,k+1] (and probs [B,k,2] when
+    asked), all on the device; nothing is synchronised.
+    """
+    lib = load_library()
+    tc, (tsb, tsp, _) = _logits(target, 3, "target")
+    dc, (dsb, dsp, _) = _logits(draft, 3, "draft")
+    B, kp1, V = target.shape
+    k = kp1 - 1
+    if tuple(draft.shape) != (B, k, V) or draft.device != target.device:
+        raise ValueError("draft must be [B, k, V] on the target's device")
+    dev = target.device
+    tok = _tokens(draft_tokens, (B, k), dev, "draft_tokens")
+    res = {"accepted_len": _out(out, "accepted_len", (B,), torch.int32, dev),
+           "out_tokens": _out(out, "out_tokens", (B, k + 1), torch.int32, dev)}
+    if probs:
+        res["probs"] = _out(out, "probs", (B, k, 2), torch.float32, dev)
+    ws = workspace or default_workspace(dev)
+    ws.ensure(workspace_size(B, 1, k, V), stream)
+    with torch.cuda.device(dev):
+        code = lib.spec_verify_stochastic(
+            target.data_ptr(), tc, tsb, tsp, draft.data_ptr(), dc, dsb, dsp, tok.data_ptr(),
+            B, k, V, float(temperature), int(seed) & (2**64 - 1), int(seq_offset) & 0xFFFFFFFF,
+            res["accepted_len"].data_ptr(), res["out_tokens"].data_ptr(),
+            res["probs"].data_ptr() if probs else None, ws.buf.data_ptr(), ws.nbytes,
+            _stream_ptr(stream, dev))
+    _check(code, "spec_verify_stochastic")
+    _count()
+    return res
+
+
+def greedy(target: torch.Tensor, draft_tokens: torch.Tensor, *, out: dict | None = None,
+           workspace: Workspace | None = None, stream=None) -> dict:
+    """Greedy verify: target [B,k+1,V], draft_tokens [B,k]."""
+    lib = load_library()
+    tc, (tsb, tsp, _) = _logits(target, 3, "target")
+    B, kp1, V = target.shape
+    k = kp1 - 1
+    dev = target.device
+    tok = _tokens(draft_tokens, (B, k), dev, "draft_tokens")
+    res = {"accepted_len": _out(out, "accepted_len", (B,), torch.int32, dev),
+           "out_tokens": _out(out, "out_tokens", (B, k + 1), torch.int32, dev)}
+    ws = workspace or default_workspace(dev)
+    ws.ensure(workspace_size(B, 1, k, V), stream)
+    with torch.cuda.device(dev):
+        code = lib.spec_verify_greedy(
+            target.data_ptr(), tc, tsb, tsp, tok.data_ptr(), B, k, V,
+            res["accepted_len"].data_ptr(), res["out_tokens"].data_ptr(), ws.buf.data_ptr(),
+            ws.nbytes, _stream_ptr(stream, dev))
+    _check(code, "spec_verify_greedy")
+    _count()
+    return res
+
+
+def multi_candidate(target: torch.Tensor, cand_tokens: torch.Tensor, *, out: dict | None = None,
+                    workspace: Workspace | None = None, stream=None) -> dict:
+    """Multi-candidate verify: target [B,G,k+1,V], cand_tokens [B,G,k]."""
+    lib = load_library()
+    tc, (tsb, tsg, tsp, _) = _logits(target, 4, "target")
+    B, G, kp1, V = target.shape
+    k = kp1 - 1
+    dev = target.device
+    tok = _tokens(cand_tokens, (B, G, k), dev, "cand_tokens")
+    res = {"best_candidate": _out(out, "best_candidate", (B,), torch.int32, dev),
+           "accepted_len": _out(out, "accepted_len", (B,), torch.int32, dev),
+           "out_tokens": _out(out, "out_tokens", (B, k + 1), torch.int32, dev)}
+    ws = workspace or default_workspace(dev)
+    ws.ensure(workspace_size(B, G, k, V), stream)
+    with torch.cuda.device(dev):
+        code = lib.spec_verify_multi_candidate(
+            target.data_ptr(), tc, tsb, tsg, tsp, tok.data_ptr(), B, G, k, V,
+            res["best_candidate"].data_ptr(), res["accepted_len"].data_ptr(),
+            res["out_tokens"].data_ptr(), ws.buf.data_ptr(), ws.nbytes, _stream_ptr(stream, dev))
+    _check(code, "spec_verify_multi_candidate")
+    _count()
+    return res
+
+
+def philox4x32_10(counters: torch.Tensor, seed: int, stream=None) -> torch.Tensor:
+    """Device Philox4x32-10 of each counter row ([n,4] int32 bit patterns)."""
+    lib = load_library()
+    if counters.dtype != torch.int32 or counters.dim() != 2 or counters.shape[1] != 4:
+        raise TypeError("counters must be an int32 tensor [n, 4] (uint32 bit patterns)")
+    c = counters.contiguous()
+    out = torch.empty_like(c)
+    with torch.cuda.device(c.device):
+        code = lib.spec_verify_philox4x32_10(c.data_ptr(), c.shape[0], int(seed) & (2**64 - 1),
+                                              out.data_ptr(), _stream_ptr(stream, c.device))
+    _check(code, "spec_verify_philox4x32_10")
+    _count()
+    return out

@@ -1,0 +1,293 @@
+// sv_api.cu -- the C ABI of libspecverify.so (include/spec_verify.h):
+// argument validation, chunk planning, workspace layout and kernel dispatch.
+// Host code only; every step of the verify path runs in sv_kernels.cu.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "spec_verify.h"
+#include "sv_internal.h"
+
+namespace sv {
+
+Plan plan_chunks(long long rows, int V, int bpe) {
+  // Largest chunk (multiple of 8 entries) whose unit of work fits one stage.
+  int chmax = (kStageBytes / bpe) & ~7;
+  if (chmax < 8) chmax = 8;
+  long long nch = (V + chmax - 1) / chmax;
+  // Small calls: split rows finer (chunks of >= 512 entries) so that about
+  // 2048 chunks spread over the SMs.
+  const long long want = 2048;
+  if (rows > 0 && rows * nch < want) {
+    const long long finer = (want + rows - 1) / rows;
+    const long long most = (V + 511) / 512;
+    const long long n2 = finer < most ? finer : most;
+    if (n2 > nch) nch = n2;
+  }
+  long long ch = (V + nch - 1) / nch;
+  ch = (ch + 7) / 8 * 8;
+  nch = (V + ch - 1) / ch;
+  return Plan{static_cast<int>(ch), static_cast<int>(nch)};
+}
+
+namespace {
+
+constexpr size_t kCtrlBytes = sizeof(Ctrl);
+
+int elem_bytes(int dtype) { return dtype == SV_BF16 ? 2 : 4; }
+bool dtype_ok(int dtype) { return dtype == SV_F32 || dtype == SV_BF16; }
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+bool stride16(long long stride, int es) { return ((stride * es) % 16) == 0; }
+
+size_t seq_bytes(int B) { return static_cast<size_t>(B) * sizeof(SeqRec); }
+
+size_t stochastic_part_bytes(int B, int k, int V, int bpe) {
+  const Plan pl = plan_chunks(static_cast<long long>(B) * k, V, bpe);
+  return static_cast<size_t>(B) * k * pl.nch * sizeof(float4);
+}
+
+size_t argmax_key_bytes(int B, int G, int k) {
+  return static_cast<size_t>(B) * G * (k + 1) * sizeof(unsigned long long);
+}
+
+bool sizes_ok(int B, int G, int k, int V) {
+  return B >= 0 && G >= 1 && G <= 64 && k >= 0 && k <= 32 && V >= 1;
+}
+
+int sm_count() {
+  static int cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+  if (dev >= 0 && dev < 64) cached[dev] = n;
+  return n;
+}
+
+struct WsView {
+  Ctrl* ctrl;
+  SeqRec* seq;
+  void* tail;
+};
+
+WsView carve(void* ws, int B) {
+  unsigned char* base = static_cast<unsigned char*>(ws);
+  return WsView{reinterpret_cast<Ctrl*>(base), reinterpret_cast<SeqRec*>(base + kCtrlBytes),
+                base + kCtrlBytes + seq_bytes(B)};
+}
+
+}  // namespace
+}  // namespace sv
+
+using namespace sv;
+
+extern "C" size_t spec_verify_workspace_size(int B, int G, int k, int V) {
+  if (!sizes_ok(B, G, k, V)) return 0;
+  size_t tail = argmax_key_bytes(B, G, k);
+  if (G == 1) {
+    for (int bpe : {4, 6, 8}) {
+      const size_t s = stochastic_part_bytes(B, k, V, bpe);
+      if (s > tail) tail = s;
+    }
+  }
+  const size_t total = kCtrlBytes + seq_bytes(B) + tail;
+  return (total + 255) / 256 * 256;
+}
+
+extern "C" const char* spec_verify_status_string(int status) {
+  switch (status) {
+    case SV_OK: return "SV_OK";
+    case SV_ERR_INVALID_ARG: return "SV_ERR_INVALID_ARG: invalid argument";
+    case SV_ERR_MISALIGNED: return "SV_ERR_MISALIGNED: pointer not aligned";
+    case SV_ERR_WORKSPACE: return "SV_ERR_WORKSPACE: workspace too small";
+    case SV_ERR_CUDA: return "SV_ERR_CUDA: CUDA runtime error";
+    case SV_ERR_DEVICE_TIMEOUT: return "SV_ERR_DEVICE_TIMEOUT: a device wait timed out";
+    default: return "unknown spec_verify status";
+  }
+}
+
+extern "C" int spec_verify_workspace_init(void* workspace, size_t workspace_bytes,
+                                          void* stream) {
+  if (!workspace) return SV_ERR_INVALID_ARG;
+  if (!aligned(workspace, 16)) return SV_ERR_MISALIGNED;
+  if (cudaMemsetAsync(workspace, 0, workspace_bytes, static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return SV_ERR_CUDA;
+  return SV_OK;
+}
+
+extern "C" int spec_verify_read_device_status(void* workspace, uint32_t* flags_host, int clear,
+                                              void* stream) {
+  if (!workspace || !flags_host) return SV_ERR_INVALID_ARG;
+  if (!aligned(workspace, 16)) return SV_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Ctrl* ctrl = static_cast<Ctrl*>(workspace);
+  uint32_t v = 0;
+  if (cudaMemcpyAsync(&v, &ctrl->flags, sizeof v, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return SV_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return SV_ERR_CUDA;
+  *flags_host = v;
+  if (clear && cudaMemsetAsync(&ctrl->flags, 0, sizeof v, st) != cudaSuccess) return SV_ERR_CUDA;
+  return SV_OK;
+}
+
+extern "C" int spec_verify_stochastic(const void* target_logits, int t_dtype,
+                                      int64_t t_stride_b, int64_t t_stride_pos,
+                                      const void* draft_logits, int d_dtype, int64_t d_stride_b,
+                                      int64_t d_stride_pos, const int32_t* draft_tokens, int B,
+                                      int k, int V, float temperature, uint64_t seed,
+                                      uint32_t seq_offset, int32_t* accepted_len,
+                                      int32_t* out_tokens, float* probs_out, void* workspace,
+                                      size_t workspace_bytes, void* stream) {
+  if (!sizes_ok(B, 1, k, V)) return SV_ERR_INVALID_ARG;
+  if (B == 0) return SV_OK;
+  if (!target_logits || !accepted_len || !out_tokens || !workspace) return SV_ERR_INVALID_ARG;
+  if (k > 0 && (!draft_logits || !draft_tokens)) return SV_ERR_INVALID_ARG;
+  if (!dtype_ok(t_dtype) || !dtype_ok(d_dtype)) return SV_ERR_INVALID_ARG;
+  if (!(temperature > 0.0f) || !std::isfinite(temperature) || !std::isnormal(temperature))
+    return SV_ERR_INVALID_ARG;
+  if (t_stride_b < 0 || t_stride_pos < 0 || d_stride_b < 0 || d_stride_pos < 0)
+    return SV_ERR_INVALID_ARG;
+  const int st = elem_bytes(t_dtype), sd = elem_bytes(d_dtype);
+  if (!aligned(target_logits, st) || (k > 0 && !aligned(draft_logits, sd)) ||
+      !aligned(accepted_len, 4) || !aligned(out_tokens, 4) ||
+      (k > 0 && !aligned(draft_tokens, 4)) || (probs_out && !aligned(probs_out, 4)) ||
+      !aligned(workspace, 16))
+    return SV_ERR_MISALIGNED;
+  if (workspace_bytes < spec_verify_workspace_size(B, 1, k, V)) return SV_ERR_WORKSPACE;
+
+  const int grid = sm_count();
+  if (grid <= 0) return SV_ERR_CUDA;
+  const Plan pl = plan_chunks(static_cast<long long>(B) * k, V, st + sd);
+  const long long p1 = static_cast<long long>(k) * pl.nch;
+  long long lag = 0;
+  if (p1 > 0) {
+    lag = (static_cast<long long>(kStages) * grid + p1 - 1) / p1 + 1;
+    if (lag > B) lag = B;
+  }
+  const long long slot_items = static_cast<long long>(k + 1) * pl.nch;
+  const long long total = (static_cast<long long>(B) + lag) * slot_items;
+  if (total >= (1ll << 31)) return SV_ERR_INVALID_ARG;
+
+  const bool tma = aligned(target_logits, 16) && stride16(t_stride_b, st) &&
+                   stride16(t_stride_pos, st) &&
+                   (k == 0 || (aligned(draft_logits, 16) && stride16(d_stride_b, sd) &&
+                               stride16(d_stride_pos, sd)));
+
+  const WsView ws = carve(workspace, B);
+  StochParams p{};
+  p.tgt = target_logits;
+  p.t_sb = t_stride_b;
+  p.t_sp = t_stride_pos;
+  p.drf = draft_logits;
+  p.d_sb = d_stride_b;
+  p.d_sp = d_stride_pos;
+  p.tokens = draft_tokens;
+  p.B = B;
+  p.k = k;
+  p.V = V;
+  p.invT = 1.0f / temperature;
+  p.c2 = 1.4426950408889634f / temperature;
+  p.key0 = static_cast<unsigned int>(seed & 0xffffffffull);
+  p.key1 = static_cast<unsigned int>(seed >> 32);
+  p.seq_offset = seq_offset;
+  p.accepted_len = accepted_len;
+  p.out_tokens = out_tokens;
+  p.probs = probs_out;
+  p.ch = pl.ch;
+  p.nch = pl.nch;
+  p.lag = static_cast<int>(lag);
+  p.slot_items = static_cast<unsigned int>(slot_items);
+  p.total = static_cast<unsigned int>(total);
+  p.ctrl = ws.ctrl;
+  p.seq = ws.seq;
+  p.part = static_cast<float4*>(ws.tail);
+  const cudaError_t e = launch_stochastic(p, t_dtype, d_dtype, tma, grid, kernel_smem_bytes(),
+                                          static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SV_OK : SV_ERR_CUDA;
+}
+
+static int argmax_call(const void* target_logits, int t_dtype, int64_t sb, int64_t sg,
+                       int64_t sp, const int32_t* tokens, int B, int G, int k, int V,
+                       int32_t* best_g, int32_t* accepted_len, int32_t* out_tokens,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+  if (!sizes_ok(B, G, k, V)) return SV_ERR_INVALID_ARG;
+  if (B == 0) return SV_OK;
+  if (!target_logits || !accepted_len || !out_tokens || !workspace) return SV_ERR_INVALID_ARG;
+  if (k > 0 && !tokens) return SV_ERR_INVALID_ARG;
+  if (!dtype_ok(t_dtype)) return SV_ERR_INVALID_ARG;
+  if (sb < 0 || sg < 0 || sp < 0) return SV_ERR_INVALID_ARG;
+  const int st = elem_bytes(t_dtype);
+  if (!aligned(target_logits, st) || !aligned(accepted_len, 4) || !aligned(out_tokens, 4) ||
+      (k > 0 && !aligned(tokens, 4)) || (best_g && !aligned(best_g, 4)) ||
+      !aligned(workspace, 16))
+    return SV_ERR_MISALIGNED;
+  if (workspace_bytes < spec_verify_workspace_size(B, G, k, V)) return SV_ERR_WORKSPACE;
+
+  const int grid = sm_count();
+  if (grid <= 0) return SV_ERR_CUDA;
+  const long long rows = static_cast<long long>(B) * G * (k + 1);
+  const Plan pl = plan_chunks(rows, V, st);
+  const long long total = rows * pl.nch;
+  if (total >= (1ll << 31)) return SV_ERR_INVALID_ARG;
+  const bool tma =
+      aligned(target_logits, 16) && stride16(sb, st) && stride16(sg, st) && stride16(sp, st);
+
+  const WsView ws = carve(workspace, B);
+  ArgmaxParams p{};
+  p.tgt = target_logits;
+  p.sb = sb;
+  p.sg = sg;
+  p.sp = sp;
+  p.tokens = tokens;
+  p.B = B;
+  p.G = G;
+  p.k = k;
+  p.V = V;
+  p.best_g = best_g;
+  p.accepted_len = accepted_len;
+  p.out_tokens = out_tokens;
+  p.ch = pl.ch;
+  p.nch = pl.nch;
+  p.total = static_cast<unsigned int>(total);
+  p.ctrl = ws.ctrl;
+  p.seq = ws.seq;
+  p.rowkey = static_cast<unsigned long long*>(ws.tail);
+  const cudaError_t e = launch_argmax(p, t_dtype, tma, grid, kernel_smem_bytes(),
+                                      static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SV_OK : SV_ERR_CUDA;
+}
+
+extern "C" int spec_verify_greedy(const void* target_logits, int t_dtype, int64_t t_stride_b,
+                                  int64_t t_stride_pos, const int32_t* draft_tokens, int B, int k,
+                                  int V, int32_t* accepted_len, int32_t* out_tokens,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+  return argmax_call(target_logits, t_dtype, t_stride_b, 0, t_stride_pos, draft_tokens, B, 1, k,
+                     V, nullptr, accepted_len, out_tokens, workspace, workspace_bytes, stream);
+}
+
+extern "C" int spec_verify_multi_candidate(const void* target_logits, int t_dtype,
+                                           int64_t t_stride_b, int64_t t_stride_g,
+                                           int64_t t_stride_pos, const int32_t* cand_tokens,
+                                           int B, int G, int k, int V, int32_t* best_candidate,
+                                           int32_t* accepted_len, int32_t* out_tokens,
+                                           void* workspace, size_t workspace_bytes,
+                                           void* stream) {
+  if (!best_candidate && B > 0) return SV_ERR_INVALID_ARG;
+  return argmax_call(target_logits, t_dtype, t_stride_b, t_stride_g, t_stride_pos, cand_tokens, B,
+                     G, k, V, best_candidate, accepted_len, out_tokens, workspace,
+                     workspace_bytes, stream);
+}
+
+extern "C" int spec_verify_philox4x32_10(const uint32_t* counters, int64_t n, uint64_t seed,
+                                         uint32_t* out, void* stream) {
+  if (n < 0 || (n > 0 && (!counters || !out))) return SV_ERR_INVALID_ARG;
+  if (n == 0) return SV_OK;
+  if (!aligned(counters, 16) || !aligned(out, 16)) return SV_ERR_MISALIGNED;
+  const cudaError_t e = launch_philox(
+      reinterpret_cast<const uint4*>(counters), n, static_cast<unsigned int>(seed & 0xffffffffull),
+      static_cast<unsigned int>(seed >> 32), reinterpret_cast<uint4*>(out),
+      static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SV_OK : SV_ERR_CUDA;
+}

@@ -1,0 +1,99 @@
+// sv_internal.h -- parameter blocks and work plan shared by the C ABI layer
+// (sv_api.cu) and the kernels (sv_kernels.cu).  Not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+
+namespace sv {
+
+// ---- CTA shape of the persistent verify kernels -------------------------
+// warp 0: producer (one thread: ticket, waits, bulk copies)
+// warps 1..kComputeWarps: compute (reduce one chunk held in shared memory)
+// last warp: epilogue (publish chunk partials, finalize sequences)
+constexpr int kComputeWarps = 8;
+constexpr int kThreads = 32 * (kComputeWarps + 2);
+constexpr int kStages = 4;
+constexpr int kStageBytes = 48 * 1024;
+
+// Device-wide control words at the start of the workspace (256 bytes).
+struct Ctrl {
+  unsigned int ticket;  // next work ticket (reset by the last CTA to leave)
+  unsigned int exits;   // CTAs that took their last ticket
+  unsigned int flags;   // sticky SV_FLAG_* bits
+  unsigned int pad[61];
+};
+static_assert(sizeof(Ctrl) == 256, "Ctrl must be 256 bytes");
+
+// Per-sequence record (64 bytes).  Counters, flag and key are zero between
+// calls; the kernel that raises them also lowers them.
+struct SeqRec {
+  unsigned int cnt1;       // phase-1 chunk arrivals
+  unsigned int cnt2;       // phase-2 chunk arrivals
+  unsigned int ready;      // phase 1 finalized (accepted length known)
+  int n;                   // accepted length
+  float mt, ist, md, isd;  // row n: max (log2 units) and 1/sum of p and q
+  unsigned long long key;  // phase-2 Gumbel-max key (score, ~index)
+  unsigned int pad[6];
+};
+static_assert(sizeof(SeqRec) == 64, "SeqRec must be 64 bytes");
+
+// Chunking of the vocabulary axis: `nch` chunks of `ch` elements (the last
+// one shorter); ch is a multiple of 8 so that every chunk of a 16-byte
+// aligned row starts 16-byte aligned for both 2- and 4-byte elements.
+struct Plan {
+  int ch;
+  int nch;
+};
+
+// rows: rows (or row pairs) a call reduces; bpe: bytes per vocab entry of
+// one unit of work (target + draft bytes for a stochastic pair).
+Plan plan_chunks(long long rows, int V, int bpe);
+
+struct StochParams {
+  const void* tgt;
+  long long t_sb, t_sp;
+  const void* drf;
+  long long d_sb, d_sp;
+  const int* tokens;  // [B, k]
+  int B, k, V;
+  float invT;  // 1 / T
+  float c2;    // log2(e) / T: logit -> log2-domain scale
+  unsigned int key0, key1, seq_offset;
+  int* accepted_len;
+  int* out_tokens;
+  float* probs;  // nullable
+  int ch, nch, lag;
+  unsigned int slot_items;  // (k + 1) * nch tickets per slot
+  unsigned int total;       // tickets
+  Ctrl* ctrl;
+  SeqRec* seq;
+  float4* part;  // [B][k][nch] chunk partials (mt, st, md, sd)
+};
+
+struct ArgmaxParams {
+  const void* tgt;
+  long long sb, sg, sp;
+  const int* tokens;  // [B, G, k]
+  int B, G, k, V;
+  int* best_g;  // nullable
+  int* accepted_len;
+  int* out_tokens;
+  int ch, nch;
+  unsigned int total;
+  Ctrl* ctrl;
+  SeqRec* seq;
+  unsigned long long* rowkey;  // [B][G][k+1] argmax keys
+};
+
+// dtype codes follow sv_dtype (0 = f32, 1 = bf16).  Return cudaError_t.
+cudaError_t launch_stochastic(const StochParams& p, int t_dtype, int d_dtype, bool tma,
+                              int grid, size_t smem, cudaStream_t stream);
+cudaError_t launch_argmax(const ArgmaxParams& p, int t_dtype, bool tma, int grid, size_t smem,
+                          cudaStream_t stream);
+cudaError_t launch_philox(const uint4* ctr, long long n, unsigned int key0, unsigned int key1,
+                          uint4* out, cudaStream_t stream);
+size_t kernel_smem_bytes();
+
+}  // namespace sv

@@ -1,0 +1,311 @@
+"""GPU parity: the CUDA library (through its C ABI) against the CPU oracle.
+
+Greedy, multi-candidate and Philox results must be bit-exact.  Stochastic
+results: accepted lengths and tokens must match exactly, except for
+sequences where a decision the oracle took was a near tie (an acceptance
+margin |u - p/q| < 1e-5 at a position the oracle examined, or a Gumbel-max
+score gap < 1e-5 in the sampled row); those are counted.  p_i(x_i) and
+q_i(x_i) must agree within 1e-5 absolute.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import speculative_decoding_verification_88_b200 as sv
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+TOL_PROB = 1e-5
+TOL_MARGIN = 1e-5
+TOL_GAP = 1e-5
+THREADS = os.cpu_count() or 1
+
+
+@pytest.fixture(scope="module")
+def dev():
+    from speculative_decoding_verification_88_b200 import build
+
+    build.build()
+    assert torch.cuda.is_available(), "the GPU tests need a CUDA device"
+    return torch.device("cuda:0")
+
+
+def to_dev(arr, dtype, dev):
+    return workloads.as_torch(arr, dtype).to(dev)
+
+
+def near_ties(o, k):
+    n = o["accepted_len"]
+    near = o["gaps"] < TOL_GAP
+    if k > 0:
+        for b in range(len(n)):
+            upto = min(int(n[b]), k - 1)
+            near[b] |= bool((o["margins"][b, : upto + 1] < TOL_MARGIN).any())
+    return near
+
+
+def compare_stochastic(r, o, k, what=""):
+    acc = r["accepted_len"].cpu().numpy()
+    tok = r["out_tokens"].cpu().numpy()
+    if "probs" in r and k > 0:
+        np.testing.assert_allclose(r["probs"].cpu().numpy(), o["probs"], atol=TOL_PROB, rtol=0,
+                                   err_msg=what)
+    near = near_ties(o, k)
+    mism = (acc != o["accepted_len"]) | (tok != o["out_tokens"]).any(axis=1)
+    bad = np.nonzero(mism & ~near)[0]
+    assert bad.size == 0, (
+        f"{what}: {bad.size} mismatches outside near ties, first b={bad[0]}: gpu n={acc[bad[0]]} "
+        f"tok={tok[bad[0]]} oracle n={o['accepted_len'][bad[0]]} tok={o['out_tokens'][bad[0]]} "
+        f"margins={o['margins'][bad[0]]} gap={o['gaps'][bad[0]]}")
+    return int(near.sum()), int((mism & near).sum())
+
+
+def run_stochastic(w, dev, seed=None, seq_offset=0, **views):
+    T = w["temperature"]
+    seed = w["seed"] if seed is None else seed
+    t = views.get("t", to_dev(w["target"], w["t_dtype"], dev))
+    d = views.get("d", to_dev(w["draft"], w["d_dtype"], dev))
+    tok = torch.from_numpy(w["tokens"]).to(dev)
+    r = sv.stochastic(t, d, tok, T, seed, seq_offset, probs=True)
+    o = oracle.verify_stochastic(views.get("t_np", w["target"]), w["t_dtype"],
+                                 views.get("d_np", w["draft"]), w["d_dtype"], w["tokens"], T,
+                                 seed, seq_offset, threads=THREADS)
+    torch.cuda.synchronize()
+    return r, o
+
+
+# ------------------------------------------------------------------ Philox
+
+def test_philox_matches_oracle(dev):
+    rng = np.random.default_rng(0)
+    ctr = rng.integers(0, 2**32, size=(1 << 20, 4), dtype=np.uint64).astype(np.uint32)
+    ctr[:4] = [[0, 0, 0, 0], [0xFFFFFFFF] * 4, [1, 2, 3, 4], [0, 7, 9, 2]]
+    for seed in (0, 1, 0xFFFFFFFFFFFFFFFF, 0xA4093822299F31D0):
+        want = oracle.philox4x32_10(ctr, seed)
+        got = sv.philox4x32_10(torch.from_numpy(ctr.view(np.int32)).to(dev), seed)
+        assert np.array_equal(got.cpu().numpy().view(np.uint32), want)
+
+
+# ------------------------------------------------------------------ greedy
+
+def tie_heavy(rng, shape):
+    x = rng.integers(-4, 5, size=shape).astype(np.float32)
+    x[rng.random(shape) < 0.03] = -np.inf
+    z = x == 0
+    x[z & (rng.random(shape) < 0.5)] = -0.0
+    return x
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("B,k,V", [(1, 0, 1), (3, 1, 2), (129, 4, 7), (3, 8, 8), (1, 4, 9),
+                                   (3, 32, 31), (129, 2, 33), (3, 4, 4095), (1, 8, 4097),
+                                   (5, 3, 32000), (2, 4, 128256)])
+def test_greedy_parity_shapes(dev, dtype, B, k, V):
+    rng = np.random.default_rng(B * 1000 + k * 10 + V)
+    if V <= 64:
+        x = tie_heavy(rng, (B, k + 1, V))
+    else:
+        x = rng.standard_normal((B, k + 1, V)).astype(np.float32) * 3
+    arr = workloads.f32_to_bf16_bits(x) if dtype == "bf16" else x
+    xv = workloads.to_f32(arr, dtype)
+    am = np.argmax(xv, -1)
+    tok = np.where(rng.random((B, k)) < 0.75, am[:, :k], rng.integers(-2, V + 2, (B, k)))
+    tok = tok.astype(np.int32)
+    r = sv.greedy(to_dev(arr, dtype, dev), torch.from_numpy(tok).to(dev))
+    o = oracle.verify_greedy(arr, dtype, tok, threads=THREADS)
+    np.testing.assert_array_equal(r["accepted_len"].cpu().numpy(), o["accepted_len"])
+    np.testing.assert_array_equal(r["out_tokens"].cpu().numpy(), o["out_tokens"])
+
+
+def test_greedy_strided_unaligned_and_broadcast(dev):
+    rng = np.random.default_rng(3)
+    B, k, V = 6, 4, 1001
+    big = workloads.f32_to_bf16_bits(rng.standard_normal((B, k + 2, V + 3)).astype(np.float32))
+    tok = rng.integers(0, V, (B, k)).astype(np.int32)
+    tok_d = torch.from_numpy(tok).to(dev)
+    big_d = to_dev(big, "bf16", dev)
+    # offset by one element: rows are not 16-byte aligned (plain-load path)
+    r = sv.greedy(big_d[:, 1:, 1:1 + V], tok_d)
+    o = oracle.verify_greedy(big[:, 1:, 1:1 + V], "bf16", tok)
+    np.testing.assert_array_equal(r["out_tokens"].cpu().numpy(), o["out_tokens"])
+    np.testing.assert_array_equal(r["accepted_len"].cpu().numpy(), o["accepted_len"])
+    # stride-0 broadcast of one sequence over the batch
+    one = big[:1, :k + 1, :V]
+    bc = big_d[:1, :k + 1, :V].expand(B, k + 1, V)
+    r = sv.greedy(bc, tok_d)
+    o = oracle.verify_greedy(np.broadcast_to(one, (B, k + 1, V)), "bf16", tok)
+    np.testing.assert_array_equal(r["out_tokens"].cpu().numpy(), o["out_tokens"])
+
+
+def test_greedy_all_accepted_and_none(dev):
+    rng = np.random.default_rng(4)
+    B, k, V = 40, 6, 5000
+    x = workloads.f32_to_bf16_bits(rng.standard_normal((B, k + 1, V)).astype(np.float32))
+    am = np.argmax(workloads.to_f32(x, "bf16"), -1).astype(np.int32)
+    t = to_dev(x, "bf16", dev)
+    r = sv.greedy(t, torch.from_numpy(am[:, :k].copy()).to(dev))
+    assert (r["accepted_len"].cpu().numpy() == k).all()
+    np.testing.assert_array_equal(r["out_tokens"].cpu().numpy(), am)
+    bad = ((am[:, :k] + 1) % V).astype(np.int32)
+    r = sv.greedy(t, torch.from_numpy(bad).to(dev))
+    assert (r["accepted_len"].cpu().numpy() == 0).all()
+    np.testing.assert_array_equal(r["out_tokens"].cpu().numpy()[:, 0], am[:, 0])
+
+
+# ---------------------------------------------------------- multi-candidate
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("B,G,k,V", [(1, 1, 4, 100), (3, 3, 2, 17), (16, 8, 4, 3001),
+                                     (2, 64, 3, 50), (4, 5, 32, 40), (2, 2, 0, 10)])
+def test_multi_parity_shapes(dev, dtype, B, G, k, V):
+    rng = np.random.default_rng(B + G * 7 + k * 13 + V)
+    x = tie_heavy(rng, (B, G, k + 1, V)) if V < 64 else \
+        rng.standard_normal((B, G, k + 1, V)).astype(np.float32) * 3
+    arr = workloads.f32_to_bf16_bits(x) if dtype == "bf16" else x
+    am = np.argmax(workloads.to_f32(arr, dtype), -1)
+    cand = np.where(rng.random((B, G, k)) < 0.7, am[..., :k], rng.integers(0, V, (B, G, k)))
+    cand = cand.astype(np.int32)
+    r = sv.multi_candidate(to_dev(arr, dtype, dev), torch.from_numpy(cand).to(dev))
+    o = oracle.verify_multi(arr, dtype, cand, threads=THREADS)
+    for key in ("best_candidate", "accepted_len", "out_tokens"):
+        np.testing.assert_array_equal(r[key].cpu().numpy(), o[key], err_msg=key)
+
+
+# --------------------------------------------------------------- stochastic
+
+@pytest.mark.parametrize("t_dtype,d_dtype", [("bf16", "bf16"), ("bf16", "f32"), ("f32", "f32"),
+                                             ("f32", "bf16")])
+@pytest.mark.parametrize("B,k,V,T", [(1, 1, 1, 1.0), (3, 1, 2, 1.0), (129, 4, 7, 0.7),
+                                     (3, 8, 9, 1.3), (3, 32, 33, 1.0), (5, 4, 4095, 0.7),
+                                     (3, 8, 4097, 1.0), (4, 4, 32000, 0.5),
+                                     (2, 3, 128256, 1.0)])
+def test_stochastic_parity_shapes(dev, t_dtype, d_dtype, B, k, V, T):
+    w = workloads.make_stochastic(B, k, V, t_dtype, d_dtype, t_std=3.0, d_noise=1.0,
+                                  temperature=T, seed=B * 100 + k * 10 + V)
+    r, o = run_stochastic(w, dev)
+    compare_stochastic(r, o, k, f"{t_dtype}/{d_dtype} B={B} k={k} V={V}")
+
+
+def test_stochastic_zero_drafts_samples_bonus(dev):
+    w = workloads.make_stochastic(50, 0, 3000, "bf16", "bf16", seed=8)
+    r, o = run_stochastic(w, dev)
+    assert (r["accepted_len"].cpu().numpy() == 0).all()
+    compare_stochastic(r, o, 0, "k=0")
+
+
+def test_stochastic_sharp_and_flat_temperatures(dev):
+    for T in (0.05, 4.0):
+        w = workloads.make_stochastic(24, 4, 5000, "bf16", "f32", t_std=3.0, d_noise=0.5,
+                                      temperature=T, seed=9)
+        r, o = run_stochastic(w, dev)
+        compare_stochastic(r, o, 4, f"T={T}")
+
+
+def test_stochastic_neg_inf_logits(dev):
+    w = workloads.make_stochastic(16, 4, 3000, "f32", "f32", seed=10)
+    rng = np.random.default_rng(1)
+    w["target"][rng.random(w["target"].shape) < 0.2] = -np.inf
+    w["draft"][rng.random(w["draft"].shape) < 0.2] = -np.inf
+    r, o = run_stochastic(w, dev)
+    compare_stochastic(r, o, 4, "-inf")
+
+
+def test_stochastic_strided_unaligned_views(dev):
+    """Rows not 16-byte aligned take the plain-load path; same results."""
+    B, k, V = 7, 4, 2500
+    w = workloads.make_stochastic(B, k, V, "bf16", "f32", seed=12)
+    big_t = np.zeros((B, k + 2, V + 5), np.uint16)
+    big_t[:, 1:, 3:3 + V] = w["target"]
+    big_d = np.zeros((B, k, V + 1), np.float32)
+    big_d[:, :, 1:] = w["draft"]
+    t = to_dev(big_t, "bf16", dev)[:, 1:, 3:3 + V]
+    d = to_dev(big_d, "f32", dev)[:, :, 1:]
+    r, o = run_stochastic(w, dev, t=t, d=d)
+    compare_stochastic(r, o, k, "unaligned")
+    # aligned but padded rows (strides larger than V): bulk-copy path
+    big_t = np.zeros((B, k + 1, V + 12), np.uint16)
+    big_t[:, :, :V] = w["target"]
+    t = to_dev(big_t, "bf16", dev)[:, :, :V]
+    r, o = run_stochastic(w, dev, t=t)
+    compare_stochastic(r, o, k, "padded")
+
+
+def test_stochastic_broadcast_rows_statistics(dev):
+    """Stride-0 batch of one tiny p/q set: 200k independent trials; the
+    GPU's first committed token follows p_0 and matches the oracle."""
+    rng = np.random.default_rng(13)
+    k, V, T, trials = 3, 6, 0.8, 200_000
+    tl = (rng.standard_normal((k + 1, V)) * 1.5).astype(np.float32)
+    dl = (tl[:k] + rng.standard_normal((k, V))).astype(np.float32)
+    q = np.exp(dl / np.float32(T))
+    q /= q.sum(-1, keepdims=True)
+    g = np.random.default_rng(5)
+    tok = np.stack([g.choice(V, trials, p=q[i]) for i in range(k)], 1).astype(np.int32)
+    t = torch.from_numpy(tl).to(dev).expand(trials, k + 1, V)
+    d = torch.from_numpy(dl).to(dev).expand(trials, k, V)
+    r = sv.stochastic(t, d, torch.from_numpy(tok).to(dev), T, 31, probs=True)
+    o = oracle.verify_stochastic(np.broadcast_to(tl, (trials, k + 1, V)), "f32",
+                                 np.broadcast_to(dl, (trials, k, V)), "f32", tok, T, 31,
+                                 threads=THREADS)
+    near, flipped = compare_stochastic(r, o, k, "broadcast")
+    assert flipped <= max(5, trials // 10000)
+
+
+def test_stochastic_invalid_token_and_residual_fallback(dev):
+    B, k, V = 10, 3, 700
+    w = workloads.make_stochastic(B, k, V, "f32", "f32", seed=14)
+    w["draft"] = w["target"][:, :k].copy()  # p == q: every valid draft is accepted
+    w["tokens"][:, 1] = np.where(np.arange(B) % 2 == 0, V, -3)
+    ws = sv.Workspace(dev)
+    t = to_dev(w["target"], "f32", dev)
+    d = to_dev(w["draft"], "f32", dev)
+    r = sv.stochastic(t, d, torch.from_numpy(w["tokens"]).to(dev), 1.0, 3, probs=True,
+                      workspace=ws)
+    o = oracle.verify_stochastic(w["target"], "f32", w["draft"], "f32", w["tokens"], 1.0, 3)
+    assert (o["flags"] == 3).all()
+    compare_stochastic(r, o, k, "fallback")
+    flags = ws.device_status(clear=True)
+    assert flags == (sv.SV_FLAG_INVALID_TOKEN | sv.SV_FLAG_RESIDUAL_FALLBACK)
+    assert ws.device_status() == 0
+
+
+def test_stochastic_seq_offset_and_repeat(dev):
+    w = workloads.make_stochastic(12, 4, 6000, "bf16", "bf16", seed=15)
+    r0, o0 = run_stochastic(w, dev, seq_offset=1000)
+    compare_stochastic(r0, o0, 4, "offset")
+    t = to_dev(w["target"], "bf16", dev)
+    d = to_dev(w["draft"], "bf16", dev)
+    tok = torch.from_numpy(w["tokens"]).to(dev)
+    for _ in range(3):  # the workspace is left clean: repeated calls agree
+        r = sv.stochastic(t, d, tok, w["temperature"], w["seed"], 1000, probs=True)
+        assert torch.equal(r["out_tokens"], r0["out_tokens"])
+        assert torch.equal(r["probs"], r0["probs"])
+
+
+# ------------------------------------------------------- named workloads
+
+@pytest.mark.parametrize("name", list(workloads.WORKLOADS))
+def test_named_workload_full_size(dev, name):
+    """Every sequence of the full-size workload against the oracle, in the
+    same launch configuration the benchmark times."""
+    w = workloads.make(name, threads=THREADS)
+    mode = w["mode"]
+    if mode == "stochastic":
+        r, o = run_stochastic(w, dev)
+        near, flipped = compare_stochastic(r, o, w["k"], name)
+        print(f"{name}: near ties {near}, of which differing {flipped}")
+    elif mode == "greedy":
+        r = sv.greedy(to_dev(w["target"], "bf16", dev), torch.from_numpy(w["tokens"]).to(dev))
+        o = oracle.verify_greedy(w["target"], "bf16", w["tokens"], threads=THREADS)
+        np.testing.assert_array_equal(r["accepted_len"].cpu().numpy(), o["accepted_len"])
+        np.testing.assert_array_equal(r["out_tokens"].cpu().numpy(), o["out_tokens"])
+    else:
+        r = sv.multi_candidate(to_dev(w["target"], "bf16", dev),
+                               torch.from_numpy(w["tokens"]).to(dev))
+        o = oracle.verify_multi(w["target"], "bf16", w["tokens"], threads=THREADS)
+        for key in ("best_candidate", "accepted_len", "out_tokens"):
+            np.testing.assert_array_equal(r[key].cpu().numpy(), o[key], err_msg=key)
