@@ -199,6 +199,13 @@ __device__ __forceinline__ uint4 vocab_words(const Draw& d, uint32_t c0) {
   return philox10(make_uint4(c0, d.pos, d.seq, d.tag), d.key0, d.key1);
 }
 
+// p(x) - q(x) from the logits and the row statistics.  Both products are
+// rounded on their own (no fused multiply-add), so identical target and
+// draft rows give exactly zero.
+__device__ __forceinline__ float residual(float lt, float ld, float c2, const Hdr& h) {
+  return __fmul_rn(ex2f(fmaf(lt, c2, -h.mt)), h.ist) - __fmul_rn(ex2f(fmaf(ld, c2, -h.md)), h.isd);
+}
+
 // Gumbel-max over the positive residual r(x) = p(x) - q(x) of one chunk:
 // score ln r(x) + g(x).  Returns the warp's best (score, x); x = INT_MAX if
 // the warp saw no positive residual.
@@ -217,7 +224,7 @@ __device__ __forceinline__ void chunk_residual(const unsigned char* ts, const un
     bool any = false;
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      r[e] = ex2f(fmaf(lt[e], c2, -h.mt)) * h.ist - ex2f(fmaf(ld[e], c2, -h.md)) * h.isd;
+      r[e] = residual(lt[e], ld[e], c2, h);
       any |= r[e] > 0.0f;
     }
     if (any) {
@@ -238,8 +245,7 @@ __device__ __forceinline__ void chunk_residual(const unsigned char* ts, const un
   }
   for (int e = 8 * ng + tid; e < h.len; e += kComputeThreads) {
     const int x = h.x0 + e;
-    const float r = ex2f(fmaf(load_elem<TT>(tgt, h.toff + e), c2, -h.mt)) * h.ist -
-                    ex2f(fmaf(load_elem<TD>(drf, h.doff + e), c2, -h.md)) * h.isd;
+    const float r = residual(load_elem<TT>(tgt, h.toff + e), load_elem<TD>(drf, h.doff + e), c2, h);
     if (r > 0.0f) {
       const float sc = lg2f(r) * kLn2 +
                        gumbel(word_of(vocab_words(d, static_cast<uint32_t>(x) >> 2), x & 3));
@@ -357,7 +363,9 @@ __device__ void stoch_producer(const StochParams& p, Shared& sh, unsigned char* 
             ok = false;
             break;
           }
-          n = __ldcg(&p.seq[b].n);
+          // clamped so that no workspace content can steer a read outside
+          // the tensors
+          n = min(max(__ldcg(&p.seq[b].n), 0), p.k);
         }
         h.i = n;
         if (n < p.k) {
@@ -446,11 +454,14 @@ __device__ void finalize_accept(const StochParams& p, int b, int lane) {
   float MT = -INFINITY, ST = 0.0f, MD = -INFINITY, SD = 0.0f;
   bool acc = true;
   if (lane < k) {
-    const float4* part = p.part + (static_cast<size_t>(b) * k + lane) * p.nch;
+    // merge this position's chunk partials, then clear them: every call
+    // leaves the workspace zeroed, whatever sizes the next call uses
+    float4* part = p.part + (static_cast<size_t>(b) * k + lane) * p.nch;
     for (int c = 0; c < p.nch; ++c) {
       const float4 v = __ldcg(part + c);
       merge_stats(MT, ST, v.x, v.y);
       merge_stats(MD, SD, v.z, v.w);
+      part[c] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     }
     const int x = __ldg(p.tokens + static_cast<size_t>(b) * k + lane);
     const bool valid = x >= 0 && x < p.V;
@@ -532,8 +543,11 @@ __device__ void finalize_sample(const StochParams& p, const Hdr& h, int lane) {
   if (lane == 0) {
     p.out_tokens[static_cast<size_t>(b) * (k + 1) + n] = tok;
     p.accepted_len[b] = n;
-    p.seq[b].cnt2 = 0u;
-    p.seq[b].ready = 0u;
+    SeqRec* r = p.seq + b;
+    r->n = 0;
+    r->mt = r->ist = r->md = r->isd = 0.0f;
+    r->cnt2 = 0u;
+    r->ready = 0u;
   }
 }
 

@@ -286,6 +286,43 @@ def test_stochastic_seq_offset_and_repeat(dev):
         assert torch.equal(r["probs"], r0["probs"])
 
 
+def test_one_workspace_across_modes_and_sizes(dev):
+    """Calls of every mode and many sizes share one workspace; each call must
+    leave it clean for the next."""
+    ws = sv.Workspace(dev)
+    rng = np.random.default_rng(16)
+    for step in range(12):
+        mode = ("stochastic", "greedy", "multi")[step % 3]
+        B = int(rng.integers(1, 40))
+        k = int(rng.integers(0, 9))
+        V = int(rng.integers(2, 3000))
+        if mode == "stochastic":
+            w = workloads.make_stochastic(B, k, V, "bf16", "f32", seed=step)
+            t = to_dev(w["target"], "bf16", dev)
+            d = to_dev(w["draft"], "f32", dev)
+            r = sv.stochastic(t, d, torch.from_numpy(w["tokens"]).to(dev), w["temperature"], 7,
+                              probs=True, workspace=ws)
+            o = oracle.verify_stochastic(w["target"], "bf16", w["draft"], "f32", w["tokens"],
+                                         w["temperature"], 7)
+            compare_stochastic(r, o, k, f"step {step}")
+        elif mode == "greedy":
+            w = workloads.make_greedy(B, k, V, seed=step)
+            r = sv.greedy(to_dev(w["target"], "bf16", dev), torch.from_numpy(w["tokens"]).to(dev),
+                          workspace=ws)
+            o = oracle.verify_greedy(w["target"], "bf16", w["tokens"])
+            np.testing.assert_array_equal(r["out_tokens"].cpu().numpy(), o["out_tokens"])
+        else:
+            w = workloads.make_multi(B, 3, k, V, seed=step)
+            r = sv.multi_candidate(to_dev(w["target"], "bf16", dev),
+                                   torch.from_numpy(w["tokens"]).to(dev), workspace=ws)
+            o = oracle.verify_multi(w["target"], "bf16", w["tokens"])
+            np.testing.assert_array_equal(r["out_tokens"].cpu().numpy(), o["out_tokens"])
+        torch.cuda.synchronize()
+        body = ws.buf[256:].cpu()
+        assert int(body.count_nonzero()) == 0, f"workspace not clean after step {step} ({mode})"
+    assert ws.device_status() == 0
+
+
 # ------------------------------------------------------- named workloads
 
 @pytest.mark.parametrize("name", list(workloads.WORKLOADS))
