@@ -41,13 +41,42 @@ bool stride16(long long stride, int es) { return ((stride * es) % 16) == 0; }
 
 size_t seq_bytes(int B) { return static_cast<size_t>(B) * sizeof(SeqRec); }
 
-size_t stochastic_part_bytes(int B, int k, int V, int bpe) {
-  const Plan pl = plan_chunks(static_cast<long long>(B) * k, V, bpe);
-  return static_cast<size_t>(B) * k * pl.nch * sizeof(float4);
+// Partial slots (8 bytes each) and row counters (4 bytes each):
+//   stochastic: chunk [B][k][nch][2], row [B][k][2], phase-2 [B][nch], rc [B][k]
+//   argmax:     chunk [B][R][nch], row [B][R], rc [B][R]   (R = G (k+1))
+struct StochLayout {
+  size_t p1, r1, p2, rc, bytes;  // offsets from the tail, in bytes
+};
+StochLayout stochastic_layout(int B, int k, int nch) {
+  StochLayout l;
+  const size_t bk = static_cast<size_t>(B) * k;
+  l.p1 = 0;
+  l.r1 = l.p1 + bk * nch * 2 * 8;
+  l.p2 = l.r1 + bk * 2 * 8;
+  l.rc = l.p2 + static_cast<size_t>(B) * nch * 8;
+  l.bytes = l.rc + (bk * 4 + 15) / 16 * 16;
+  return l;
+}
+struct ArgLayout {
+  size_t slots, rkey, rc, bytes;
+};
+ArgLayout argmax_layout(long long rows, int nch) {
+  ArgLayout l;
+  l.slots = 0;
+  l.rkey = static_cast<size_t>(rows) * nch * 8;
+  l.rc = l.rkey + static_cast<size_t>(rows) * 8;
+  l.bytes = l.rc + (static_cast<size_t>(rows) * 4 + 15) / 16 * 16;
+  return l;
 }
 
-size_t argmax_key_bytes(int B, int G, int k) {
-  return static_cast<size_t>(B) * G * (k + 1) * sizeof(unsigned long long);
+size_t stochastic_part_bytes(int B, int k, int V, int bpe) {
+  const Plan pl = plan_chunks(static_cast<long long>(B) * k, V, bpe);
+  return stochastic_layout(B, k, pl.nch).bytes;
+}
+
+size_t argmax_key_bytes(int B, int G, int k, int V, int es) {
+  const long long rows = static_cast<long long>(B) * G * (k + 1);
+  return argmax_layout(rows, plan_chunks(rows, V, es).nch).bytes;
 }
 
 bool sizes_ok(int B, int G, int k, int V) {
@@ -84,7 +113,11 @@ using namespace sv;
 
 extern "C" size_t spec_verify_workspace_size(int B, int G, int k, int V) {
   if (!sizes_ok(B, G, k, V)) return 0;
-  size_t tail = argmax_key_bytes(B, G, k);
+  size_t tail = 0;
+  for (int es : {2, 4}) {
+    const size_t a = argmax_key_bytes(B, G, k, V, es);
+    if (a > tail) tail = a;
+  }
   if (G == 1) {
     for (int bpe : {4, 6, 8}) {
       const size_t s = stochastic_part_bytes(B, k, V, bpe);
@@ -163,7 +196,9 @@ extern "C" int spec_verify_stochastic(const void* target_logits, int t_dtype,
   const long long p1 = static_cast<long long>(k) * pl.nch;
   long long lag = 0;
   if (p1 > 0) {
-    lag = (static_cast<long long>(kStages) * grid + p1 - 1) / p1 + 1;
+    // phase-2 chunks of a sequence come about 1.5 ring-fulls of the whole
+    // grid after its phase-1 chunks
+    lag = (static_cast<long long>(3 * kStages) * grid / 2 + p1 - 1) / p1 + 1;
     if (lag > B) lag = B;
   }
   const long long slot_items = static_cast<long long>(k + 1) * pl.nch;
@@ -202,7 +237,12 @@ extern "C" int spec_verify_stochastic(const void* target_logits, int t_dtype,
   p.total = static_cast<unsigned int>(total);
   p.ctrl = ws.ctrl;
   p.seq = ws.seq;
-  p.part = static_cast<float4*>(ws.tail);
+  const StochLayout lay = stochastic_layout(B, k, pl.nch);
+  unsigned char* tail = static_cast<unsigned char*>(ws.tail);
+  p.p1 = reinterpret_cast<unsigned long long*>(tail + lay.p1);
+  p.r1 = reinterpret_cast<unsigned long long*>(tail + lay.r1);
+  p.p2 = reinterpret_cast<unsigned long long*>(tail + lay.p2);
+  p.rc = reinterpret_cast<unsigned int*>(tail + lay.rc);
   const cudaError_t e = launch_stochastic(p, t_dtype, d_dtype, tma, grid, kernel_smem_bytes(),
                                           static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? SV_OK : SV_ERR_CUDA;
@@ -253,7 +293,11 @@ static int argmax_call(const void* target_logits, int t_dtype, int64_t sb, int64
   p.total = static_cast<unsigned int>(total);
   p.ctrl = ws.ctrl;
   p.seq = ws.seq;
-  p.rowkey = static_cast<unsigned long long*>(ws.tail);
+  const ArgLayout lay = argmax_layout(rows, pl.nch);
+  unsigned char* tail = static_cast<unsigned char*>(ws.tail);
+  p.slots = reinterpret_cast<unsigned long long*>(tail + lay.slots);
+  p.rkey = reinterpret_cast<unsigned long long*>(tail + lay.rkey);
+  p.rc = reinterpret_cast<unsigned int*>(tail + lay.rc);
   const cudaError_t e = launch_argmax(p, t_dtype, tma, grid, kernel_smem_bytes(),
                                       static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? SV_OK : SV_ERR_CUDA;

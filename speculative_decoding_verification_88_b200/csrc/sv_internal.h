@@ -12,7 +12,10 @@ namespace sv {
 // warp 0: producer (one thread: ticket, waits, bulk copies)
 // warps 1..kComputeWarps: compute (reduce one chunk held in shared memory)
 // last warp: epilogue (publish chunk partials, finalize sequences)
-constexpr int kComputeWarps = 8;
+#ifndef SV_COMPUTE_WARPS
+#define SV_COMPUTE_WARPS 16
+#endif
+constexpr int kComputeWarps = SV_COMPUTE_WARPS;
 constexpr int kThreads = 32 * (kComputeWarps + 2);
 constexpr int kStages = 4;
 constexpr int kStageBytes = 48 * 1024;
@@ -26,16 +29,15 @@ struct Ctrl {
 };
 static_assert(sizeof(Ctrl) == 256, "Ctrl must be 256 bytes");
 
-// Per-sequence record (64 bytes).  Counters, flag and key are zero between
-// calls; the kernel that raises them also lowers them.
+// Per-sequence record (64 bytes), zero between calls: the kernel that sets
+// a field also clears it.
 struct SeqRec {
-  unsigned int cnt1;       // phase-1 chunk arrivals
-  unsigned int cnt2;       // phase-2 chunk arrivals
+  unsigned int cnt1;       // rows merged (phase 1, or all rows for argmax)
+  unsigned int cnt2;       // phase-2 chunks published
   unsigned int ready;      // phase 1 finalized (accepted length known)
   int n;                   // accepted length
   float mt, ist, md, isd;  // row n: max (log2 units) and 1/sum of p and q
-  unsigned long long key;  // phase-2 Gumbel-max key (score, ~index)
-  unsigned int pad[6];
+  unsigned int pad[8];
 };
 static_assert(sizeof(SeqRec) == 64, "SeqRec must be 64 bytes");
 
@@ -69,7 +71,12 @@ struct StochParams {
   unsigned int total;       // tickets
   Ctrl* ctrl;
   SeqRec* seq;
-  float4* part;  // [B][k][nch] chunk partials (mt, st, md, sd)
+  // Partials, published with one 64-bit store each and never zero once
+  // written (so the value is its own "ready" flag):
+  unsigned long long* p1;  // [B][k][nch][2]: chunk (max, sum) of target, of draft
+  unsigned long long* r1;  // [B][k][2]: row (max, sum) of target, of draft
+  unsigned long long* p2;  // [B][nch]: chunk Gumbel-max key, 1 = no candidate
+  unsigned int* rc;        // [B][k]: chunks of a row published
 };
 
 struct ArgmaxParams {
@@ -84,7 +91,9 @@ struct ArgmaxParams {
   unsigned int total;
   Ctrl* ctrl;
   SeqRec* seq;
-  unsigned long long* rowkey;  // [B][G][k+1] argmax keys
+  unsigned long long* slots;  // [B][G][k+1][nch] chunk argmax keys
+  unsigned long long* rkey;   // [B][G][k+1] row argmax keys
+  unsigned int* rc;           // [B][G][k+1] chunks of a row published
 };
 
 // dtype codes follow sv_dtype (0 = f32, 1 = bf16).  Return cudaError_t.

@@ -1,46 +1,60 @@
 // sv_kernels.cu -- persistent verify kernels for sm_100a.
 //
 // One CTA per SM runs until the work tickets run out.  A ticket names one
-// chunk of one row (or row pair); the vocabulary of every row is split into
-// `nch` chunks so that a (sequence, position) row is reduced by many CTAs.
+// chunk of one row (or row pair): the vocabulary of every row is split into
+// `nch` chunks, so each (sequence, position) row is reduced by many CTAs.
 //
-//   warp 0, lane 0   producer: takes tickets (atomicAdd), waits where a chunk
-//                    depends on an earlier result, and streams the chunk into
-//                    a 4-stage shared-memory ring with 1-D bulk copies (TMA,
-//                    cp.async.bulk) that complete on an mbarrier.
-//   warps 1..8       compute: reduce the chunk held in shared memory (softmax
+//   warp 0, lane 0   producer: takes tickets (atomicAdd, two at a time, one
+//                    grab ahead) and streams each chunk into a 4-stage shared-
+//                    memory ring with 1-D bulk copies (TMA, cp.async.bulk)
+//                    that complete on an mbarrier.  A chunk whose sequence is
+//                    not ready yet (phase 2 below) is set aside in a short
+//                    queue and issued once it is, so the ring keeps flowing.
+//   warps 1..16      compute: reduce the chunk held in shared memory (softmax
 //                    statistics, Gumbel-max, or argmax) to one record per warp.
-//   last warp        epilogue: merges the warp records, publishes the chunk's
-//                    partial to the workspace, counts arrivals per sequence,
-//                    and, in the CTA that completes a sequence, finalizes it.
+//   last warp        epilogue: merges the warp records, publishes the
+//                    chunk's partial with one 64-bit store and counts it with
+//                    a relaxed atomicAdd on its row's counter.  A published
+//                    partial is never zero, so the value is its own "ready"
+//                    flag and no fence is needed.  The counter's old value is
+//                    checked one chunk later (or at once when no chunk is
+//                    waiting), so its round trip overlaps work.  Merging is
+//                    two-level: the CTA that completes a row merges the row's
+//                    chunk partials (one lane per chunk, one round trip) into
+//                    a row record and counts the row on the sequence; the CTA
+//                    that completes a sequence finalizes it from its row
+//                    records.  Every slot and counter is cleared after use.
 //
 // Stochastic verify ("Accelerating Sonar through speculation", section
 // "Draft-Target": acceptance compares the full draft and target
 // distributions; the target's logits after the accepted prefix are sampled)
-// runs in two phases keyed on the same ticket counter:
+// runs in two phases on the same ticket counter:
 //   phase 1  chunks of row pairs (target i, draft i), i < k: per-chunk
-//            online softmax statistics (max, sum of 2^(x*log2e/T - max)).
-//            The last chunk of a sequence merges them, gathers p_i(x_i) and
-//            q_i(x_i), draws u_i (Philox, tag ACCEPT), finds the first
-//            rejection n with a warp ballot and publishes n.
+//            softmax statistics (max and sum of 2^(x log2(e)/T - max)).  The
+//            finalizer merges them, gathers p_i(x_i) and q_i(x_i), draws u_i
+//            (Philox, tag ACCEPT), finds the first rejection n with a warp
+//            ballot and publishes n (release store of a ready flag).
 //   phase 2  the `nch` chunks of the row that gives the next token: the row
-//            pair n (correction, Gumbel-max over ln max(0, p_n - q_n)) or
-//            target row k (bonus, Gumbel-max over l_k / T).  They are placed
-//            `lag` sequences after their phase-1 chunks, so the pair is
-//            usually still in L2 and the producer rarely waits.
+//            pair n (correction: Gumbel-max over ln max(0, p_n - q_n)) or
+//            target row k (bonus: Gumbel-max over l_k / T).  They sit `lag`
+//            sequences after their phase-1 chunks in ticket order, so the
+//            pair is usually still in L2 and the producer rarely waits.
 // Target row k is read only for sequences that accept all k drafts.
 //
 // Greedy and multi-candidate verify ("Lookahead decoding" news piece,
 // section "Lookahead decoding breaks the order dependency") are one phase:
-// per-chunk argmax keys merged with a 64-bit atomicMax per row; the last
-// chunk of a sequence compares every branch's drafts with its row argmaxes
-// (warp ballot) and commits the longest branch.
+// per-chunk argmax keys; the finalizer takes each row's maximum key, compares
+// every branch's drafts with its row argmaxes (warp ballot) and commits the
+// longest branch.
 //
 // Every wait is bounded (kWaitLimitNs); on expiry the kernel raises
 // kFlagTimeout, every role leaves its loop, and the producer waits for its
-// bulk copies in flight before the CTA exits.  A CTA only ever waits for
-// tickets smaller than the one it holds, and those are held by running CTAs,
-// so the waits end.
+// bulk copies in flight before the CTA exits.  A producer only waits for a
+// sequence whose phase-1 chunks all carry smaller tickets than the one it
+// waits with; those are held by running CTAs, which issue their fresh
+// tickets in order and never hold a set-aside ticket smaller than a fresh
+// one, and an epilogue settles every arrival before it blocks again, so
+// every wait ends.
 #include <climits>
 
 #include "sv_device.cuh"
@@ -50,6 +64,8 @@ namespace sv {
 enum : int { kKindEnd = 0, kKindStats = 1, kKindCorrection = 2, kKindBonus = 3, kKindArgmax = 4 };
 
 constexpr int kComputeThreads = kComputeWarps * 32;
+constexpr unsigned int kGrab = 2;                 // tickets per atomicAdd
+constexpr unsigned long long kNoCandidate = 1ull;  // phase-2 key: no positive residual
 
 struct Hdr {
   int kind;
@@ -76,6 +92,55 @@ struct Shared {
 constexpr size_t kSharedHead = (sizeof(Shared) + 127) / 128 * 128;
 
 size_t kernel_smem_bytes() { return kSharedHead + static_cast<size_t>(kStages) * kStageBytes; }
+
+// ----------------------------------------------------------- publish/poll
+
+__device__ __forceinline__ void st_relaxed_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Wait (bounded) until a published partial appears; 0 on timeout/abort.
+__device__ __forceinline__ unsigned long long poll_u64(const unsigned long long* p, Ctrl* ctrl) {
+  unsigned long long v = ld_relaxed_u64(p);
+  if (v) return v;
+  const unsigned long long t0 = global_ns();
+  for (unsigned int spin = 1;; ++spin) {
+    v = ld_relaxed_u64(p);
+    if (v) return v;
+    if ((spin & 63u) == 0u) {
+      if (aborted(ctrl)) return 0ull;
+      if (global_ns() - t0 > kWaitLimitNs) {
+        atomicOr(&ctrl->flags, kFlagTimeout);
+        return 0ull;
+      }
+    }
+  }
+}
+
+// (max, sum) packed in 64 bits.  sum >= 1 for any chunk with a finite max
+// and max = -inf otherwise, so a published pair is never all-zero bits.
+__device__ __forceinline__ unsigned long long pack_stats(float m, float s) {
+  return (static_cast<unsigned long long>(__float_as_uint(s)) << 32) | __float_as_uint(m);
+}
+__device__ __forceinline__ void unpack_stats(unsigned long long v, float& m, float& s) {
+  m = __uint_as_float(static_cast<uint32_t>(v & 0xffffffffull));
+  s = __uint_as_float(static_cast<uint32_t>(v >> 32));
+}
+
+__device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const unsigned long long w = __shfl_xor_sync(0xffffffffu, v, o);
+    v = w > v ? w : v;
+  }
+  return v;
+}
 
 // ------------------------------------------------------------------ waits
 
@@ -139,6 +204,15 @@ __device__ __forceinline__ void issue_chunk(Shared& sh, unsigned char* stage, in
   }
 }
 
+// Push the end marker into the next stage.
+__device__ __forceinline__ void push_end(Shared& sh, uint32_t use, Ctrl* ctrl) {
+  const int s = use % kStages;
+  if (mbar_wait(&sh.empty[s], ((use / kStages) & 1u) ^ 1u, ctrl)) {
+    sh.hdr[s].kind = kKindEnd;
+    mbar_arrive(&sh.full[s]);
+  }
+}
+
 // ------------------------------------------------------- chunk reductions
 
 // Softmax statistics of one chunk, per warp: m = max(x) * c2 (log2 units)
@@ -156,19 +230,23 @@ __device__ __forceinline__ void chunk_stats(const unsigned char* smem, int nvec,
   for (int e = nvec * EPV + tid; e < len; e += kComputeThreads)
     m = fmaxf(m, load_elem<T>(g, goff + e));
   m = warp_max(m);
-  float s = 0.0f, mc = -INFINITY;
+  float mc = -INFINITY, s = 0.0f;
   if (m != -INFINITY) {
     mc = m * c2;
-#pragma unroll 4
+    float s0 = 0.0f, s1 = 0.0f;
+#pragma unroll 2
     for (int v = tid; v < nvec; v += kComputeThreads) {
       float f[EPV];
       unpack(sv[v], f);
 #pragma unroll
-      for (int j = 0; j < EPV; ++j) s += ex2f(fmaf(f[j], c2, -mc));
+      for (int j = 0; j < EPV; j += 2) {
+        s0 += ex2f(fmaf(f[j], c2, -mc));
+        s1 += ex2f(fmaf(f[j + 1], c2, -mc));
+      }
     }
     for (int e = nvec * EPV + tid; e < len; e += kComputeThreads)
-      s += ex2f(fmaf(load_elem<T>(g, goff + e), c2, -mc));
-    s = warp_sum(s);
+      s0 += ex2f(fmaf(load_elem<T>(g, goff + e), c2, -mc));
+    s = warp_sum(s0 + s1);
   }
   m_out = mc;
   s_out = s;
@@ -245,7 +323,8 @@ __device__ __forceinline__ void chunk_residual(const unsigned char* ts, const un
   }
   for (int e = 8 * ng + tid; e < h.len; e += kComputeThreads) {
     const int x = h.x0 + e;
-    const float r = residual(load_elem<TT>(tgt, h.toff + e), load_elem<TD>(drf, h.doff + e), c2, h);
+    const float r =
+        residual(load_elem<TT>(tgt, h.toff + e), load_elem<TD>(drf, h.doff + e), c2, h);
     if (r > 0.0f) {
       const float sc = lg2f(r) * kLn2 +
                        gumbel(word_of(vocab_words(d, static_cast<uint32_t>(x) >> 2), x & 3));
@@ -331,76 +410,129 @@ __device__ __forceinline__ void chunk_argmax(const unsigned char* smem, const Hd
 
 // ============================================================ stochastic
 
+// Place a chunk in the next ring stage (waits for the stage to be free).
+template <typename TT, typename TD, bool kTma>
+__device__ __forceinline__ bool stoch_issue(const StochParams& p, Shared& sh,
+                                            unsigned char* stages, uint32_t& use, Hdr& h) {
+  h.x0 = h.c * p.ch;
+  h.len = min(p.ch, p.V - h.x0);
+  h.toff = static_cast<long long>(h.b) * p.t_sb + static_cast<long long>(h.i) * p.t_sp + h.x0;
+  h.doff = static_cast<long long>(h.b) * p.d_sb + static_cast<long long>(h.i) * p.d_sp + h.x0;
+  const int s = use % kStages;
+  if (!mbar_wait(&sh.empty[s], ((use / kStages) & 1u) ^ 1u, p.ctrl)) return false;
+  issue_chunk<TT, TD, kTma>(sh, stages + static_cast<size_t>(s) * kStageBytes, s, h, p.tgt,
+                            p.drf, p.ch, h.kind != kKindBonus);
+  ++use;
+  return true;
+}
+
+// Phase-2 chunk c of sequence b, whose accepted length is published.
+template <typename TT, typename TD, bool kTma>
+__device__ __forceinline__ bool stoch_issue_phase2(const StochParams& p, Shared& sh,
+                                                   unsigned char* stages, uint32_t& use, int b,
+                                                   int c) {
+  Hdr h;
+  h.b = b;
+  h.c = c;
+  // clamped so that no workspace content can steer a read outside the tensors
+  const int n = p.k > 0 ? min(max(__ldcg(&p.seq[b].n), 0), p.k) : 0;
+  h.i = n;
+  if (n < p.k) {
+    h.kind = kKindCorrection;
+    h.mt = __ldcg(&p.seq[b].mt);
+    h.ist = __ldcg(&p.seq[b].ist);
+    h.md = __ldcg(&p.seq[b].md);
+    h.isd = __ldcg(&p.seq[b].isd);
+  } else {
+    h.kind = kKindBonus;
+  }
+  return stoch_issue<TT, TD, kTma>(p, sh, stages, use, h);
+}
+
 template <typename TT, typename TD, bool kTma>
 __device__ void stoch_producer(const StochParams& p, Shared& sh, unsigned char* stages) {
+  constexpr int kDefer = 4;
   Ctrl* ctrl = p.ctrl;
   const unsigned int p1_items = static_cast<unsigned int>(p.k) * static_cast<unsigned int>(p.nch);
   uint32_t use = 0;
   bool ok = true;
-  unsigned int t = atomicAdd(&ctrl->ticket, 1u);
-  while (t < p.total) {
-    const unsigned int tn = atomicAdd(&ctrl->ticket, 1u);  // overlaps this chunk
-    const unsigned int slot = t / p.slot_items, o = t % p.slot_items;
-    Hdr h;
-    bool real = false;
-    if (o < p1_items) {
-      if (static_cast<int>(slot) < p.B) {
-        real = true;
-        h.kind = kKindStats;
-        h.b = static_cast<int>(slot);
-        h.i = static_cast<int>(o) / p.nch;
-        h.c = static_cast<int>(o) % p.nch;
-      }
-    } else {
-      const int b = static_cast<int>(slot) - p.lag;
-      if (b >= 0 && b < p.B) {
-        real = true;
-        h.b = b;
-        h.c = static_cast<int>(o - p1_items);
-        int n = 0;
-        if (p.k > 0) {
-          if (!wait_flag(&p.seq[b].ready, ctrl)) {
-            ok = false;
-            break;
-          }
-          // clamped so that no workspace content can steer a read outside
-          // the tensors
-          n = min(max(__ldcg(&p.seq[b].n), 0), p.k);
-        }
-        h.i = n;
-        if (n < p.k) {
-          h.kind = kKindCorrection;
-          h.mt = __ldcg(&p.seq[b].mt);
-          h.ist = __ldcg(&p.seq[b].ist);
-          h.md = __ldcg(&p.seq[b].md);
-          h.isd = __ldcg(&p.seq[b].isd);
+  int db[kDefer], dc[kDefer];  // set-aside phase-2 chunks, oldest first
+  int nd = 0;
+  unsigned int base = atomicAdd(&ctrl->ticket, kGrab), next = 0u, j = 0u;
+  bool prefetched = false;
+  while (ok) {
+    // set-aside chunks whose sequence became ready go first
+    int keep = 0;
+#pragma unroll
+    for (int d = 0; d < kDefer; ++d) {
+      if (d < nd) {
+        if (ok && ld_acquire_u32(&p.seq[db[d]].ready)) {
+          ok = stoch_issue_phase2<TT, TD, kTma>(p, sh, stages, use, db[d], dc[d]);
         } else {
-          h.kind = kKindBonus;
+          db[keep] = db[d];
+          dc[keep] = dc[d];
+          ++keep;
         }
       }
     }
-    if (real) {
-      h.x0 = h.c * p.ch;
-      h.len = min(p.ch, p.V - h.x0);
-      h.toff = static_cast<long long>(h.b) * p.t_sb + static_cast<long long>(h.i) * p.t_sp + h.x0;
-      h.doff = static_cast<long long>(h.b) * p.d_sb + static_cast<long long>(h.i) * p.d_sp + h.x0;
-      const int s = use % kStages;
-      if (!mbar_wait(&sh.empty[s], ((use / kStages) & 1u) ^ 1u, ctrl)) {
+    nd = keep;
+    if (!ok) break;
+    if (base >= p.total) {  // no fresh tickets left
+      if (nd == 0) break;
+      if (!wait_flag(&p.seq[db[0]].ready, ctrl)) {
         ok = false;
         break;
       }
-      issue_chunk<TT, TD, kTma>(sh, stages + static_cast<size_t>(s) * kStageBytes, s, h, p.tgt,
-                                p.drf, p.ch, h.kind != kKindBonus);
-      ++use;
+      continue;
     }
-    t = tn;
+    if (!prefetched) {
+      next = atomicAdd(&ctrl->ticket, kGrab);  // overlaps the chunks of this grab
+      prefetched = true;
+    }
+    const unsigned int t = base + j;
+    if (++j == kGrab) {
+      j = 0u;
+      base = next;
+      prefetched = false;
+    }
+    if (t >= p.total) continue;
+    const unsigned int slot = t / p.slot_items, o = t % p.slot_items;
+    if (o < p1_items) {
+      if (static_cast<int>(slot) >= p.B) continue;
+      Hdr h;
+      h.kind = kKindStats;
+      h.b = static_cast<int>(slot);
+      h.i = static_cast<int>(o) / p.nch;
+      h.c = static_cast<int>(o) % p.nch;
+      ok = stoch_issue<TT, TD, kTma>(p, sh, stages, use, h);
+    } else {
+      const int b = static_cast<int>(slot) - p.lag;
+      if (b < 0 || b >= p.B) continue;
+      const int c = static_cast<int>(o - p1_items);
+      if (p.k == 0 || ld_acquire_u32(&p.seq[b].ready)) {
+        ok = stoch_issue_phase2<TT, TD, kTma>(p, sh, stages, use, b, c);
+      } else {
+        if (nd == kDefer) {  // queue full: the oldest must go first
+          if (!wait_flag(&p.seq[db[0]].ready, ctrl)) {
+            ok = false;
+            break;
+          }
+          ok = stoch_issue_phase2<TT, TD, kTma>(p, sh, stages, use, db[0], dc[0]);
+#pragma unroll
+          for (int d = 1; d < kDefer; ++d) {
+            db[d - 1] = db[d];
+            dc[d - 1] = dc[d];
+          }
+          --nd;
+        }
+        db[nd] = b;
+        dc[nd] = c;
+        ++nd;
+      }
+    }
   }
   if (ok) {
-    const int s = use % kStages;
-    if (mbar_wait(&sh.empty[s], ((use / kStages) & 1u) ^ 1u, ctrl)) {
-      sh.hdr[s].kind = kKindEnd;
-      mbar_arrive(&sh.full[s]);
-    }
+    push_end(sh, use, ctrl);
     leave_grid(ctrl);
   } else if (kTma) {
     drain_stages(sh, use);
@@ -446,24 +578,28 @@ __device__ void stoch_compute(const StochParams& p, Shared& sh, unsigned char* s
   }
 }
 
-// Phase-1 finalize of sequence b (one warp): merge chunk statistics per
-// position, gather p_i(x_i), q_i(x_i), accept while u_i q < p, publish n.
+// Read a published partial: the load is issued at once; only a slot whose
+// store is not visible yet is polled.
+__device__ __forceinline__ unsigned long long take(unsigned long long* slot, unsigned long long v,
+                                                   Ctrl* ctrl) {
+  if (v == 0ull) v = poll_u64(slot, ctrl);
+  *slot = 0ull;
+  return v;
+}
+
+// Phase-1 finalize of sequence b (one warp): row statistics of every
+// position, p_i(x_i), q_i(x_i), accept while u_i q < p, publish n.
 template <typename TT, typename TD>
 __device__ void finalize_accept(const StochParams& p, int b, int lane) {
   const int k = p.k;
   float MT = -INFINITY, ST = 0.0f, MD = -INFINITY, SD = 0.0f;
   bool acc = true;
   if (lane < k) {
-    // merge this position's chunk partials, then clear them: every call
-    // leaves the workspace zeroed, whatever sizes the next call uses
-    float4* part = p.part + (static_cast<size_t>(b) * k + lane) * p.nch;
-    for (int c = 0; c < p.nch; ++c) {
-      const float4 v = __ldcg(part + c);
-      merge_stats(MT, ST, v.x, v.y);
-      merge_stats(MD, SD, v.z, v.w);
-      part[c] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-    }
+    unsigned long long* row = p.r1 + (static_cast<size_t>(b) * k + lane) * 2;
+    const unsigned long long vt0 = ld_relaxed_u64(row), vd0 = ld_relaxed_u64(row + 1);
     const int x = __ldg(p.tokens + static_cast<size_t>(b) * k + lane);
+    unpack_stats(take(row, vt0, p.ctrl), MT, ST);
+    unpack_stats(take(row + 1, vd0, p.ctrl), MD, SD);
     const bool valid = x >= 0 && x < p.V;
     float pt = 0.0f, qd = 0.0f;
     if (valid) {
@@ -510,17 +646,57 @@ __device__ void finalize_accept(const StochParams& p, int b, int lane) {
   }
 }
 
-// Phase-2 finalize of sequence b (one warp): the merged Gumbel-max key gives
-// the token at position n.  With no positive residual mass the token is drawn
+// Row merge of position i of sequence b (one warp, one lane per chunk):
+// publish the row statistics and count the row; the last row finalizes.
+template <typename TT, typename TD>
+__device__ void merge_row(const StochParams& p, int b, int i, int lane) {
+  unsigned long long* slot = p.p1 + (static_cast<size_t>(b) * p.k + i) * p.nch * 2;
+  float MT = -INFINITY, ST = 0.0f, MD = -INFINITY, SD = 0.0f;
+  for (int c = lane; c < p.nch; c += 32) {
+    const unsigned long long vt0 = ld_relaxed_u64(slot + 2 * c);
+    const unsigned long long vd0 = ld_relaxed_u64(slot + 2 * c + 1);
+    float m, s;
+    unpack_stats(take(slot + 2 * c, vt0, p.ctrl), m, s);
+    merge_stats(MT, ST, m, s);
+    unpack_stats(take(slot + 2 * c + 1, vd0, p.ctrl), m, s);
+    merge_stats(MD, SD, m, s);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float a = __shfl_xor_sync(0xffffffffu, MT, o);
+    const float bb = __shfl_xor_sync(0xffffffffu, ST, o);
+    const float c = __shfl_xor_sync(0xffffffffu, MD, o);
+    const float d = __shfl_xor_sync(0xffffffffu, SD, o);
+    merge_stats(MT, ST, a, bb);
+    merge_stats(MD, SD, c, d);
+  }
+  unsigned int old = 0u;
+  if (lane == 0) {
+    unsigned long long* row = p.r1 + (static_cast<size_t>(b) * p.k + i) * 2;
+    st_relaxed_u64(row, pack_stats(MT, ST));
+    st_relaxed_u64(row + 1, pack_stats(MD, SD));
+    p.rc[static_cast<size_t>(b) * p.k + i] = 0u;
+    old = atomicAdd(&p.seq[b].cnt1, 1u);
+  }
+  if (__shfl_sync(0xffffffffu, old == static_cast<unsigned int>(p.k) - 1u ? 1 : 0, 0))
+    finalize_accept<TT, TD>(p, b, lane);
+}
+
+// Phase-2 finalize of sequence b (one warp): the largest chunk key gives the
+// token at position n.  With no positive residual mass the token is drawn
 // from p_n with the same CORRECTION stream (slow path, one warp).
 template <typename TT>
-__device__ void finalize_sample(const StochParams& p, const Hdr& h, int lane) {
-  const int b = h.b, n = h.i, k = p.k;
+__device__ void finalize_sample(const StochParams& p, int b, int n, int lane) {
+  const int k = p.k;
   unsigned long long key = 0ull;
-  if (lane == 0) key = atomicExch(&p.seq[b].key, 0ull);
-  key = __shfl_sync(0xffffffffu, key, 0);
+  unsigned long long* slot = p.p2 + static_cast<size_t>(b) * p.nch;
+  for (int c = lane; c < p.nch; c += 32) {
+    const unsigned long long v = take(slot + c, ld_relaxed_u64(slot + c), p.ctrl);
+    key = v > key ? v : key;
+  }
+  key = warp_max_u64(key);
   int tok;
-  if (key == 0ull) {
+  if (key <= kNoCandidate) {
     if (lane == 0) atomicOr(&p.ctrl->flags, kFlagResidualFallback);
     const Draw d{p.key0, p.key1, static_cast<uint32_t>(n),
                  static_cast<uint32_t>(b) + p.seq_offset, kTagCorrection};
@@ -551,18 +727,43 @@ __device__ void finalize_sample(const StochParams& p, const Hdr& h, int lane) {
   }
 }
 
+// An arrival whose counter value is checked later.
+struct Pending {
+  int kind;           // 0: none, kKindStats (row counter) or kKindCorrection (cnt2)
+  int b, i;           // sequence; position (phase-1 row, or phase-2 row n)
+  unsigned int old;   // counter value before this arrival (lane 0)
+};
+
+template <typename TT, typename TD>
+__device__ __forceinline__ void resolve(const StochParams& p, Pending& pd, int lane) {
+  if (pd.kind == 0) return;
+  const unsigned int last = static_cast<unsigned int>(p.nch) - 1u;
+  if (__shfl_sync(0xffffffffu, pd.old == last ? 1 : 0, 0)) {
+    if (pd.kind == kKindStats)
+      merge_row<TT, TD>(p, pd.b, pd.i, lane);
+    else
+      finalize_sample<TT>(p, pd.b, pd.i, lane);
+  }
+  pd.kind = 0;
+}
+
 template <typename TT, typename TD>
 __device__ void stoch_epilogue(const StochParams& p, Shared& sh, int lane) {
+  Pending pd{0, 0, 0, 0u};
   for (uint32_t use = 0;; ++use) {
     const int s = use % kStages;
-    if (!mbar_wait(&sh.rfull[s], (use / kStages) & 1u, p.ctrl)) break;
+    const uint32_t parity = (use / kStages) & 1u;
+    // nothing to overlap with: settle the previous arrival before blocking
+    if (pd.kind != 0 && !mbar_try_wait(&sh.rfull[s], parity)) resolve<TT, TD>(p, pd, lane);
+    if (!mbar_wait(&sh.rfull[s], parity, p.ctrl)) break;
     const Hdr h = sh.hdr[s];
     if (h.kind == kKindEnd) break;
     float4 r = lane < kComputeWarps ? sh.res[s][lane]
                                     : make_float4(-INFINITY, __int_as_float(INT_MAX), 0.f, 0.f);
     __syncwarp();
     if (lane == 0) mbar_arrive(&sh.empty[s]);
-    bool last = false;
+    unsigned int old = 0u;
+    Pending next;
     if (h.kind == kKindStats) {
       if (lane >= kComputeWarps) r = make_float4(-INFINITY, 0.0f, -INFINITY, 0.0f);
 #pragma unroll
@@ -575,32 +776,28 @@ __device__ void stoch_epilogue(const StochParams& p, Shared& sh, int lane) {
         merge_stats(r.z, r.w, c, d);
       }
       if (lane == 0) {
-        p.part[(static_cast<size_t>(h.b) * p.k + h.i) * p.nch + h.c] = r;
-        __threadfence();
-        last = atomicAdd(&p.seq[h.b].cnt1, 1u) ==
-               static_cast<unsigned int>(p.k) * static_cast<unsigned int>(p.nch) - 1u;
+        unsigned long long* slot =
+            p.p1 + ((static_cast<size_t>(h.b) * p.k + h.i) * p.nch + h.c) * 2;
+        st_relaxed_u64(slot, pack_stats(r.x, r.y));
+        st_relaxed_u64(slot + 1, pack_stats(r.z, r.w));
+        old = atomicAdd(&p.rc[static_cast<size_t>(h.b) * p.k + h.i], 1u);
       }
-      last = __shfl_sync(0xffffffffu, last, 0);
-      if (last) {
-        __threadfence();
-        finalize_accept<TT, TD>(p, h.b, lane);
-      }
+      next = Pending{kKindStats, h.b, h.i, old};
     } else {
       float v = r.x;
       int i = __float_as_int(r.y);
       warp_argmax(v, i);
       if (lane == 0) {
-        if (i != INT_MAX) atomicMax(&p.seq[h.b].key, make_key(v, i));
-        __threadfence();
-        last = atomicAdd(&p.seq[h.b].cnt2, 1u) == static_cast<unsigned int>(p.nch) - 1u;
+        st_relaxed_u64(p.p2 + static_cast<size_t>(h.b) * p.nch + h.c,
+                       i == INT_MAX ? kNoCandidate : make_key(v, i));
+        old = atomicAdd(&p.seq[h.b].cnt2, 1u);
       }
-      last = __shfl_sync(0xffffffffu, last, 0);
-      if (last) {
-        __threadfence();
-        finalize_sample<TT>(p, h, lane);
-      }
+      next = Pending{kKindCorrection, h.b, h.i, old};
     }
+    resolve<TT, TD>(p, pd, lane);
+    pd = next;
   }
+  resolve<TT, TD>(p, pd, lane);
 }
 
 template <typename TT, typename TD, bool kTma>
@@ -637,37 +834,37 @@ __device__ void argmax_producer(const ArgmaxParams& p, Shared& sh, unsigned char
   const unsigned int per_seq = R * static_cast<unsigned int>(p.nch);
   uint32_t use = 0;
   bool ok = true;
-  unsigned int t = atomicAdd(&ctrl->ticket, 1u);
-  while (t < p.total) {
-    const unsigned int tn = atomicAdd(&ctrl->ticket, 1u);
-    Hdr h;
-    h.kind = kKindArgmax;
-    h.b = static_cast<int>(t / per_seq);
-    const unsigned int rem = t % per_seq;
-    h.i = static_cast<int>(rem / p.nch);
-    h.c = static_cast<int>(rem % p.nch);
-    const int g = h.i / (p.k + 1), pos = h.i % (p.k + 1);
-    h.x0 = h.c * p.ch;
-    h.len = min(p.ch, p.V - h.x0);
-    h.toff = static_cast<long long>(h.b) * p.sb + static_cast<long long>(g) * p.sg +
-             static_cast<long long>(pos) * p.sp + h.x0;
-    h.doff = 0;
-    const int s = use % kStages;
-    if (!mbar_wait(&sh.empty[s], ((use / kStages) & 1u) ^ 1u, ctrl)) {
-      ok = false;
-      break;
+  unsigned int base = atomicAdd(&ctrl->ticket, kGrab);
+  while (ok && base < p.total) {
+    const unsigned int next = atomicAdd(&ctrl->ticket, kGrab);
+    for (unsigned int j = 0; j < kGrab; ++j) {
+      const unsigned int t = base + j;
+      if (t >= p.total) break;
+      Hdr h;
+      h.kind = kKindArgmax;
+      h.b = static_cast<int>(t / per_seq);
+      const unsigned int rem = t % per_seq;
+      h.i = static_cast<int>(rem / p.nch);
+      h.c = static_cast<int>(rem % p.nch);
+      const int g = h.i / (p.k + 1), pos = h.i % (p.k + 1);
+      h.x0 = h.c * p.ch;
+      h.len = min(p.ch, p.V - h.x0);
+      h.toff = static_cast<long long>(h.b) * p.sb + static_cast<long long>(g) * p.sg +
+               static_cast<long long>(pos) * p.sp + h.x0;
+      h.doff = 0;
+      const int s = use % kStages;
+      if (!mbar_wait(&sh.empty[s], ((use / kStages) & 1u) ^ 1u, ctrl)) {
+        ok = false;
+        break;
+      }
+      issue_chunk<TT, TT, kTma>(sh, stages + static_cast<size_t>(s) * kStageBytes, s, h, p.tgt,
+                                nullptr, p.ch, false);
+      ++use;
     }
-    issue_chunk<TT, TT, kTma>(sh, stages + static_cast<size_t>(s) * kStageBytes, s, h, p.tgt,
-                              nullptr, p.ch, false);
-    ++use;
-    t = tn;
+    base = next;
   }
   if (ok) {
-    const int s = use % kStages;
-    if (mbar_wait(&sh.empty[s], ((use / kStages) & 1u) ^ 1u, ctrl)) {
-      sh.hdr[s].kind = kKindEnd;
-      mbar_arrive(&sh.full[s]);
-    }
+    push_end(sh, use, ctrl);
     leave_grid(ctrl);
   } else if (kTma) {
     drain_stages(sh, use);
@@ -701,23 +898,35 @@ __device__ void argmax_compute(const ArgmaxParams& p, Shared& sh, unsigned char*
 // longest branch (lowest g on a tie) is committed.
 __device__ void finalize_argmax(const ArgmaxParams& p, int b, int lane) {
   const int k = p.k, G = p.G;
-  unsigned long long* keys = p.rowkey + static_cast<size_t>(b) * G * (k + 1);
+  unsigned long long* keys = p.rkey + static_cast<size_t>(b) * G * (k + 1);
   int best_n = -1, best_g = 0, best_next = -1;
-  for (int g = 0; g < G; ++g) {
-    unsigned long long* gk = keys + static_cast<size_t>(g) * (k + 1);
-    int a = -1, a32 = -1;
-    if (lane <= k) a = key_index(atomicExch(gk + lane, 0ull));
-    if (k == 32 && lane == 0) a32 = key_index(atomicExch(gk + 32, 0ull));
-    const int* cand = p.tokens + (static_cast<size_t>(b) * G + g) * k;
-    const bool miss = lane < k && __ldg(cand + lane) != a;
-    const unsigned int mm = __ballot_sync(0xffffffffu, miss);
-    const int n = mm ? __ffs(mm) - 1 : k;
-    const int an = __shfl_sync(0xffffffffu, a, n & 31);
-    const int a32b = __shfl_sync(0xffffffffu, a32, 0);
-    if (n > best_n) {
-      best_n = n;
-      best_g = g;
-      best_next = (n == 32) ? a32b : an;
+  for (int g0 = 0; g0 < G; g0 += 4) {
+    // row keys of up to four branches: loads issued together
+    unsigned long long v[4], v32[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int g = g0 + q;
+      v[q] = (g < G && lane <= k) ? ld_relaxed_u64(keys + g * (k + 1) + lane) : 0ull;
+      v32[q] = (g < G && k == 32 && lane == 0) ? ld_relaxed_u64(keys + g * (k + 1) + 32) : 0ull;
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int g = g0 + q;
+      if (g >= G) break;
+      const int a = lane <= k ? key_index(take(keys + g * (k + 1) + lane, v[q], p.ctrl)) : -1;
+      const int a32 =
+          (k == 32 && lane == 0) ? key_index(take(keys + g * (k + 1) + 32, v32[q], p.ctrl)) : -1;
+      const int* cand = p.tokens + (static_cast<size_t>(b) * G + g) * k;
+      const bool miss = lane < k && __ldg(cand + lane) != a;
+      const unsigned int mm = __ballot_sync(0xffffffffu, miss);
+      const int n = mm ? __ffs(mm) - 1 : k;
+      const int an = __shfl_sync(0xffffffffu, a, n & 31);
+      const int a32b = __shfl_sync(0xffffffffu, a32, 0);
+      if (n > best_n) {
+        best_n = n;
+        best_g = g;
+        best_next = (n == 32) ? a32b : an;
+      }
     }
   }
   const int* cand = p.tokens + (static_cast<size_t>(b) * G + best_g) * k;
@@ -731,11 +940,40 @@ __device__ void finalize_argmax(const ArgmaxParams& p, int b, int lane) {
   }
 }
 
+// Row merge (one warp, one lane per chunk): the row's argmax key is the
+// largest chunk key; count the row, and the last row finalizes.
+__device__ void merge_argmax_row(const ArgmaxParams& p, int b, int r, int lane) {
+  const unsigned int R = static_cast<unsigned int>(p.G) * static_cast<unsigned int>(p.k + 1);
+  unsigned long long* slot = p.slots + (static_cast<size_t>(b) * R + r) * p.nch;
+  unsigned long long key = 0ull;
+  for (int c = lane; c < p.nch; c += 32) {
+    const unsigned long long v = take(slot + c, ld_relaxed_u64(slot + c), p.ctrl);
+    key = v > key ? v : key;
+  }
+  key = warp_max_u64(key);
+  unsigned int old = 0u;
+  if (lane == 0) {
+    st_relaxed_u64(p.rkey + static_cast<size_t>(b) * R + r, key);
+    p.rc[static_cast<size_t>(b) * R + r] = 0u;
+    old = atomicAdd(&p.seq[b].cnt1, 1u);
+  }
+  if (__shfl_sync(0xffffffffu, old == R - 1u ? 1 : 0, 0)) finalize_argmax(p, b, lane);
+}
+
 __device__ void argmax_epilogue(const ArgmaxParams& p, Shared& sh, int lane) {
   const unsigned int R = static_cast<unsigned int>(p.G) * static_cast<unsigned int>(p.k + 1);
+  const unsigned int last = static_cast<unsigned int>(p.nch) - 1u;
+  int pend_b = -1, pend_r = 0;  // unresolved arrival (sequence, row), or -1
+  unsigned int pend_old = 0u;
   for (uint32_t use = 0;; ++use) {
     const int s = use % kStages;
-    if (!mbar_wait(&sh.rfull[s], (use / kStages) & 1u, p.ctrl)) break;
+    const uint32_t parity = (use / kStages) & 1u;
+    if (pend_b >= 0 && !mbar_try_wait(&sh.rfull[s], parity)) {
+      if (__shfl_sync(0xffffffffu, pend_old == last ? 1 : 0, 0))
+        merge_argmax_row(p, pend_b, pend_r, lane);
+      pend_b = -1;
+    }
+    if (!mbar_wait(&sh.rfull[s], parity, p.ctrl)) break;
     const Hdr h = sh.hdr[s];
     if (h.kind == kKindEnd) break;
     float v = -INFINITY;
@@ -748,18 +986,20 @@ __device__ void argmax_epilogue(const ArgmaxParams& p, Shared& sh, int lane) {
     __syncwarp();
     if (lane == 0) mbar_arrive(&sh.empty[s]);
     warp_argmax(v, i);
-    bool last = false;
+    unsigned int old = 0u;
     if (lane == 0) {
-      atomicMax(p.rowkey + static_cast<size_t>(h.b) * R + h.i, make_key(v, i));
-      __threadfence();
-      last = atomicAdd(&p.seq[h.b].cnt1, 1u) == R * static_cast<unsigned int>(p.nch) - 1u;
+      st_relaxed_u64(p.slots + (static_cast<size_t>(h.b) * R + h.i) * p.nch + h.c,
+                     make_key(v, i));
+      old = atomicAdd(&p.rc[static_cast<size_t>(h.b) * R + h.i], 1u);
     }
-    last = __shfl_sync(0xffffffffu, last, 0);
-    if (last) {
-      __threadfence();
-      finalize_argmax(p, h.b, lane);
-    }
+    if (pend_b >= 0 && __shfl_sync(0xffffffffu, pend_old == last ? 1 : 0, 0))
+      merge_argmax_row(p, pend_b, pend_r, lane);
+    pend_b = h.b;
+    pend_r = h.i;
+    pend_old = old;
   }
+  if (pend_b >= 0 && __shfl_sync(0xffffffffu, pend_old == last ? 1 : 0, 0))
+    merge_argmax_row(p, pend_b, pend_r, lane);
 }
 
 template <typename TT, bool kTma>
