@@ -44,6 +44,29 @@ __device__ __forceinline__ float lg2f(float x) {
   return y;
 }
 
+// Packed fp32 pairs (Blackwell f32x2 FMA / add): two lanes of arithmetic per
+// instruction.
+__device__ __forceinline__ unsigned long long pack2(float lo, float hi) {
+  unsigned long long d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(lo), "f"(hi));
+  return d;
+}
+__device__ __forceinline__ void unpack2(unsigned long long v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b,
+                                                   unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ unsigned long long add2(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
                : "memory");
@@ -146,15 +169,32 @@ __device__ __forceinline__ float accept_uniform(uint32_t w) {
   return static_cast<float>(w >> 8) * 0x1p-24f;
 }
 
-// Gumbel noise -ln(-ln u'), u' = ((w >> 9) + 0.5) 2^-23 in (0, 1) (exact in
-// fp32).  The inner log must be accurate relative to its small result for u'
-// near 1, so it is the full-precision logf; the outer one is the hardware
-// approximation (absolute error ~1e-7).
-__device__ __forceinline__ float gumbel(uint32_t w) {
-  const float u = (static_cast<float>(w >> 9) + 0.5f) * 0x1p-23f;
-  const float e = -logf(u);
-  return -lg2f(e) * kLn2;
+// Exponential variate E = -ln u', u' = ((w >> 9) + 0.5) 2^-23 in (0, 1).  Both
+// u' and v = 1 - u' are exact in fp32.  E must be accurate relative to its own
+// size, also when it is tiny (u' near 1), because small E are the ones that win
+// a Gumbel-max.  So:
+//   v <  1/8:  -ln(1 - v) = v + v^2/2 + ... + v^7/7, Taylor series written in
+//              Horner form (truncation below 7e-8 relative);
+//   v >= 1/8:  -ln(u') = -lg2(u') ln 2 with the hardware lg2, whose absolute
+//              error (about 2^-22.6) is below 1e-6 relative here, since
+//              |lg2 u'| >= 0.19.
+__device__ __forceinline__ float exp1_variate(uint32_t w) {
+  const uint32_t j = w >> 9;
+  const float u = (static_cast<float>(j) + 0.5f) * 0x1p-23f;
+  const float v = (static_cast<float>(0x7fffffu - j) + 0.5f) * 0x1p-23f;
+  float t = fmaf(v, 1.0f / 7.0f, 1.0f / 6.0f);
+  t = fmaf(v, t, 0.2f);
+  t = fmaf(v, t, 0.25f);
+  t = fmaf(v, t, 1.0f / 3.0f);
+  t = fmaf(v, t, 0.5f);
+  t = fmaf(v, t, 1.0f);
+  const float series = v * t;
+  const float viaLog = -lg2f(u) * kLn2;
+  return v < 0.125f ? series : viaLog;
 }
+
+// Gumbel noise g = -ln(-ln u') = -ln E.
+__device__ __forceinline__ float gumbel(uint32_t w) { return -lg2f(exp1_variate(w)) * kLn2; }
 
 __device__ __forceinline__ uint32_t word_of(const uint4& v, int j) {
   return j == 0 ? v.x : (j == 1 ? v.y : (j == 2 ? v.z : v.w));

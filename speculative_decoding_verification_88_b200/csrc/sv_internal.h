@@ -16,6 +16,10 @@ namespace sv {
 #define SV_COMPUTE_WARPS 16
 #endif
 constexpr int kComputeWarps = SV_COMPUTE_WARPS;
+// The compute warps form two groups that take alternate ring stages, so one
+// group's load and reduction latency overlaps the other group's arithmetic.
+constexpr int kComputeGroups = 2;
+constexpr int kGroupWarps = kComputeWarps / kComputeGroups;
 constexpr int kThreads = 32 * (kComputeWarps + 2);
 constexpr int kStages = 4;
 constexpr int kStageBytes = 48 * 1024;

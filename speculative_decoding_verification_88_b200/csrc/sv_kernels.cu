@@ -63,7 +63,7 @@ namespace sv {
 
 enum : int { kKindEnd = 0, kKindStats = 1, kKindCorrection = 2, kKindBonus = 3, kKindArgmax = 4 };
 
-constexpr int kComputeThreads = kComputeWarps * 32;
+constexpr int kComputeThreads = kGroupWarps * 32;  // threads that share one chunk
 constexpr unsigned int kGrab = 2;                 // tickets per atomicAdd
 constexpr unsigned long long kNoCandidate = 1ull;  // phase-2 key: no positive residual
 
@@ -86,7 +86,7 @@ struct Shared {
   uint64_t empty[kStages];  // epilogue -> producer (slot free)
   uint64_t rfull[kStages];  // compute -> epilogue (warp records written)
   Hdr hdr[kStages];
-  float4 res[kStages][kComputeWarps];
+  float4 res[kStages][kGroupWarps];
 };
 
 constexpr size_t kSharedHead = (sizeof(Shared) + 127) / 128 * 128;
@@ -204,10 +204,11 @@ __device__ __forceinline__ void issue_chunk(Shared& sh, unsigned char* stage, in
   }
 }
 
-// Push the end marker into the next stage.
+// Push one end marker per compute group into the next stages.
 __device__ __forceinline__ void push_end(Shared& sh, uint32_t use, Ctrl* ctrl) {
-  const int s = use % kStages;
-  if (mbar_wait(&sh.empty[s], ((use / kStages) & 1u) ^ 1u, ctrl)) {
+  for (int g = 0; g < kComputeGroups; ++g, ++use) {
+    const int s = use % kStages;
+    if (!mbar_wait(&sh.empty[s], ((use / kStages) & 1u) ^ 1u, ctrl)) return;
     sh.hdr[s].kind = kKindEnd;
     mbar_arrive(&sh.full[s]);
   }
@@ -252,6 +253,156 @@ __device__ __forceinline__ void chunk_stats(const unsigned char* smem, int nvec,
   s_out = s;
 }
 
+// --- register-resident reductions (bulk-copy path) -----------------------
+// Every thread loads all of its 16-byte vectors of the chunk at once
+// (vectors tid, tid + 512, ...), padding with -inf, so each warp has a
+// whole chunk's worth of independent loads, exps and maxima in flight and
+// no reduction sits between the max and the sum.
+
+// Most vectors one thread holds for a tensor of element type T when the
+// stage is shared with a partner tensor of element size `partner` bytes
+// (0: the tensor has the stage to itself).
+template <typename T, int partner>
+__host__ __device__ constexpr int max_vecs() {
+  return ((kStageBytes / (Elem<T>::kBytes + partner)) * Elem<T>::kBytes / 16 + kComputeThreads - 1) /
+         kComputeThreads;
+}
+
+template <typename T>
+__device__ __forceinline__ uint4 neg_inf_vec();
+template <>
+__device__ __forceinline__ uint4 neg_inf_vec<uint16_t>() {
+  return make_uint4(0xff80ff80u, 0xff80ff80u, 0xff80ff80u, 0xff80ff80u);
+}
+template <>
+__device__ __forceinline__ uint4 neg_inf_vec<float>() {
+  return make_uint4(0xff800000u, 0xff800000u, 0xff800000u, 0xff800000u);
+}
+
+template <typename T, int N>
+__device__ __forceinline__ void load_vecs(const unsigned char* smem, int nvec, int tid,
+                                          uint4 (&v)[N]) {
+  const uint4* sv = reinterpret_cast<const uint4*>(smem);
+#pragma unroll
+  for (int j = 0; j < N; ++j) {
+    const int idx = tid + j * kComputeThreads;
+    v[j] = idx < nvec ? sv[idx] : neg_inf_vec<T>();
+  }
+}
+
+// Thread-local (m, s): m = max * c2 (log2 units), s = sum 2^(x c2 - m)
+// over the thread's vectors plus its share of the ragged end in global
+// memory (entries [tail0, len)).
+template <typename T, int N>
+__device__ __forceinline__ void thread_stats(const uint4 (&v)[N], const void* g, long long goff,
+                                             int tail0, int len, float c2, int tid, float& m_out,
+                                             float& s_out) {
+  constexpr int EPV = Elem<T>::kPerVec;
+  float m = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < N; ++j) m = fmaxf(m, vec_max<T>(v[j]));
+  float tail = -INFINITY;
+  const int e = tail0 + tid;  // the ragged end is shorter than one vector
+  if (e < len) tail = load_elem<T>(g, goff + e);
+  m = fmaxf(m, tail);
+  float s = 0.0f, mc = -INFINITY;
+  if (m != -INFINITY) {
+    mc = m * c2;
+    // pairs of entries: one f32x2 FMA for the exponents, one f32x2 add
+    const unsigned long long cc = pack2(c2, c2), mm = pack2(-mc, -mc);
+    unsigned long long acc0 = 0ull, acc1 = 0ull;  // +0.0f pairs
+#pragma unroll
+    for (int j = 0; j < N; ++j) {
+      float f[EPV];
+      unpack(v[j], f);
+#pragma unroll
+      for (int q = 0; q < EPV; q += 2) {
+        float a, b;
+        unpack2(fma2(pack2(f[q], f[q + 1]), cc, mm), a, b);
+        const unsigned long long e = pack2(ex2f(a), ex2f(b));
+        if ((q & 2) == 0) acc0 = add2(acc0, e);
+        else acc1 = add2(acc1, e);
+      }
+    }
+    float a0, a1, b0, b1;
+    unpack2(acc0, a0, a1);
+    unpack2(acc1, b0, b1);
+    s = ((a0 + a1) + (b0 + b1)) + ex2f(fmaf(tail, c2, -mc));
+  }
+  m_out = mc;
+  s_out = s;
+}
+
+// Softmax statistics of a (target, draft) chunk pair, merged over the warp.
+template <typename TT, typename TD>
+__device__ __forceinline__ float4 chunk_stats_pair(const unsigned char* ts,
+                                                   const unsigned char* ds, const Hdr& h,
+                                                   const void* tgt, const void* drf, float c2,
+                                                   int tid) {
+  constexpr int NT = max_vecs<TT, Elem<TD>::kBytes>();
+  constexpr int ND = max_vecs<TD, Elem<TT>::kBytes>();
+  uint4 vt[NT], vd[ND];
+  load_vecs<TT>(ts, h.nvec_t, tid, vt);
+  load_vecs<TD>(ds, h.nvec_d, tid, vd);
+  float4 r;
+  thread_stats<TT>(vt, tgt, h.toff, h.nvec_t * Elem<TT>::kPerVec, h.len, c2, tid, r.x, r.y);
+  thread_stats<TD>(vd, drf, h.doff, h.nvec_d * Elem<TD>::kPerVec, h.len, c2, tid, r.z, r.w);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float a = __shfl_xor_sync(0xffffffffu, r.x, o);
+    const float b = __shfl_xor_sync(0xffffffffu, r.y, o);
+    const float c = __shfl_xor_sync(0xffffffffu, r.z, o);
+    const float d = __shfl_xor_sync(0xffffffffu, r.w, o);
+    merge_stats(r.x, r.y, a, b);
+    merge_stats(r.z, r.w, c, d);
+  }
+  return r;
+}
+
+// Argmax (first maximum) of a chunk held in shared memory, merged over the
+// warp.
+template <typename T>
+__device__ __forceinline__ void chunk_argmax_regs(const unsigned char* smem, const Hdr& h,
+                                                  const void* g, int tid, float& bv, int& bi) {
+  constexpr int EPV = Elem<T>::kPerVec;
+  constexpr int N = max_vecs<T, 0>();
+  uint4 v[N];
+  load_vecs<T>(smem, h.nvec_t, tid, v);
+  float best = -INFINITY;
+  int bj = -1;
+#pragma unroll
+  for (int j = 0; j < N; ++j) {
+    const float m = vec_max<T>(v[j]);
+    if (tid + j * kComputeThreads < h.nvec_t && (bj < 0 || m > best)) {
+      best = m;
+      bj = j;
+    }
+  }
+  int idx = INT_MAX;
+#pragma unroll
+  for (int j = 0; j < N; ++j) {
+    if (j == bj) {
+      float f[EPV];
+      unpack(v[j], f);
+      const int x = h.x0 + (tid + j * kComputeThreads) * EPV;
+#pragma unroll
+      for (int q = EPV - 1; q >= 0; --q)
+        if (f[q] == best) idx = x + q;
+    }
+  }
+  const int e = h.nvec_t * EPV + tid;  // the ragged end is shorter than one vector
+  if (e < h.len) {
+    const float t = load_elem<T>(g, h.toff + e);
+    if (better(t, h.x0 + e, best, idx)) {
+      best = t;
+      idx = h.x0 + e;
+    }
+  }
+  warp_argmax(best, idx);
+  bv = best;
+  bi = idx;
+}
+
 // Eight consecutive entries (group j of the chunk) from shared memory.
 template <typename T>
 __device__ __forceinline__ void load8(const unsigned char* smem, int j, float (&f)[8]);
@@ -281,43 +432,69 @@ __device__ __forceinline__ uint4 vocab_words(const Draw& d, uint32_t c0) {
 // rounded on their own (no fused multiply-add), so identical target and
 // draft rows give exactly zero.
 __device__ __forceinline__ float residual(float lt, float ld, float c2, const Hdr& h) {
-  return __fmul_rn(ex2f(fmaf(lt, c2, -h.mt)), h.ist) - __fmul_rn(ex2f(fmaf(ld, c2, -h.md)), h.isd);
+  return __fsub_rn(__fmul_rn(ex2f(fmaf(lt, c2, -h.mt)), h.ist),
+                   __fmul_rn(ex2f(fmaf(ld, c2, -h.md)), h.isd));
 }
 
-// Gumbel-max over the positive residual r(x) = p(x) - q(x) of one chunk:
-// score ln r(x) + g(x).  Returns the warp's best (score, x); x = INT_MAX if
-// the warp saw no positive residual.
+// The same for eight entries: the exponents two at a time (f32x2 FMA), the
+// products and the difference as scalar round-to-nearest operations.  (The
+// assembler may fuse a packed multiply with a following packed subtract into
+// one FMA, which leaves the product's rounding error behind, so p - q of
+// identical rows would not be zero.)
+__device__ __forceinline__ void residual8(const float (&lt)[8], const float (&ld)[8], float c2,
+                                          const Hdr& h, float (&r)[8]) {
+  const unsigned long long cc = pack2(c2, c2);
+  const unsigned long long mt = pack2(-h.mt, -h.mt), md = pack2(-h.md, -h.md);
+#pragma unroll
+  for (int e = 0; e < 8; e += 2) {
+    float a0, a1, b0, b1;
+    unpack2(fma2(pack2(lt[e], lt[e + 1]), cc, mt), a0, a1);
+    unpack2(fma2(pack2(ld[e], ld[e + 1]), cc, md), b0, b1);
+    r[e] = __fsub_rn(__fmul_rn(ex2f(a0), h.ist), __fmul_rn(ex2f(b0), h.isd));
+    r[e + 1] = __fsub_rn(__fmul_rn(ex2f(a1), h.ist), __fmul_rn(ex2f(b1), h.isd));
+  }
+}
+
+// Exponential race: argmax_x r(x)/E(x) with E = -ln u'(x) is the Gumbel-max
+// argmax_x ln r(x) + g(x).  Keeps the best (r, E, x) of one thread.
+struct Race {
+  float r, e;
+  int x;
+};
+
+__device__ __forceinline__ void race_push(Race& b, float r, uint32_t w, int x) {
+  const float e = exp1_variate(w);
+  if (r * b.e > b.r * e) {  // r/e > b.r/b.e, first x kept on a tie
+    b.r = r;
+    b.e = e;
+    b.x = x;
+  }
+}
+
+// Gumbel-max over the positive residual r(x) = p(x) - q(x) of one chunk.
+// Returns the warp's best (score ln r - ln E, x); x = INT_MAX if the warp saw
+// no positive residual.
 template <typename TT, typename TD, bool kTma>
 __device__ __forceinline__ void chunk_residual(const unsigned char* ts, const unsigned char* ds,
                                                const Hdr& h, const void* tgt, const void* drf,
                                                float c2, const Draw& d, int tid, float& bv,
                                                int& bi) {
-  bv = -INFINITY;
-  bi = INT_MAX;
+  Race best{0.0f, 1.0f, INT_MAX};
   const int ng = kTma ? h.len / 8 : 0;
   for (int j = tid; j < ng; j += kComputeThreads) {
     float lt[8], ld[8], r[8];
     load8<TT>(ts, j, lt);
     load8<TD>(ds, j, ld);
-    bool any = false;
+    residual8(lt, ld, c2, h, r);
+    const int xg = h.x0 + 8 * j;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      r[e] = residual(lt[e], ld[e], c2, h);
-      any |= r[e] > 0.0f;
-    }
-    if (any) {
-      const int xg = h.x0 + 8 * j;
-      const uint4 w0 = vocab_words(d, static_cast<uint32_t>(xg) >> 2);
-      const uint4 w1 = vocab_words(d, (static_cast<uint32_t>(xg) >> 2) + 1u);
+    for (int half = 0; half < 2; ++half) {
+      const int e0 = 4 * half;
+      if (r[e0] > 0.0f || r[e0 + 1] > 0.0f || r[e0 + 2] > 0.0f || r[e0 + 3] > 0.0f) {
+        const uint4 w = vocab_words(d, (static_cast<uint32_t>(xg) >> 2) + half);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        if (r[e] > 0.0f) {
-          const float sc = lg2f(r[e]) * kLn2 + gumbel(word_of(e < 4 ? w0 : w1, e & 3));
-          if (better(sc, xg + e, bv, bi)) {
-            bv = sc;
-            bi = xg + e;
-          }
-        }
+        for (int q = 0; q < 4; ++q)
+          if (r[e0 + q] > 0.0f) race_push(best, r[e0 + q], word_of(w, q), xg + e0 + q);
       }
     }
   }
@@ -325,15 +502,11 @@ __device__ __forceinline__ void chunk_residual(const unsigned char* ts, const un
     const int x = h.x0 + e;
     const float r =
         residual(load_elem<TT>(tgt, h.toff + e), load_elem<TD>(drf, h.doff + e), c2, h);
-    if (r > 0.0f) {
-      const float sc = lg2f(r) * kLn2 +
-                       gumbel(word_of(vocab_words(d, static_cast<uint32_t>(x) >> 2), x & 3));
-      if (better(sc, x, bv, bi)) {
-        bv = sc;
-        bi = x;
-      }
-    }
+    if (r > 0.0f)
+      race_push(best, r, word_of(vocab_words(d, static_cast<uint32_t>(x) >> 2), x & 3), x);
   }
+  bv = best.x == INT_MAX ? -INFINITY : (lg2f(best.r) - lg2f(best.e)) * kLn2;
+  bi = best.x;
   warp_argmax(bv, bi);
 }
 
@@ -542,8 +715,10 @@ __device__ void stoch_producer(const StochParams& p, Shared& sh, unsigned char* 
 template <typename TT, typename TD, bool kTma>
 __device__ void stoch_compute(const StochParams& p, Shared& sh, unsigned char* stages, int w,
                               int lane) {
+  const int group = w / kGroupWarps;
+  w %= kGroupWarps;
   const int tid = w * 32 + lane;
-  for (uint32_t use = 0;; ++use) {
+  for (uint32_t use = group;; use += kComputeGroups) {
     const int s = use % kStages;
     if (!mbar_wait(&sh.full[s], (use / kStages) & 1u, p.ctrl)) break;
     const Hdr h = sh.hdr[s];
@@ -555,10 +730,14 @@ __device__ void stoch_compute(const StochParams& p, Shared& sh, unsigned char* s
     const unsigned char* ds = ts + static_cast<size_t>(p.ch) * Elem<TT>::kBytes;
     float4 r;
     if (h.kind == kKindStats) {
-      float m1, s1, m2, s2;
-      chunk_stats<TT>(ts, h.nvec_t, p.tgt, h.toff, h.len, p.c2, tid, m1, s1);
-      chunk_stats<TD>(ds, h.nvec_d, p.drf, h.doff, h.len, p.c2, tid, m2, s2);
-      r = make_float4(m1, s1, m2, s2);
+      if (kTma) {
+        r = chunk_stats_pair<TT, TD>(ts, ds, h, p.tgt, p.drf, p.c2, tid);
+      } else {
+        float m1, s1, m2, s2;
+        chunk_stats<TT>(ts, h.nvec_t, p.tgt, h.toff, h.len, p.c2, tid, m1, s1);
+        chunk_stats<TD>(ds, h.nvec_d, p.drf, h.doff, h.len, p.c2, tid, m2, s2);
+        r = make_float4(m1, s1, m2, s2);
+      }
     } else {
       const Draw d{p.key0, p.key1, static_cast<uint32_t>(h.i),
                    static_cast<uint32_t>(h.b) + p.seq_offset,
@@ -758,14 +937,14 @@ __device__ void stoch_epilogue(const StochParams& p, Shared& sh, int lane) {
     if (!mbar_wait(&sh.rfull[s], parity, p.ctrl)) break;
     const Hdr h = sh.hdr[s];
     if (h.kind == kKindEnd) break;
-    float4 r = lane < kComputeWarps ? sh.res[s][lane]
-                                    : make_float4(-INFINITY, __int_as_float(INT_MAX), 0.f, 0.f);
+    float4 r = lane < kGroupWarps ? sh.res[s][lane]
+                                  : make_float4(-INFINITY, __int_as_float(INT_MAX), 0.f, 0.f);
     __syncwarp();
     if (lane == 0) mbar_arrive(&sh.empty[s]);
     unsigned int old = 0u;
     Pending next;
     if (h.kind == kKindStats) {
-      if (lane >= kComputeWarps) r = make_float4(-INFINITY, 0.0f, -INFINITY, 0.0f);
+      if (lane >= kGroupWarps) r = make_float4(-INFINITY, 0.0f, -INFINITY, 0.0f);
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) {
         const float a = __shfl_xor_sync(0xffffffffu, r.x, o);
@@ -811,7 +990,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sh.full[s], 1);
       mbar_init(&sh.empty[s], 1);
-      mbar_init(&sh.rfull[s], kComputeWarps);
+      mbar_init(&sh.rfull[s], kGroupWarps);
     }
     mbar_fence_init();
   }
@@ -871,11 +1050,13 @@ __device__ void argmax_producer(const ArgmaxParams& p, Shared& sh, unsigned char
   }
 }
 
-template <typename TT>
+template <typename TT, bool kTma>
 __device__ void argmax_compute(const ArgmaxParams& p, Shared& sh, unsigned char* stages, int w,
                                int lane) {
+  const int group = w / kGroupWarps;
+  w %= kGroupWarps;
   const int tid = w * 32 + lane;
-  for (uint32_t use = 0;; ++use) {
+  for (uint32_t use = group;; use += kComputeGroups) {
     const int s = use % kStages;
     if (!mbar_wait(&sh.full[s], (use / kStages) & 1u, p.ctrl)) break;
     const Hdr h = sh.hdr[s];
@@ -885,7 +1066,10 @@ __device__ void argmax_compute(const ArgmaxParams& p, Shared& sh, unsigned char*
     }
     float bv;
     int bi;
-    chunk_argmax<TT>(stages + static_cast<size_t>(s) * kStageBytes, h, p.tgt, tid, bv, bi);
+    if (kTma)
+      chunk_argmax_regs<TT>(stages + static_cast<size_t>(s) * kStageBytes, h, p.tgt, tid, bv, bi);
+    else
+      chunk_argmax<TT>(stages + static_cast<size_t>(s) * kStageBytes, h, p.tgt, tid, bv, bi);
     if (lane == 0) {
       sh.res[s][w] = make_float4(bv, __int_as_float(bi), 0.0f, 0.0f);
       mbar_arrive(&sh.rfull[s]);
@@ -978,7 +1162,7 @@ __device__ void argmax_epilogue(const ArgmaxParams& p, Shared& sh, int lane) {
     if (h.kind == kKindEnd) break;
     float v = -INFINITY;
     int i = INT_MAX;
-    if (lane < kComputeWarps) {
+    if (lane < kGroupWarps) {
       const float4 r = sh.res[s][lane];
       v = r.x;
       i = __float_as_int(r.y);
@@ -1013,7 +1197,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sh.full[s], 1);
       mbar_init(&sh.empty[s], 1);
-      mbar_init(&sh.rfull[s], kComputeWarps);
+      mbar_init(&sh.rfull[s], kGroupWarps);
     }
     mbar_fence_init();
   }
@@ -1021,7 +1205,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     if (lane == 0) argmax_producer<TT, kTma>(p, sh, stages);
   } else if (warp <= kComputeWarps) {
-    argmax_compute<TT>(p, sh, stages, warp - 1, lane);
+    argmax_compute<TT, kTma>(p, sh, stages, warp - 1, lane);
   } else {
     argmax_epilogue(p, sh, lane);
   }
