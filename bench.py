@@ -1,0 +1,470 @@
+#!/usr/bin/env python
+"""Throughput benchmark of the speculative-decoding verify step on B200.
+
+One step = one verify call on each of the four full-size workloads, in this
+order (every row of the hot path: stochastic accept/correct/bonus, greedy,
+multi-candidate):
+
+  greedy_b64_k4_v128256    greedy,          bf16 [64,5,128256]
+  stoch_b64_k4_v128256     stochastic,      bf16 [64,5,128256] + fp32 [64,4,128256]
+  stoch_b256_k8_v128256    stochastic,      bf16 [256,9,128256] + bf16 [256,8,128256]
+  multi_b16_g8_k4_v32000   multi-candidate, bf16 [16,8,5,32000]
+
+Metric: verified positions per second (positions = B (k+1), or B G (k+1)),
+whole job over all GPUs.  Inputs are resident in HBM and 1.45 GB are
+streamed per step, more than L2 (126 MB), so no buffer is re-read from L2
+across steps.  Usage:
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1, launch one process per GPU with torch.distributed.run; every
+rank verifies its own batch (weak scaling, no collective on the data path).
+`--impl reference` times the CPU oracle (the only reference this method has)
+on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import glob
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+STEP = ["greedy_b64_k4_v128256", "stoch_b64_k4_v128256", "stoch_b256_k8_v128256",
+        "multi_b16_g8_k4_v32000"]
+DOMINANT = "stoch_b256_k8_v128256"
+HBM_FALLBACK_GBS = 6650.0
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic_stochastic_verify_b256_k8.json")
+
+
+# ------------------------------------------------------------------ helpers
+
+def positions(w: dict) -> int:
+    return w["B"] * w.get("G", 1) * (w["k"] + 1)
+
+
+def algorithmic_bytes(w: dict, accepted_len: np.ndarray | None) -> int:
+    """Bytes the method must move for one call (logits + tokens + outputs).
+
+    Stochastic: rows 0..k-1 of target and draft always; target row k only for
+    sequences that accept all k drafts (it feeds nothing else).  The re-read
+    of the rejected pair for the correction is not counted.
+    """
+    from workloads import ELEM_BYTES
+
+    B, k, V = w["B"], w["k"], w["V"]
+    st = ELEM_BYTES[w["t_dtype"]]
+    if w["mode"] == "greedy":
+        return B * (k + 1) * V * st + 4 * B * k + 4 * B * (k + 2)
+    if w["mode"] == "multi":
+        G = w["G"]
+        return B * G * (k + 1) * V * st + 4 * B * G * k + 4 * B * (k + 3)
+    sd = ELEM_BYTES[w["d_dtype"]]
+    n_full = int((accepted_len == k).sum()) if accepted_len is not None else B
+    return B * k * V * (st + sd) + n_full * V * st + 4 * B * k + 4 * B * (k + 2)
+
+
+def measured_hbm_peak() -> tuple[float, str]:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return HBM_FALLBACK_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "speculative_decoding_verification_88_b200", "csrc")
+    for p in sorted(glob.glob(os.path.join(csrc, "*"))) + [os.path.join(ROOT, "include",
+                                                                         "spec_verify.h")]:
+        with open(p, "rb") as f:
+            h.update(os.path.basename(p).encode())
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def recorded_traffic() -> float | None:
+    """DRAM bytes per launch of the dominant kernel from an ncu capture of the
+    current kernel sources, or None if the sources changed since."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    if rec.get("kernel_source_sha256") != kernel_source_hash():
+        return None
+    return float(rec["dram_bytes_per_launch"])
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples of one GPU while it runs."""
+
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.lines: list[str] = []
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", gpu_id], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self, t0: float, t1: float) -> dict | None:
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, reasons, n = [], [], set(), 0
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            except ValueError:
+                continue
+            if not (t0 <= ts <= t1):
+                continue
+            n += 1
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                pass
+            for name, val in zip(self.REASONS, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": n}
+
+
+# --------------------------------------------------------------- reference
+
+def run_reference(args, rank: int) -> None:
+    """The CPU oracle timed on the host cores: each step verifies one sequence
+    of each step workload (rotating through the batch), the four in parallel."""
+    if rank != 0:
+        return
+    import oracle
+    import workloads
+
+    oracle.build()
+    ws = {n: workloads.make(n) for n in STEP}
+    cores = min(len(STEP), os.cpu_count() or 1)
+
+    def one(name, b):
+        w = ws[name]
+        if w["mode"] == "stochastic":
+            oracle.verify_stochastic(w["target"][b:b + 1], w["t_dtype"], w["draft"][b:b + 1],
+                                     w["d_dtype"], w["tokens"][b:b + 1], w["temperature"],
+                                     w["seed"], seq_offset=b)
+        elif w["mode"] == "greedy":
+            oracle.verify_greedy(w["target"][b:b + 1], w["t_dtype"], w["tokens"][b:b + 1])
+        else:
+            oracle.verify_multi(w["target"][b:b + 1], w["t_dtype"], w["tokens"][b:b + 1])
+
+    def step(s):
+        ts = [threading.Thread(target=one, args=(n, s % ws[n]["B"])) for n in STEP]
+        for t in ts:
+            t.start()
+        for t in ts:
+            t.join()
+
+    for s in range(args.warmup):
+        step(s)
+    t0 = time.perf_counter()
+    for s in range(args.steps):
+        step(args.warmup + s)
+    dt = time.perf_counter() - t0
+    pos = sum(ws[n]["k"] + 1 if ws[n]["mode"] != "multi" else ws[n]["G"] * (ws[n]["k"] + 1)
+              for n in STEP)
+    value = pos * args.steps / dt
+    sample = "one sequence of each of the four step workloads per step, in parallel threads"
+    print(json.dumps({
+        "impl": "reference", "metric": "verified positions/s", "value": value,
+        "unit": "positions/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "spec_verify step: " + " + ".join(STEP),
+                   "positions_per_step": pos, "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "positions/s", "cores": cores,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "positions/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }))
+
+
+# --------------------------------------------------------------------- ours
+
+def oracle_baseline(ws: dict) -> dict:
+    """The CPU oracle on one full step (all sequences of the four workloads),
+    all host cores; repeated while under 5 s of wall time (at most 3 times)."""
+    import oracle
+
+    oracle.build()
+    cores = os.cpu_count() or 1
+    reps, t_total = 0, 0.0
+    while reps < 3 and t_total < 5.0:
+        t0 = time.perf_counter()
+        for name in STEP:
+            w = ws[name]
+            if w["mode"] == "stochastic":
+                oracle.verify_stochastic(w["target"], w["t_dtype"], w["draft"], w["d_dtype"],
+                                         w["tokens"], w["temperature"], w["seed"],
+                                         threads=cores)
+            elif w["mode"] == "greedy":
+                oracle.verify_greedy(w["target"], w["t_dtype"], w["tokens"], threads=cores)
+            else:
+                oracle.verify_multi(w["target"], w["t_dtype"], w["tokens"], threads=cores)
+        t_total += time.perf_counter() - t0
+        reps += 1
+    pos = sum(positions(ws[n]) for n in STEP) * reps
+    return {"value": pos / t_total, "unit": "positions/s", "cores": cores, "kind": "oracle",
+            "sample": f"{reps} full step(s): every sequence of the four workloads "
+                      f"({pos // reps} positions per step), {t_total:.1f} s"}
+
+
+def run_ours(args, rank: int, world: int, dist) -> None:
+    import torch
+
+    import speculative_decoding_verification_88_b200 as sv
+    import workloads
+    from speculative_decoding_verification_88_b200 import build as libbuild
+
+    if rank == 0:
+        libbuild.build()
+    if dist is not None:
+        dist.barrier()
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+
+    # inputs (seeded, synthetic; each rank its own batch through seq_offset)
+    threads = max(1, (os.cpu_count() or 1) // max(1, world))
+    ws = {n: workloads.make(n, threads=threads) for n in STEP}
+    calls, host, devbuf = {}, {}, {}
+    for name in STEP:
+        w = ws[name]
+        t_h = workloads.as_torch(w["target"], w["t_dtype"]).pin_memory()
+        tok_h = torch.from_numpy(w["tokens"]).pin_memory()
+        d_h = workloads.as_torch(w["draft"], w["d_dtype"]).pin_memory() if "draft" in w else None
+        t_d, tok_d = t_h.to(dev), tok_h.to(dev)
+        d_d = d_h.to(dev) if d_h is not None else None
+        wsp = sv.Workspace(dev)
+        B, k = w["B"], w["k"]
+        if w["mode"] == "multi":
+            out = {"best_candidate": torch.empty(B, dtype=torch.int32, device=dev)}
+        else:
+            out = {}
+        out["accepted_len"] = torch.empty(B, dtype=torch.int32, device=dev)
+        out["out_tokens"] = torch.empty((B, k + 1), dtype=torch.int32, device=dev)
+        if w["mode"] == "stochastic":
+            off = rank * B
+            fn = (lambda w=w, t=t_d, d=d_d, tok=tok_d, o=out, wsp=wsp, off=off:
+                  sv.stochastic(t, d, tok, w["temperature"], w["seed"], off, out=o, workspace=wsp))
+        elif w["mode"] == "greedy":
+            fn = lambda t=t_d, tok=tok_d, o=out, wsp=wsp: sv.greedy(t, tok, out=o, workspace=wsp)
+        else:
+            fn = (lambda t=t_d, tok=tok_d, o=out, wsp=wsp:
+                  sv.multi_candidate(t, tok, out=o, workspace=wsp))
+        calls[name] = fn
+        host[name] = (t_h, d_h, tok_h, {kk: torch.empty_like(v, device="cpu").pin_memory()
+                                        for kk, v in out.items()})
+        devbuf[name] = (t_d, d_d, tok_d, out)
+
+    # warm-up, then the accepted lengths that fix the stochastic byte counts
+    for _ in range(max(1, args.warmup)):
+        for name in STEP:
+            calls[name]()
+    torch.cuda.synchronize()
+    alg = {n: algorithmic_bytes(ws[n], devbuf[n][3]["accepted_len"].cpu().numpy())
+           for n in STEP}
+
+    # timed region: device-resident inputs, CUDA events on the launching stream
+    K = args.steps
+    ev = {n: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(K)] for n in STEP}
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+    time.sleep(1.0 if sampler.proc is not None else 0.0)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    launches0 = sv.launch_count()
+    t0 = time.time()
+    e_start.record(stream)
+    for s in range(K):
+        for name in STEP:
+            a, b = ev[name][s]
+            a.record(stream)
+            calls[name]()
+            b.record(stream)
+    e_end.record(stream)
+    torch.cuda.synchronize()
+    t1 = time.time()
+    launches = sv.launch_count() - launches0
+    clocks = sampler.stop(t0, t1)
+    elapsed_ms = e_start.elapsed_time(e_end)
+    if dist is not None:
+        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+        dist.barrier()
+    ms_step = elapsed_ms / K
+    pos_step = sum(positions(ws[n]) for n in STEP)
+    value = pos_step * world / (ms_step * 1e-3)
+
+    per = {}
+    for name in STEP:
+        us = statistics.fmean(a.elapsed_time(b) for a, b in ev[name]) * 1e3
+        per[name] = {"us_per_call": round(us, 2),
+                     "positions_per_s": positions(ws[name]) / (us * 1e-6),
+                     "algorithmic_bytes": alg[name],
+                     "alg_gbs": alg[name] / (us * 1e-6) / 1e9}
+    peak, peak_kind = measured_hbm_peak()
+    for name in STEP:
+        per[name]["frac_of_hbm_peak"] = per[name]["alg_gbs"] / peak
+    d = per[DOMINANT]
+    roofline = {"bound": "hbm", "achieved": d["alg_gbs"], "peak": peak, "unit": "GB/s",
+                "frac": d["alg_gbs"] / peak, "traffic": recorded_traffic(),
+                "kernel": "stochastic_verify_kernel (" + DOMINANT + ")",
+                "peak_source": peak_kind + " (MEASURED_PEAKS.json hbm_gbs)"
+                if peak_kind == "measured" else "fallback 6.65 TB/s"}
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if args.e2e_steps > 0:
+        h2d = d2h = 0
+        for name in STEP:
+            t_h, d_h, tok_h, out_h = host[name]
+            h2d += t_h.numel() * t_h.element_size() + tok_h.numel() * 4
+            h2d += d_h.numel() * d_h.element_size() if d_h is not None else 0
+            d2h += sum(v.numel() * 4 for v in out_h.values())
+
+        def e2e_step():
+            for name in STEP:
+                t_h, d_h, tok_h, out_h = host[name]
+                t_d, d_d, tok_d, out = devbuf[name]
+                t_d.copy_(t_h, non_blocking=True)
+                tok_d.copy_(tok_h, non_blocking=True)
+                if d_h is not None:
+                    d_d.copy_(d_h, non_blocking=True)
+                calls[name]()
+                for kk, v in out.items():
+                    out_h[kk].copy_(v, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = a.elapsed_time(b) / args.e2e_steps
+        if dist is not None:
+            t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": pos_step * world / (e_ms * 1e-3), "unit": "positions/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": e_ms}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.skip_cpu_baseline:
+        cpu = oracle_baseline(ws)
+
+    if rank == 0:
+        total_bytes = sum(alg.values())
+        print(json.dumps({
+            "metric": "verified positions/s", "value": value, "unit": "positions/s",
+            "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic (seeded numpy Philox; logits N(0, sigma^2), "
+                                    "draft = target + noise, tokens from the draft softmax)",
+            "config": {"workload": "spec_verify step: " + " + ".join(STEP),
+                       "global_batch": sum(ws[n]["B"] for n in STEP) * world,
+                       "positions_per_step": pos_step * world,
+                       "algorithmic_bytes_per_step": total_bytes,
+                       "step_alg_gbs": total_bytes / (ms_step * 1e-3) / 1e9,
+                       "l2": "inputs larger than L2: 1.45 GB streamed per step, no buffer "
+                             "re-read across steps from L2",
+                       "parallelism": f"weak: {world} GPU(s), each its own batch, no collective"},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": launches, "clocks": clocks, "per_workload": per,
+        }))
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__,
+                                 formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--skip-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if world != args.gpus:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}: launch N>1 with "
+                 "python -m torch.distributed.run --nproc-per-node N")
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    dist = None
+    if world > 1:
+        import torch
+        import torch.distributed as tdist
+
+        local = int(os.environ.get("LOCAL_RANK", "0"))
+        torch.cuda.set_device(local)
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                 device_id=torch.device("cuda", local))
+        dist = tdist
+    try:
+        run_ours(args, rank, world, dist)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

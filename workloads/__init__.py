@@ -110,60 +110,25 @@ def from_torch(t) -> tuple[np.ndarray, str]:
     raise TypeError(f"unsupported logit dtype {t.dtype}")
 
 
-# -------------------------------------------------------------- primitives
-
-def normal_rows(seed: int, stream: int, rows: int, V: int, std: float,
-                threads: int | None = None) -> np.ndarray:
-    """[rows, V] float32, row r drawn from its own Philox stream (seed, stream, r)."""
-    out = np.empty((rows, V), np.float32)
-
-    def fill(r):
-        g = _rng(seed, stream, r)
-        g.standard_normal(V, dtype=np.float32, out=out[r])
-        out[r] *= np.float32(std)
-
-    _pmap(fill, rows, threads)
-    return out
-
-
-def sample_from_softmax(logits_f32: np.ndarray, temperature: float, seed: int, stream: int,
-                        threads: int | None = None) -> np.ndarray:
-    """One token per row from softmax(row / T), by inverse CDF (draft-model sampler)."""
-    rows, V = logits_f32.shape
-    T = float(np.float32(temperature))
-    out = np.empty(rows, np.int32)
-
-    def draw(r):
-        z = logits_f32[r].astype(np.float64) / T
-        w = np.exp(z - z.max())
-        c = np.cumsum(w)
-        u = _rng(seed, stream, r).random() * c[-1]
-        out[r] = min(int(np.searchsorted(c, u, side="right")), V - 1)
-
-    _pmap(draw, rows, threads)
-    return out
-
-
-def argmax_or_uniform(logits_f32: np.ndarray, p_match: float, seed: int, stream: int,
-                      threads: int | None = None) -> np.ndarray:
-    """Per row: the row's argmax with probability p_match, else a uniform token."""
-    rows, V = logits_f32.shape
-    am = np.empty(rows, np.int64)
-
-    def f(r):
-        am[r] = int(np.argmax(logits_f32[r]))
-
-    _pmap(f, rows, threads)
-    g = _rng(seed, stream)
-    hit = g.random(rows) < p_match
-    uni = g.integers(0, V, rows)
-    return np.where(hit, am, uni).astype(np.int32)
-
-
 # ------------------------------------------------------------- generators
 
 # stream ids inside one seed
 _S_TARGET, _S_DRAFT, _S_TOKENS, _S_SHARE = 1, 2, 3, 4
+
+
+def _target_rows(seed: int, rows: int, V: int, std: float, dtype: str,
+                 threads: int | None) -> np.ndarray:
+    """[rows, V] target rows ~ N(0, std^2), row r from stream (seed, 1, r),
+    stored as `dtype` (bf16 rounded to nearest even)."""
+    out = np.empty((rows, V), np.uint16 if dtype == "bf16" else np.float32)
+
+    def fill(r):
+        x = _rng(seed, _S_TARGET, r).standard_normal(V, dtype=np.float32)
+        x *= np.float32(std)
+        out[r] = f32_to_bf16_bits(x) if dtype == "bf16" else x
+
+    _pmap(fill, rows, threads)
+    return out
 
 
 def make_stochastic(B: int, k: int, V: int, t_dtype: str = "bf16", d_dtype: str = "bf16",
@@ -171,43 +136,59 @@ def make_stochastic(B: int, k: int, V: int, t_dtype: str = "bf16", d_dtype: str 
                     seed: int = 0, threads: int | None = None) -> dict:
     """Target [B,k+1,V] ~ N(0, t_std^2); draft [B,k,V] = target + N(0, d_noise^2);
     draft tokens [B,k] drawn from softmax(draft / T)."""
-    t32 = normal_rows(seed, _S_TARGET, B * (k + 1), V, t_std, threads)
-    if t_dtype == "bf16":
-        target = f32_to_bf16_bits(t32)
-        t32 = bf16_bits_to_f32(target)
-    else:
-        target = t32
-    target = target.reshape(B, k + 1, V)
-    tv = t32.reshape(B, k + 1, V)[:, :k, :].reshape(B * k, V)
-    noise = normal_rows(seed, _S_DRAFT, B * k, V, d_noise, threads)
-    d32 = tv + noise
-    if d_dtype == "bf16":
-        draft = f32_to_bf16_bits(d32)
-        d32 = bf16_bits_to_f32(draft)
-    else:
-        draft = d32
-    draft = draft.reshape(B, k, V)
-    tokens = (sample_from_softmax(d32, temperature, seed, _S_TOKENS, threads).reshape(B, k)
-              if B * k else np.zeros((B, k), np.int32))
+    target = _target_rows(seed, B * (k + 1), V, t_std, t_dtype, threads).reshape(B, k + 1, V)
+    draft = np.empty((B, k, V), np.uint16 if d_dtype == "bf16" else np.float32)
+    tokens = np.zeros((B, k), np.int32)
+    T = float(np.float32(temperature))
+
+    def fill(r):
+        b, i = divmod(r, k)
+        noise = _rng(seed, _S_DRAFT, r).standard_normal(V, dtype=np.float32)
+        noise *= np.float32(d_noise)
+        d32 = to_f32(target[b, i], t_dtype) + noise
+        if d_dtype == "bf16":
+            draft[b, i] = f32_to_bf16_bits(d32)
+            d32 = bf16_bits_to_f32(draft[b, i])
+        else:
+            draft[b, i] = d32
+        tokens[b, i] = _inverse_cdf(d32, T, _rng(seed, _S_TOKENS, r).random())
+
+    _pmap(fill, B * k, threads)
     return dict(mode="stochastic", target=target, t_dtype=t_dtype, draft=draft,
-                d_dtype=d_dtype, tokens=tokens, temperature=float(np.float32(temperature)),
-                seed=seed, B=B, k=k, V=V)
+                d_dtype=d_dtype, tokens=tokens, temperature=T, seed=seed, B=B, k=k, V=V)
+
+
+def _inverse_cdf(row_f32: np.ndarray, T: float, u: float) -> int:
+    """Token drawn from softmax(row / T) by inverse CDF with uniform u."""
+    z = row_f32.astype(np.float64) / T
+    c = np.cumsum(np.exp(z - z.max()))
+    return min(int(np.searchsorted(c, u * c[-1], side="right")), row_f32.size - 1)
 
 
 def make_greedy(B: int, k: int, V: int, t_dtype: str = "bf16", t_std: float = 3.0,
                 p_match: float = 0.7, seed: int = 0, threads: int | None = None) -> dict:
     """Target [B,k+1,V] ~ N(0, t_std^2); draft token = row argmax w.p. p_match."""
-    t32 = normal_rows(seed, _S_TARGET, B * (k + 1), V, t_std, threads)
-    if t_dtype == "bf16":
-        target = f32_to_bf16_bits(t32)
-        t32 = bf16_bits_to_f32(target)
-    else:
-        target = t32
-    rows = t32.reshape(B, k + 1, V)[:, :k, :].reshape(B * k, V)
-    tokens = (argmax_or_uniform(rows, p_match, seed, _S_TOKENS, threads).reshape(B, k)
+    target = _target_rows(seed, B * (k + 1), V, t_std, t_dtype, threads).reshape(B, k + 1, V)
+    rows = target[:, :k, :].reshape(B * k, V)
+    tokens = (_argmax_or_uniform(rows, t_dtype, p_match, seed, threads).reshape(B, k)
               if B * k else np.zeros((B, k), np.int32))
-    return dict(mode="greedy", target=target.reshape(B, k + 1, V), t_dtype=t_dtype,
-                tokens=tokens, seed=seed, B=B, k=k, V=V)
+    return dict(mode="greedy", target=target, t_dtype=t_dtype, tokens=tokens, seed=seed,
+                B=B, k=k, V=V)
+
+
+def _argmax_or_uniform(rows: np.ndarray, dtype: str, p_match: float, seed: int,
+                       threads: int | None) -> np.ndarray:
+    n, V = rows.shape
+    am = np.empty(n, np.int64)
+
+    def f(r):
+        am[r] = int(np.argmax(to_f32(rows[r], dtype)))
+
+    _pmap(f, n, threads)
+    g = _rng(seed, _S_TOKENS)
+    hit = g.random(n) < p_match
+    uni = g.integers(0, V, n)
+    return np.where(hit, am, uni).astype(np.int32)
 
 
 def make_multi(B: int, G: int, k: int, V: int, t_dtype: str = "bf16", t_std: float = 3.0,
@@ -219,14 +200,10 @@ def make_multi(B: int, G: int, k: int, V: int, t_dtype: str = "bf16", t_std: flo
     1..G-1 copy branch 0's first s tokens; every other token is its own row's
     argmax with probability p_match, else uniform.
     """
-    t32 = normal_rows(seed, _S_TARGET, B * G * (k + 1), V, t_std, threads)
-    if t_dtype == "bf16":
-        target = f32_to_bf16_bits(t32)
-        t32 = bf16_bits_to_f32(target)
-    else:
-        target = t32
-    rows = t32.reshape(B, G, k + 1, V)[:, :, :k, :].reshape(B * G * k, V)
-    cand = (argmax_or_uniform(rows, p_match, seed, _S_TOKENS, threads).reshape(B, G, k)
+    target = _target_rows(seed, B * G * (k + 1), V, t_std, t_dtype, threads)
+    target = target.reshape(B, G, k + 1, V)
+    rows = target[:, :, :k, :].reshape(B * G * k, V)
+    cand = (_argmax_or_uniform(rows, t_dtype, p_match, seed, threads).reshape(B, G, k)
             if B * G * k else np.zeros((B, G, k), np.int32))
     g = _rng(seed, _S_SHARE)
     shared = g.random(B) < p_shared
@@ -235,8 +212,8 @@ def make_multi(B: int, G: int, k: int, V: int, t_dtype: str = "bf16", t_std: flo
         if shared[b] and k > 0:
             m = min(int(s[b]), k)
             cand[b, 1:, :m] = cand[b, 0, :m]
-    return dict(mode="multi", target=target.reshape(B, G, k + 1, V), t_dtype=t_dtype,
-                tokens=cand, seed=seed, B=B, G=G, k=k, V=V)
+    return dict(mode="multi", target=target, t_dtype=t_dtype, tokens=cand, seed=seed,
+                B=B, G=G, k=k, V=V)
 
 
 def make(name: str, threads: int | None = None, **overrides) -> dict:
