@@ -169,7 +169,7 @@ def _logits(t: torch.Tensor, ndim: int, name: str):
         raise TypeError(f"{name} must be a CUDA tensor")
     if t.dim() != ndim:
         raise ValueError(f"{name} must be {ndim}-d, got shape {tuple(t.shape)}")
-    if t.shape[-1] > 1 and t.stride(-1) != 1:
+    if t.numel() > 0 and t.shape[-1] > 1 and t.stride(-1) != 1:
         raise ValueError(f"{name}: the vocabulary axis must be contiguous")
     return _dtype_code(t), t.stride()
 
