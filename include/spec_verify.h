@@ -172,6 +172,35 @@ int spec_verify_multi_candidate(const void *target_logits, int t_dtype, int64_t 
 int spec_verify_philox4x32_10(const uint32_t *counters, int64_t n, uint64_t seed,
                               uint32_t *out, void *stream);
 
+/*
+ * Greedy verify without any allocation.  The pages have no counterpart: this
+ * is a library convenience for callers that cannot allocate device memory on
+ * the verify path (an external allocator or pool owns the device, the call
+ * runs in a real-time loop where an allocation may block or fail) and cannot
+ * keep a workspace of their own.
+ *
+ * Same arguments, layouts and results as spec_verify_greedy, minus the
+ * workspace: the library uses a fixed device array of
+ * SV_NOALLOC_SCRATCH_BYTES that it carries in its image (every GPU that loads
+ * the library holds it until the process exits).  Each call clears the part
+ * it needs with cudaMemsetAsync on `stream`, then runs greedy verify on it;
+ * nothing is allocated or freed.
+ *  - Returns SV_ERR_WORKSPACE when spec_verify_workspace_size(B, 1, k, V)
+ *    exceeds SV_NOALLOC_SCRATCH_BYTES (about B <= 512 at k = 8, V = 128256),
+ *    SV_ERR_INVALID_ARG for sizes outside the limits, and otherwise what
+ *    spec_verify_greedy returns.
+ *  - The first call on each device looks up the array's address
+ *    (cudaGetSymbolAddress with that device current); make it before any
+ *    stream capture.
+ *  - All calls share the array: calls whose kernels may overlap on the GPU
+ *    (unordered streams) race.  Order them on one stream.
+ */
+#define SV_NOALLOC_SCRATCH_BYTES ((size_t)2 << 20)
+
+int spec_verify_greedy_noalloc(const void *target_logits, int t_dtype, int64_t t_stride_b,
+                               int64_t t_stride_pos, const int32_t *draft_tokens, int B, int k,
+                               int V, int32_t *accepted_len, int32_t *out_tokens, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -28,7 +28,7 @@ SV_FLAG_INVALID_TOKEN, SV_FLAG_RESIDUAL_FALLBACK, SV_FLAG_TIMEOUT = 1, 2, 4
 EXPORTS = (
     "spec_verify_workspace_size", "spec_verify_status_string", "spec_verify_workspace_init",
     "spec_verify_read_device_status", "spec_verify_stochastic", "spec_verify_greedy",
-    "spec_verify_multi_candidate", "spec_verify_philox4x32_10",
+    "spec_verify_multi_candidate", "spec_verify_philox4x32_10", "spec_verify_greedy_noalloc",
 )
 
 _lib = None
@@ -76,6 +76,8 @@ def load_library():
         lib.spec_verify_multi_candidate.restype = I
         lib.spec_verify_philox4x32_10.argtypes = [P, I64, U64, P, P]
         lib.spec_verify_philox4x32_10.restype = I
+        lib.spec_verify_greedy_noalloc.argtypes = [P, I, I64, I64, P, I, I, I, P, P, P]
+        lib.spec_verify_greedy_noalloc.restype = I
         _lib = lib
         return lib
 
@@ -270,6 +272,35 @@ def multi_candidate(target: torch.Tensor, cand_tokens: torch.Tensor, *, out: dic
             res["best_candidate"].data_ptr(), res["accepted_len"].data_ptr(),
             res["out_tokens"].data_ptr(), ws.buf.data_ptr(), ws.nbytes, _stream_ptr(stream, dev))
     _check(code, "spec_verify_multi_candidate")
+    _count()
+    return res
+
+
+def greedy_noalloc(target: torch.Tensor, draft_tokens: torch.Tensor, *,
+                   out: dict | None = None, stream=None) -> dict:
+    """Greedy verify that allocates no device memory inside the library.
+
+    For callers that cannot allocate on the verify path (an external
+    allocator or pool owns the device, or the call runs where an allocation
+    may block or fail): the library uses its own fixed 2 MiB device array
+    instead of a workspace.  Pass preallocated `out` tensors to keep this
+    wrapper free of allocations as well.  Calls share that array, so order
+    them on one stream; the first call on a device should come before any
+    stream capture.
+    """
+    lib = load_library()
+    tc, (tsb, tsp, _) = _logits(target, 3, "target")
+    B, kp1, V = target.shape
+    k = kp1 - 1
+    dev = target.device
+    tok = _tokens(draft_tokens, (B, k), dev, "draft_tokens")
+    res = {"accepted_len": _out(out, "accepted_len", (B,), torch.int32, dev),
+           "out_tokens": _out(out, "out_tokens", (B, k + 1), torch.int32, dev)}
+    with torch.cuda.device(dev):
+        code = lib.spec_verify_greedy_noalloc(
+            target.data_ptr(), tc, tsb, tsp, tok.data_ptr(), B, k, V,
+            res["accepted_len"].data_ptr(), res["out_tokens"].data_ptr(), _stream_ptr(stream, dev))
+    _check(code, "spec_verify_greedy_noalloc")
     _count()
     return res
 
