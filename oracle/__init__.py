@@ -85,7 +85,7 @@ def _logits(arr: np.ndarray, dtype: str, ndim: int):
         raise TypeError("bf16 logits must be a uint16/int16 array of bit patterns")
     if arr.ndim != ndim:
         raise ValueError(f"expected {ndim}-d logits, got shape {arr.shape}")
-    if arr.strides[-1] != arr.itemsize:
+    if arr.size > 0 and arr.strides[-1] != arr.itemsize:
         raise ValueError("vocabulary axis must be contiguous")
     strides = tuple(s // arr.itemsize for s in arr.strides[:-1])
     return DTYPE_CODES[dtype], strides
