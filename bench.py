@@ -271,7 +271,8 @@ def run_ours(args, rank: int, world: int, dist) -> None:
 
     # inputs (seeded, synthetic; each rank its own batch through seq_offset)
     threads = max(1, (os.cpu_count() or 1) // max(1, world))
-    ws = {n: workloads.make(n, threads=threads) for n in STEP}
+    over = {"B": args.batch} if args.batch else {}
+    ws = {n: workloads.make(n, threads=threads, **over) for n in STEP}
     calls, host, devbuf = {}, {}, {}
     for name in STEP:
         w = ws[name]
@@ -428,6 +429,16 @@ def run_ours(args, rank: int, world: int, dist) -> None:
         }))
 
 
+def select_workloads(only: str | None) -> None:
+    """Restrict the step to one workload (profiling runs)."""
+    global STEP, DOMINANT
+    if only:
+        if only not in STEP:
+            raise SystemExit(f"--only must be one of {STEP}")
+        STEP = [only]
+        DOMINANT = only
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__,
                                  formatter_class=argparse.RawDescriptionHelpFormatter)
@@ -437,7 +448,11 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--skip-cpu-baseline", action="store_true")
+    ap.add_argument("--only", help="profiling: time only this workload of the step")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="profiling: override the batch size B of the workloads")
     args = ap.parse_args()
+    select_workloads(args.only)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
 
