@@ -11,16 +11,18 @@ namespace sv {
 // ---- CTA shape of the persistent verify kernels -------------------------
 // warp 0: producer (one thread: ticket, waits, bulk copies)
 // warps 1..kComputeWarps: compute (reduce one chunk held in shared memory)
-// last warp: epilogue (publish chunk partials, finalize sequences)
+// last kComputeGroups warps: epilogues, one per compute group (publish chunk
+// partials, merge rows, finalize sequences)
 #ifndef SV_COMPUTE_WARPS
 #define SV_COMPUTE_WARPS 16
 #endif
 constexpr int kComputeWarps = SV_COMPUTE_WARPS;
 // The compute warps form two groups that take alternate ring stages, so one
-// group's load and reduction latency overlaps the other group's arithmetic.
+// group's load and reduction latency overlaps the other group's arithmetic;
+// each group has its own epilogue warp.
 constexpr int kComputeGroups = 2;
 constexpr int kGroupWarps = kComputeWarps / kComputeGroups;
-constexpr int kThreads = 32 * (kComputeWarps + 2);
+constexpr int kThreads = 32 * (1 + kComputeWarps + kComputeGroups);
 constexpr int kStages = 4;
 constexpr int kStageBytes = 48 * 1024;
 

@@ -12,7 +12,7 @@
 //                    queue and issued once it is, so the ring keeps flowing.
 //   warps 1..16      compute: reduce the chunk held in shared memory (softmax
 //                    statistics, Gumbel-max, or argmax) to one record per warp.
-//   last warp        epilogue: merges the warp records, publishes the
+//   last 2 warps     epilogues, one per compute group: merge the warp records, publish the
 //                    chunk's partial with one 64-bit store and counts it with
 //                    a relaxed atomicAdd on its row's counter.  A published
 //                    partial is never zero, so the value is its own "ready"
@@ -464,11 +464,11 @@ struct Race {
 
 __device__ __forceinline__ void race_push(Race& b, float r, uint32_t w, int x) {
   const float e = exp1_variate(w);
-  if (r * b.e > b.r * e) {  // r/e > b.r/b.e, first x kept on a tie
-    b.r = r;
-    b.e = e;
-    b.x = x;
-  }
+  // a candidate needs r > 0; r/e > b.r/b.e, the first x kept on a tie
+  const bool win = r > 0.0f && r * b.e > b.r * e;
+  b.r = win ? r : b.r;
+  b.e = win ? e : b.e;
+  b.x = win ? x : b.x;
 }
 
 // Gumbel-max over the positive residual r(x) = p(x) - q(x) of one chunk.
@@ -487,23 +487,20 @@ __device__ __forceinline__ void chunk_residual(const unsigned char* ts, const un
     load8<TD>(ds, j, ld);
     residual8(lt, ld, c2, h, r);
     const int xg = h.x0 + 8 * j;
+    // both Philox words in straight-line code, so their round chains
+    // interleave; candidates are selected without branches
+    const uint4 w0 = vocab_words(d, static_cast<uint32_t>(xg) >> 2);
+    const uint4 w1 = vocab_words(d, (static_cast<uint32_t>(xg) >> 2) + 1u);
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const int e0 = 4 * half;
-      if (r[e0] > 0.0f || r[e0 + 1] > 0.0f || r[e0 + 2] > 0.0f || r[e0 + 3] > 0.0f) {
-        const uint4 w = vocab_words(d, (static_cast<uint32_t>(xg) >> 2) + half);
+    for (int q = 0; q < 4; ++q) race_push(best, r[q], word_of(w0, q), xg + q);
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          if (r[e0 + q] > 0.0f) race_push(best, r[e0 + q], word_of(w, q), xg + e0 + q);
-      }
-    }
+    for (int q = 0; q < 4; ++q) race_push(best, r[4 + q], word_of(w1, q), xg + 4 + q);
   }
   for (int e = 8 * ng + tid; e < h.len; e += kComputeThreads) {
     const int x = h.x0 + e;
     const float r =
         residual(load_elem<TT>(tgt, h.toff + e), load_elem<TD>(drf, h.doff + e), c2, h);
-    if (r > 0.0f)
-      race_push(best, r, word_of(vocab_words(d, static_cast<uint32_t>(x) >> 2), x & 3), x);
+    race_push(best, r, word_of(vocab_words(d, static_cast<uint32_t>(x) >> 2), x & 3), x);
   }
   bv = best.x == INT_MAX ? -INFINITY : (lg2f(best.r) - lg2f(best.e)) * kLn2;
   bi = best.x;
@@ -527,10 +524,9 @@ __device__ __forceinline__ void chunk_bonus(const unsigned char* ts, const Hdr& 
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       const float sc = fmaf(lt[e], invT, gumbel(word_of(e < 4 ? w0 : w1, e & 3)));
-      if (better(sc, xg + e, bv, bi)) {
-        bv = sc;
-        bi = xg + e;
-      }
+      const bool win = sc > bv;  // entries arrive in increasing x: first maximum kept
+      bv = win ? sc : bv;
+      bi = win ? xg + e : bi;
     }
   }
   for (int e = 8 * ng + tid; e < h.len; e += kComputeThreads) {
@@ -927,9 +923,9 @@ __device__ __forceinline__ void resolve(const StochParams& p, Pending& pd, int l
 }
 
 template <typename TT, typename TD>
-__device__ void stoch_epilogue(const StochParams& p, Shared& sh, int lane) {
+__device__ void stoch_epilogue(const StochParams& p, Shared& sh, int group, int lane) {
   Pending pd{0, 0, 0, 0u};
-  for (uint32_t use = 0;; ++use) {
+  for (uint32_t use = group;; use += kComputeGroups) {
     const int s = use % kStages;
     const uint32_t parity = (use / kStages) & 1u;
     // nothing to overlap with: settle the previous arrival before blocking
@@ -1000,7 +996,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp <= kComputeWarps) {
     stoch_compute<TT, TD, kTma>(p, sh, stages, warp - 1, lane);
   } else {
-    stoch_epilogue<TT, TD>(p, sh, lane);
+    stoch_epilogue<TT, TD>(p, sh, warp - 1 - kComputeWarps, lane);
   }
 }
 
@@ -1144,12 +1140,12 @@ __device__ void merge_argmax_row(const ArgmaxParams& p, int b, int r, int lane) 
   if (__shfl_sync(0xffffffffu, old == R - 1u ? 1 : 0, 0)) finalize_argmax(p, b, lane);
 }
 
-__device__ void argmax_epilogue(const ArgmaxParams& p, Shared& sh, int lane) {
+__device__ void argmax_epilogue(const ArgmaxParams& p, Shared& sh, int group, int lane) {
   const unsigned int R = static_cast<unsigned int>(p.G) * static_cast<unsigned int>(p.k + 1);
   const unsigned int last = static_cast<unsigned int>(p.nch) - 1u;
   int pend_b = -1, pend_r = 0;  // unresolved arrival (sequence, row), or -1
   unsigned int pend_old = 0u;
-  for (uint32_t use = 0;; ++use) {
+  for (uint32_t use = group;; use += kComputeGroups) {
     const int s = use % kStages;
     const uint32_t parity = (use / kStages) & 1u;
     if (pend_b >= 0 && !mbar_try_wait(&sh.rfull[s], parity)) {
@@ -1207,7 +1203,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp <= kComputeWarps) {
     argmax_compute<TT, kTma>(p, sh, stages, warp - 1, lane);
   } else {
-    argmax_epilogue(p, sh, lane);
+    argmax_epilogue(p, sh, warp - 1 - kComputeWarps, lane);
   }
 }
 
