@@ -222,7 +222,6 @@ extern "C" int spec_verify_stochastic(const void* target_logits, int t_dtype,
   p.B = B;
   p.k = k;
   p.V = V;
-  p.invT = 1.0f / temperature;
   p.c2 = 1.4426950408889634f / temperature;
   p.key0 = static_cast<unsigned int>(seed & 0xffffffffull);
   p.key1 = static_cast<unsigned int>(seed >> 32);

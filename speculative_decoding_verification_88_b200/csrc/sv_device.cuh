@@ -65,6 +65,24 @@ __device__ __forceinline__ unsigned long long add2(unsigned long long a, unsigne
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
+__device__ __forceinline__ unsigned long long sub2(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ unsigned long long splat2(float x) { return pack2(x, x); }
+
+// Largest of three (sm_100 three-input max; a NaN operand is ignored, like fmaxf).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
 
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
@@ -151,11 +169,11 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 __device__ __forceinline__ uint4 philox10(uint4 c, uint32_t k0, uint32_t k1) {
 #pragma unroll
   for (int r = 0; r < 10; ++r) {
-    const uint32_t lo0 = 0xD2511F53u * c.x;
-    const uint32_t hi0 = __umulhi(0xD2511F53u, c.x);
-    const uint32_t lo1 = 0xCD9E8D57u * c.z;
-    const uint32_t hi1 = __umulhi(0xCD9E8D57u, c.z);
-    c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+    // one 32x32->64 multiply per product gives both halves
+    const unsigned long long p0 = static_cast<unsigned long long>(c.x) * 0xD2511F53u;
+    const unsigned long long p1 = static_cast<unsigned long long>(c.z) * 0xCD9E8D57u;
+    c = make_uint4(static_cast<uint32_t>(p1 >> 32) ^ c.y ^ k0, static_cast<uint32_t>(p1),
+                   static_cast<uint32_t>(p0 >> 32) ^ c.w ^ k1, static_cast<uint32_t>(p0));
     k0 += 0x9E3779B9u;
     k1 += 0xBB67AE85u;
   }
@@ -169,32 +187,68 @@ __device__ __forceinline__ float accept_uniform(uint32_t w) {
   return static_cast<float>(w >> 8) * 0x1p-24f;
 }
 
-// Exponential variate E = -ln u', u' = ((w >> 9) + 0.5) 2^-23 in (0, 1).  Both
-// u' and v = 1 - u' are exact in fp32.  E must be accurate relative to its own
-// size, also when it is tiny (u' near 1), because small E are the ones that win
-// a Gumbel-max.  So:
-//   v <  1/8:  -ln(1 - v) = v + v^2/2 + ... + v^7/7, Taylor series written in
-//              Horner form (truncation below 7e-8 relative);
-//   v >= 1/8:  -ln(u') = -lg2(u') ln 2 with the hardware lg2, whose absolute
-//              error (about 2^-22.6) is below 1e-6 relative here, since
-//              |lg2 u'| >= 0.19.
-__device__ __forceinline__ float exp1_variate(uint32_t w) {
-  const uint32_t j = w >> 9;
-  const float u = (static_cast<float>(j) + 0.5f) * 0x1p-23f;
-  const float v = (static_cast<float>(0x7fffffu - j) + 0.5f) * 0x1p-23f;
-  float t = fmaf(v, 1.0f / 7.0f, 1.0f / 6.0f);
-  t = fmaf(v, t, 0.2f);
-  t = fmaf(v, t, 0.25f);
-  t = fmaf(v, t, 1.0f / 3.0f);
-  t = fmaf(v, t, 0.5f);
-  t = fmaf(v, t, 1.0f);
-  const float series = v * t;
-  const float viaLog = -lg2f(u) * kLn2;
-  return v < 0.125f ? series : viaLog;
+// Exponential variates for the Gumbel-max draws, kept in NEGATIVE LOG2 UNITS:
+//   e = lg2 u' = -E / ln 2,   E = -ln u',   u' = ((w >> 9) + 1/2) 2^-23 in (0, 1).
+// Every comparison the draws enter (r / E of the exponential race, l/T - ln E
+// of a Gumbel score) is invariant under this fixed rescaling, so no ln 2
+// factor is ever applied.
+//
+// u' and v = 1 - u' are formed exactly from bits: the float with exponent 0
+// and mantissa j is 1 + j 2^-23, and subtracting 1 - 2^-24 from a float in
+// [1, 2) is exact (Sterbenz); the complemented mantissa 2^23 - 1 - j gives v.
+//
+// e must be accurate relative to its own size, also when it is tiny (u' near
+// 1), because small E are the ones that win.  So:
+//   v <  1/8 (w >= 0xE0000000):  lg2(1 - v) = -(v + v^2/2 + ... + v^7/7) / ln 2,
+//              Taylor series in Horner form (truncation below 7e-8 relative);
+//   v >= 1/8:  the hardware lg2 of u', whose absolute error (about 2^-22.6)
+//              is below 1e-6 relative here, since |lg2 u'| >= 0.19.
+constexpr float kOneMinusHalfUlp = 1.0f - 0x1p-24f;
+constexpr float kSeries1 = static_cast<float>(-1.4426950408889634 / 1.0);
+constexpr float kSeries2 = static_cast<float>(-1.4426950408889634 / 2.0);
+constexpr float kSeries3 = static_cast<float>(-1.4426950408889634 / 3.0);
+constexpr float kSeries4 = static_cast<float>(-1.4426950408889634 / 4.0);
+constexpr float kSeries5 = static_cast<float>(-1.4426950408889634 / 5.0);
+constexpr float kSeries6 = static_cast<float>(-1.4426950408889634 / 6.0);
+constexpr float kSeries7 = static_cast<float>(-1.4426950408889634 / 7.0);
+constexpr uint32_t kSeriesWords = 0xE0000000u;  // w >= this  <=>  v < 1/8
+
+__device__ __forceinline__ float bits_1j(uint32_t w) { return __uint_as_float(0x3f800000u + (w >> 9)); }
+__device__ __forceinline__ float bits_1jc(uint32_t w) { return __uint_as_float(0x3fffffffu - (w >> 9)); }
+
+__device__ __forceinline__ float neg_exp1_log2(uint32_t w) {
+  const float u = bits_1j(w) - kOneMinusHalfUlp;
+  const float v = bits_1jc(w) - kOneMinusHalfUlp;
+  float t = fmaf(v, kSeries7, kSeries6);
+  t = fmaf(v, t, kSeries5);
+  t = fmaf(v, t, kSeries4);
+  t = fmaf(v, t, kSeries3);
+  t = fmaf(v, t, kSeries2);
+  t = fmaf(v, t, kSeries1);
+  return w >= kSeriesWords ? v * t : lg2f(u);
 }
 
-// Gumbel noise g = -ln(-ln u') = -ln E.
-__device__ __forceinline__ float gumbel(uint32_t w) { return -lg2f(exp1_variate(w)) * kLn2; }
+// The same for two words at once (f32x2 arithmetic; identical values).
+__device__ __forceinline__ void neg_exp1_log2_x2(uint32_t w0, uint32_t w1, float& e0, float& e1) {
+  const unsigned long long c = splat2(-kOneMinusHalfUlp);
+  float u0, u1;
+  unpack2(add2(pack2(bits_1j(w0), bits_1j(w1)), c), u0, u1);
+  const unsigned long long v = add2(pack2(bits_1jc(w0), bits_1jc(w1)), c);
+  unsigned long long t = fma2(v, splat2(kSeries7), splat2(kSeries6));
+  t = fma2(v, t, splat2(kSeries5));
+  t = fma2(v, t, splat2(kSeries4));
+  t = fma2(v, t, splat2(kSeries3));
+  t = fma2(v, t, splat2(kSeries2));
+  t = fma2(v, t, splat2(kSeries1));
+  float s0, s1;
+  unpack2(mul2(v, t), s0, s1);
+  e0 = w0 >= kSeriesWords ? s0 : lg2f(u0);
+  e1 = w1 >= kSeriesWords ? s1 : lg2f(u1);
+}
+
+// Gumbel noise in log2 units: g / ln 2 = -lg2 E = -lg2(-e ln 2); the constant
+// -lg2(ln 2) is dropped, as it shifts every score of a row alike.
+__device__ __forceinline__ float gumbel_log2(float e) { return -lg2f(-e); }
 
 __device__ __forceinline__ uint32_t word_of(const uint4& v, int j) {
   return j == 0 ? v.x : (j == 1 ? v.y : (j == 2 ? v.z : v.w));

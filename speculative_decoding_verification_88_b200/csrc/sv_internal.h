@@ -66,7 +66,6 @@ struct StochParams {
   long long d_sb, d_sp;
   const int* tokens;  // [B, k]
   int B, k, V;
-  float invT;  // 1 / T
   float c2;    // log2(e) / T: logit -> log2-domain scale
   unsigned int key0, key1, seq_offset;
   int* accepted_len;

@@ -290,6 +290,26 @@ __device__ __forceinline__ void load_vecs(const unsigned char* smem, int nvec, i
   }
 }
 
+// Largest element of N vectors (the -inf padding included).
+template <typename T, int N>
+__device__ __forceinline__ float vecs_max(const uint4 (&v)[N]) {
+  if constexpr (Elem<T>::kBytes == 2) {
+    // bf16: a running packed maximum, one max.bf16x2 per two elements
+    uint32_t m = 0xff80ff80u;
+#pragma unroll
+    for (int j = 0; j < N; ++j) m = bmax2(m, bmax2(bmax2(v[j].x, v[j].y), bmax2(v[j].z, v[j].w)));
+    return fmaxf(bf16_lo(m), bf16_hi(m));
+  } else {
+    float m = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < N; ++j) {
+      m = fmax3(m, __uint_as_float(v[j].x), __uint_as_float(v[j].y));
+      m = fmax3(m, __uint_as_float(v[j].z), __uint_as_float(v[j].w));
+    }
+    return m;
+  }
+}
+
 // Thread-local (m, s): m = max * c2 (log2 units), s = sum 2^(x c2 - m)
 // over the thread's vectors plus its share of the ragged end in global
 // memory (entries [tail0, len)).
@@ -298,9 +318,7 @@ __device__ __forceinline__ void thread_stats(const uint4 (&v)[N], const void* g,
                                              int tail0, int len, float c2, int tid, float& m_out,
                                              float& s_out) {
   constexpr int EPV = Elem<T>::kPerVec;
-  float m = -INFINITY;
-#pragma unroll
-  for (int j = 0; j < N; ++j) m = fmaxf(m, vec_max<T>(v[j]));
+  float m = vecs_max<T>(v);
   float tail = -INFINITY;
   const int e = tail0 + tid;  // the ragged end is shorter than one vector
   if (e < len) tail = load_elem<T>(g, goff + e);
@@ -428,89 +446,99 @@ __device__ __forceinline__ uint4 vocab_words(const Draw& d, uint32_t c0) {
   return philox10(make_uint4(c0, d.pos, d.seq, d.tag), d.key0, d.key1);
 }
 
-// p(x) - q(x) from the logits and the row statistics.  Both products are
-// rounded on their own (no fused multiply-add), so identical target and
-// draft rows give exactly zero.
-__device__ __forceinline__ float residual(float lt, float ld, float c2, const Hdr& h) {
-  return __fsub_rn(__fmul_rn(ex2f(fmaf(lt, c2, -h.mt)), h.ist),
-                   __fmul_rn(ex2f(fmaf(ld, c2, -h.md)), h.isd));
+// Residual of the correction race, rescaled by the row's target sum s_t:
+//   r'(x) = 2^(l_t(x) c2 - m_t) - 2^(l_d(x) c2 - m_d + o),   o = lg2(1/s_d) - lg2(1/s_t),
+// which is s_t (p(x) - q(x)).  s_t is one positive constant per row, so the
+// winner of the race over r'/E is the winner over (p - q)/E.  Identical
+// target and draft rows have equal statistics, o = 0 exactly, and r' = 0
+// exactly.
+struct ResidualTerms {
+  float c2, mt, mdo;  // c2, m_t, m_d - o
+};
+__device__ __forceinline__ ResidualTerms residual_terms(float c2, const Hdr& h) {
+  return ResidualTerms{c2, h.mt, h.md - (lg2f(h.isd) - lg2f(h.ist))};
+}
+__device__ __forceinline__ float residual(float lt, float ld, const ResidualTerms& rt) {
+  return ex2f(fmaf(lt, rt.c2, -rt.mt)) - ex2f(fmaf(ld, rt.c2, -rt.mdo));
 }
 
-// The same for eight entries: the exponents two at a time (f32x2 FMA), the
-// products and the difference as scalar round-to-nearest operations.  (The
-// assembler may fuse a packed multiply with a following packed subtract into
-// one FMA, which leaves the product's rounding error behind, so p - q of
-// identical rows would not be zero.)
-__device__ __forceinline__ void residual8(const float (&lt)[8], const float (&ld)[8], float c2,
-                                          const Hdr& h, float (&r)[8]) {
-  const unsigned long long cc = pack2(c2, c2);
-  const unsigned long long mt = pack2(-h.mt, -h.mt), md = pack2(-h.md, -h.md);
+// The same for eight entries, two at a time (f32x2 exponents and difference).
+__device__ __forceinline__ void residual8(const float (&lt)[8], const float (&ld)[8],
+                                          const ResidualTerms& rt, float (&r)[8]) {
+  const unsigned long long cc = splat2(rt.c2);
+  const unsigned long long mt = splat2(-rt.mt), md = splat2(-rt.mdo);
 #pragma unroll
   for (int e = 0; e < 8; e += 2) {
     float a0, a1, b0, b1;
     unpack2(fma2(pack2(lt[e], lt[e + 1]), cc, mt), a0, a1);
     unpack2(fma2(pack2(ld[e], ld[e + 1]), cc, md), b0, b1);
-    r[e] = __fsub_rn(__fmul_rn(ex2f(a0), h.ist), __fmul_rn(ex2f(b0), h.isd));
-    r[e + 1] = __fsub_rn(__fmul_rn(ex2f(a1), h.ist), __fmul_rn(ex2f(b1), h.isd));
+    unpack2(sub2(pack2(ex2f(a0), ex2f(a1)), pack2(ex2f(b0), ex2f(b1))), r[e], r[e + 1]);
   }
 }
 
 // Exponential race: argmax_x r(x)/E(x) with E = -ln u'(x) is the Gumbel-max
-// argmax_x ln r(x) + g(x).  Keeps the best (r, E, x) of one thread.
+// argmax_x ln r(x) + g(x).  Keeps the best (r, e, x) of one thread, with e the
+// draw in negative log2 units (e = -E / ln 2 < 0).  r/E > b.r/b.E is
+// r b.e < b.r e; a candidate with r <= 0 never passes it (its left side is
+// >= 0 > the right side once b.r > 0, and -r < -0 fails for the initial
+// b = (0, -1)), and the first x is kept on a tie.
 struct Race {
   float r, e;
   int x;
 };
 
-__device__ __forceinline__ void race_push(Race& b, float r, uint32_t w, int x) {
-  const float e = exp1_variate(w);
-  // a candidate needs r > 0; r/e > b.r/b.e, the first x kept on a tie
-  const bool win = r > 0.0f && r * b.e > b.r * e;
+__device__ __forceinline__ void race_push(Race& b, float r, float e, int x) {
+  const bool win = r * b.e < b.r * e;
   b.r = win ? r : b.r;
   b.e = win ? e : b.e;
   b.x = win ? x : b.x;
 }
 
-// Gumbel-max over the positive residual r(x) = p(x) - q(x) of one chunk.
-// Returns the warp's best (score ln r - ln E, x); x = INT_MAX if the warp saw
-// no positive residual.
+// Gumbel-max over the positive residual of one chunk.  Returns the warp's
+// best (score lg2 r' - lg2 E + const, x); x = INT_MAX if the warp saw no
+// positive residual.
 template <typename TT, typename TD, bool kTma>
 __device__ __forceinline__ void chunk_residual(const unsigned char* ts, const unsigned char* ds,
                                                const Hdr& h, const void* tgt, const void* drf,
                                                float c2, const Draw& d, int tid, float& bv,
                                                int& bi) {
-  Race best{0.0f, 1.0f, INT_MAX};
+  const ResidualTerms rt = residual_terms(c2, h);
+  Race best{0.0f, -1.0f, INT_MAX};
   const int ng = kTma ? h.len / 8 : 0;
   for (int j = tid; j < ng; j += kComputeThreads) {
     float lt[8], ld[8], r[8];
     load8<TT>(ts, j, lt);
     load8<TD>(ds, j, ld);
-    residual8(lt, ld, c2, h, r);
+    residual8(lt, ld, rt, r);
     const int xg = h.x0 + 8 * j;
     // both Philox words in straight-line code, so their round chains
     // interleave; candidates are selected without branches
     const uint4 w0 = vocab_words(d, static_cast<uint32_t>(xg) >> 2);
     const uint4 w1 = vocab_words(d, (static_cast<uint32_t>(xg) >> 2) + 1u);
+    float e[8];
+    neg_exp1_log2_x2(w0.x, w0.y, e[0], e[1]);
+    neg_exp1_log2_x2(w0.z, w0.w, e[2], e[3]);
+    neg_exp1_log2_x2(w1.x, w1.y, e[4], e[5]);
+    neg_exp1_log2_x2(w1.z, w1.w, e[6], e[7]);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) race_push(best, r[q], word_of(w0, q), xg + q);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) race_push(best, r[4 + q], word_of(w1, q), xg + 4 + q);
+    for (int q = 0; q < 8; ++q) race_push(best, r[q], e[q], xg + q);
   }
   for (int e = 8 * ng + tid; e < h.len; e += kComputeThreads) {
     const int x = h.x0 + e;
-    const float r =
-        residual(load_elem<TT>(tgt, h.toff + e), load_elem<TD>(drf, h.doff + e), c2, h);
-    race_push(best, r, word_of(vocab_words(d, static_cast<uint32_t>(x) >> 2), x & 3), x);
+    const float r = residual(load_elem<TT>(tgt, h.toff + e), load_elem<TD>(drf, h.doff + e), rt);
+    race_push(best, r,
+              neg_exp1_log2(word_of(vocab_words(d, static_cast<uint32_t>(x) >> 2), x & 3)), x);
   }
-  bv = best.x == INT_MAX ? -INFINITY : (lg2f(best.r) - lg2f(best.e)) * kLn2;
+  bv = best.x == INT_MAX ? -INFINITY : lg2f(best.r) - lg2f(-best.e);
   bi = best.x;
   warp_argmax(bv, bi);
 }
 
-// Gumbel-max over l(x) / T of one chunk of the bonus row.
+// Gumbel-max over l(x) / T of one chunk of the bonus row, in log2 units:
+// the score is l(x) c2 + g(x) / ln 2 (c2 = log2(e) / T).
 template <typename TT, bool kTma>
 __device__ __forceinline__ void chunk_bonus(const unsigned char* ts, const Hdr& h,
-                                            const void* tgt, float invT, const Draw& d, int tid,
+                                            const void* tgt, float c2, const Draw& d, int tid,
                                             float& bv, int& bi) {
   bv = -INFINITY;
   bi = INT_MAX;
@@ -521,18 +549,24 @@ __device__ __forceinline__ void chunk_bonus(const unsigned char* ts, const Hdr& 
     const int xg = h.x0 + 8 * j;
     const uint4 w0 = vocab_words(d, static_cast<uint32_t>(xg) >> 2);
     const uint4 w1 = vocab_words(d, (static_cast<uint32_t>(xg) >> 2) + 1u);
+    float e[8];
+    neg_exp1_log2_x2(w0.x, w0.y, e[0], e[1]);
+    neg_exp1_log2_x2(w0.z, w0.w, e[2], e[3]);
+    neg_exp1_log2_x2(w1.x, w1.y, e[4], e[5]);
+    neg_exp1_log2_x2(w1.z, w1.w, e[6], e[7]);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const float sc = fmaf(lt[e], invT, gumbel(word_of(e < 4 ? w0 : w1, e & 3)));
+    for (int q = 0; q < 8; ++q) {
+      const float sc = fmaf(lt[q], c2, gumbel_log2(e[q]));
       const bool win = sc > bv;  // entries arrive in increasing x: first maximum kept
       bv = win ? sc : bv;
-      bi = win ? xg + e : bi;
+      bi = win ? xg + q : bi;
     }
   }
   for (int e = 8 * ng + tid; e < h.len; e += kComputeThreads) {
     const int x = h.x0 + e;
-    const float sc = fmaf(load_elem<TT>(tgt, h.toff + e), invT,
-                          gumbel(word_of(vocab_words(d, static_cast<uint32_t>(x) >> 2), x & 3)));
+    const float sc =
+        fmaf(load_elem<TT>(tgt, h.toff + e), c2,
+             gumbel_log2(neg_exp1_log2(word_of(vocab_words(d, static_cast<uint32_t>(x) >> 2), x & 3))));
     if (better(sc, x, bv, bi)) {
       bv = sc;
       bi = x;
@@ -743,7 +777,7 @@ __device__ void stoch_compute(const StochParams& p, Shared& sh, unsigned char* s
       if (h.kind == kKindCorrection)
         chunk_residual<TT, TD, kTma>(ts, ds, h, p.tgt, p.drf, p.c2, d, tid, bv, bi);
       else
-        chunk_bonus<TT, kTma>(ts, h, p.tgt, p.invT, d, tid, bv, bi);
+        chunk_bonus<TT, kTma>(ts, h, p.tgt, p.c2, d, tid, bv, bi);
       r = make_float4(bv, __int_as_float(bi), 0.0f, 0.0f);
     }
     if (lane == 0) {
@@ -879,8 +913,9 @@ __device__ void finalize_sample(const StochParams& p, int b, int n, int lane) {
     float bv = -INFINITY;
     int bi = INT_MAX;
     for (int x = lane; x < p.V; x += 32) {
-      const float sc = fmaf(load_elem<TT>(p.tgt, off + x), p.invT,
-                            gumbel(word_of(vocab_words(d, static_cast<uint32_t>(x) >> 2), x & 3)));
+      const float sc = fmaf(load_elem<TT>(p.tgt, off + x), p.c2,
+                            gumbel_log2(neg_exp1_log2(
+                                word_of(vocab_words(d, static_cast<uint32_t>(x) >> 2), x & 3))));
       if (better(sc, x, bv, bi)) {
         bv = sc;
         bi = x;
