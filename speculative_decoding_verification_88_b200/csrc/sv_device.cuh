@@ -199,18 +199,15 @@ __device__ __forceinline__ float accept_uniform(uint32_t w) {
 //
 // e must be accurate relative to its own size, also when it is tiny (u' near
 // 1), because small E are the ones that win.  So:
-//   v <  1/8 (w >= 0xE0000000):  lg2(1 - v) = -(v + v^2/2 + ... + v^7/7) / ln 2,
-//              Taylor series in Horner form (truncation below 7e-8 relative);
+//   v <  1/8 (w >= 0xE0000000):  lg2(1 - v) = -v g(v), g(v) = -ln(1 - v) / (v ln 2),
+//              with g the degree-4 polynomial that interpolates it at the five
+//              Chebyshev nodes of [0, 1/8] (relative error 1.4e-8, 8e-8 with
+//              fp32 rounding);
 //   v >= 1/8:  the hardware lg2 of u', whose absolute error (about 2^-22.6)
 //              is below 1e-6 relative here, since |lg2 u'| >= 0.19.
 constexpr float kOneMinusHalfUlp = 1.0f - 0x1p-24f;
-constexpr float kSeries1 = static_cast<float>(-1.4426950408889634 / 1.0);
-constexpr float kSeries2 = static_cast<float>(-1.4426950408889634 / 2.0);
-constexpr float kSeries3 = static_cast<float>(-1.4426950408889634 / 3.0);
-constexpr float kSeries4 = static_cast<float>(-1.4426950408889634 / 4.0);
-constexpr float kSeries5 = static_cast<float>(-1.4426950408889634 / 5.0);
-constexpr float kSeries6 = static_cast<float>(-1.4426950408889634 / 6.0);
-constexpr float kSeries7 = static_cast<float>(-1.4426950408889634 / 7.0);
+constexpr float kG0 = -1.44269506f, kG1 = -0.72133995f, kG2 = -0.48137748f,
+                kG3 = -0.35020793f, kG4 = -0.37898599f;  // -g(v) coefficients
 constexpr uint32_t kSeriesWords = 0xE0000000u;  // w >= this  <=>  v < 1/8
 
 __device__ __forceinline__ float bits_1j(uint32_t w) { return __uint_as_float(0x3f800000u + (w >> 9)); }
@@ -219,12 +216,10 @@ __device__ __forceinline__ float bits_1jc(uint32_t w) { return __uint_as_float(0
 __device__ __forceinline__ float neg_exp1_log2(uint32_t w) {
   const float u = bits_1j(w) - kOneMinusHalfUlp;
   const float v = bits_1jc(w) - kOneMinusHalfUlp;
-  float t = fmaf(v, kSeries7, kSeries6);
-  t = fmaf(v, t, kSeries5);
-  t = fmaf(v, t, kSeries4);
-  t = fmaf(v, t, kSeries3);
-  t = fmaf(v, t, kSeries2);
-  t = fmaf(v, t, kSeries1);
+  float t = fmaf(v, kG4, kG3);
+  t = fmaf(v, t, kG2);
+  t = fmaf(v, t, kG1);
+  t = fmaf(v, t, kG0);
   return w >= kSeriesWords ? v * t : lg2f(u);
 }
 
@@ -234,16 +229,39 @@ __device__ __forceinline__ void neg_exp1_log2_x2(uint32_t w0, uint32_t w1, float
   float u0, u1;
   unpack2(add2(pack2(bits_1j(w0), bits_1j(w1)), c), u0, u1);
   const unsigned long long v = add2(pack2(bits_1jc(w0), bits_1jc(w1)), c);
-  unsigned long long t = fma2(v, splat2(kSeries7), splat2(kSeries6));
-  t = fma2(v, t, splat2(kSeries5));
-  t = fma2(v, t, splat2(kSeries4));
-  t = fma2(v, t, splat2(kSeries3));
-  t = fma2(v, t, splat2(kSeries2));
-  t = fma2(v, t, splat2(kSeries1));
+  unsigned long long t = fma2(v, splat2(kG4), splat2(kG3));
+  t = fma2(v, t, splat2(kG2));
+  t = fma2(v, t, splat2(kG1));
+  t = fma2(v, t, splat2(kG0));
   float s0, s1;
   unpack2(mul2(v, t), s0, s1);
   e0 = w0 >= kSeriesWords ? s0 : lg2f(u0);
   e1 = w1 >= kSeriesWords ? s1 : lg2f(u1);
+}
+
+// 2^y for y <= 0, two at a time on the FMA pipe, to take part of the
+// exponentials off the special-function unit.  y is clamped at -126 (2^-126
+// is negligible against a sum that holds a term equal to 1), split as
+// y = j + f with j = rint(y) (adding and removing 1.5 * 2^23 rounds to an
+// integer) and f in [-1/2, 1/2]; 2^f is the degree-5 polynomial that
+// interpolates it at the six Chebyshev nodes of [-1/2, 1/2] (relative error
+// 1.0e-7, 2.2e-7 with fp32 rounding); 2^j enters by adding j to the exponent
+// field (the low bits of y + 1.5 * 2^23 hold j, shifted up by 23).
+__device__ __forceinline__ unsigned long long ex2_poly_x2(float y0, float y1) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  const unsigned long long y = pack2(fmaxf(y0, -126.0f), fmaxf(y1, -126.0f));
+  const unsigned long long t = add2(y, splat2(kRound));
+  const unsigned long long f = sub2(y, sub2(t, splat2(kRound)));
+  unsigned long long q = fma2(f, splat2(1.339086337e-03f), splat2(9.676031918e-03f));
+  q = fma2(f, q, splat2(5.550357114e-02f));
+  q = fma2(f, q, splat2(2.402210749e-01f));
+  q = fma2(f, q, splat2(6.931471880e-01f));
+  q = fma2(f, q, splat2(1.000000075e+00f));
+  float q0, q1, t0, t1;
+  unpack2(q, q0, q1);
+  unpack2(t, t0, t1);
+  return pack2(__uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23)),
+               __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23)));
 }
 
 // Gumbel noise in log2 units: g / ln 2 = -lg2 E = -lg2(-e ln 2); the constant

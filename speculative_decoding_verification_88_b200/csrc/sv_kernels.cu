@@ -283,11 +283,40 @@ template <typename T, int N>
 __device__ __forceinline__ void load_vecs(const unsigned char* smem, int nvec, int tid,
                                           uint4 (&v)[N]) {
   const uint4* sv = reinterpret_cast<const uint4*>(smem);
+  if (nvec == N * kComputeThreads) {  // a full chunk (uniform): no padding
 #pragma unroll
-  for (int j = 0; j < N; ++j) {
-    const int idx = tid + j * kComputeThreads;
-    v[j] = idx < nvec ? sv[idx] : neg_inf_vec<T>();
+    for (int j = 0; j < N; ++j) v[j] = sv[tid + j * kComputeThreads];
+  } else {
+#pragma unroll
+    for (int j = 0; j < N; ++j) {
+      const int idx = tid + j * kComputeThreads;
+      v[j] = idx < nvec ? sv[idx] : neg_inf_vec<T>();
+    }
   }
+}
+
+// One pair in kPolyEvery of the register-resident exponentials runs on the FMA
+// pipe (ex2_poly_x2) instead of the special-function unit, which the
+// statistics otherwise saturate.
+constexpr int kPolyEvery = 8;
+
+// Warp merge of per-thread (m, s) pairs of two tensors: the maxima first,
+// then one rescale per thread and a plain sum.
+__device__ __forceinline__ float4 warp_stats2(float4 r) {
+  float Mt = r.x, Md = r.z;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    Mt = fmaxf(Mt, __shfl_xor_sync(0xffffffffu, Mt, o));
+    Md = fmaxf(Md, __shfl_xor_sync(0xffffffffu, Md, o));
+  }
+  float st = Mt == -INFINITY ? 0.0f : r.y * ex2f(r.x - Mt);
+  float sd = Md == -INFINITY ? 0.0f : r.w * ex2f(r.z - Md);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    st += __shfl_xor_sync(0xffffffffu, st, o);
+    sd += __shfl_xor_sync(0xffffffffu, sd, o);
+  }
+  return make_float4(Mt, st, Md, sd);
 }
 
 // Largest element of N vectors (the -inf padding included).
@@ -337,7 +366,9 @@ __device__ __forceinline__ void thread_stats(const uint4 (&v)[N], const void* g,
       for (int q = 0; q < EPV; q += 2) {
         float a, b;
         unpack2(fma2(pack2(f[q], f[q + 1]), cc, mm), a, b);
-        const unsigned long long e = pack2(ex2f(a), ex2f(b));
+        const unsigned long long e = ((j * EPV + q) / 2) % kPolyEvery == kPolyEvery - 1
+                                         ? ex2_poly_x2(a, b)
+                                         : pack2(ex2f(a), ex2f(b));
         if ((q & 2) == 0) acc0 = add2(acc0, e);
         else acc1 = add2(acc1, e);
       }
@@ -365,16 +396,7 @@ __device__ __forceinline__ float4 chunk_stats_pair(const unsigned char* ts,
   float4 r;
   thread_stats<TT>(vt, tgt, h.toff, h.nvec_t * Elem<TT>::kPerVec, h.len, c2, tid, r.x, r.y);
   thread_stats<TD>(vd, drf, h.doff, h.nvec_d * Elem<TD>::kPerVec, h.len, c2, tid, r.z, r.w);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const float a = __shfl_xor_sync(0xffffffffu, r.x, o);
-    const float b = __shfl_xor_sync(0xffffffffu, r.y, o);
-    const float c = __shfl_xor_sync(0xffffffffu, r.z, o);
-    const float d = __shfl_xor_sync(0xffffffffu, r.w, o);
-    merge_stats(r.x, r.y, a, b);
-    merge_stats(r.z, r.w, c, d);
-  }
-  return r;
+  return warp_stats2(r);
 }
 
 // Argmax (first maximum) of a chunk held in shared memory, merged over the
@@ -386,27 +408,27 @@ __device__ __forceinline__ void chunk_argmax_regs(const unsigned char* smem, con
   constexpr int N = max_vecs<T, 0>();
   uint4 v[N];
   load_vecs<T>(smem, h.nvec_t, tid, v);
+  // one pass: the first vector holding the thread's maximum, kept whole
   float best = -INFINITY;
   int bj = -1;
+  uint4 bvec = v[0];
+  const bool full = h.nvec_t == N * kComputeThreads;
 #pragma unroll
   for (int j = 0; j < N; ++j) {
     const float m = vec_max<T>(v[j]);
-    if (tid + j * kComputeThreads < h.nvec_t && (bj < 0 || m > best)) {
-      best = m;
-      bj = j;
-    }
+    const bool take = (full || tid + j * kComputeThreads < h.nvec_t) && (bj < 0 || m > best);
+    best = take ? m : best;
+    bj = take ? j : bj;
+    bvec = take ? v[j] : bvec;
   }
   int idx = INT_MAX;
+  if (bj >= 0) {
+    float f[EPV];
+    unpack(bvec, f);
+    const int x = h.x0 + (tid + bj * kComputeThreads) * EPV;
 #pragma unroll
-  for (int j = 0; j < N; ++j) {
-    if (j == bj) {
-      float f[EPV];
-      unpack(v[j], f);
-      const int x = h.x0 + (tid + j * kComputeThreads) * EPV;
-#pragma unroll
-      for (int q = EPV - 1; q >= 0; --q)
-        if (f[q] == best) idx = x + q;
-    }
+    for (int q = EPV - 1; q >= 0; --q)
+      if (f[q] == best) idx = x + q;
   }
   const int e = h.nvec_t * EPV + tid;  // the ragged end is shorter than one vector
   if (e < h.len) {
