@@ -129,6 +129,24 @@ __device__ __forceinline__ void st_release_u32(unsigned int* p, unsigned int v) 
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
+__device__ __forceinline__ unsigned int ld_relaxed_u32(const unsigned int* p) {
+  unsigned int v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// With a preceding relaxed load that saw a release store, makes the writer's
+// earlier stores visible to this thread's later accesses.
+__device__ __forceinline__ void fence_acq_rel_gpu() {
+  asm volatile("fence.acq_rel.gpu;" ::: "memory");
+}
+
+// Orders this thread's generic-proxy accesses to global memory before its
+// later async-proxy (bulk copy) accesses, and the reverse.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 __device__ __forceinline__ bool aborted(const Ctrl* ctrl) {
   return (*reinterpret_cast<const volatile unsigned int*>(&ctrl->flags) & kFlagTimeout) != 0;
 }

@@ -64,7 +64,13 @@ namespace sv {
 enum : int { kKindEnd = 0, kKindStats = 1, kKindCorrection = 2, kKindBonus = 3, kKindArgmax = 4 };
 
 constexpr int kComputeThreads = kGroupWarps * 32;  // threads that share one chunk
-constexpr unsigned int kGrab = 2;                 // tickets per atomicAdd
+// Tickets per atomicAdd (the next grab's atomic is always in flight).
+// Argmax chunks are uniform work, so larger grabs save atomics; stochastic
+// tickets are taken one at a time, which balances the uneven phase-1 and
+// phase-2 chunks best (grabs of 2 and 3 measured 3% and 19% slower on
+// B = 256, k = 8, V = 128256).
+constexpr unsigned int kGrabStoch = 1;
+constexpr unsigned int kGrabArgmax = 8;
 constexpr unsigned long long kNoCandidate = 1ull;  // phase-2 key: no positive residual
 
 struct Hdr {
@@ -76,7 +82,6 @@ struct Hdr {
   int len;     // entries in the chunk
   int nvec_t;  // full 16-byte target vectors in shared memory
   int nvec_d;  // full 16-byte draft vectors in shared memory
-  float mt, ist, md, isd;  // correction: row-n statistics
   long long toff;          // element offset of entry x0 in the target
   long long doff;          // element offset of entry x0 in the draft
 };
@@ -87,6 +92,7 @@ struct Shared {
   uint64_t rfull[kStages];  // compute -> epilogue (warp records written)
   Hdr hdr[kStages];
   float4 res[kStages][kGroupWarps];
+  float4 rstat[kStages];  // correction: row-n (m_t, 1/s_t, m_d, 1/s_d), bulk-copied
 };
 
 constexpr size_t kSharedHead = (sizeof(Shared) + 127) / 128 * 128;
@@ -144,17 +150,21 @@ __device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v)
 
 // ------------------------------------------------------------------ waits
 
-__device__ __forceinline__ bool wait_flag(const unsigned int* flag, Ctrl* ctrl) {
-  if (ld_acquire_u32(flag)) return true;
+// Waits (bounded) for a nonzero flag; returns its value, or 0 on abort or
+// timeout.  Acquire: the flag's writer's earlier stores are visible after.
+__device__ __forceinline__ unsigned int wait_flag(const unsigned int* flag, Ctrl* ctrl) {
+  unsigned int v = ld_acquire_u32(flag);
+  if (v) return v;
   const unsigned long long t0 = global_ns();
   for (unsigned int spin = 1;; ++spin) {
     __nanosleep(32);
-    if (ld_acquire_u32(flag)) return true;
+    v = ld_acquire_u32(flag);
+    if (v) return v;
     if ((spin & 63u) == 0u) {
-      if (aborted(ctrl)) return false;
+      if (aborted(ctrl)) return 0u;
       if (global_ns() - t0 > kWaitLimitNs) {
         atomicOr(&ctrl->flags, kFlagTimeout);
-        return false;
+        return 0u;
       }
     }
   }
@@ -184,22 +194,26 @@ __device__ __forceinline__ void leave_grid(Ctrl* ctrl) {
 
 // Fill stage `s` with the chunk described by `h` (bulk copies of the full
 // 16-byte vectors; the ragged end is read by the compute warps directly).
+// `stat` (nullable, 16-byte aligned, global): a row-statistics record that
+// goes to sh.rstat[s] with the chunk.
 template <typename TT, typename TD, bool kTma>
 __device__ __forceinline__ void issue_chunk(Shared& sh, unsigned char* stage, int s, Hdr& h,
                                             const void* tgt, const void* drf, int ch,
-                                            bool with_draft) {
+                                            bool with_draft, const float4* stat) {
   h.nvec_t = kTma ? (h.len * Elem<TT>::kBytes) / 16 : 0;
   h.nvec_d = (kTma && with_draft) ? (h.len * Elem<TD>::kBytes) / 16 : 0;
   sh.hdr[s] = h;
   if (kTma) {
     const uint32_t bt = static_cast<uint32_t>(h.nvec_t) * 16u;
     const uint32_t bd = static_cast<uint32_t>(h.nvec_d) * 16u;
-    mbar_arrive_expect_tx(&sh.full[s], bt + bd);
+    mbar_arrive_expect_tx(&sh.full[s], bt + bd + (stat ? 16u : 0u));
     if (bt) bulk_load(stage, reinterpret_cast<const TT*>(tgt) + h.toff, bt, &sh.full[s]);
     if (bd)
       bulk_load(stage + static_cast<size_t>(ch) * Elem<TT>::kBytes,
                 reinterpret_cast<const TD*>(drf) + h.doff, bd, &sh.full[s]);
+    if (stat) bulk_load(&sh.rstat[s], stat, 16u, &sh.full[s]);
   } else {
+    if (stat) sh.rstat[s] = __ldcg(stat);
     mbar_arrive(&sh.full[s]);
   }
 }
@@ -477,8 +491,8 @@ __device__ __forceinline__ uint4 vocab_words(const Draw& d, uint32_t c0) {
 struct ResidualTerms {
   float c2, mt, mdo;  // c2, m_t, m_d - o
 };
-__device__ __forceinline__ ResidualTerms residual_terms(float c2, const Hdr& h) {
-  return ResidualTerms{c2, h.mt, h.md - (lg2f(h.isd) - lg2f(h.ist))};
+__device__ __forceinline__ ResidualTerms residual_terms(float c2, const float4& st) {
+  return ResidualTerms{c2, st.x, st.z - (lg2f(st.w) - lg2f(st.y))};
 }
 __device__ __forceinline__ float residual(float lt, float ld, const ResidualTerms& rt) {
   return ex2f(fmaf(lt, rt.c2, -rt.mt)) - ex2f(fmaf(ld, rt.c2, -rt.mdo));
@@ -521,10 +535,10 @@ __device__ __forceinline__ void race_push(Race& b, float r, float e, int x) {
 // positive residual.
 template <typename TT, typename TD, bool kTma>
 __device__ __forceinline__ void chunk_residual(const unsigned char* ts, const unsigned char* ds,
-                                               const Hdr& h, const void* tgt, const void* drf,
-                                               float c2, const Draw& d, int tid, float& bv,
-                                               int& bi) {
-  const ResidualTerms rt = residual_terms(c2, h);
+                                               const Hdr& h, const float4& st, const void* tgt,
+                                               const void* drf, float c2, const Draw& d, int tid,
+                                               float& bv, int& bi) {
+  const ResidualTerms rt = residual_terms(c2, st);
   Race best{0.0f, -1.0f, INT_MAX};
   const int ng = kTma ? h.len / 8 : 0;
   for (int j = tid; j < ng; j += kComputeThreads) {
@@ -638,7 +652,8 @@ __device__ __forceinline__ void chunk_argmax(const unsigned char* smem, const Hd
 // Place a chunk in the next ring stage (waits for the stage to be free).
 template <typename TT, typename TD, bool kTma>
 __device__ __forceinline__ bool stoch_issue(const StochParams& p, Shared& sh,
-                                            unsigned char* stages, uint32_t& use, Hdr& h) {
+                                            unsigned char* stages, uint32_t& use, Hdr& h,
+                                            const float4* stat) {
   h.x0 = h.c * p.ch;
   h.len = min(p.ch, p.V - h.x0);
   h.toff = static_cast<long long>(h.b) * p.t_sb + static_cast<long long>(h.i) * p.t_sp + h.x0;
@@ -646,63 +661,84 @@ __device__ __forceinline__ bool stoch_issue(const StochParams& p, Shared& sh,
   const int s = use % kStages;
   if (!mbar_wait(&sh.empty[s], ((use / kStages) & 1u) ^ 1u, p.ctrl)) return false;
   issue_chunk<TT, TD, kTma>(sh, stages + static_cast<size_t>(s) * kStageBytes, s, h, p.tgt,
-                            p.drf, p.ch, h.kind != kKindBonus);
+                            p.drf, p.ch, h.kind != kKindBonus, stat);
   ++use;
   return true;
 }
 
-// Phase-2 chunk c of sequence b, whose accepted length is published.
+// Phase-2 chunk c of sequence b.  `ready` is the sequence's published flag,
+// n + 1, already acquired (load + fence) by the caller.  The correction's row
+// statistics travel with the chunk as a 16-byte bulk copy.
 template <typename TT, typename TD, bool kTma>
 __device__ __forceinline__ bool stoch_issue_phase2(const StochParams& p, Shared& sh,
                                                    unsigned char* stages, uint32_t& use, int b,
-                                                   int c) {
+                                                   int c, unsigned int ready) {
   Hdr h;
   h.b = b;
   h.c = c;
   // clamped so that no workspace content can steer a read outside the tensors
-  const int n = p.k > 0 ? min(max(__ldcg(&p.seq[b].n), 0), p.k) : 0;
+  const int n = p.k > 0 ? min(max(static_cast<int>(ready) - 1, 0), p.k) : 0;
   h.i = n;
+  const float4* stat = nullptr;
   if (n < p.k) {
     h.kind = kKindCorrection;
-    h.mt = __ldcg(&p.seq[b].mt);
-    h.ist = __ldcg(&p.seq[b].ist);
-    h.md = __ldcg(&p.seq[b].md);
-    h.isd = __ldcg(&p.seq[b].isd);
+    stat = reinterpret_cast<const float4*>(&p.seq[b].mt);
+    if (kTma) fence_proxy_async_global();
   } else {
     h.kind = kKindBonus;
   }
-  return stoch_issue<TT, TD, kTma>(p, sh, stages, use, h);
+  return stoch_issue<TT, TD, kTma>(p, sh, stages, use, h, stat);
 }
 
+// The producer takes tickets kGrabStoch at a time (the next grab's atomic in
+// flight meanwhile) and decodes them incrementally: ticket t is slot
+// t / slot_items, offset o = t % slot_items; offsets below k * nch are
+// phase-1 chunks (i, c) = (o / nch, o % nch) of sequence `slot`, the rest
+// phase-2 chunks of sequence slot - lag.  A phase-2 chunk whose sequence is
+// not ready yet is set aside (at most kDefer); set-aside chunks are polled
+// together with relaxed loads and issued once ready.
 template <typename TT, typename TD, bool kTma>
 __device__ void stoch_producer(const StochParams& p, Shared& sh, unsigned char* stages) {
   constexpr int kDefer = 4;
   Ctrl* ctrl = p.ctrl;
-  const unsigned int p1_items = static_cast<unsigned int>(p.k) * static_cast<unsigned int>(p.nch);
+  const unsigned int nch = static_cast<unsigned int>(p.nch);
+  const unsigned int p1_items = static_cast<unsigned int>(p.k) * nch;
   uint32_t use = 0;
   bool ok = true;
   int db[kDefer], dc[kDefer];  // set-aside phase-2 chunks, oldest first
   int nd = 0;
-  unsigned int base = atomicAdd(&ctrl->ticket, kGrab), next = 0u, j = 0u;
+  unsigned int base = atomicAdd(&ctrl->ticket, kGrabStoch), next = 0u, j = 0u;
   bool prefetched = false;
+  unsigned int slot = 0u, o = 0u, ci = 0u, cc = 0u;  // decoded ticket base + j
   while (ok) {
-    // set-aside chunks whose sequence became ready go first
-    int keep = 0;
+    if (nd > 0) {
+      unsigned int rd[kDefer];
+      bool any = false;
 #pragma unroll
-    for (int d = 0; d < kDefer; ++d) {
-      if (d < nd) {
-        if (ok && ld_acquire_u32(&p.seq[db[d]].ready)) {
-          ok = stoch_issue_phase2<TT, TD, kTma>(p, sh, stages, use, db[d], dc[d]);
-        } else {
-          db[keep] = db[d];
-          dc[keep] = dc[d];
-          ++keep;
+      for (int d = 0; d < kDefer; ++d) {
+        rd[d] = d < nd ? ld_relaxed_u32(&p.seq[db[d]].ready) : 0u;
+        any |= rd[d] != 0u;
+      }
+      if (any) {
+        fence_acq_rel_gpu();
+        int keep = 0;
+#pragma unroll
+        for (int d = 0; d < kDefer; ++d) {
+          if (d < nd) {
+            if (ok && rd[d]) {
+              ok = stoch_issue_phase2<TT, TD, kTma>(p, sh, stages, use, db[d], dc[d], rd[d]);
+            } else {
+              db[keep] = db[d];
+              dc[keep] = dc[d];
+              ++keep;
+            }
+          }
         }
+        nd = keep;
+        if (!ok) break;
       }
     }
-    nd = keep;
-    if (!ok) break;
-    if (base >= p.total) {  // no fresh tickets left
+    if (base >= p.total) {  // no fresh tickets left: wait for the oldest set-aside chunk
       if (nd == 0) break;
       if (!wait_flag(&p.seq[db[0]].ready, ctrl)) {
         ok = false;
@@ -711,38 +747,54 @@ __device__ void stoch_producer(const StochParams& p, Shared& sh, unsigned char* 
       continue;
     }
     if (!prefetched) {
-      next = atomicAdd(&ctrl->ticket, kGrab);  // overlaps the chunks of this grab
+      next = atomicAdd(&ctrl->ticket, kGrabStoch);  // overlaps the chunks of this grab
       prefetched = true;
     }
     const unsigned int t = base + j;
-    if (++j == kGrab) {
+    if (j == 0u) {
+      slot = t / p.slot_items;
+      o = t % p.slot_items;
+      ci = o < p1_items ? o / nch : 0u;
+      cc = o < p1_items ? o % nch : 0u;
+    } else if (++o == p.slot_items) {
+      o = 0u;
+      ++slot;
+      ci = 0u;
+      cc = 0u;
+    } else if (o < p1_items && ++cc == nch) {
+      cc = 0u;
+      ++ci;
+    }
+    if (++j == kGrabStoch) {
       j = 0u;
       base = next;
       prefetched = false;
     }
     if (t >= p.total) continue;
-    const unsigned int slot = t / p.slot_items, o = t % p.slot_items;
     if (o < p1_items) {
       if (static_cast<int>(slot) >= p.B) continue;
       Hdr h;
       h.kind = kKindStats;
       h.b = static_cast<int>(slot);
-      h.i = static_cast<int>(o) / p.nch;
-      h.c = static_cast<int>(o) % p.nch;
-      ok = stoch_issue<TT, TD, kTma>(p, sh, stages, use, h);
+      h.i = static_cast<int>(ci);
+      h.c = static_cast<int>(cc);
+      ok = stoch_issue<TT, TD, kTma>(p, sh, stages, use, h, nullptr);
     } else {
       const int b = static_cast<int>(slot) - p.lag;
       if (b < 0 || b >= p.B) continue;
       const int c = static_cast<int>(o - p1_items);
-      if (p.k == 0 || ld_acquire_u32(&p.seq[b].ready)) {
-        ok = stoch_issue_phase2<TT, TD, kTma>(p, sh, stages, use, b, c);
+      const unsigned int rd = p.k == 0 ? 1u : ld_relaxed_u32(&p.seq[b].ready);
+      if (rd) {
+        if (p.k > 0) fence_acq_rel_gpu();
+        ok = stoch_issue_phase2<TT, TD, kTma>(p, sh, stages, use, b, c, rd);
       } else {
         if (nd == kDefer) {  // queue full: the oldest must go first
-          if (!wait_flag(&p.seq[db[0]].ready, ctrl)) {
+          const unsigned int r0 = wait_flag(&p.seq[db[0]].ready, ctrl);
+          if (!r0) {
             ok = false;
             break;
           }
-          ok = stoch_issue_phase2<TT, TD, kTma>(p, sh, stages, use, db[0], dc[0]);
+          ok = stoch_issue_phase2<TT, TD, kTma>(p, sh, stages, use, db[0], dc[0], r0);
 #pragma unroll
           for (int d = 1; d < kDefer; ++d) {
             db[d - 1] = db[d];
@@ -797,7 +849,8 @@ __device__ void stoch_compute(const StochParams& p, Shared& sh, unsigned char* s
       float bv;
       int bi;
       if (h.kind == kKindCorrection)
-        chunk_residual<TT, TD, kTma>(ts, ds, h, p.tgt, p.drf, p.c2, d, tid, bv, bi);
+        chunk_residual<TT, TD, kTma>(ts, ds, h, sh.rstat[s], p.tgt, p.drf, p.c2, d, tid, bv,
+                                     bi);
       else
         chunk_bonus<TT, kTma>(ts, h, p.tgt, p.c2, d, tid, bv, bi);
       r = make_float4(bv, __int_as_float(bi), 0.0f, 0.0f);
@@ -873,7 +926,8 @@ __device__ void finalize_accept(const StochParams& p, int b, int lane) {
     r->isd = 1.0f / ssd;
     r->cnt1 = 0u;
     __threadfence();
-    st_release_u32(&r->ready, 1u);
+    fence_proxy_async_global();
+    st_release_u32(&r->ready, static_cast<unsigned int>(n) + 1u);
   }
 }
 
@@ -1066,10 +1120,10 @@ __device__ void argmax_producer(const ArgmaxParams& p, Shared& sh, unsigned char
   const unsigned int per_seq = R * static_cast<unsigned int>(p.nch);
   uint32_t use = 0;
   bool ok = true;
-  unsigned int base = atomicAdd(&ctrl->ticket, kGrab);
+  unsigned int base = atomicAdd(&ctrl->ticket, kGrabArgmax);
   while (ok && base < p.total) {
-    const unsigned int next = atomicAdd(&ctrl->ticket, kGrab);
-    for (unsigned int j = 0; j < kGrab; ++j) {
+    const unsigned int next = atomicAdd(&ctrl->ticket, kGrabArgmax);
+    for (unsigned int j = 0; j < kGrabArgmax; ++j) {
       const unsigned int t = base + j;
       if (t >= p.total) break;
       Hdr h;
@@ -1090,7 +1144,7 @@ __device__ void argmax_producer(const ArgmaxParams& p, Shared& sh, unsigned char
         break;
       }
       issue_chunk<TT, TT, kTma>(sh, stages + static_cast<size_t>(s) * kStageBytes, s, h, p.tgt,
-                                nullptr, p.ch, false);
+                                nullptr, p.ch, false, nullptr);
       ++use;
     }
     base = next;
