@@ -218,6 +218,66 @@ __device__ __forceinline__ void issue_chunk(Shared& sh, unsigned char* stage, in
   }
 }
 
+// --- per-group rings (stochastic kernel) -----------------------------------
+// Compute group g owns stages g and g + 2; its j-th use is stage
+// g + 2 (j % 2), phase (j / 2) & 1 -- the order in which its compute warps and
+// its epilogue warp walk them.  The producer keeps one use counter per group
+// and gives each chunk to whichever group frees a stage first, so a group
+// busy with a long chunk does not hold the other back.
+constexpr int kGroupStages = kStages / kComputeGroups;
+static_assert(kGroupStages * kComputeGroups == kStages, "stages split evenly over groups");
+
+__device__ __forceinline__ int group_stage(int g, uint32_t j) {
+  return g + kComputeGroups * static_cast<int>(j % kGroupStages);
+}
+__device__ __forceinline__ uint32_t group_phase(uint32_t j) { return (j / kGroupStages) & 1u; }
+
+// Waits (bounded) until some group's next stage is free; returns that group,
+// trying `pref` first, or -1 on abort or timeout.
+__device__ int take_group_stage(Shared& sh, const uint32_t (&used)[kComputeGroups], int pref,
+                                Ctrl* ctrl) {
+  const unsigned long long t0 = global_ns();
+  for (unsigned int spin = 0;; ++spin) {
+#pragma unroll
+    for (int q = 0; q < kComputeGroups; ++q) {
+      const int g = (pref + q) % kComputeGroups;
+      if (mbar_test_wait(&sh.empty[group_stage(g, used[g])], group_phase(used[g]) ^ 1u)) return g;
+    }
+    if ((spin & 255u) == 255u) {
+      if (aborted(ctrl)) return -1;
+      if (global_ns() - t0 > kWaitLimitNs) {
+        atomicOr(&ctrl->flags, kFlagTimeout);
+        return -1;
+      }
+    }
+  }
+}
+
+// One end marker into each group's next stage.
+__device__ __forceinline__ void push_group_ends(Shared& sh, const uint32_t (&used)[kComputeGroups],
+                                                Ctrl* ctrl) {
+  for (int g = 0; g < kComputeGroups; ++g) {
+    const int s = group_stage(g, used[g]);
+    if (!mbar_wait(&sh.empty[s], group_phase(used[g]) ^ 1u, ctrl)) return;
+    sh.hdr[s].kind = kKindEnd;
+    mbar_arrive(&sh.full[s]);
+  }
+}
+
+// After an abort: wait (bounded) until the last bulk copy issued into each
+// group's stages has landed.
+__device__ void drain_group_stages(Shared& sh, const uint32_t (&used)[kComputeGroups]) {
+  for (int g = 0; g < kComputeGroups; ++g) {
+    for (uint32_t r = 0; r < static_cast<uint32_t>(kGroupStages) && r < used[g]; ++r) {
+      const uint32_t last = r + ((used[g] - 1 - r) / kGroupStages) * kGroupStages;
+      const unsigned long long t0 = global_ns();
+      while (!mbar_try_wait(&sh.full[group_stage(g, r)], group_phase(last))) {
+        if (global_ns() - t0 > 100000000ull) break;
+      }
+    }
+  }
+}
+
 // Push one end marker per compute group into the next stages.
 __device__ __forceinline__ void push_end(Shared& sh, uint32_t use, Ctrl* ctrl) {
   for (int g = 0; g < kComputeGroups; ++g, ++use) {
@@ -652,17 +712,20 @@ __device__ __forceinline__ void chunk_argmax(const unsigned char* smem, const Hd
 // Place a chunk in the next ring stage (waits for the stage to be free).
 template <typename TT, typename TD, bool kTma>
 __device__ __forceinline__ bool stoch_issue(const StochParams& p, Shared& sh,
-                                            unsigned char* stages, uint32_t& use, Hdr& h,
+                                            unsigned char* stages,
+                                            uint32_t (&used)[kComputeGroups], int& pref, Hdr& h,
                                             const float4* stat) {
   h.x0 = h.c * p.ch;
   h.len = min(p.ch, p.V - h.x0);
   h.toff = static_cast<long long>(h.b) * p.t_sb + static_cast<long long>(h.i) * p.t_sp + h.x0;
   h.doff = static_cast<long long>(h.b) * p.d_sb + static_cast<long long>(h.i) * p.d_sp + h.x0;
-  const int s = use % kStages;
-  if (!mbar_wait(&sh.empty[s], ((use / kStages) & 1u) ^ 1u, p.ctrl)) return false;
+  const int g = take_group_stage(sh, used, pref, p.ctrl);
+  if (g < 0) return false;
+  const int s = group_stage(g, used[g]);
   issue_chunk<TT, TD, kTma>(sh, stages + static_cast<size_t>(s) * kStageBytes, s, h, p.tgt,
                             p.drf, p.ch, h.kind != kKindBonus, stat);
-  ++use;
+  ++used[g];
+  pref = (g + 1) % kComputeGroups;  // alternate while both have room
   return true;
 }
 
@@ -671,8 +734,9 @@ __device__ __forceinline__ bool stoch_issue(const StochParams& p, Shared& sh,
 // statistics travel with the chunk as a 16-byte bulk copy.
 template <typename TT, typename TD, bool kTma>
 __device__ __forceinline__ bool stoch_issue_phase2(const StochParams& p, Shared& sh,
-                                                   unsigned char* stages, uint32_t& use, int b,
-                                                   int c, unsigned int ready) {
+                                                   unsigned char* stages,
+                                                   uint32_t (&used)[kComputeGroups], int& pref,
+                                                   int b, int c, unsigned int ready) {
   Hdr h;
   h.b = b;
   h.c = c;
@@ -687,7 +751,7 @@ __device__ __forceinline__ bool stoch_issue_phase2(const StochParams& p, Shared&
   } else {
     h.kind = kKindBonus;
   }
-  return stoch_issue<TT, TD, kTma>(p, sh, stages, use, h, stat);
+  return stoch_issue<TT, TD, kTma>(p, sh, stages, used, pref, h, stat);
 }
 
 // The producer takes tickets kGrabStoch at a time (the next grab's atomic in
@@ -703,7 +767,8 @@ __device__ void stoch_producer(const StochParams& p, Shared& sh, unsigned char* 
   Ctrl* ctrl = p.ctrl;
   const unsigned int nch = static_cast<unsigned int>(p.nch);
   const unsigned int p1_items = static_cast<unsigned int>(p.k) * nch;
-  uint32_t use = 0;
+  uint32_t used[kComputeGroups] = {};  // uses issued per group
+  int pref = 0;
   bool ok = true;
   int db[kDefer], dc[kDefer];  // set-aside phase-2 chunks, oldest first
   int nd = 0;
@@ -726,7 +791,7 @@ __device__ void stoch_producer(const StochParams& p, Shared& sh, unsigned char* 
         for (int d = 0; d < kDefer; ++d) {
           if (d < nd) {
             if (ok && rd[d]) {
-              ok = stoch_issue_phase2<TT, TD, kTma>(p, sh, stages, use, db[d], dc[d], rd[d]);
+              ok = stoch_issue_phase2<TT, TD, kTma>(p, sh, stages, used, pref, db[d], dc[d], rd[d]);
             } else {
               db[keep] = db[d];
               dc[keep] = dc[d];
@@ -778,7 +843,7 @@ __device__ void stoch_producer(const StochParams& p, Shared& sh, unsigned char* 
       h.b = static_cast<int>(slot);
       h.i = static_cast<int>(ci);
       h.c = static_cast<int>(cc);
-      ok = stoch_issue<TT, TD, kTma>(p, sh, stages, use, h, nullptr);
+      ok = stoch_issue<TT, TD, kTma>(p, sh, stages, used, pref, h, nullptr);
     } else {
       const int b = static_cast<int>(slot) - p.lag;
       if (b < 0 || b >= p.B) continue;
@@ -786,7 +851,7 @@ __device__ void stoch_producer(const StochParams& p, Shared& sh, unsigned char* 
       const unsigned int rd = p.k == 0 ? 1u : ld_relaxed_u32(&p.seq[b].ready);
       if (rd) {
         if (p.k > 0) fence_acq_rel_gpu();
-        ok = stoch_issue_phase2<TT, TD, kTma>(p, sh, stages, use, b, c, rd);
+        ok = stoch_issue_phase2<TT, TD, kTma>(p, sh, stages, used, pref, b, c, rd);
       } else {
         if (nd == kDefer) {  // queue full: the oldest must go first
           const unsigned int r0 = wait_flag(&p.seq[db[0]].ready, ctrl);
@@ -794,7 +859,7 @@ __device__ void stoch_producer(const StochParams& p, Shared& sh, unsigned char* 
             ok = false;
             break;
           }
-          ok = stoch_issue_phase2<TT, TD, kTma>(p, sh, stages, use, db[0], dc[0], r0);
+          ok = stoch_issue_phase2<TT, TD, kTma>(p, sh, stages, used, pref, db[0], dc[0], r0);
 #pragma unroll
           for (int d = 1; d < kDefer; ++d) {
             db[d - 1] = db[d];
@@ -809,10 +874,10 @@ __device__ void stoch_producer(const StochParams& p, Shared& sh, unsigned char* 
     }
   }
   if (ok) {
-    push_end(sh, use, ctrl);
+    push_group_ends(sh, used, ctrl);
     leave_grid(ctrl);
   } else if (kTma) {
-    drain_stages(sh, use);
+    drain_group_stages(sh, used);
   }
 }
 
