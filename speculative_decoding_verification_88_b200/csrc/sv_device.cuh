@@ -387,22 +387,22 @@ __device__ __forceinline__ bool better(float v, int i, float bv, int bi) {
   return v > bv || (v == bv && i < bi);
 }
 
-__device__ __forceinline__ void warp_argmax(float& v, int& i) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const float ov = __shfl_xor_sync(0xffffffffu, v, o);
-    const int oi = __shfl_xor_sync(0xffffffffu, i, o);
-    if (better(ov, oi, v, i)) {
-      v = ov;
-      i = oi;
-    }
-  }
+// Warp-wide maximum of a float (sm_100 redux; a NaN operand is ignored).
+__device__ __forceinline__ float warp_max(float v) {
+  float m;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(m) : "f"(v));
+  return m;
 }
 
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
+// Warp-wide argmax in the order of better(): the largest value, and among
+// lanes holding it (-0 and +0 alike) the lowest index.  Every lane gets it.
+__device__ __forceinline__ void warp_argmax(float& v, int& i) {
+  const float m = warp_max(v);
+  const unsigned int cand = v == m ? static_cast<unsigned int>(i) : 0xffffffffu;
+  unsigned int r;
+  asm volatile("redux.sync.min.u32 %0, %1, 0xffffffff;" : "=r"(r) : "r"(cand));
+  v = m;
+  i = static_cast<int>(r);
 }
 
 __device__ __forceinline__ float warp_sum(float v) {

@@ -377,12 +377,7 @@ constexpr int kPolyEvery = 8;
 // Warp merge of per-thread (m, s) pairs of two tensors: the maxima first,
 // then one rescale per thread and a plain sum.
 __device__ __forceinline__ float4 warp_stats2(float4 r) {
-  float Mt = r.x, Md = r.z;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    Mt = fmaxf(Mt, __shfl_xor_sync(0xffffffffu, Mt, o));
-    Md = fmaxf(Md, __shfl_xor_sync(0xffffffffu, Md, o));
-  }
+  const float Mt = warp_max(r.x), Md = warp_max(r.z);
   float st = Mt == -INFINITY ? 0.0f : r.y * ex2f(r.x - Mt);
   float sd = Md == -INFINITY ? 0.0f : r.w * ex2f(r.z - Md);
 #pragma unroll
@@ -1011,15 +1006,11 @@ __device__ void merge_row(const StochParams& p, int b, int i, int lane) {
     unpack_stats(take(slot + 2 * c + 1, vd0, p.ctrl), m, s);
     merge_stats(MD, SD, m, s);
   }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const float a = __shfl_xor_sync(0xffffffffu, MT, o);
-    const float bb = __shfl_xor_sync(0xffffffffu, ST, o);
-    const float c = __shfl_xor_sync(0xffffffffu, MD, o);
-    const float d = __shfl_xor_sync(0xffffffffu, SD, o);
-    merge_stats(MT, ST, a, bb);
-    merge_stats(MD, SD, c, d);
-  }
+  const float4 w = warp_stats2(make_float4(MT, ST, MD, SD));
+  MT = w.x;
+  ST = w.y;
+  MD = w.z;
+  SD = w.w;
   unsigned int old = 0u;
   if (lane == 0) {
     unsigned long long* row = p.r1 + (static_cast<size_t>(b) * p.k + i) * 2;
@@ -1117,15 +1108,7 @@ __device__ void stoch_epilogue(const StochParams& p, Shared& sh, int group, int 
     Pending next;
     if (h.kind == kKindStats) {
       if (lane >= kGroupWarps) r = make_float4(-INFINITY, 0.0f, -INFINITY, 0.0f);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float a = __shfl_xor_sync(0xffffffffu, r.x, o);
-        const float b = __shfl_xor_sync(0xffffffffu, r.y, o);
-        const float c = __shfl_xor_sync(0xffffffffu, r.z, o);
-        const float d = __shfl_xor_sync(0xffffffffu, r.w, o);
-        merge_stats(r.x, r.y, a, b);
-        merge_stats(r.z, r.w, c, d);
-      }
+      r = warp_stats2(r);
       if (lane == 0) {
         unsigned long long* slot =
             p.p1 + ((static_cast<size_t>(h.b) * p.k + h.i) * p.nch + h.c) * 2;
