@@ -10,11 +10,10 @@
 
 namespace sv {
 
-Plan plan_chunks(long long rows, int V, int bpe) {
-  // Largest chunk (multiple of 8 entries) whose unit of work fits one stage.
-  int chmax = (kStageBytes / bpe) & ~7;
-  if (chmax < 8) chmax = 8;
-  long long nch = (V + chmax - 1) / chmax;
+Plan plan_chunks(long long rows, int V, int bpe, int es_min, int chunk_bytes) {
+  const int ch = full_chunk_entries(chunk_bytes < kStageBytes ? chunk_bytes : kStageBytes, bpe,
+                                    es_min);
+  long long nch = (V + ch - 1) / ch;
   // Small calls: split rows finer (chunks of >= 512 entries) so that about
   // 2048 chunks spread over the SMs.
   const long long want = 2048;
@@ -22,12 +21,13 @@ Plan plan_chunks(long long rows, int V, int bpe) {
     const long long finer = (want + rows - 1) / rows;
     const long long most = (V + 511) / 512;
     const long long n2 = finer < most ? finer : most;
-    if (n2 > nch) nch = n2;
+    if (n2 > nch) {
+      long long c = (V + n2 - 1) / n2;
+      c = (c + 7) / 8 * 8;
+      return Plan{static_cast<int>(c), static_cast<int>((V + c - 1) / c)};
+    }
   }
-  long long ch = (V + nch - 1) / nch;
-  ch = (ch + 7) / 8 * 8;
-  nch = (V + ch - 1) / ch;
-  return Plan{static_cast<int>(ch), static_cast<int>(nch)};
+  return Plan{ch, static_cast<int>(nch)};
 }
 
 namespace {
@@ -69,14 +69,14 @@ ArgLayout argmax_layout(long long rows, int nch) {
   return l;
 }
 
-size_t stochastic_part_bytes(int B, int k, int V, int bpe) {
-  const Plan pl = plan_chunks(static_cast<long long>(B) * k, V, bpe);
+size_t stochastic_part_bytes(int B, int k, int V, int bpe, int es_min) {
+  const Plan pl = plan_chunks(static_cast<long long>(B) * k, V, bpe, es_min, kStochChunkBytes);
   return stochastic_layout(B, k, pl.nch).bytes;
 }
 
 size_t argmax_key_bytes(int B, int G, int k, int V, int es) {
   const long long rows = static_cast<long long>(B) * G * (k + 1);
-  return argmax_layout(rows, plan_chunks(rows, V, es).nch).bytes;
+  return argmax_layout(rows, plan_chunks(rows, V, es, es, kArgmaxChunkBytes).nch).bytes;
 }
 
 bool sizes_ok(int B, int G, int k, int V) {
@@ -119,8 +119,11 @@ extern "C" size_t spec_verify_workspace_size(int B, int G, int k, int V) {
     if (a > tail) tail = a;
   }
   if (G == 1) {
-    for (int bpe : {4, 6, 8}) {
-      const size_t s = stochastic_part_bytes(B, k, V, bpe);
+    // (bytes per entry, narrowest element) of bf16/bf16, bf16/fp32 (either
+    // way round) and fp32/fp32 pairs
+    static const int kPairs[3][2] = {{4, 2}, {6, 2}, {8, 4}};
+    for (const auto& pr : kPairs) {
+      const size_t s = stochastic_part_bytes(B, k, V, pr[0], pr[1]);
       if (s > tail) tail = s;
     }
   }
@@ -192,7 +195,7 @@ extern "C" int spec_verify_stochastic(const void* target_logits, int t_dtype,
 
   const int grid = sm_count();
   if (grid <= 0) return SV_ERR_CUDA;
-  const Plan pl = plan_chunks(static_cast<long long>(B) * k, V, st + sd);
+  const Plan pl = plan_chunks(static_cast<long long>(B) * k, V, st + sd, st < sd ? st : sd, kStochChunkBytes);
   const long long p1 = static_cast<long long>(k) * pl.nch;
   long long lag = 0;
   if (p1 > 0) {
@@ -271,7 +274,7 @@ static int argmax_call(const void* target_logits, int t_dtype, int64_t sb, int64
   const int grid = sm_count();
   if (grid <= 0) return SV_ERR_CUDA;
   const long long rows = static_cast<long long>(B) * G * (k + 1);
-  const Plan pl = plan_chunks(rows, V, st);
+  const Plan pl = plan_chunks(rows, V, st, st, kArgmaxChunkBytes);
   const long long total = rows * pl.nch;
   if (total >= (1ll << 31)) return SV_ERR_INVALID_ARG;
   const bool tma =

@@ -23,8 +23,20 @@ constexpr int kComputeWarps = SV_COMPUTE_WARPS;
 constexpr int kComputeGroups = 2;
 constexpr int kGroupWarps = kComputeWarps / kComputeGroups;
 constexpr int kThreads = 32 * (1 + kComputeWarps + kComputeGroups);
+constexpr int kComputeThreads = kGroupWarps * 32;  // threads that share one chunk
 constexpr int kStages = 4;
-constexpr int kStageBytes = 48 * 1024;
+constexpr int kStageBytes = 56 * 1024;
+
+// Entries of a full chunk: as many as fit `bytes` at `bpe` bytes per entry,
+// rounded down to whole rounds of 16-byte vectors over the kComputeThreads
+// threads of a group for the narrowest tensor (es_min bytes per element), so
+// that every thread holds the same number of vectors and no -inf padding is
+// needed; a budget below one round falls back to a multiple of 8 entries.
+__host__ __device__ constexpr int full_chunk_entries(int bytes, int bpe, int es_min) {
+  return bytes / bpe >= kComputeThreads * 16 / es_min
+             ? bytes / bpe / (kComputeThreads * 16 / es_min) * (kComputeThreads * 16 / es_min)
+             : ((bytes / bpe) & ~7) > 8 ? (bytes / bpe) & ~7 : 8;
+}
 
 // Device-wide control words at the start of the workspace (256 bytes).
 struct Ctrl {
@@ -56,8 +68,19 @@ struct Plan {
 };
 
 // rows: rows (or row pairs) a call reduces; bpe: bytes per vocab entry of
-// one unit of work (target + draft bytes for a stochastic pair).
-Plan plan_chunks(long long rows, int V, int bpe);
+// one unit of work (target + draft bytes for a stochastic pair); es_min: the
+// narrowest element size in it; chunk_bytes: most bytes one chunk may take
+// (at most a stage).  Chunks are full_chunk_entries long, the last one of a
+// row shorter; small calls split rows finer.
+Plan plan_chunks(long long rows, int V, int bpe, int es_min, int chunk_bytes);
+
+// Chunk budgets.  Stochastic chunks fill a stage (56 KB measured faster than
+// 48 KB: 230 -> 224 us on B = 256, k = 8, V = 128256); argmax chunks are
+// smaller, since an argmax chunk is cheap to reduce and its calls are small
+// enough that the ramp of the ring dominates (greedy B = 64, k = 4,
+// V = 128256: 40 KB chunks 15.9 us, 48 KB 16.9 us, 54 KB 18.1 us).
+constexpr int kStochChunkBytes = kStageBytes;
+constexpr int kArgmaxChunkBytes = 40 * 1024;
 
 struct StochParams {
   const void* tgt;

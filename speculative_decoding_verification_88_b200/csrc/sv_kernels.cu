@@ -63,7 +63,6 @@ namespace sv {
 
 enum : int { kKindEnd = 0, kKindStats = 1, kKindCorrection = 2, kKindBonus = 3, kKindArgmax = 4 };
 
-constexpr int kComputeThreads = kGroupWarps * 32;  // threads that share one chunk
 // Tickets per atomicAdd (the next grab's atomic is always in flight).
 // Argmax chunks are uniform work, so larger grabs save atomics; stochastic
 // tickets are taken one at a time, which balances the uneven phase-1 and
@@ -333,12 +332,16 @@ __device__ __forceinline__ void chunk_stats(const unsigned char* smem, int nvec,
 // whole chunk's worth of independent loads, exps and maxima in flight and
 // no reduction sits between the max and the sum.
 
-// Most vectors one thread holds for a tensor of element type T when the
-// stage is shared with a partner tensor of element size `partner` bytes
-// (0: the tensor has the stage to itself).
-template <typename T, int partner>
+// Most vectors one thread holds for a tensor of element type T in a chunk of
+// a `bytes` budget shared with a partner tensor of element size `partner`
+// bytes (0: the tensor has the chunk to itself); a full chunk gives every
+// thread exactly this many.
+template <typename T, int partner, int bytes>
 __host__ __device__ constexpr int max_vecs() {
-  return ((kStageBytes / (Elem<T>::kBytes + partner)) * Elem<T>::kBytes / 16 + kComputeThreads - 1) /
+  return (full_chunk_entries(bytes, Elem<T>::kBytes + partner,
+                             partner > 0 && partner < Elem<T>::kBytes ? partner : Elem<T>::kBytes) *
+              Elem<T>::kBytes / 16 +
+          kComputeThreads - 1) /
          kComputeThreads;
 }
 
@@ -457,8 +460,8 @@ __device__ __forceinline__ float4 chunk_stats_pair(const unsigned char* ts,
                                                    const unsigned char* ds, const Hdr& h,
                                                    const void* tgt, const void* drf, float c2,
                                                    int tid) {
-  constexpr int NT = max_vecs<TT, Elem<TD>::kBytes>();
-  constexpr int ND = max_vecs<TD, Elem<TT>::kBytes>();
+  constexpr int NT = max_vecs<TT, Elem<TD>::kBytes, kStochChunkBytes>();
+  constexpr int ND = max_vecs<TD, Elem<TT>::kBytes, kStochChunkBytes>();
   uint4 vt[NT], vd[ND];
   load_vecs<TT>(ts, h.nvec_t, tid, vt);
   load_vecs<TD>(ds, h.nvec_d, tid, vd);
@@ -474,7 +477,7 @@ template <typename T>
 __device__ __forceinline__ void chunk_argmax_regs(const unsigned char* smem, const Hdr& h,
                                                   const void* g, int tid, float& bv, int& bi) {
   constexpr int EPV = Elem<T>::kPerVec;
-  constexpr int N = max_vecs<T, 0>();
+  constexpr int N = max_vecs<T, 0, kArgmaxChunkBytes>();
   uint4 v[N];
   load_vecs<T>(smem, h.nvec_t, tid, v);
   // one pass: the first vector holding the thread's maximum, kept whole
