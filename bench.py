@@ -70,6 +70,10 @@ def algorithmic_bytes(w: dict, accepted_len: np.ndarray | None) -> int:
     if w["mode"] == "multi":
         G = w["G"]
         return B * G * (k + 1) * V * st + 4 * B * G * k + 4 * B * (k + 3)
+    if w["mode"] == "multi_rows":  # each distinct prefix row once, plus the row map
+        G = w["G"]
+        distinct = sum(len(np.unique(w["row_of"][b])) for b in range(B))
+        return distinct * V * st + 4 * B * G * (k + 1) + 4 * B * G * k + 4 * B * (k + 3)
     sd = ELEM_BYTES[w["d_dtype"]]
     n_full = int((accepted_len == k).sum()) if accepted_len is not None else B
     return B * k * V * (st + sd) + n_full * V * st + 4 * B * k + 4 * B * (k + 2)
@@ -189,6 +193,9 @@ def run_reference(args, rank: int) -> None:
                                      w["seed"], seq_offset=b)
         elif w["mode"] == "greedy":
             oracle.verify_greedy(w["target"][b:b + 1], w["t_dtype"], w["tokens"][b:b + 1])
+        elif w["mode"] == "multi_rows":
+            oracle.verify_multi_rows(w["rows"][b:b + 1], w["t_dtype"], w["row_of"][b:b + 1],
+                                     w["tokens"][b:b + 1])
         else:
             oracle.verify_multi(w["target"][b:b + 1], w["t_dtype"], w["tokens"][b:b + 1])
 
@@ -243,6 +250,9 @@ def oracle_baseline(ws: dict) -> dict:
                                          threads=cores)
             elif w["mode"] == "greedy":
                 oracle.verify_greedy(w["target"], w["t_dtype"], w["tokens"], threads=cores)
+            elif w["mode"] == "multi_rows":
+                oracle.verify_multi_rows(w["rows"], w["t_dtype"], w["row_of"], w["tokens"],
+                                         threads=cores)
             else:
                 oracle.verify_multi(w["target"], w["t_dtype"], w["tokens"], threads=cores)
         t_total += time.perf_counter() - t0
@@ -276,14 +286,15 @@ def run_ours(args, rank: int, world: int, dist) -> None:
     calls, host, devbuf = {}, {}, {}
     for name in STEP:
         w = ws[name]
-        t_h = workloads.as_torch(w["target"], w["t_dtype"]).pin_memory()
+        t_h = workloads.as_torch(w["rows"] if "rows" in w else w["target"],
+                                 w["t_dtype"]).pin_memory()
         tok_h = torch.from_numpy(w["tokens"]).pin_memory()
         d_h = workloads.as_torch(w["draft"], w["d_dtype"]).pin_memory() if "draft" in w else None
         t_d, tok_d = t_h.to(dev), tok_h.to(dev)
         d_d = d_h.to(dev) if d_h is not None else None
         wsp = sv.Workspace(dev)
         B, k = w["B"], w["k"]
-        if w["mode"] == "multi":
+        if w["mode"] in ("multi", "multi_rows"):
             out = {"best_candidate": torch.empty(B, dtype=torch.int32, device=dev)}
         else:
             out = {}
@@ -295,6 +306,10 @@ def run_ours(args, rank: int, world: int, dist) -> None:
                   sv.stochastic(t, d, tok, w["temperature"], w["seed"], off, out=o, workspace=wsp))
         elif w["mode"] == "greedy":
             fn = lambda t=t_d, tok=tok_d, o=out, wsp=wsp: sv.greedy(t, tok, out=o, workspace=wsp)
+        elif w["mode"] == "multi_rows":
+            rmap = torch.from_numpy(w["row_of"]).to(dev)
+            fn = (lambda t=t_d, rm=rmap, tok=tok_d, o=out, wsp=wsp:
+                  sv.multi_candidate_rows(t, rm, tok, out=o, workspace=wsp))
         else:
             fn = (lambda t=t_d, tok=tok_d, o=out, wsp=wsp:
                   sv.multi_candidate(t, tok, out=o, workspace=wsp))
@@ -461,8 +476,10 @@ def select_workloads(only: str | None) -> None:
     """Restrict the step to one workload (profiling runs)."""
     global STEP, DOMINANT
     if only:
-        if only not in STEP:
-            raise SystemExit(f"--only must be one of {STEP}")
+        import workloads
+
+        if only not in workloads.WORKLOADS:
+            raise SystemExit(f"--only must be one of {list(workloads.WORKLOADS)}")
         STEP = [only]
         DOMINANT = only
 

@@ -62,6 +62,7 @@ typedef enum {
 #define SV_FLAG_INVALID_TOKEN 1u     /* a draft token was outside [0, V); it was rejected */
 #define SV_FLAG_RESIDUAL_FALLBACK 2u /* no positive residual mass; correction drawn from p_n */
 #define SV_FLAG_TIMEOUT 4u           /* a bounded device wait gave up; outputs are invalid */
+#define SV_FLAG_INVALID_ROW 8u       /* a row map entry was outside [0, R); see the rows form */
 
 /*
  * Bytes of workspace that calls with these sizes need (any mode, any dtype).
@@ -163,6 +164,36 @@ int spec_verify_multi_candidate(const void *target_logits, int t_dtype, int64_t 
                                 int32_t *best_candidate, int32_t *accepted_len,
                                 int32_t *out_tokens, void *workspace, size_t workspace_bytes,
                                 void *stream);
+
+/*
+ * Multi-candidate greedy verify on deduplicated rows.
+ *
+ * "Lookahead decoding" news piece, steps 3-4: one decoding step verifies many
+ * captured n-grams at once (the verification branch of the 2-in-1 attention
+ * mask).  Candidates that share a prefix share the target rows of that prefix
+ * (row i of a branch conditions on the context plus its first i tokens), so a
+ * caller that evaluates each distinct prefix once passes the distinct rows and
+ * a map instead of G(k+1) rows per sequence; each distinct row is then read
+ * once.
+ *
+ * Results are exactly those of spec_verify_multi_candidate on the expanded
+ * logits E[b,g,i,:] = row_logits[b, row_of[b,g,i], :].
+ *
+ * row_logits [B, R, V], element (b,r,x) at b*r_stride_b + r*r_stride_row + x;
+ * row_of [B, G, k+1] int32 in [0, R); cand_tokens [B, G, k]; outputs as in
+ * spec_verify_multi_candidate.  Requires 1 <= R <= G*(k+1) (so the workspace
+ * of spec_verify_workspace_size(B, G, k, V) suffices), else
+ * SV_ERR_INVALID_ARG.  A map entry outside [0, R) is not read through: that
+ * row counts as one whose argmax is -1 (no candidate token matches it, and a
+ * branch that stops there commits -1), and the device flag
+ * SV_FLAG_INVALID_ROW is set.
+ */
+int spec_verify_multi_candidate_rows(const void *row_logits, int t_dtype, int64_t r_stride_b,
+                                     int64_t r_stride_row, const int32_t *row_of,
+                                     const int32_t *cand_tokens, int B, int G, int k, int R,
+                                     int V, int32_t *best_candidate, int32_t *accepted_len,
+                                     int32_t *out_tokens, void *workspace,
+                                     size_t workspace_bytes, void *stream);
 
 /*
  * Philox4x32-10 (Salmon et al., SC'11) on the device, as the verify kernels

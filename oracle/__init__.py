@@ -207,3 +207,48 @@ def verify_multi(target: np.ndarray, t_dtype: str, cand: np.ndarray,
 
     _run_parallel(fn, B, threads)
     return out
+
+
+def verify_multi_rows(rows: np.ndarray, t_dtype: str, row_of: np.ndarray, cand: np.ndarray,
+                      threads: int = 1) -> dict:
+    """Multi-candidate verify on deduplicated rows [B,R,V] with row_of [B,G,k+1].
+
+    By definition the result of verify_multi on the gathered logits
+    E[b,g,i] = rows[b, row_of[b,g,i]].  A map entry outside [0, R) stands for
+    a row whose argmax is -1; then the gather is impossible and the same
+    decision (per branch the longest prefix equal to the row argmaxes, the
+    longest branch, lowest g on a tie) is taken on the row argmaxes directly.
+    Also returns "invalid_row": whether such an entry occurred.
+    """
+    B, R, V = rows.shape
+    rmap = np.ascontiguousarray(row_of, dtype=np.int32)
+    G, kp1 = rmap.shape[1], rmap.shape[2]
+    k = kp1 - 1
+    c = np.ascontiguousarray(cand, dtype=np.int32).reshape(B, G, k)
+    valid = (rmap >= 0) & (rmap < R)
+    if valid.all():
+        gathered = np.ascontiguousarray(rows[np.arange(B)[:, None, None], rmap])
+        out = verify_multi(gathered, t_dtype, c, threads=threads)
+        out["invalid_row"] = False
+        return out
+    # argmax of every distinct row (first maximum), through the greedy oracle
+    flat = np.ascontiguousarray(rows.reshape(B * R, 1, V))
+    amax = verify_greedy(flat, t_dtype, np.zeros((B * R, 0), np.int32),
+                         threads=threads)["row_argmax"].reshape(B, R)
+    out = {"best_candidate": np.zeros(B, np.int32), "accepted_len": np.zeros(B, np.int32),
+           "out_tokens": np.full((B, kp1), -1, np.int32), "invalid_row": True}
+    for b in range(B):
+        a = np.where(valid[b], amax[b][np.clip(rmap[b], 0, R - 1)], -1)  # [G, k+1]
+        best_n, best_g = -1, 0
+        for g in range(G):
+            n = 0
+            while n < k and c[b, g, n] == a[g, n]:
+                n += 1
+            if n > best_n:
+                best_n, best_g = n, g
+        out["best_candidate"][b] = best_g
+        out["accepted_len"][b] = best_n
+        out["out_tokens"][b, :best_n] = c[b, best_g, :best_n]
+        out["out_tokens"][b, best_n] = a[best_g, best_n]
+    return out
+

@@ -23,12 +23,14 @@ from .build import LIB_PATH
 
 SV_F32, SV_BF16 = 0, 1
 SV_FLAG_INVALID_TOKEN, SV_FLAG_RESIDUAL_FALLBACK, SV_FLAG_TIMEOUT = 1, 2, 4
+SV_FLAG_INVALID_ROW = 8
 
 # Entry points declared in include/spec_verify.h.
 EXPORTS = (
     "spec_verify_workspace_size", "spec_verify_status_string", "spec_verify_workspace_init",
     "spec_verify_read_device_status", "spec_verify_stochastic", "spec_verify_greedy",
-    "spec_verify_multi_candidate", "spec_verify_philox4x32_10", "spec_verify_greedy_noalloc",
+    "spec_verify_multi_candidate", "spec_verify_multi_candidate_rows",
+    "spec_verify_philox4x32_10", "spec_verify_greedy_noalloc",
 )
 
 _lib = None
@@ -74,6 +76,9 @@ def load_library():
         lib.spec_verify_multi_candidate.argtypes = [
             P, I, I64, I64, I64, P, I, I, I, I, P, P, P, P, SZ, P]
         lib.spec_verify_multi_candidate.restype = I
+        lib.spec_verify_multi_candidate_rows.argtypes = [
+            P, I, I64, I64, P, P, I, I, I, I, I, P, P, P, P, SZ, P]
+        lib.spec_verify_multi_candidate_rows.restype = I
         lib.spec_verify_philox4x32_10.argtypes = [P, I64, U64, P, P]
         lib.spec_verify_philox4x32_10.restype = I
         lib.spec_verify_greedy_noalloc.argtypes = [P, I, I64, I64, P, I, I, I, P, P, P]
@@ -272,6 +277,37 @@ def multi_candidate(target: torch.Tensor, cand_tokens: torch.Tensor, *, out: dic
             res["best_candidate"].data_ptr(), res["accepted_len"].data_ptr(),
             res["out_tokens"].data_ptr(), ws.buf.data_ptr(), ws.nbytes, _stream_ptr(stream, dev))
     _check(code, "spec_verify_multi_candidate")
+    _count()
+    return res
+
+
+def multi_candidate_rows(rows: torch.Tensor, row_of: torch.Tensor, cand_tokens: torch.Tensor, *,
+                         out: dict | None = None, workspace: Workspace | None = None,
+                         stream=None) -> dict:
+    """Multi-candidate verify on deduplicated rows: rows [B,R,V], row_of
+    [B,G,k+1] (int32, the row of each (b, g, i)), cand_tokens [B,G,k].  Same
+    results as multi_candidate on rows gathered to [B,G,k+1,V]."""
+    lib = load_library()
+    tc, (tsb, tsr, _) = _logits(rows, 3, "rows")
+    B, R, V = rows.shape
+    if row_of.dim() != 3 or row_of.shape[0] != B:
+        raise ValueError(f"row_of must be [B, G, k+1], got {tuple(row_of.shape)}")
+    G, kp1 = int(row_of.shape[1]), int(row_of.shape[2])
+    k = kp1 - 1
+    dev = rows.device
+    rmap = _tokens(row_of, (B, G, kp1), dev, "row_of")
+    tok = _tokens(cand_tokens, (B, G, k), dev, "cand_tokens")
+    res = {"best_candidate": _out(out, "best_candidate", (B,), torch.int32, dev),
+           "accepted_len": _out(out, "accepted_len", (B,), torch.int32, dev),
+           "out_tokens": _out(out, "out_tokens", (B, k + 1), torch.int32, dev)}
+    ws = workspace or default_workspace(dev)
+    ws.ensure(workspace_size(B, G, k, V), stream)
+    with torch.cuda.device(dev):
+        code = lib.spec_verify_multi_candidate_rows(
+            rows.data_ptr(), tc, tsb, tsr, rmap.data_ptr(), tok.data_ptr(), B, G, k, R, V,
+            res["best_candidate"].data_ptr(), res["accepted_len"].data_ptr(),
+            res["out_tokens"].data_ptr(), ws.buf.data_ptr(), ws.nbytes, _stream_ptr(stream, dev))
+    _check(code, "spec_verify_multi_candidate_rows")
     _count()
     return res
 

@@ -254,11 +254,16 @@ extern "C" int spec_verify_stochastic(const void* target_logits, int t_dtype,
   return e == cudaSuccess ? SV_OK : SV_ERR_CUDA;
 }
 
+// R == 0: rows g*(k+1)+i of a [B, G, k+1, V] tensor; R > 0: the rows form
+// (row_of maps (b, g, i) to one of R rows per sequence, sg is the row stride).
 static int argmax_call(const void* target_logits, int t_dtype, int64_t sb, int64_t sg,
-                       int64_t sp, const int32_t* tokens, int B, int G, int k, int V,
-                       int32_t* best_g, int32_t* accepted_len, int32_t* out_tokens,
-                       void* workspace, size_t workspace_bytes, void* stream) {
+                       int64_t sp, const int32_t* tokens, int B, int G, int k, int V, int R,
+                       const int32_t* row_of, int32_t* best_g, int32_t* accepted_len,
+                       int32_t* out_tokens, void* workspace, size_t workspace_bytes,
+                       void* stream) {
   if (!sizes_ok(B, G, k, V)) return SV_ERR_INVALID_ARG;
+  const long long full_rows = static_cast<long long>(G) * (k + 1);
+  if (R < 0 || R > full_rows || (R > 0) != (row_of != nullptr)) return SV_ERR_INVALID_ARG;
   if (B == 0) return SV_OK;
   if (!target_logits || !accepted_len || !out_tokens || !workspace) return SV_ERR_INVALID_ARG;
   if (k > 0 && !tokens) return SV_ERR_INVALID_ARG;
@@ -267,18 +272,19 @@ static int argmax_call(const void* target_logits, int t_dtype, int64_t sb, int64
   const int st = elem_bytes(t_dtype);
   if (!aligned(target_logits, st) || !aligned(accepted_len, 4) || !aligned(out_tokens, 4) ||
       (k > 0 && !aligned(tokens, 4)) || (best_g && !aligned(best_g, 4)) ||
-      !aligned(workspace, 16))
+      (row_of && !aligned(row_of, 4)) || !aligned(workspace, 16))
     return SV_ERR_MISALIGNED;
   if (workspace_bytes < spec_verify_workspace_size(B, G, k, V)) return SV_ERR_WORKSPACE;
 
   const int grid = sm_count();
   if (grid <= 0) return SV_ERR_CUDA;
-  const long long rows = static_cast<long long>(B) * G * (k + 1);
+  const int rows_per_seq = R > 0 ? R : static_cast<int>(full_rows);
+  const long long rows = static_cast<long long>(B) * rows_per_seq;
   const Plan pl = plan_chunks(rows, V, st, st, kArgmaxChunkBytes);
   const long long total = rows * pl.nch;
   if (total >= (1ll << 31)) return SV_ERR_INVALID_ARG;
-  const bool tma =
-      aligned(target_logits, 16) && stride16(sb, st) && stride16(sg, st) && stride16(sp, st);
+  const bool tma = aligned(target_logits, 16) && stride16(sb, st) && stride16(sg, st) &&
+                   (R > 0 || stride16(sp, st));
 
   const WsView ws = carve(workspace, B);
   ArgmaxParams p{};
@@ -291,6 +297,8 @@ static int argmax_call(const void* target_logits, int t_dtype, int64_t sb, int64
   p.G = G;
   p.k = k;
   p.V = V;
+  p.R = rows_per_seq;
+  p.row_of = row_of;
   p.best_g = best_g;
   p.accepted_len = accepted_len;
   p.out_tokens = out_tokens;
@@ -314,7 +322,8 @@ extern "C" int spec_verify_greedy(const void* target_logits, int t_dtype, int64_
                                   int V, int32_t* accepted_len, int32_t* out_tokens,
                                   void* workspace, size_t workspace_bytes, void* stream) {
   return argmax_call(target_logits, t_dtype, t_stride_b, 0, t_stride_pos, draft_tokens, B, 1, k,
-                     V, nullptr, accepted_len, out_tokens, workspace, workspace_bytes, stream);
+                     V, 0, nullptr, nullptr, accepted_len, out_tokens, workspace,
+                     workspace_bytes, stream);
 }
 
 extern "C" int spec_verify_multi_candidate(const void* target_logits, int t_dtype,
@@ -326,8 +335,22 @@ extern "C" int spec_verify_multi_candidate(const void* target_logits, int t_dtyp
                                            void* stream) {
   if (!best_candidate && B > 0) return SV_ERR_INVALID_ARG;
   return argmax_call(target_logits, t_dtype, t_stride_b, t_stride_g, t_stride_pos, cand_tokens, B,
-                     G, k, V, best_candidate, accepted_len, out_tokens, workspace,
+                     G, k, V, 0, nullptr, best_candidate, accepted_len, out_tokens, workspace,
                      workspace_bytes, stream);
+}
+
+extern "C" int spec_verify_multi_candidate_rows(const void* row_logits, int t_dtype,
+                                                int64_t r_stride_b, int64_t r_stride_row,
+                                                const int32_t* row_of,
+                                                const int32_t* cand_tokens, int B, int G, int k,
+                                                int R, int V, int32_t* best_candidate,
+                                                int32_t* accepted_len, int32_t* out_tokens,
+                                                void* workspace, size_t workspace_bytes,
+                                                void* stream) {
+  if (B > 0 && (!best_candidate || !row_of || R < 1)) return SV_ERR_INVALID_ARG;
+  return argmax_call(row_logits, t_dtype, r_stride_b, r_stride_row, 0, cand_tokens, B, G, k, V,
+                     B > 0 ? R : 0, B > 0 ? row_of : nullptr, best_candidate, accepted_len,
+                     out_tokens, workspace, workspace_bytes, stream);
 }
 
 extern "C" int spec_verify_philox4x32_10(const uint32_t* counters, int64_t n, uint64_t seed,

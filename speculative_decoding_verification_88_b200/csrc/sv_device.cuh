@@ -13,6 +13,7 @@ namespace sv {
 constexpr unsigned int kFlagInvalidToken = 1u;
 constexpr unsigned int kFlagResidualFallback = 2u;
 constexpr unsigned int kFlagTimeout = 4u;
+constexpr unsigned int kFlagInvalidRow = 8u;
 
 // A device wait gives up after this long (ns) and raises kFlagTimeout.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;

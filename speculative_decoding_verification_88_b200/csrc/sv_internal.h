@@ -109,9 +109,11 @@ struct StochParams {
 
 struct ArgmaxParams {
   const void* tgt;
-  long long sb, sg, sp;
-  const int* tokens;  // [B, G, k]
+  long long sb, sg, sp;  // rows form: sg is the row stride, sp unused
+  const int* tokens;     // [B, G, k]
   int B, G, k, V;
+  int R;                 // rows per sequence: G * (k + 1), or the distinct rows of the rows form
+  const int* row_of;     // rows form: [B, G, k+1] row of (b, g, i); nullptr: row g*(k+1)+i
   int* best_g;  // nullable
   int* accepted_len;
   int* out_tokens;
@@ -119,9 +121,9 @@ struct ArgmaxParams {
   unsigned int total;
   Ctrl* ctrl;
   SeqRec* seq;
-  unsigned long long* slots;  // [B][G][k+1][nch] chunk argmax keys
-  unsigned long long* rkey;   // [B][G][k+1] row argmax keys
-  unsigned int* rc;           // [B][G][k+1] chunks of a row published
+  unsigned long long* slots;  // [B][R][nch] chunk argmax keys
+  unsigned long long* rkey;   // [B][R] row argmax keys
+  unsigned int* rc;           // [B][R] chunks of a row published
 };
 
 // dtype codes follow sv_dtype (0 = f32, 1 = bf16).  Return cudaError_t.

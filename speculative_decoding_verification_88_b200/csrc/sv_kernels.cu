@@ -1167,8 +1167,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <typename TT, bool kTma>
 __device__ void argmax_producer(const ArgmaxParams& p, Shared& sh, unsigned char* stages) {
   Ctrl* ctrl = p.ctrl;
-  const unsigned int R = static_cast<unsigned int>(p.G) * static_cast<unsigned int>(p.k + 1);
-  const unsigned int per_seq = R * static_cast<unsigned int>(p.nch);
+  const unsigned int per_seq = static_cast<unsigned int>(p.R) * static_cast<unsigned int>(p.nch);
   uint32_t use = 0;
   bool ok = true;
   unsigned int base = atomicAdd(&ctrl->ticket, kGrabArgmax);
@@ -1183,11 +1182,15 @@ __device__ void argmax_producer(const ArgmaxParams& p, Shared& sh, unsigned char
       const unsigned int rem = t % per_seq;
       h.i = static_cast<int>(rem / p.nch);
       h.c = static_cast<int>(rem % p.nch);
-      const int g = h.i / (p.k + 1), pos = h.i % (p.k + 1);
       h.x0 = h.c * p.ch;
       h.len = min(p.ch, p.V - h.x0);
-      h.toff = static_cast<long long>(h.b) * p.sb + static_cast<long long>(g) * p.sg +
-               static_cast<long long>(pos) * p.sp + h.x0;
+      if (p.row_of) {  // rows form: row h.i of the sequence's distinct rows
+        h.toff = static_cast<long long>(h.b) * p.sb + static_cast<long long>(h.i) * p.sg + h.x0;
+      } else {
+        const int g = h.i / (p.k + 1), pos = h.i % (p.k + 1);
+        h.toff = static_cast<long long>(h.b) * p.sb + static_cast<long long>(g) * p.sg +
+                 static_cast<long long>(pos) * p.sp + h.x0;
+      }
       h.doff = 0;
       const int s = use % kStages;
       if (!mbar_wait(&sh.empty[s], ((use / kStages) & 1u) ^ 1u, ctrl)) {
@@ -1232,6 +1235,60 @@ __device__ void argmax_compute(const ArgmaxParams& p, Shared& sh, unsigned char*
       sh.res[s][w] = make_float4(bv, __int_as_float(bi), 0.0f, 0.0f);
       mbar_arrive(&sh.rfull[s]);
     }
+  }
+}
+
+// Rows form of the finalize: the row keys of sequence b are read without
+// clearing (several (g, i) may share a row), looked up through row_of, and
+// cleared at the end.
+__device__ void finalize_argmax_rows(const ArgmaxParams& p, int b, int lane) {
+  const int k = p.k, G = p.G, R = p.R;
+  unsigned long long* keys = p.rkey + static_cast<size_t>(b) * R;
+  for (int r = lane; r < R; r += 32)
+    if (ld_relaxed_u64(keys + r) == 0ull) poll_u64(keys + r, p.ctrl);  // published by now
+  __syncwarp();
+  const int* map = p.row_of + static_cast<size_t>(b) * G * (k + 1);
+  int best_n = -1, best_g = 0, best_next = -1;
+  bool bad = false;
+  for (int g = 0; g < G; ++g) {
+    // a[i] for i = lane and i = lane + 32 (k + 1 <= 33 rows per branch)
+    int a[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int i = lane + 32 * h;
+      a[h] = -1;
+      if (i <= k) {
+        const int r = __ldg(map + g * (k + 1) + i);
+        if (r >= 0 && r < R) {
+          a[h] = key_index(ld_relaxed_u64(keys + r));
+        } else {
+          bad = true;
+        }
+      }
+    }
+    const int* cand = p.tokens + (static_cast<size_t>(b) * G + g) * k;
+    const bool miss = lane < k && __ldg(cand + lane) != a[0];
+    const unsigned int mm = __ballot_sync(0xffffffffu, miss);
+    const int n = mm ? __ffs(mm) - 1 : k;
+    const int an = __shfl_sync(0xffffffffu, a[0], n & 31);
+    const int a32 = __shfl_sync(0xffffffffu, a[1], 0);
+    if (n > best_n) {
+      best_n = n;
+      best_g = g;
+      best_next = (n == 32) ? a32 : an;
+    }
+  }
+  if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(&p.ctrl->flags, kFlagInvalidRow);
+  const int* cand = p.tokens + (static_cast<size_t>(b) * G + best_g) * k;
+  int* out = p.out_tokens + static_cast<size_t>(b) * (k + 1);
+  for (int i = lane; i <= k; i += 32)
+    out[i] = i < best_n ? __ldg(cand + i) : (i == best_n ? best_next : -1);
+  __syncwarp();
+  for (int r = lane; r < R; r += 32) keys[r] = 0ull;
+  if (lane == 0) {
+    p.accepted_len[b] = best_n;
+    if (p.best_g) p.best_g[b] = best_g;
+    p.seq[b].cnt1 = 0u;
   }
 }
 
@@ -1285,7 +1342,7 @@ __device__ void finalize_argmax(const ArgmaxParams& p, int b, int lane) {
 // Row merge (one warp, one lane per chunk): the row's argmax key is the
 // largest chunk key; count the row, and the last row finalizes.
 __device__ void merge_argmax_row(const ArgmaxParams& p, int b, int r, int lane) {
-  const unsigned int R = static_cast<unsigned int>(p.G) * static_cast<unsigned int>(p.k + 1);
+  const unsigned int R = static_cast<unsigned int>(p.R);
   unsigned long long* slot = p.slots + (static_cast<size_t>(b) * R + r) * p.nch;
   unsigned long long key = 0ull;
   for (int c = lane; c < p.nch; c += 32) {
@@ -1299,11 +1356,16 @@ __device__ void merge_argmax_row(const ArgmaxParams& p, int b, int r, int lane) 
     p.rc[static_cast<size_t>(b) * R + r] = 0u;
     old = atomicAdd(&p.seq[b].cnt1, 1u);
   }
-  if (__shfl_sync(0xffffffffu, old == R - 1u ? 1 : 0, 0)) finalize_argmax(p, b, lane);
+  if (__shfl_sync(0xffffffffu, old == R - 1u ? 1 : 0, 0)) {
+    if (p.row_of)
+      finalize_argmax_rows(p, b, lane);
+    else
+      finalize_argmax(p, b, lane);
+  }
 }
 
 __device__ void argmax_epilogue(const ArgmaxParams& p, Shared& sh, int group, int lane) {
-  const unsigned int R = static_cast<unsigned int>(p.G) * static_cast<unsigned int>(p.k + 1);
+  const unsigned int R = static_cast<unsigned int>(p.R);
   const unsigned int last = static_cast<unsigned int>(p.nch) - 1u;
   int pend_b = -1, pend_r = 0;  // unresolved arrival (sequence, row), or -1
   unsigned int pend_old = 0u;

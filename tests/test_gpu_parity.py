@@ -175,6 +175,90 @@ def test_multi_parity_shapes(dev, dtype, B, G, k, V):
         np.testing.assert_array_equal(r[key].cpu().numpy(), o[key], err_msg=key)
 
 
+# ------------------------------------------ multi-candidate, rows form
+
+def random_rows_case(rng, B, G, k, V, dtype, share=0.6):
+    """Candidates with shared prefixes, their prefix row map and one row of
+    logits per distinct prefix."""
+    cand = rng.integers(0, max(V, 1), (B, G, k)).astype(np.int32)
+    for b in range(B):
+        for g in range(1, G):
+            if rng.random() < share and k > 0:
+                m = int(rng.integers(1, k + 1))
+                src = int(rng.integers(0, g))
+                cand[b, g, :m] = cand[b, src, :m]
+    row_of, R = workloads.prefix_rows(cand)
+    x = tie_heavy(rng, (B, R, V)) if V < 64 else \
+        rng.standard_normal((B, R, V)).astype(np.float32) * 3
+    arr = workloads.f32_to_bf16_bits(x) if dtype == "bf16" else x
+    # steer some candidates onto their row's argmax so that prefixes get accepted
+    am = np.argmax(workloads.to_f32(arr, dtype), -1)
+    for b in range(B):
+        for g in range(G):
+            for i in range(k):
+                if rng.random() < 0.5:
+                    cand[b, g, i] = am[b, row_of[b, g, i]]
+    row_of, R2 = workloads.prefix_rows(cand)
+    if R2 > R:  # steering created new prefixes: give them rows too
+        extra = rng.standard_normal((B, R2 - R, V)).astype(np.float32) * 3
+        extra = workloads.f32_to_bf16_bits(extra) if dtype == "bf16" else extra
+        arr = np.concatenate([arr, extra], axis=1)
+    return arr, row_of, cand
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("B,G,k,V", [(1, 1, 4, 100), (3, 3, 2, 17), (16, 8, 4, 3001),
+                                     (2, 64, 3, 50), (4, 5, 32, 40), (2, 2, 0, 10),
+                                     (3, 6, 5, 20480 + 17)])
+def test_multi_rows_parity_shapes(dev, dtype, B, G, k, V):
+    rng = np.random.default_rng(B * 3 + G * 5 + k * 11 + V)
+    arr, row_of, cand = random_rows_case(rng, B, G, k, V, dtype)
+    r = sv.multi_candidate_rows(to_dev(arr, dtype, dev), torch.from_numpy(row_of).to(dev),
+                                torch.from_numpy(cand).to(dev))
+    o = oracle.verify_multi_rows(arr, dtype, row_of, cand, threads=THREADS)
+    for key in ("best_candidate", "accepted_len", "out_tokens"):
+        np.testing.assert_array_equal(r[key].cpu().numpy(), o[key], err_msg=key)
+
+
+def test_multi_rows_equals_expanded_multi(dev):
+    """The rows form and the expanded form give the same results."""
+    rng = np.random.default_rng(21)
+    arr, row_of, cand = random_rows_case(rng, 9, 7, 6, 2000, "bf16")
+    t = to_dev(arr, "bf16", dev)
+    rm = torch.from_numpy(row_of).to(dev)
+    c = torch.from_numpy(cand).to(dev)
+    r = sv.multi_candidate_rows(t, rm, c)
+    expanded = t[torch.arange(9, device=dev)[:, None, None], rm.long()]
+    e = sv.multi_candidate(expanded.contiguous(), c)
+    for key in ("best_candidate", "accepted_len", "out_tokens"):
+        assert torch.equal(r[key], e[key]), key
+
+
+def test_multi_rows_invalid_entries_and_limits(dev):
+    rng = np.random.default_rng(22)
+    arr, row_of, cand = random_rows_case(rng, 5, 4, 3, 300, "bf16")
+    R = arr.shape[1]
+    bad = row_of.copy()
+    bad[1, 2, 1] = R + 5
+    bad[3, 0, 0] = -1
+    ws = sv.Workspace(dev)
+    r = sv.multi_candidate_rows(to_dev(arr, "bf16", dev), torch.from_numpy(bad).to(dev),
+                                torch.from_numpy(cand).to(dev), workspace=ws)
+    o = oracle.verify_multi_rows(arr, "bf16", bad, cand)
+    assert o["invalid_row"]
+    for key in ("best_candidate", "accepted_len", "out_tokens"):
+        np.testing.assert_array_equal(r[key].cpu().numpy(), o[key], err_msg=key)
+    assert ws.device_status(clear=True) == sv.SV_FLAG_INVALID_ROW
+    torch.cuda.synchronize()
+    assert int(ws.buf[256:].cpu().count_nonzero()) == 0
+    # more rows than G * (k + 1) is refused
+    big = np.zeros((1, 2 * 2 + 1, 64), np.uint16)
+    with pytest.raises(sv.SpecVerifyError):
+        sv.multi_candidate_rows(to_dev(big, "bf16", dev),
+                                torch.zeros((1, 2, 2), dtype=torch.int32, device=dev),
+                                torch.zeros((1, 2, 1), dtype=torch.int32, device=dev))
+
+
 # --------------------------------------------------------------- stochastic
 
 @pytest.mark.parametrize("t_dtype,d_dtype", [("bf16", "bf16"), ("bf16", "f32"), ("f32", "f32"),
@@ -292,7 +376,7 @@ def test_one_workspace_across_modes_and_sizes(dev):
     ws = sv.Workspace(dev)
     rng = np.random.default_rng(16)
     for step in range(12):
-        mode = ("stochastic", "greedy", "multi")[step % 3]
+        mode = ("stochastic", "greedy", "multi", "rows")[step % 4]
         B = int(rng.integers(1, 40))
         k = int(rng.integers(0, 9))
         V = int(rng.integers(2, 3000))
@@ -311,11 +395,18 @@ def test_one_workspace_across_modes_and_sizes(dev):
                           workspace=ws)
             o = oracle.verify_greedy(w["target"], "bf16", w["tokens"])
             np.testing.assert_array_equal(r["out_tokens"].cpu().numpy(), o["out_tokens"])
-        else:
+        elif mode == "multi":
             w = workloads.make_multi(B, 3, k, V, seed=step)
             r = sv.multi_candidate(to_dev(w["target"], "bf16", dev),
                                    torch.from_numpy(w["tokens"]).to(dev), workspace=ws)
             o = oracle.verify_multi(w["target"], "bf16", w["tokens"])
+            np.testing.assert_array_equal(r["out_tokens"].cpu().numpy(), o["out_tokens"])
+        else:
+            w = workloads.make_multi_rows(B, 3, k, V, seed=step)
+            r = sv.multi_candidate_rows(to_dev(w["rows"], "bf16", dev),
+                                        torch.from_numpy(w["row_of"]).to(dev),
+                                        torch.from_numpy(w["tokens"]).to(dev), workspace=ws)
+            o = oracle.verify_multi_rows(w["rows"], "bf16", w["row_of"], w["tokens"])
             np.testing.assert_array_equal(r["out_tokens"].cpu().numpy(), o["out_tokens"])
         torch.cuda.synchronize()
         body = ws.buf[256:].cpu()
@@ -340,9 +431,16 @@ def test_named_workload_full_size(dev, name):
         o = oracle.verify_greedy(w["target"], "bf16", w["tokens"], threads=THREADS)
         np.testing.assert_array_equal(r["accepted_len"].cpu().numpy(), o["accepted_len"])
         np.testing.assert_array_equal(r["out_tokens"].cpu().numpy(), o["out_tokens"])
-    else:
+    elif mode == "multi":
         r = sv.multi_candidate(to_dev(w["target"], "bf16", dev),
                                torch.from_numpy(w["tokens"]).to(dev))
         o = oracle.verify_multi(w["target"], "bf16", w["tokens"], threads=THREADS)
+        for key in ("best_candidate", "accepted_len", "out_tokens"):
+            np.testing.assert_array_equal(r[key].cpu().numpy(), o[key], err_msg=key)
+    else:
+        r = sv.multi_candidate_rows(to_dev(w["rows"], "bf16", dev),
+                                    torch.from_numpy(w["row_of"]).to(dev),
+                                    torch.from_numpy(w["tokens"]).to(dev))
+        o = oracle.verify_multi_rows(w["rows"], "bf16", w["row_of"], w["tokens"], threads=THREADS)
         for key in ("best_candidate", "accepted_len", "out_tokens"):
             np.testing.assert_array_equal(r[key].cpu().numpy(), o[key], err_msg=key)

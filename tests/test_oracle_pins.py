@@ -413,6 +413,59 @@ def test_multi_all_branches_empty_picks_branch_zero():
     assert r["out_tokens"].tolist() == [[2, -1]]
 
 
+# ------------------------------------------------ multi-candidate, rows form
+
+def test_prefix_rows_hand_case():
+    # branch 0: 5 6 ; branch 1: 5 7 ; branch 2: 9 6
+    cand = np.array([[[5, 6], [5, 7], [9, 6]]], np.int32)
+    row_of, R = workloads.prefix_rows(cand)
+    # i = 0: all share the empty prefix -> row 0
+    # i = 1: prefixes (5,) (5,) (9,) -> rows 1, 1, 2
+    # i = 2: prefixes (5,6) (5,7) (9,6) -> rows 3, 4, 5
+    assert R == 6
+    assert row_of.tolist() == [[[0, 1, 3], [0, 1, 4], [0, 2, 5]]]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_multi_rows_bruteforce(dtype):
+    """Rows form against a plain argmax decision on the gathered rows."""
+    rng = np.random.default_rng(31)
+    B, G, k, R, V = 40, 5, 3, 9, 13
+    x = tie_heavy_rows(rng, (B, R, V))
+    arr = workloads.f32_to_bf16_bits(x) if dtype == "bf16" else x
+    row_of = rng.integers(0, R, (B, G, k + 1)).astype(np.int32)
+    a = np.argmax(x, axis=-1)
+    gathered = x[np.arange(B)[:, None, None], row_of]
+    ga = np.argmax(gathered, -1)
+    cand = np.where(rng.random((B, G, k)) < 0.7, ga[:, :, :k], rng.integers(0, V, (B, G, k)))
+    cand = cand.astype(np.int32)
+    r = oracle.verify_multi_rows(arr, dtype, row_of, cand)
+    bg, n, out = plain_multi(gathered, cand)
+    assert not r["invalid_row"]
+    np.testing.assert_array_equal(r["best_candidate"], bg)
+    np.testing.assert_array_equal(r["accepted_len"], n)
+    np.testing.assert_array_equal(r["out_tokens"], out)
+    assert a.shape == (B, R)
+
+
+def test_multi_rows_invalid_entry_hand_case():
+    # rows: argmax of row 0 is 1, of row 1 is 2
+    rows = np.array([[[0.0, 5.0, 1.0], [0.0, 1.0, 5.0]]], np.float32)
+    cand = np.array([[[1, 2], [1, 2]]], np.int32)
+    # branch 0: rows 0, 1, 1 -> accepts 1 (=argmax row 0), 2 (=argmax row 1), next = 2
+    # branch 1: rows 0, 7 (invalid), 1 -> accepts 1, stops at the invalid row
+    row_of = np.array([[[0, 1, 1], [0, 7, 1]]], np.int32)
+    r = oracle.verify_multi_rows(rows, "f32", row_of, cand)
+    assert r["invalid_row"]
+    assert r["best_candidate"].tolist() == [0]
+    assert r["accepted_len"].tolist() == [2]
+    assert r["out_tokens"].tolist() == [[1, 2, 2]]
+    # only the invalid branch left: it commits -1 where it stops
+    r = oracle.verify_multi_rows(rows, "f32", row_of[:, 1:], cand[:, 1:])
+    assert r["accepted_len"].tolist() == [1]
+    assert r["out_tokens"].tolist() == [[1, -1, -1]]
+
+
 # ------------------------------------------------------------------ strides
 
 def test_strided_views_equal_contiguous():

@@ -49,6 +49,10 @@ WORKLOADS = {
                                   seed=3),
     "multi_b16_g8_k4_v32000": dict(mode="multi", B=16, G=8, k=4, V=32000, t_dtype="bf16",
                                    t_std=3.0, p_match=0.6, p_shared=0.5, seed=4),
+    # the same lookahead step with each distinct candidate prefix's row once
+    "multi_rows_b16_g8_k4_v32000": dict(mode="multi_rows", B=16, G=8, k=4, V=32000,
+                                        t_dtype="bf16", t_std=3.0, p_match=0.6,
+                                        p_shared=0.5, seed=4),
 }
 
 ELEM_BYTES = {"f32": 4, "bf16": 2}
@@ -216,6 +220,49 @@ def make_multi(B: int, G: int, k: int, V: int, t_dtype: str = "bf16", t_std: flo
                 B=B, G=G, k=k, V=V)
 
 
+def prefix_rows(cand: np.ndarray) -> tuple[np.ndarray, int]:
+    """Row map of lookahead candidates [B,G,k]: row (b, g, i) conditions on
+    the context plus cand[b,g,:i], so (g, i) pairs with equal prefixes share
+    one row.  Returns row_of [B,G,k+1] (int32, rows numbered per sequence in
+    order of first appearance, i-major) and R, the most rows any sequence
+    needs."""
+    B, G, k = cand.shape
+    row_of = np.zeros((B, G, k + 1), np.int32)
+    R = 1
+    for b in range(B):
+        seen = {}
+        for i in range(k + 1):
+            for g in range(G):
+                key = tuple(int(t) for t in cand[b, g, :i])
+                if key not in seen:
+                    seen[key] = len(seen)
+                row_of[b, g, i] = seen[key]
+        R = max(R, len(seen))
+    return row_of, R
+
+
+def make_multi_rows(B: int, G: int, k: int, V: int, t_dtype: str = "bf16", t_std: float = 3.0,
+                    p_match: float = 0.6, p_shared: float = 0.5, seed: int = 0,
+                    threads: int | None = None) -> dict:
+    """The multi-candidate workload in deduplicated form: the candidates of
+    make_multi (same seed), rows [B,R,V] holding one row per distinct prefix
+    (the row of the first (g, i) with that prefix), and row_of [B,G,k+1].
+    Unused row slots of a sequence repeat its last row."""
+    w = make_multi(B, G, k, V, t_dtype, t_std, p_match, p_shared, seed, threads)
+    row_of, R = prefix_rows(w["tokens"])
+    rows = np.empty((B, R, V), w["target"].dtype)
+    for b in range(B):
+        first = {}
+        for i in range(k + 1):
+            for g in range(G):
+                first.setdefault(int(row_of[b, g, i]), (g, i))
+        for r in range(R):
+            g, i = first.get(r, first[max(first)])
+            rows[b, r] = w["target"][b, g, i]
+    return dict(mode="multi_rows", rows=rows, row_of=row_of, t_dtype=t_dtype,
+                tokens=w["tokens"], seed=seed, B=B, G=G, k=k, R=R, V=V)
+
+
 def make(name: str, threads: int | None = None, **overrides) -> dict:
     """Inputs of a named workload (``WORKLOADS``), with optional overrides
     (e.g. ``B=4`` for a bounded sample of the same workload)."""
@@ -228,12 +275,14 @@ def make(name: str, threads: int | None = None, **overrides) -> dict:
         return make_greedy(threads=threads, **cfg)
     if mode == "multi":
         return make_multi(threads=threads, **cfg)
+    if mode == "multi_rows":
+        return make_multi_rows(threads=threads, **cfg)
     raise ValueError(mode)
 
 
 def logit_bytes(w: dict) -> int:
     """Bytes of logits a verify call over workload ``w`` streams (all rows)."""
-    n = w["target"].size * ELEM_BYTES[w["t_dtype"]]
+    n = (w["rows"] if "rows" in w else w["target"]).size * ELEM_BYTES[w["t_dtype"]]
     if "draft" in w:
         n += w["draft"].size * ELEM_BYTES[w["d_dtype"]]
     return n
