@@ -63,6 +63,7 @@ typedef enum {
 #define SV_FLAG_RESIDUAL_FALLBACK 2u /* no positive residual mass; correction drawn from p_n */
 #define SV_FLAG_TIMEOUT 4u           /* a bounded device wait gave up; outputs are invalid */
 #define SV_FLAG_INVALID_ROW 8u       /* a row map entry was outside [0, R); see the rows form */
+#define SV_FLAG_CAPACITY 16u         /* spec_verify_commit: a token buffer was full */
 
 /*
  * Bytes of workspace that calls with these sizes need (any mode, any dtype).
@@ -194,6 +195,33 @@ int spec_verify_multi_candidate_rows(const void *row_logits, int t_dtype, int64_
                                      int V, int32_t *best_candidate, int32_t *accepted_len,
                                      int32_t *out_tokens, void *workspace,
                                      size_t workspace_bytes, void *stream);
+
+/*
+ * Device-side commit: the step after verify, with no host synchronisation.
+ *
+ * "Accelerating Sonar through speculation", section "Single-token MTP
+ * scheduling": a small amount of extra GPU work spares the CPU-GPU sync after
+ * acceptance -- the next tokens are written into place on the device, and
+ * the host schedules the next step without waiting for the accepted lengths.
+ *
+ * For every sequence b, with n = accepted_len[b] (clamped to [0, k]) and
+ * L = seq_len[b]: the n + 1 committed tokens out_tokens[b, 0..n] are written
+ * to token_buf[b*buf_stride + L .. L+n]; seq_len[b] becomes L + n + 1; and
+ * next_input[b] (nullable) receives out_tokens[b, n], the input of the next
+ * decoding step (the position shift of an MTP draft is the caller's
+ * indexing).  Tokens are copied as they are, -1 included.
+ *
+ * accepted_len [B], out_tokens [B, k+1] (as the verify calls write them),
+ * seq_len [B] in/out, token_buf [B, >= capacity] (row stride buf_stride >=
+ * capacity, in elements), next_input [B] or NULL: int32 device arrays.
+ * Tokens that would land at or past `capacity` are dropped, seq_len stops at
+ * capacity, and SV_FLAG_CAPACITY is set in `workspace` (a verify workspace,
+ * nullable: then the flag is not reported).  A negative seq_len is read as 0.
+ * One small launch on `stream`; B == 0 does nothing.
+ */
+int spec_verify_commit(const int32_t *accepted_len, const int32_t *out_tokens, int B, int k,
+                       int32_t *seq_len, int32_t *token_buf, int64_t buf_stride, int capacity,
+                       int32_t *next_input, void *workspace, void *stream);
 
 /*
  * Philox4x32-10 (Salmon et al., SC'11) on the device, as the verify kernels

@@ -252,3 +252,31 @@ def verify_multi_rows(rows: np.ndarray, t_dtype: str, row_of: np.ndarray, cand: 
         out["out_tokens"][b, best_n] = a[best_g, best_n]
     return out
 
+
+def commit(accepted_len: np.ndarray, out_tokens: np.ndarray, seq_len: np.ndarray,
+           token_buf: np.ndarray) -> dict:
+    """Device-side commit, written out: for each sequence, n = accepted_len
+    clamped to [0, k], L = max(seq_len, 0); tokens out_tokens[b, :n+1] go to
+    token_buf[b, L:L+n+1] (those at or past the capacity are dropped), the
+    length becomes min(L + n + 1, capacity), the next input is out_tokens[b, n].
+    Returns copies: seq_len, token_buf, next_input, capacity_hit."""
+    out = np.asarray(out_tokens, np.int32)
+    B, kp1 = out.shape
+    k = kp1 - 1
+    buf = np.array(token_buf, np.int32, copy=True)
+    cap = buf.shape[1]
+    lens = np.array(seq_len, np.int32, copy=True)
+    nxt = np.zeros(B, np.int32)
+    hit = False
+    for b in range(B):
+        n = min(max(int(accepted_len[b]), 0), k)
+        L = max(int(lens[b]), 0)
+        for j in range(n + 1):
+            if L + j < cap:
+                buf[b, L + j] = out[b, j]
+            else:
+                hit = True
+        lens[b] = min(L + n + 1, cap)
+        nxt[b] = out[b, n]
+    return {"seq_len": lens, "token_buf": buf, "next_input": nxt, "capacity_hit": hit}
+

@@ -23,13 +23,13 @@ from .build import LIB_PATH
 
 SV_F32, SV_BF16 = 0, 1
 SV_FLAG_INVALID_TOKEN, SV_FLAG_RESIDUAL_FALLBACK, SV_FLAG_TIMEOUT = 1, 2, 4
-SV_FLAG_INVALID_ROW = 8
+SV_FLAG_INVALID_ROW, SV_FLAG_CAPACITY = 8, 16
 
 # Entry points declared in include/spec_verify.h.
 EXPORTS = (
     "spec_verify_workspace_size", "spec_verify_status_string", "spec_verify_workspace_init",
     "spec_verify_read_device_status", "spec_verify_stochastic", "spec_verify_greedy",
-    "spec_verify_multi_candidate", "spec_verify_multi_candidate_rows",
+    "spec_verify_multi_candidate", "spec_verify_multi_candidate_rows", "spec_verify_commit",
     "spec_verify_philox4x32_10", "spec_verify_greedy_noalloc",
 )
 
@@ -79,6 +79,8 @@ def load_library():
         lib.spec_verify_multi_candidate_rows.argtypes = [
             P, I, I64, I64, P, P, I, I, I, I, I, P, P, P, P, SZ, P]
         lib.spec_verify_multi_candidate_rows.restype = I
+        lib.spec_verify_commit.argtypes = [P, P, I, I, P, P, I64, I, P, P, P]
+        lib.spec_verify_commit.restype = I
         lib.spec_verify_philox4x32_10.argtypes = [P, I64, U64, P, P]
         lib.spec_verify_philox4x32_10.restype = I
         lib.spec_verify_greedy_noalloc.argtypes = [P, I, I64, I64, P, I, I, I, P, P, P]
@@ -310,6 +312,44 @@ def multi_candidate_rows(rows: torch.Tensor, row_of: torch.Tensor, cand_tokens: 
     _check(code, "spec_verify_multi_candidate_rows")
     _count()
     return res
+
+
+def commit(result: dict, seq_len: torch.Tensor, token_buf: torch.Tensor, *,
+           next_input: torch.Tensor | None = None, workspace: Workspace | None = None,
+           stream=None) -> None:
+    """Device-side commit after a verify call: append each sequence's n + 1
+    committed tokens (result["out_tokens"][b, :n+1], n = result["accepted_len"][b])
+    to token_buf[b, seq_len[b]:], advance seq_len and write the next step's
+    input token, all on the GPU (no host synchronisation).  token_buf is an
+    int32 [B, capacity] tensor whose rows may be strided; tokens past capacity
+    are dropped and flagged (SV_FLAG_CAPACITY) in `workspace` if given."""
+    lib = load_library()
+    acc, out = result["accepted_len"], result["out_tokens"]
+    dev = acc.device
+    B = int(acc.shape[0])
+    k = int(out.shape[1]) - 1
+    acc = _tokens(acc, (B,), dev, "accepted_len")
+    out = _tokens(out, (B, k + 1), dev, "out_tokens")
+    if (not isinstance(seq_len, torch.Tensor) or seq_len.dtype != torch.int32 or
+            seq_len.device != dev or tuple(seq_len.shape) != (B,) or not seq_len.is_contiguous()):
+        raise ValueError("seq_len must be a contiguous int32 [B] tensor on the verify device")
+    if (token_buf.dtype != torch.int32 or token_buf.device != dev or token_buf.dim() != 2 or
+            token_buf.shape[0] != B or (token_buf.shape[1] > 1 and token_buf.stride(1) != 1)):
+        raise ValueError("token_buf must be an int32 [B, capacity] tensor with contiguous rows")
+    if next_input is not None and (next_input.dtype != torch.int32 or next_input.device != dev or
+                                   tuple(next_input.shape) != (B,) or
+                                   not next_input.is_contiguous()):
+        raise ValueError("next_input must be a contiguous int32 [B] tensor")
+    cap = int(token_buf.shape[1])
+    stride = int(token_buf.stride(0)) if B > 1 else cap
+    with torch.cuda.device(dev):
+        code = lib.spec_verify_commit(
+            acc.data_ptr(), out.data_ptr(), B, k, seq_len.data_ptr(), token_buf.data_ptr(),
+            max(stride, cap), cap, next_input.data_ptr() if next_input is not None else None,
+            workspace.buf.data_ptr() if workspace is not None and workspace.buf is not None
+            else None, _stream_ptr(stream, dev))
+    _check(code, "spec_verify_commit")
+    _count()
 
 
 def greedy_noalloc(target: torch.Tensor, draft_tokens: torch.Tensor, *,

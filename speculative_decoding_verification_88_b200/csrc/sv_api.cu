@@ -353,6 +353,24 @@ extern "C" int spec_verify_multi_candidate_rows(const void* row_logits, int t_dt
                      out_tokens, workspace, workspace_bytes, stream);
 }
 
+extern "C" int spec_verify_commit(const int32_t* accepted_len, const int32_t* out_tokens, int B,
+                                  int k, int32_t* seq_len, int32_t* token_buf,
+                                  int64_t buf_stride, int capacity, int32_t* next_input,
+                                  void* workspace, void* stream) {
+  if (B < 0 || k < 0 || k > 32 || capacity < 0 || buf_stride < capacity) return SV_ERR_INVALID_ARG;
+  if (B == 0) return SV_OK;
+  if (!accepted_len || !out_tokens || !seq_len || (capacity > 0 && !token_buf))
+    return SV_ERR_INVALID_ARG;
+  if (!aligned(accepted_len, 4) || !aligned(out_tokens, 4) || !aligned(seq_len, 4) ||
+      (token_buf && !aligned(token_buf, 4)) || (next_input && !aligned(next_input, 4)) ||
+      (workspace && !aligned(workspace, 16)))
+    return SV_ERR_MISALIGNED;
+  const cudaError_t e = launch_commit(
+      accepted_len, out_tokens, B, k, seq_len, token_buf, buf_stride, capacity, next_input,
+      workspace ? reinterpret_cast<Ctrl*>(workspace) : nullptr, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SV_OK : SV_ERR_CUDA;
+}
+
 extern "C" int spec_verify_philox4x32_10(const uint32_t* counters, int64_t n, uint64_t seed,
                                          uint32_t* out, void* stream) {
   if (n < 0 || (n > 0 && (!counters || !out))) return SV_ERR_INVALID_ARG;

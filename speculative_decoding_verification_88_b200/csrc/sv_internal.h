@@ -131,6 +131,9 @@ cudaError_t launch_stochastic(const StochParams& p, int t_dtype, int d_dtype, bo
                               int grid, size_t smem, cudaStream_t stream);
 cudaError_t launch_argmax(const ArgmaxParams& p, int t_dtype, bool tma, int grid, size_t smem,
                           cudaStream_t stream);
+cudaError_t launch_commit(const int* accepted_len, const int* out_tokens, int B, int k,
+                          int* seq_len, int* token_buf, long long buf_stride, int capacity,
+                          int* next_input, Ctrl* ctrl, cudaStream_t st);
 cudaError_t launch_philox(const uint4* ctr, long long n, unsigned int key0, unsigned int key1,
                           uint4* out, cudaStream_t stream);
 size_t kernel_smem_bytes();

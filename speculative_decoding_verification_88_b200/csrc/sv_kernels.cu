@@ -1440,6 +1440,40 @@ __global__ void philox_kernel(const uint4* __restrict__ ctr, long long n, uint32
     out[j] = philox10(ctr[j], k0, k1);
 }
 
+// ================================================================ commit
+
+// One warp per sequence: lane 0 reads the length, every lane copies up to two
+// of the n + 1 committed tokens (k + 1 <= 33), then lane 0 advances the
+// length and writes the next input.
+__global__ void commit_kernel(const int* __restrict__ accepted_len,
+                              const int* __restrict__ out_tokens, int B, int k,
+                              int* __restrict__ seq_len, int* __restrict__ token_buf,
+                              long long buf_stride, int capacity, int* __restrict__ next_input,
+                              Ctrl* ctrl) {
+  const int b = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (b >= B) return;
+  const int n = min(max(__ldg(accepted_len + b), 0), k);
+  const int L = max(seq_len[b], 0);
+  const int* out = out_tokens + static_cast<size_t>(b) * (k + 1);
+  int* buf = token_buf + static_cast<size_t>(b) * buf_stride;
+  bool full = false;
+  for (int j = lane; j <= n; j += 32) {
+    const long long pos = static_cast<long long>(L) + j;
+    if (pos < capacity)
+      buf[pos] = __ldg(out + j);
+    else
+      full = true;
+  }
+  full = __any_sync(0xffffffffu, full);
+  if (lane == 0) {
+    const long long end = static_cast<long long>(L) + n + 1;
+    seq_len[b] = static_cast<int>(end < capacity ? end : capacity);
+    if (next_input) next_input[b] = __ldg(out + n);
+    if (full && ctrl) atomicOr(&ctrl->flags, kFlagCapacity);
+  }
+}
+
 // ============================================================== launchers
 
 // The shared-memory opt-in is per function and device; setting it again is
@@ -1498,6 +1532,16 @@ cudaError_t launch_argmax(const ArgmaxParams& p, int t_dtype, bool tma, int grid
                : launch_argmax_t<uint16_t, false>(p, grid, smem, st);
   return tma ? launch_argmax_t<float, true>(p, grid, smem, st)
              : launch_argmax_t<float, false>(p, grid, smem, st);
+}
+
+cudaError_t launch_commit(const int* accepted_len, const int* out_tokens, int B, int k,
+                          int* seq_len, int* token_buf, long long buf_stride, int capacity,
+                          int* next_input, Ctrl* ctrl, cudaStream_t st) {
+  if (B <= 0) return cudaSuccess;
+  constexpr int kWarps = 8;
+  commit_kernel<<<(B + kWarps - 1) / kWarps, 32 * kWarps, 0, st>>>(
+      accepted_len, out_tokens, B, k, seq_len, token_buf, buf_stride, capacity, next_input, ctrl);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_philox(const uint4* ctr, long long n, unsigned int key0, unsigned int key1,

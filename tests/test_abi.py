@@ -125,6 +125,42 @@ def test_greedy_and_multi_validation(lib):
     assert m(wb=64) == WORKSPACE
 
 
+def test_multi_rows_validation(lib):
+    def r(**kw):
+        a = dict(rows=A16, t=1, sb=80, sr=8, rmap=A16, tok=A16, B=2, G=2, k=4, R=3, V=8,
+                 best=A16, acc=A16, out=A16, ws=A16, wb=1 << 20, st=None)
+        a.update(kw)
+        return lib.spec_verify_multi_candidate_rows(*a.values())
+
+    assert r(B=0, rows=None, rmap=None) == OK
+    assert r(R=0) == INVALID
+    assert r(R=2 * 5 + 1) == INVALID  # more rows than G * (k + 1)
+    assert r(rmap=None) == INVALID
+    assert r(best=None) == INVALID
+    assert r(rmap=A16 + 2) == MISALIGNED
+    assert r(wb=64) == WORKSPACE
+
+
+def test_commit_validation(lib):
+    def c(**kw):
+        a = dict(acc=A16, out=A16, B=2, k=4, lens=A16, buf=A16, stride=16, cap=16, nxt=A16,
+                 ws=None, st=None)
+        a.update(kw)
+        return lib.spec_verify_commit(*a.values())
+
+    assert c(B=0, acc=None, out=None, lens=None, buf=None) == OK
+    assert c(B=-1) == INVALID
+    assert c(k=33) == INVALID
+    assert c(cap=-1) == INVALID
+    assert c(stride=8) == INVALID  # row stride below the capacity
+    assert c(acc=None) == INVALID
+    assert c(lens=None) == INVALID
+    assert c(buf=None) == INVALID
+    assert c(out=A16 + 2) == MISALIGNED
+    assert c(nxt=A16 + 1) == MISALIGNED
+    assert c(ws=A16 + 4) == MISALIGNED
+
+
 def test_philox_and_workspace_validation(lib):
     assert lib.spec_verify_philox4x32_10(None, 0, 0, None, None) == OK
     assert lib.spec_verify_philox4x32_10(None, 4, 0, A16, None) == INVALID

@@ -259,6 +259,55 @@ def test_multi_rows_invalid_entries_and_limits(dev):
                                 torch.zeros((1, 2, 1), dtype=torch.int32, device=dev))
 
 
+# ------------------------------------------------------------ device commit
+
+@pytest.mark.parametrize("B,k,cap", [(1, 0, 4), (7, 1, 9), (300, 8, 40), (33, 32, 100),
+                                     (20, 4, 3)])
+def test_commit_parity(dev, B, k, cap):
+    rng = np.random.default_rng(B + k + cap)
+    out = rng.integers(-1, 32000, (B, k + 1)).astype(np.int32)
+    acc = rng.integers(-1, k + 2, B).astype(np.int32)
+    lens = rng.integers(-2, cap + 1, B).astype(np.int32)
+    buf = rng.integers(0, 9, (B, cap + 5)).astype(np.int32)  # row stride cap + 5
+    o = oracle.commit(acc, out, lens, buf[:, :cap])
+    seq = torch.from_numpy(lens).to(dev)
+    tb = torch.from_numpy(buf).to(dev)
+    nxt = torch.full((B,), -7, dtype=torch.int32, device=dev)
+    ws = sv.Workspace(dev)
+    ws.ensure(256)
+    sv.commit({"accepted_len": torch.from_numpy(acc).to(dev),
+               "out_tokens": torch.from_numpy(out).to(dev)},
+              seq, tb[:, :cap], next_input=nxt, workspace=ws)
+    np.testing.assert_array_equal(seq.cpu().numpy(), o["seq_len"])
+    np.testing.assert_array_equal(tb[:, :cap].cpu().numpy(), o["token_buf"])
+    np.testing.assert_array_equal(tb[:, cap:].cpu().numpy(), buf[:, cap:])  # untouched
+    np.testing.assert_array_equal(nxt.cpu().numpy(), o["next_input"])
+    assert ws.device_status(clear=True) == (sv.SV_FLAG_CAPACITY if o["capacity_hit"] else 0)
+
+
+def test_verify_then_commit_without_host_sync(dev):
+    """Greedy verify and the commit enqueued back to back on one stream, twice;
+    the host reads nothing in between."""
+    B, k, V, cap = 24, 4, 3000, 64
+    w = workloads.make_greedy(B, k, V, seed=31)
+    w2 = workloads.make_greedy(B, k, V, seed=32)
+    seq = torch.zeros(B, dtype=torch.int32, device=dev)
+    tb = torch.full((B, cap), -9, dtype=torch.int32, device=dev)
+    nxt = torch.empty(B, dtype=torch.int32, device=dev)
+    for ww in (w, w2):
+        r = sv.greedy(to_dev(ww["target"], "bf16", dev), torch.from_numpy(ww["tokens"]).to(dev))
+        sv.commit(r, seq, tb, next_input=nxt)
+    lens = np.zeros(B, np.int32)
+    buf = np.full((B, cap), -9, np.int32)
+    for ww in (w, w2):
+        o = oracle.verify_greedy(ww["target"], "bf16", ww["tokens"])
+        c = oracle.commit(o["accepted_len"], o["out_tokens"], lens, buf)
+        lens, buf, last = c["seq_len"], c["token_buf"], c["next_input"]
+    np.testing.assert_array_equal(seq.cpu().numpy(), lens)
+    np.testing.assert_array_equal(tb.cpu().numpy(), buf)
+    np.testing.assert_array_equal(nxt.cpu().numpy(), last)
+
+
 # --------------------------------------------------------------- stochastic
 
 @pytest.mark.parametrize("t_dtype,d_dtype", [("bf16", "bf16"), ("bf16", "f32"), ("f32", "f32"),

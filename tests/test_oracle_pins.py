@@ -466,6 +466,40 @@ def test_multi_rows_invalid_entry_hand_case():
     assert r["out_tokens"].tolist() == [[1, -1, -1]]
 
 
+# ------------------------------------------------------------ device commit
+
+def test_commit_hand_case():
+    out = np.array([[7, 8, 9, -1], [1, 2, 3, 4]], np.int32)
+    acc = np.array([1, 3], np.int32)
+    buf = np.full((2, 6), -5, np.int32)
+    r = oracle.commit(acc, out, np.array([2, 5], np.int32), buf)
+    # sequence 0: n = 1 -> tokens 7, 8 at 2..3; next input 8
+    # sequence 1: n = 3 -> tokens 1..4 at 5..8, only position 5 fits
+    assert r["token_buf"].tolist() == [[-5, -5, 7, 8, -5, -5], [-5, -5, -5, -5, -5, 1]]
+    assert r["seq_len"].tolist() == [4, 6]
+    assert r["next_input"].tolist() == [8, 4]
+    assert r["capacity_hit"]
+
+
+def test_commit_clamps_and_appends_the_commit():
+    rng = np.random.default_rng(5)
+    B, k, cap = 50, 6, 40
+    out = rng.integers(0, 1000, (B, k + 1)).astype(np.int32)
+    acc = rng.integers(-2, k + 3, B).astype(np.int32)  # includes values outside [0, k]
+    lens = rng.integers(-3, 20, B).astype(np.int32)
+    buf = rng.integers(0, 1000, (B, cap)).astype(np.int32)
+    r = oracle.commit(acc, out, lens, buf)
+    for b in range(B):
+        n = min(max(int(acc[b]), 0), k)
+        L = max(int(lens[b]), 0)
+        assert r["seq_len"][b] == L + n + 1
+        assert r["token_buf"][b, L:L + n + 1].tolist() == out[b, :n + 1].tolist()
+        assert r["token_buf"][b, :L].tolist() == buf[b, :L].tolist()
+        assert r["token_buf"][b, L + n + 1:].tolist() == buf[b, L + n + 1:].tolist()
+        assert r["next_input"][b] == out[b, n]
+    assert not r["capacity_hit"]
+
+
 # ------------------------------------------------------------------ strides
 
 def test_strided_views_equal_contiguous():
