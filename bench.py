@@ -51,6 +51,8 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic_stochastic_verify_b256_k8
 # ------------------------------------------------------------------ helpers
 
 def positions(w: dict) -> int:
+    if w["mode"] == "tree":  # every drafted node is a verified position
+        return w["B"] * w["N"]
     return w["B"] * w.get("G", 1) * (w["k"] + 1)
 
 
@@ -63,8 +65,11 @@ def algorithmic_bytes(w: dict, accepted_len: np.ndarray | None) -> int:
     """
     from workloads import ELEM_BYTES
 
-    B, k, V = w["B"], w["k"], w["V"]
     st = ELEM_BYTES[w["t_dtype"]]
+    if w["mode"] == "tree":  # every node row, parents and tokens, path and tokens out
+        B, N, V = w["B"], w["N"], w["V"]
+        return B * N * V * st + 8 * B * N + 4 * B + 8 * B * N
+    B, k, V = w["B"], w["k"], w["V"]
     if w["mode"] == "greedy":
         return B * (k + 1) * V * st + 4 * B * k + 4 * B * (k + 2)
     if w["mode"] == "multi":
@@ -196,6 +201,9 @@ def run_reference(args, rank: int) -> None:
         elif w["mode"] == "multi_rows":
             oracle.verify_multi_rows(w["rows"][b:b + 1], w["t_dtype"], w["row_of"][b:b + 1],
                                      w["tokens"][b:b + 1])
+        elif w["mode"] == "tree":
+            oracle.verify_tree_greedy(w["node_logits"][b:b + 1], w["t_dtype"],
+                                      w["parent"][b:b + 1], w["tokens"][b:b + 1])
         else:
             oracle.verify_multi(w["target"][b:b + 1], w["t_dtype"], w["tokens"][b:b + 1])
 
@@ -212,8 +220,7 @@ def run_reference(args, rank: int) -> None:
     for s in range(args.steps):
         step(args.warmup + s)
     dt = time.perf_counter() - t0
-    pos = sum(ws[n]["k"] + 1 if ws[n]["mode"] != "multi" else ws[n]["G"] * (ws[n]["k"] + 1)
-              for n in STEP)
+    pos = sum(positions(ws[n]) // ws[n]["B"] for n in STEP)  # one sequence of each
     value = pos * args.steps / dt
     sample = "one sequence of each of the four step workloads per step, in parallel threads"
     print(json.dumps({
@@ -253,6 +260,9 @@ def oracle_baseline(ws: dict) -> dict:
             elif w["mode"] == "multi_rows":
                 oracle.verify_multi_rows(w["rows"], w["t_dtype"], w["row_of"], w["tokens"],
                                          threads=cores)
+            elif w["mode"] == "tree":
+                oracle.verify_tree_greedy(w["node_logits"], w["t_dtype"], w["parent"],
+                                          w["tokens"], threads=cores)
             else:
                 oracle.verify_multi(w["target"], w["t_dtype"], w["tokens"], threads=cores)
         t_total += time.perf_counter() - t0
@@ -286,26 +296,33 @@ def run_ours(args, rank: int, world: int, dist) -> None:
     calls, host, devbuf = {}, {}, {}
     for name in STEP:
         w = ws[name]
-        t_h = workloads.as_torch(w["rows"] if "rows" in w else w["target"],
-                                 w["t_dtype"]).pin_memory()
+        key = "rows" if "rows" in w else ("node_logits" if "node_logits" in w else "target")
+        t_h = workloads.as_torch(w[key], w["t_dtype"]).pin_memory()
         tok_h = torch.from_numpy(w["tokens"]).pin_memory()
         d_h = workloads.as_torch(w["draft"], w["d_dtype"]).pin_memory() if "draft" in w else None
         t_d, tok_d = t_h.to(dev), tok_h.to(dev)
         d_d = d_h.to(dev) if d_h is not None else None
         wsp = sv.Workspace(dev)
-        B, k = w["B"], w["k"]
+        B = w["B"]
+        width = w["N"] if w["mode"] == "tree" else w["k"] + 1
         if w["mode"] in ("multi", "multi_rows"):
             out = {"best_candidate": torch.empty(B, dtype=torch.int32, device=dev)}
+        elif w["mode"] == "tree":
+            out = {"path": torch.empty((B, width), dtype=torch.int32, device=dev)}
         else:
             out = {}
         out["accepted_len"] = torch.empty(B, dtype=torch.int32, device=dev)
-        out["out_tokens"] = torch.empty((B, k + 1), dtype=torch.int32, device=dev)
+        out["out_tokens"] = torch.empty((B, width), dtype=torch.int32, device=dev)
         if w["mode"] == "stochastic":
             off = rank * B
             fn = (lambda w=w, t=t_d, d=d_d, tok=tok_d, o=out, wsp=wsp, off=off:
                   sv.stochastic(t, d, tok, w["temperature"], w["seed"], off, out=o, workspace=wsp))
         elif w["mode"] == "greedy":
             fn = lambda t=t_d, tok=tok_d, o=out, wsp=wsp: sv.greedy(t, tok, out=o, workspace=wsp)
+        elif w["mode"] == "tree":
+            par = torch.from_numpy(w["parent"]).to(dev)
+            fn = (lambda t=t_d, pa=par, tok=tok_d, o=out, wsp=wsp:
+                  sv.tree_greedy(t, pa, tok, out=o, workspace=wsp))
         elif w["mode"] == "multi_rows":
             rmap = torch.from_numpy(w["row_of"]).to(dev)
             fn = (lambda t=t_d, rm=rmap, tok=tok_d, o=out, wsp=wsp:

@@ -64,6 +64,7 @@ typedef enum {
 #define SV_FLAG_TIMEOUT 4u           /* a bounded device wait gave up; outputs are invalid */
 #define SV_FLAG_INVALID_ROW 8u       /* a row map entry was outside [0, R); see the rows form */
 #define SV_FLAG_CAPACITY 16u         /* spec_verify_commit: a token buffer was full */
+#define SV_FLAG_INVALID_TREE 32u     /* a tree node's parent was outside [0, node) */
 
 /*
  * Bytes of workspace that calls with these sizes need (any mode, any dtype).
@@ -195,6 +196,40 @@ int spec_verify_multi_candidate_rows(const void *row_logits, int t_dtype, int64_
                                      int V, int32_t *best_candidate, int32_t *accepted_len,
                                      int32_t *out_tokens, void *workspace,
                                      size_t workspace_bytes, void *stream);
+
+/*
+ * Greedy verify of a draft token tree (EAGLE-style tree drafting).
+ *
+ * "Accelerating Sonar through speculation", section "EAGLE": the draft
+ * explores a tree of likely tokens (Top-K candidates per node, fixed or
+ * dynamically shaped), the drafted sequences are scored, the longest
+ * acceptable one is kept, and one more token comes from the target.  Greedy
+ * acceptance: starting at the root, the walk moves to the child whose token
+ * equals the argmax of the current node's target row (first maximum; the
+ * lowest-index such child if several share the token), until no child
+ * matches; the target's argmax at the last node is the extra token.
+ *
+ * node_logits [B, N, V], element (b,j,x) at b*stride_b + j*stride_node + x:
+ *   row j is the target's distribution after the path to node j (node 0 is
+ *   the root: the last committed token).
+ * parent [B, N] int32: parent[b][0] is ignored; parent[b][j] in [0, j) for
+ *   j >= 1 (nodes in topological order).  A node whose parent is outside
+ *   [0, j) is never entered, and SV_FLAG_INVALID_TREE is set.
+ * tokens [B, N] int32: the draft token of node j (node 0's is ignored).
+ * Outputs: accepted_len [B] = n, the accepted nodes below the root;
+ *   path [B, N] = 0, then the n accepted nodes in order, then -1;
+ *   out_tokens [B, N] = their n tokens, then the argmax of the last accepted
+ *   node's row, then -1.
+ * 1 <= N <= 64.  Workspace: spec_verify_tree_workspace_size(B, N, V) bytes
+ * (zeroed once, as for the other calls).
+ */
+size_t spec_verify_tree_workspace_size(int B, int N, int V);
+
+int spec_verify_tree_greedy(const void *node_logits, int t_dtype, int64_t stride_b,
+                            int64_t stride_node, const int32_t *parent, const int32_t *tokens,
+                            int B, int N, int V, int32_t *accepted_len, int32_t *path,
+                            int32_t *out_tokens, void *workspace, size_t workspace_bytes,
+                            void *stream);
 
 /*
  * Device-side commit: the step after verify, with no host synchronisation.

@@ -280,3 +280,39 @@ def commit(accepted_len: np.ndarray, out_tokens: np.ndarray, seq_len: np.ndarray
         nxt[b] = out[b, n]
     return {"seq_len": lens, "token_buf": buf, "next_input": nxt, "capacity_hit": hit}
 
+
+def verify_tree_greedy(node_logits: np.ndarray, t_dtype: str, parent: np.ndarray,
+                       tokens: np.ndarray, threads: int = 1) -> dict:
+    """Greedy verify of a draft token tree [B,N,V] with parent/tokens [B,N].
+
+    From the root (node 0), step to the lowest-index child whose token equals
+    the argmax of the current node's row, until no child matches; commit the
+    tokens of the accepted nodes and the argmax of the last one.  A node whose
+    parent is outside [0, j) is never entered ("invalid_tree" reports it).
+    """
+    B, N, V = node_logits.shape
+    par = np.ascontiguousarray(parent, dtype=np.int32).reshape(B, N)
+    tok = np.ascontiguousarray(tokens, dtype=np.int32).reshape(B, N)
+    flat = np.ascontiguousarray(node_logits.reshape(B * N, 1, V))
+    amax = verify_greedy(flat, t_dtype, np.zeros((B * N, 0), np.int32),
+                         threads=threads)["row_argmax"].reshape(B, N)
+    out = {"accepted_len": np.zeros(B, np.int32), "path": np.full((B, N), -1, np.int32),
+           "out_tokens": np.full((B, N), -1, np.int32), "invalid_tree": False}
+    for b in range(B):
+        valid = [j >= 1 and 0 <= par[b, j] < j for j in range(N)]
+        if any(not valid[j] for j in range(1, N)):
+            out["invalid_tree"] = True
+        u, n = 0, 0
+        out["path"][b, 0] = 0
+        while True:
+            nxt = [j for j in range(1, N) if valid[j] and par[b, j] == u and tok[b, j] == amax[b, u]]
+            if not nxt:
+                break
+            u = nxt[0]
+            out["out_tokens"][b, n] = tok[b, u]
+            n += 1
+            out["path"][b, n] = u
+        out["out_tokens"][b, n] = amax[b, u]
+        out["accepted_len"][b] = n
+    return out
+

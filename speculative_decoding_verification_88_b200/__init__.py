@@ -23,13 +23,14 @@ from .build import LIB_PATH
 
 SV_F32, SV_BF16 = 0, 1
 SV_FLAG_INVALID_TOKEN, SV_FLAG_RESIDUAL_FALLBACK, SV_FLAG_TIMEOUT = 1, 2, 4
-SV_FLAG_INVALID_ROW, SV_FLAG_CAPACITY = 8, 16
+SV_FLAG_INVALID_ROW, SV_FLAG_CAPACITY, SV_FLAG_INVALID_TREE = 8, 16, 32
 
 # Entry points declared in include/spec_verify.h.
 EXPORTS = (
     "spec_verify_workspace_size", "spec_verify_status_string", "spec_verify_workspace_init",
     "spec_verify_read_device_status", "spec_verify_stochastic", "spec_verify_greedy",
     "spec_verify_multi_candidate", "spec_verify_multi_candidate_rows", "spec_verify_commit",
+    "spec_verify_tree_workspace_size", "spec_verify_tree_greedy",
     "spec_verify_philox4x32_10", "spec_verify_greedy_noalloc",
 )
 
@@ -81,6 +82,10 @@ def load_library():
         lib.spec_verify_multi_candidate_rows.restype = I
         lib.spec_verify_commit.argtypes = [P, P, I, I, P, P, I64, I, P, P, P]
         lib.spec_verify_commit.restype = I
+        lib.spec_verify_tree_workspace_size.argtypes = [I, I, I]
+        lib.spec_verify_tree_workspace_size.restype = SZ
+        lib.spec_verify_tree_greedy.argtypes = [P, I, I64, I64, P, P, I, I, I, P, P, P, P, SZ, P]
+        lib.spec_verify_tree_greedy.restype = I
         lib.spec_verify_philox4x32_10.argtypes = [P, I64, U64, P, P]
         lib.spec_verify_philox4x32_10.restype = I
         lib.spec_verify_greedy_noalloc.argtypes = [P, I, I64, I64, P, I, I, I, P, P, P]
@@ -310,6 +315,37 @@ def multi_candidate_rows(rows: torch.Tensor, row_of: torch.Tensor, cand_tokens: 
             res["best_candidate"].data_ptr(), res["accepted_len"].data_ptr(),
             res["out_tokens"].data_ptr(), ws.buf.data_ptr(), ws.nbytes, _stream_ptr(stream, dev))
     _check(code, "spec_verify_multi_candidate_rows")
+    _count()
+    return res
+
+
+def tree_workspace_size(B: int, N: int, V: int) -> int:
+    return int(load_library().spec_verify_tree_workspace_size(B, N, V))
+
+
+def tree_greedy(node_logits: torch.Tensor, parent: torch.Tensor, tokens: torch.Tensor, *,
+                out: dict | None = None, workspace: Workspace | None = None,
+                stream=None) -> dict:
+    """Greedy verify of a draft token tree: node_logits [B,N,V] (row j = the
+    target after the path to node j), parent [B,N] and tokens [B,N] int32.
+    Returns accepted_len [B], path [B,N] and out_tokens [B,N]."""
+    lib = load_library()
+    tc, (tsb, tsn, _) = _logits(node_logits, 3, "node_logits")
+    B, N, V = node_logits.shape
+    dev = node_logits.device
+    par = _tokens(parent, (B, N), dev, "parent")
+    tok = _tokens(tokens, (B, N), dev, "tokens")
+    res = {"accepted_len": _out(out, "accepted_len", (B,), torch.int32, dev),
+           "path": _out(out, "path", (B, N), torch.int32, dev),
+           "out_tokens": _out(out, "out_tokens", (B, N), torch.int32, dev)}
+    ws = workspace or default_workspace(dev)
+    ws.ensure(tree_workspace_size(B, N, V), stream)
+    with torch.cuda.device(dev):
+        code = lib.spec_verify_tree_greedy(
+            node_logits.data_ptr(), tc, tsb, tsn, par.data_ptr(), tok.data_ptr(), B, N, V,
+            res["accepted_len"].data_ptr(), res["path"].data_ptr(), res["out_tokens"].data_ptr(),
+            ws.buf.data_ptr(), ws.nbytes, _stream_ptr(stream, dev))
+    _check(code, "spec_verify_tree_greedy")
     _count()
     return res
 

@@ -254,17 +254,22 @@ extern "C" int spec_verify_stochastic(const void* target_logits, int t_dtype,
   return e == cudaSuccess ? SV_OK : SV_ERR_CUDA;
 }
 
-// R == 0: rows g*(k+1)+i of a [B, G, k+1, V] tensor; R > 0: the rows form
-// (row_of maps (b, g, i) to one of R rows per sequence, sg is the row stride).
+// R == 0: rows g*(k+1)+i of a [B, G, k+1, V] tensor; R > 0: R rows per
+// sequence at stride sg, either the rows form (row_of maps (b, g, i) to a
+// row) or a tree of R = k + 1 nodes (parent pointers, G = 1, path out).
 static int argmax_call(const void* target_logits, int t_dtype, int64_t sb, int64_t sg,
                        int64_t sp, const int32_t* tokens, int B, int G, int k, int V, int R,
-                       const int32_t* row_of, int32_t* best_g, int32_t* accepted_len,
-                       int32_t* out_tokens, void* workspace, size_t workspace_bytes,
-                       void* stream) {
+                       const int32_t* row_of, const int32_t* parent, int32_t* path,
+                       int32_t* best_g, int32_t* accepted_len, int32_t* out_tokens,
+                       void* workspace, size_t workspace_bytes, void* stream,
+                       size_t need_bytes) {
   if (!sizes_ok(B, G, k, V)) return SV_ERR_INVALID_ARG;
   const long long full_rows = static_cast<long long>(G) * (k + 1);
-  if (R < 0 || R > full_rows || (R > 0) != (row_of != nullptr)) return SV_ERR_INVALID_ARG;
+  if (R < 0 || R > full_rows || (R > 0) != (row_of != nullptr || parent != nullptr) ||
+      (row_of && parent))
+    return SV_ERR_INVALID_ARG;
   if (B == 0) return SV_OK;
+  if (parent && !path) return SV_ERR_INVALID_ARG;
   if (!target_logits || !accepted_len || !out_tokens || !workspace) return SV_ERR_INVALID_ARG;
   if (k > 0 && !tokens) return SV_ERR_INVALID_ARG;
   if (!dtype_ok(t_dtype)) return SV_ERR_INVALID_ARG;
@@ -272,9 +277,10 @@ static int argmax_call(const void* target_logits, int t_dtype, int64_t sb, int64
   const int st = elem_bytes(t_dtype);
   if (!aligned(target_logits, st) || !aligned(accepted_len, 4) || !aligned(out_tokens, 4) ||
       (k > 0 && !aligned(tokens, 4)) || (best_g && !aligned(best_g, 4)) ||
-      (row_of && !aligned(row_of, 4)) || !aligned(workspace, 16))
+      (row_of && !aligned(row_of, 4)) || (parent && !aligned(parent, 4)) ||
+      (path && !aligned(path, 4)) || !aligned(workspace, 16))
     return SV_ERR_MISALIGNED;
-  if (workspace_bytes < spec_verify_workspace_size(B, G, k, V)) return SV_ERR_WORKSPACE;
+  if (workspace_bytes < need_bytes) return SV_ERR_WORKSPACE;
 
   const int grid = sm_count();
   if (grid <= 0) return SV_ERR_CUDA;
@@ -299,6 +305,8 @@ static int argmax_call(const void* target_logits, int t_dtype, int64_t sb, int64
   p.V = V;
   p.R = rows_per_seq;
   p.row_of = row_of;
+  p.parent = parent;
+  p.path = path;
   p.best_g = best_g;
   p.accepted_len = accepted_len;
   p.out_tokens = out_tokens;
@@ -322,8 +330,9 @@ extern "C" int spec_verify_greedy(const void* target_logits, int t_dtype, int64_
                                   int V, int32_t* accepted_len, int32_t* out_tokens,
                                   void* workspace, size_t workspace_bytes, void* stream) {
   return argmax_call(target_logits, t_dtype, t_stride_b, 0, t_stride_pos, draft_tokens, B, 1, k,
-                     V, 0, nullptr, nullptr, accepted_len, out_tokens, workspace,
-                     workspace_bytes, stream);
+                     V, 0, nullptr, nullptr, nullptr, nullptr, accepted_len, out_tokens,
+                     workspace, workspace_bytes, stream,
+                     spec_verify_workspace_size(B, 1, k, V));
 }
 
 extern "C" int spec_verify_multi_candidate(const void* target_logits, int t_dtype,
@@ -335,8 +344,9 @@ extern "C" int spec_verify_multi_candidate(const void* target_logits, int t_dtyp
                                            void* stream) {
   if (!best_candidate && B > 0) return SV_ERR_INVALID_ARG;
   return argmax_call(target_logits, t_dtype, t_stride_b, t_stride_g, t_stride_pos, cand_tokens, B,
-                     G, k, V, 0, nullptr, best_candidate, accepted_len, out_tokens, workspace,
-                     workspace_bytes, stream);
+                     G, k, V, 0, nullptr, nullptr, nullptr, best_candidate, accepted_len,
+                     out_tokens, workspace, workspace_bytes, stream,
+                     spec_verify_workspace_size(B, G, k, V));
 }
 
 extern "C" int spec_verify_multi_candidate_rows(const void* row_logits, int t_dtype,
@@ -349,8 +359,37 @@ extern "C" int spec_verify_multi_candidate_rows(const void* row_logits, int t_dt
                                                 void* stream) {
   if (B > 0 && (!best_candidate || !row_of || R < 1)) return SV_ERR_INVALID_ARG;
   return argmax_call(row_logits, t_dtype, r_stride_b, r_stride_row, 0, cand_tokens, B, G, k, V,
-                     B > 0 ? R : 0, B > 0 ? row_of : nullptr, best_candidate, accepted_len,
-                     out_tokens, workspace, workspace_bytes, stream);
+                     B > 0 ? R : 0, B > 0 ? row_of : nullptr, nullptr, nullptr, best_candidate,
+                     accepted_len, out_tokens, workspace, workspace_bytes, stream,
+                     spec_verify_workspace_size(B, G, k, V));
+}
+
+extern "C" size_t spec_verify_tree_workspace_size(int B, int N, int V) {
+  if (B < 0 || N < 1 || N > 64 || V < 1) return 0;
+  size_t tail = 0;
+  for (int es : {2, 4}) {
+    const long long rows = static_cast<long long>(B) * N;
+    const size_t a = argmax_layout(rows, plan_chunks(rows, V, es, es, kArgmaxChunkBytes).nch).bytes;
+    if (a > tail) tail = a;
+  }
+  const size_t total = kCtrlBytes + seq_bytes(B) + tail;
+  return (total + 255) / 256 * 256;
+}
+
+extern "C" int spec_verify_tree_greedy(const void* node_logits, int t_dtype, int64_t stride_b,
+                                       int64_t stride_node, const int32_t* parent,
+                                       const int32_t* tokens, int B, int N, int V,
+                                       int32_t* accepted_len, int32_t* path,
+                                       int32_t* out_tokens, void* workspace,
+                                       size_t workspace_bytes, void* stream) {
+  if (N < 1 || N > 64 || B < 0 || V < 1) return SV_ERR_INVALID_ARG;
+  if (B == 0) return SV_OK;
+  if (!parent || !tokens || !path) return SV_ERR_INVALID_ARG;
+  // a tree of N nodes runs as one "sequence" of R = N rows of the argmax
+  // machinery (G = 2, k = 31 only bound R by 64); the finalize walks the tree
+  return argmax_call(node_logits, t_dtype, stride_b, stride_node, 0, tokens, B, 2, 31, V, N,
+                     nullptr, parent, path, nullptr, accepted_len, out_tokens, workspace,
+                     workspace_bytes, stream, spec_verify_tree_workspace_size(B, N, V));
 }
 
 extern "C" int spec_verify_commit(const int32_t* accepted_len, const int32_t* out_tokens, int B,

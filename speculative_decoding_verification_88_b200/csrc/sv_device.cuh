@@ -15,6 +15,7 @@ constexpr unsigned int kFlagResidualFallback = 2u;
 constexpr unsigned int kFlagTimeout = 4u;
 constexpr unsigned int kFlagInvalidRow = 8u;
 constexpr unsigned int kFlagCapacity = 16u;
+constexpr unsigned int kFlagInvalidTree = 32u;
 
 // A device wait gives up after this long (ns) and raises kFlagTimeout.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;

@@ -112,8 +112,12 @@ struct ArgmaxParams {
   long long sb, sg, sp;  // rows form: sg is the row stride, sp unused
   const int* tokens;     // [B, G, k]
   int B, G, k, V;
-  int R;                 // rows per sequence: G * (k + 1), or the distinct rows of the rows form
+  int R;                 // rows per sequence: G * (k + 1), the distinct rows of the rows
+                         // form, or the nodes of a tree
   const int* row_of;     // rows form: [B, G, k+1] row of (b, g, i); nullptr: row g*(k+1)+i
+  const int* parent;     // tree form: [B, R] parent of each node (tokens and out_tokens
+                         // are then [B, R]; G and k only bound R)
+  int* path;             // tree form: [B, R] accepted path out
   int* best_g;  // nullable
   int* accepted_len;
   int* out_tokens;

@@ -1184,7 +1184,7 @@ __device__ void argmax_producer(const ArgmaxParams& p, Shared& sh, unsigned char
       h.c = static_cast<int>(rem % p.nch);
       h.x0 = h.c * p.ch;
       h.len = min(p.ch, p.V - h.x0);
-      if (p.row_of) {  // rows form: row h.i of the sequence's distinct rows
+      if (p.row_of || p.parent) {  // rows or tree form: row h.i of the sequence
         h.toff = static_cast<long long>(h.b) * p.sb + static_cast<long long>(h.i) * p.sg + h.x0;
       } else {
         const int g = h.i / (p.k + 1), pos = h.i % (p.k + 1);
@@ -1235,6 +1235,72 @@ __device__ void argmax_compute(const ArgmaxParams& p, Shared& sh, unsigned char*
       sh.res[s][w] = make_float4(bv, __int_as_float(bi), 0.0f, 0.0f);
       mbar_arrive(&sh.rfull[s]);
     }
+  }
+}
+
+// Tree form of the finalize (one warp; nodes j = lane and lane + 32): from
+// the root, step to the lowest-index child whose token equals the current
+// node's row argmax, until none does; commit the path's tokens and the last
+// node's argmax.  Row keys are read without clearing and cleared at the end.
+__device__ void finalize_argmax_tree(const ArgmaxParams& p, int b, int lane) {
+  const int N = p.R;
+  unsigned long long* keys = p.rkey + static_cast<size_t>(b) * N;
+  for (int r = lane; r < N; r += 32)
+    if (ld_relaxed_u64(keys + r) == 0ull) poll_u64(keys + r, p.ctrl);  // published by now
+  __syncwarp();
+  const int* par = p.parent + static_cast<size_t>(b) * N;
+  const int* tok = p.tokens + static_cast<size_t>(b) * N;
+  int a[2], pj[2], tj[2];
+  bool bad = false;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int j = lane + 32 * h;
+    a[h] = j < N ? key_index(ld_relaxed_u64(keys + j)) : -1;
+    pj[h] = -1;
+    tj[h] = -1;
+    if (j >= 1 && j < N) {
+      const int q = __ldg(par + j);
+      if (q >= 0 && q < j) {
+        pj[h] = q;
+        tj[h] = __ldg(tok + j);
+      } else {
+        bad = true;  // never entered
+      }
+    }
+  }
+  int* path = p.path + static_cast<size_t>(b) * N;
+  int* out = p.out_tokens + static_cast<size_t>(b) * N;
+  // every step enters a child c > u (parents precede their children), so the
+  // walk ends within N - 1 steps
+  int u = 0, n = 0, au;
+  for (;;) {
+    au = __shfl_sync(0xffffffffu, u < 32 ? a[0] : a[1], u & 31);
+    const unsigned int m0 = __ballot_sync(0xffffffffu, pj[0] == u && tj[0] == au);
+    const unsigned int m1 = __ballot_sync(0xffffffffu, pj[1] == u && tj[1] == au);
+    if (m0 == 0u && m1 == 0u) break;
+    const int c = m0 ? __ffs(m0) - 1 : 32 + __ffs(m1) - 1;
+    const int tc = __shfl_sync(0xffffffffu, c < 32 ? tj[0] : tj[1], c & 31);
+    if (lane == 0) {
+      path[n + 1] = c;
+      out[n] = tc;
+    }
+    u = c;
+    ++n;
+  }
+  if (lane == 0) {
+    path[0] = 0;
+    out[n] = au;  // the target's extra token
+  }
+  for (int j = n + 1 + lane; j < N; j += 32) {
+    path[j] = -1;
+    out[j] = -1;
+  }
+  if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(&p.ctrl->flags, kFlagInvalidTree);
+  __syncwarp();
+  for (int r = lane; r < N; r += 32) keys[r] = 0ull;
+  if (lane == 0) {
+    p.accepted_len[b] = n;
+    p.seq[b].cnt1 = 0u;
   }
 }
 
@@ -1357,7 +1423,9 @@ __device__ void merge_argmax_row(const ArgmaxParams& p, int b, int r, int lane) 
     old = atomicAdd(&p.seq[b].cnt1, 1u);
   }
   if (__shfl_sync(0xffffffffu, old == R - 1u ? 1 : 0, 0)) {
-    if (p.row_of)
+    if (p.parent)
+      finalize_argmax_tree(p, b, lane);
+    else if (p.row_of)
       finalize_argmax_rows(p, b, lane);
     else
       finalize_argmax(p, b, lane);

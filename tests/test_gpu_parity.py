@@ -259,6 +259,66 @@ def test_multi_rows_invalid_entries_and_limits(dev):
                                 torch.zeros((1, 2, 1), dtype=torch.int32, device=dev))
 
 
+# ---------------------------------------------------------------- tree verify
+
+def random_tree_case(rng, B, N, V, dtype, dup=0.1):
+    x = tie_heavy(rng, (B, N, V)) if V < 64 else \
+        rng.standard_normal((B, N, V)).astype(np.float32) * 3
+    arr = workloads.f32_to_bf16_bits(x) if dtype == "bf16" else x
+    am = np.argmax(workloads.to_f32(arr, dtype), -1)
+    parent = np.zeros((B, N), np.int32)
+    tokens = rng.integers(0, V, (B, N)).astype(np.int32)
+    for b in range(B):
+        parent[b] = workloads.tree_parents(N, rng)
+        for j in range(1, N):
+            if rng.random() < 0.6:
+                tokens[b, j] = am[b, parent[b, j]]  # duplicates among siblings happen
+    return arr, parent, tokens
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("B,N,V", [(1, 1, 10), (3, 5, 17), (16, 26, 3001), (4, 64, 40),
+                                   (2, 33, 20480 + 9), (70, 12, 300)])
+def test_tree_parity_shapes(dev, dtype, B, N, V):
+    rng = np.random.default_rng(B * 7 + N * 3 + V)
+    arr, parent, tokens = random_tree_case(rng, B, N, V, dtype)
+    r = sv.tree_greedy(to_dev(arr, dtype, dev), torch.from_numpy(parent).to(dev),
+                       torch.from_numpy(tokens).to(dev))
+    o = oracle.verify_tree_greedy(arr, dtype, parent, tokens, threads=THREADS)
+    for key in ("accepted_len", "path", "out_tokens"):
+        np.testing.assert_array_equal(r[key].cpu().numpy(), o[key], err_msg=key)
+
+
+def test_tree_chain_equals_greedy_on_gpu(dev):
+    w = workloads.make_greedy(B=20, k=8, V=5000, p_match=0.8, seed=13)
+    B = w["B"]
+    t = to_dev(w["target"], "bf16", dev)
+    parent = torch.arange(-1, 8, dtype=torch.int32, device=dev).repeat(B, 1)
+    tokens = torch.cat([torch.zeros((B, 1), dtype=torch.int32),
+                        torch.from_numpy(w["tokens"])], 1).to(dev)
+    r = sv.tree_greedy(t, parent.contiguous(), tokens.contiguous())
+    g = sv.greedy(t, torch.from_numpy(w["tokens"]).to(dev))
+    assert torch.equal(r["accepted_len"], g["accepted_len"])
+    assert torch.equal(r["out_tokens"], g["out_tokens"])
+
+
+def test_tree_invalid_parent_flag(dev):
+    rng = np.random.default_rng(44)
+    arr, parent, tokens = random_tree_case(rng, 6, 10, 200, "bf16")
+    parent[2, 4] = 9   # forward pointer
+    parent[5, 7] = -3  # negative
+    ws = sv.Workspace(dev)
+    r = sv.tree_greedy(to_dev(arr, "bf16", dev), torch.from_numpy(parent).to(dev),
+                       torch.from_numpy(tokens).to(dev), workspace=ws)
+    o = oracle.verify_tree_greedy(arr, "bf16", parent, tokens)
+    assert o["invalid_tree"]
+    for key in ("accepted_len", "path", "out_tokens"):
+        np.testing.assert_array_equal(r[key].cpu().numpy(), o[key], err_msg=key)
+    assert ws.device_status(clear=True) == sv.SV_FLAG_INVALID_TREE
+    torch.cuda.synchronize()
+    assert int(ws.buf[256:].cpu().count_nonzero()) == 0
+
+
 # ------------------------------------------------------------ device commit
 
 @pytest.mark.parametrize("B,k,cap", [(1, 0, 4), (7, 1, 9), (300, 8, 40), (33, 32, 100),
@@ -425,7 +485,7 @@ def test_one_workspace_across_modes_and_sizes(dev):
     ws = sv.Workspace(dev)
     rng = np.random.default_rng(16)
     for step in range(12):
-        mode = ("stochastic", "greedy", "multi", "rows")[step % 4]
+        mode = ("stochastic", "greedy", "multi", "rows", "tree")[step % 5]
         B = int(rng.integers(1, 40))
         k = int(rng.integers(0, 9))
         V = int(rng.integers(2, 3000))
@@ -449,6 +509,13 @@ def test_one_workspace_across_modes_and_sizes(dev):
             r = sv.multi_candidate(to_dev(w["target"], "bf16", dev),
                                    torch.from_numpy(w["tokens"]).to(dev), workspace=ws)
             o = oracle.verify_multi(w["target"], "bf16", w["tokens"])
+            np.testing.assert_array_equal(r["out_tokens"].cpu().numpy(), o["out_tokens"])
+        elif mode == "tree":
+            w = workloads.make_tree(B, k + 1, V, seed=step)
+            r = sv.tree_greedy(to_dev(w["node_logits"], "bf16", dev),
+                               torch.from_numpy(w["parent"]).to(dev),
+                               torch.from_numpy(w["tokens"]).to(dev), workspace=ws)
+            o = oracle.verify_tree_greedy(w["node_logits"], "bf16", w["parent"], w["tokens"])
             np.testing.assert_array_equal(r["out_tokens"].cpu().numpy(), o["out_tokens"])
         else:
             w = workloads.make_multi_rows(B, 3, k, V, seed=step)
@@ -485,6 +552,14 @@ def test_named_workload_full_size(dev, name):
                                torch.from_numpy(w["tokens"]).to(dev))
         o = oracle.verify_multi(w["target"], "bf16", w["tokens"], threads=THREADS)
         for key in ("best_candidate", "accepted_len", "out_tokens"):
+            np.testing.assert_array_equal(r[key].cpu().numpy(), o[key], err_msg=key)
+    elif mode == "tree":
+        r = sv.tree_greedy(to_dev(w["node_logits"], "bf16", dev),
+                           torch.from_numpy(w["parent"]).to(dev),
+                           torch.from_numpy(w["tokens"]).to(dev))
+        o = oracle.verify_tree_greedy(w["node_logits"], "bf16", w["parent"], w["tokens"],
+                                      threads=THREADS)
+        for key in ("accepted_len", "path", "out_tokens"):
             np.testing.assert_array_equal(r[key].cpu().numpy(), o[key], err_msg=key)
     else:
         r = sv.multi_candidate_rows(to_dev(w["rows"], "bf16", dev),

@@ -466,6 +466,85 @@ def test_multi_rows_invalid_entry_hand_case():
     assert r["out_tokens"].tolist() == [[1, -1, -1]]
 
 
+# ---------------------------------------------------------------- tree verify
+
+def longest_matching_path(parent, tokens, amax):
+    """Independent formulation: among all root paths whose every node's token
+    equals its parent's argmax, the longest (depth-first over all nodes)."""
+    N = len(parent)
+    best = [0]
+    stack = [[0]]
+    while stack:
+        path = stack.pop()
+        if len(path) > len(best):
+            best = path
+        u = path[-1]
+        for j in range(1, N):
+            if parent[j] == u and tokens[j] == amax[u]:
+                stack.append(path + [j])
+    return best
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_tree_walk_is_the_longest_matching_path(dtype):
+    rng = np.random.default_rng(41)
+    B, N, V = 60, 20, 9
+    x = tie_heavy_rows(rng, (B, N, V))
+    arr = workloads.f32_to_bf16_bits(x) if dtype == "bf16" else x
+    amax = np.argmax(x, -1)
+    parent = np.zeros((B, N), np.int32)
+    tokens = np.zeros((B, N), np.int32)
+    for b in range(B):
+        parent[b] = workloads.tree_parents(N, rng)
+        for u in range(N):
+            kids = [j for j in range(1, N) if parent[b, j] == u]
+            toks = rng.permutation(V)[:len(kids)]  # distinct sibling tokens
+            if kids and rng.random() < 0.8:
+                toks[0] = amax[b, u] if amax[b, u] not in toks[1:] else toks[0]
+            tokens[b, kids] = toks
+    r = oracle.verify_tree_greedy(arr, dtype, parent, tokens)
+    for b in range(B):
+        best = longest_matching_path(parent[b], tokens[b], amax[b])
+        n = len(best) - 1
+        assert r["accepted_len"][b] == n
+        assert r["path"][b, :n + 1].tolist() == best
+        assert (r["path"][b, n + 1:] == -1).all()
+        assert r["out_tokens"][b, :n].tolist() == [int(tokens[b, j]) for j in best[1:]]
+        assert r["out_tokens"][b, n] == amax[b, best[-1]]
+        assert (r["out_tokens"][b, n + 1:] == -1).all()
+
+
+def test_tree_chain_equals_greedy():
+    w = workloads.make_greedy(B=10, k=6, V=400, p_match=0.8, seed=12)
+    B, kp1 = w["target"].shape[:2]
+    parent = np.tile(np.arange(-1, kp1 - 1, dtype=np.int32), (B, 1))
+    tokens = np.concatenate([np.zeros((B, 1), np.int32), w["tokens"]], axis=1)
+    r = oracle.verify_tree_greedy(w["target"], "bf16", parent, tokens)
+    g = oracle.verify_greedy(w["target"], "bf16", w["tokens"])
+    np.testing.assert_array_equal(r["accepted_len"], g["accepted_len"])
+    np.testing.assert_array_equal(r["out_tokens"], g["out_tokens"])
+
+
+def test_tree_duplicate_siblings_and_invalid_parent_hand_cases():
+    # root argmax 2; nodes 1 and 2 both carry token 2 (duplicates), node 3 under
+    # node 2 would extend the path, but the walk takes node 1 (lowest index)
+    rows = np.zeros((1, 4, 3), np.float32)
+    rows[0, :, 2] = 1.0
+    parent = np.array([[-1, 0, 0, 2]], np.int32)
+    tokens = np.array([[0, 2, 2, 2]], np.int32)
+    r = oracle.verify_tree_greedy(rows, "f32", parent, tokens)
+    assert r["accepted_len"].tolist() == [1]
+    assert r["path"].tolist() == [[0, 1, -1, -1]]
+    assert r["out_tokens"].tolist() == [[2, 2, -1, -1]]
+    assert not r["invalid_tree"]
+    # node 1's parent points forward: it is never entered
+    parent = np.array([[-1, 3, 0, 2]], np.int32)
+    r = oracle.verify_tree_greedy(rows, "f32", parent, tokens)
+    assert r["invalid_tree"]
+    assert r["path"].tolist() == [[0, 2, 3, -1]]
+    assert r["out_tokens"].tolist() == [[2, 2, 2, -1]]
+
+
 # ------------------------------------------------------------ device commit
 
 def test_commit_hand_case():

@@ -49,6 +49,9 @@ WORKLOADS = {
                                   seed=3),
     "multi_b16_g8_k4_v32000": dict(mode="multi", B=16, G=8, k=4, V=32000, t_dtype="bf16",
                                    t_std=3.0, p_match=0.6, p_shared=0.5, seed=4),
+    # an EAGLE-style draft tree per sequence (Top-K children, distinct tokens)
+    "tree_b64_n26_v128256": dict(mode="tree", B=64, N=26, V=128256, t_dtype="bf16",
+                                 t_std=3.0, p_match=0.7, seed=6),
     # the same lookahead step with each distinct candidate prefix's row once
     "multi_rows_b16_g8_k4_v32000": dict(mode="multi_rows", B=16, G=8, k=4, V=32000,
                                         t_dtype="bf16", t_std=3.0, p_match=0.6,
@@ -263,6 +266,54 @@ def make_multi_rows(B: int, G: int, k: int, V: int, t_dtype: str = "bf16", t_std
                 tokens=w["tokens"], seed=seed, B=B, G=G, k=k, R=R, V=V)
 
 
+_S_TREE = 40
+
+
+def tree_parents(N: int, rng, max_children: int = 4) -> np.ndarray:
+    """A draft tree of N nodes in topological order: breadth-first, each node
+    taking up to `max_children` children, fewer at deeper levels (a Top-K tree
+    whose K shrinks with depth).  parent[0] = -1."""
+    parent = np.full(N, -1, np.int32)
+    frontier, depth, j = [0], 0, 1
+    while j < N:
+        nxt = []
+        for u in frontier:
+            kids = max(1, max_children - depth) if depth < 2 else int(rng.integers(1, 3))
+            for _ in range(kids):
+                if j >= N:
+                    break
+                parent[j] = u
+                nxt.append(j)
+                j += 1
+        frontier, depth = (nxt or [j - 1]), depth + 1
+    return parent
+
+
+def make_tree(B: int, N: int, V: int, t_dtype: str = "bf16", t_std: float = 3.0,
+              p_match: float = 0.7, seed: int = 0, threads: int | None = None) -> dict:
+    """Node rows [B,N,V] ~ N(0, t_std^2); per sequence a tree_parents topology;
+    children of a node carry distinct tokens, the first one being the node
+    row's argmax with probability p_match (so that paths are accepted)."""
+    rows = _target_rows(seed, B * N, V, t_std, t_dtype, threads).reshape(B, N, V)
+    am = np.argmax(to_f32(rows, t_dtype), -1)
+    g = _rng(seed, _S_TREE)
+    parent = np.zeros((B, N), np.int32)
+    tokens = np.zeros((B, N), np.int32)
+    for b in range(B):
+        parent[b] = tree_parents(N, g)
+        for u in range(N):
+            kids = [j for j in range(1, N) if parent[b, j] == u]
+            used = set()
+            for r, j in enumerate(kids):
+                t = int(am[b, u]) if (r == 0 and g.random() < p_match) else int(g.integers(0, V))
+                while t in used:
+                    t = (t + 1) % V
+                used.add(t)
+                tokens[b, j] = t
+    return dict(mode="tree", node_logits=rows, parent=parent, tokens=tokens, t_dtype=t_dtype,
+                seed=seed, B=B, N=N, V=V)
+
+
 def make(name: str, threads: int | None = None, **overrides) -> dict:
     """Inputs of a named workload (``WORKLOADS``), with optional overrides
     (e.g. ``B=4`` for a bounded sample of the same workload)."""
@@ -277,12 +328,15 @@ def make(name: str, threads: int | None = None, **overrides) -> dict:
         return make_multi(threads=threads, **cfg)
     if mode == "multi_rows":
         return make_multi_rows(threads=threads, **cfg)
+    if mode == "tree":
+        return make_tree(threads=threads, **cfg)
     raise ValueError(mode)
 
 
 def logit_bytes(w: dict) -> int:
     """Bytes of logits a verify call over workload ``w`` streams (all rows)."""
-    n = (w["rows"] if "rows" in w else w["target"]).size * ELEM_BYTES[w["t_dtype"]]
+    key = "rows" if "rows" in w else ("node_logits" if "node_logits" in w else "target")
+    n = w[key].size * ELEM_BYTES[w["t_dtype"]]
     if "draft" in w:
         n += w["draft"].size * ELEM_BYTES[w["d_dtype"]]
     return n
