@@ -70,7 +70,7 @@ def algorithmic_bytes(w: dict, accepted_len: np.ndarray | None) -> int:
         B, N, V = w["B"], w["N"], w["V"]
         return B * N * V * st + 8 * B * N + 4 * B + 8 * B * N
     B, k, V = w["B"], w["k"], w["V"]
-    if w["mode"] == "greedy":
+    if w["mode"] in ("greedy", "threshold"):
         return B * (k + 1) * V * st + 4 * B * k + 4 * B * (k + 2)
     if w["mode"] == "multi":
         G = w["G"]
@@ -204,6 +204,9 @@ def run_reference(args, rank: int) -> None:
         elif w["mode"] == "tree":
             oracle.verify_tree_greedy(w["node_logits"][b:b + 1], w["t_dtype"],
                                       w["parent"][b:b + 1], w["tokens"][b:b + 1])
+        elif w["mode"] == "threshold":
+            oracle.verify_threshold(w["target"][b:b + 1], w["t_dtype"], w["tokens"][b:b + 1],
+                                    w["temperature"], w["threshold"])
         else:
             oracle.verify_multi(w["target"][b:b + 1], w["t_dtype"], w["tokens"][b:b + 1])
 
@@ -263,6 +266,9 @@ def oracle_baseline(ws: dict) -> dict:
             elif w["mode"] == "tree":
                 oracle.verify_tree_greedy(w["node_logits"], w["t_dtype"], w["parent"],
                                           w["tokens"], threads=cores)
+            elif w["mode"] == "threshold":
+                oracle.verify_threshold(w["target"], w["t_dtype"], w["tokens"],
+                                        w["temperature"], w["threshold"], threads=cores)
             else:
                 oracle.verify_multi(w["target"], w["t_dtype"], w["tokens"], threads=cores)
         t_total += time.perf_counter() - t0
@@ -319,6 +325,9 @@ def run_ours(args, rank: int, world: int, dist) -> None:
                   sv.stochastic(t, d, tok, w["temperature"], w["seed"], off, out=o, workspace=wsp))
         elif w["mode"] == "greedy":
             fn = lambda t=t_d, tok=tok_d, o=out, wsp=wsp: sv.greedy(t, tok, out=o, workspace=wsp)
+        elif w["mode"] == "threshold":
+            fn = (lambda w=w, t=t_d, tok=tok_d, o=out, wsp=wsp:
+                  sv.threshold(t, tok, w["temperature"], w["threshold"], out=o, workspace=wsp))
         elif w["mode"] == "tree":
             par = torch.from_numpy(w["parent"]).to(dev)
             fn = (lambda t=t_d, pa=par, tok=tok_d, o=out, wsp=wsp:

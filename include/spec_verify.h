@@ -145,6 +145,29 @@ int spec_verify_greedy(const void *target_logits, int t_dtype, int64_t t_stride_
                        size_t workspace_bytes, void *stream);
 
 /*
+ * Threshold acceptance (a lossy variant).
+ *
+ * "Accelerating Sonar through speculation", section "Speculative decoding":
+ * every candidate prefix is scored by probability and the longest one at or
+ * above an acceptance threshold is selected; the target gives the next token.
+ * The score of the prefix of length j is its probability under the target,
+ * prod_{i<j} p_i(x_i) with p_i = softmax(target[b,i,:] / temperature); the
+ * accepted length n is the largest j <= k whose score is >= threshold (the
+ * empty prefix scores 1), and out_tokens[b, n] is the argmax of target row n
+ * (first maximum).  A draft token outside [0, V) has probability 0.  The
+ * pages fix no threshold: the caller passes it, 0 < threshold <= 1.
+ *
+ * Arguments, layouts, outputs and workspace as spec_verify_greedy, plus
+ * temperature (> 0, finite, as for spec_verify_stochastic) and threshold;
+ * anything else is SV_ERR_INVALID_ARG.
+ */
+int spec_verify_threshold(const void *target_logits, int t_dtype, int64_t t_stride_b,
+                          int64_t t_stride_pos, const int32_t *draft_tokens, int B, int k, int V,
+                          float temperature, float threshold, int32_t *accepted_len,
+                          int32_t *out_tokens, void *workspace, size_t workspace_bytes,
+                          void *stream);
+
+/*
  * Multi-candidate (lookahead / Jacobi n-gram) greedy verify.
  *
  * "Lookahead decoding" news piece, section "Lookahead decoding breaks the

@@ -67,6 +67,9 @@ def _load():
             lib.oracle_verify_multi.argtypes = [
                 P, i32, i64, i64, i64, P, i32, i32, i32, i32, i32, i32, P, P, P]
             lib.oracle_verify_multi.restype = i32
+            lib.oracle_verify_threshold.argtypes = [
+                P, i32, i64, i64, P, i32, i32, i32, dbl, dbl, i32, i32, P, P, P]
+            lib.oracle_verify_threshold.restype = i32
             _lib = lib
     return _lib
 
@@ -314,5 +317,32 @@ def verify_tree_greedy(node_logits: np.ndarray, t_dtype: str, parent: np.ndarray
             out["path"][b, n] = u
         out["out_tokens"][b, n] = amax[b, u]
         out["accepted_len"][b] = n
+    return out
+
+
+def verify_threshold(target: np.ndarray, t_dtype: str, tokens: np.ndarray, temperature: float,
+                     threshold: float, threads: int = 1) -> dict:
+    """Threshold acceptance of target [B,k+1,V] against draft tokens [B,k]:
+    n = the longest prefix whose probability under softmax(target/T) is at
+    least `threshold`, then the argmax of row n.  temperature and threshold
+    are rounded to float32 first, as the GPU library receives them.  Returns
+    accepted_len, out_tokens and log_scores [B,k] (ln of the prefix score for
+    the examined positions, NaN after)."""
+    lib = _load()
+    tc, (t_sb, t_sp) = _logits(target, t_dtype, 3)
+    B, kp1, V = target.shape
+    k = kp1 - 1
+    tok = np.ascontiguousarray(tokens, dtype=np.int32).reshape(B, k)
+    T = float(np.float32(temperature))
+    tau = float(np.float32(threshold))
+    out = {"accepted_len": np.zeros(B, np.int32), "out_tokens": np.zeros((B, k + 1), np.int32),
+           "log_scores": np.zeros((B, k), np.float64)}
+
+    def fn(b0, b1):
+        return lib.oracle_verify_threshold(
+            _ptr(target), tc, t_sb, t_sp, _ptr(tok), B, k, V, T, tau, b0, b1,
+            _ptr(out["accepted_len"]), _ptr(out["out_tokens"]), _ptr(out["log_scores"]))
+
+    _run_parallel(fn, B, threads)
     return out
 

@@ -31,6 +31,11 @@
  *  prefix that the target accepts, plus the target's own next token.  In
  *  greedy mode "accepts" means "equals the target argmax" (first maximum).
  *
+ *  Threshold acceptance.  Same page, same section: each candidate prefix is
+ *  scored by probability and the longest at or above the acceptance threshold
+ *  is kept (the score is the prefix's probability under the target; see
+ *  oracle_verify_threshold), plus the target's argmax as the extra token.
+ *
  *  Multi-candidate (lookahead n-gram) verify.  "Lookahead decoding" news
  *  piece, section "Lookahead decoding breaks the order dependency" and
  *  steps 2-4: captured n-grams are validated against the target and the
@@ -357,6 +362,63 @@ int oracle_verify_greedy(const void *target, int t_dtype, int64_t t_sb, int64_t 
             if (i == n && a_n < 0)
                 a_n = a;
         }
+        accepted_len[b] = n;
+        for (int i = 0; i <= k; ++i) {
+            int32_t v = -1;
+            if (i < n) v = tokens[(int64_t)b * k + i];
+            else if (i == n) v = a_n;
+            out_tokens[(int64_t)b * (k + 1) + i] = v;
+        }
+    }
+    return 0;
+}
+
+/* ---------------------------------------------------- threshold acceptance */
+
+/*
+ * "Accelerating Sonar through speculation", section "Speculative decoding":
+ * each candidate prefix is scored by its probability and the longest one at
+ * or above an acceptance threshold is selected; the target gives one more
+ * token.  Reading (the pages fix no scoring rule or threshold): the score of
+ * the prefix of length j is its probability under the target,
+ *     score(j) = prod_{i<j} p_i(x_i),   p_i = softmax(target[b,i,:] / T),
+ * n = the largest j <= k with score(j) >= tau (score(0) = 1), and the extra
+ * token is the target's argmax at row n (first maximum).  A draft token
+ * outside [0, V) has p = 0.  log_scores[b*k + i] = ln score(i+1) for the
+ * examined positions i <= n (i < k), -inf after a zero, for near-tie checks.
+ */
+int oracle_verify_threshold(const void *target, int t_dtype, int64_t t_sb, int64_t t_sp,
+                            const int32_t *tokens, int B, int k, int V, double T, double tau,
+                            int b_begin, int b_end, int32_t *accepted_len,
+                            int32_t *out_tokens, double *log_scores)
+{
+    if (V < 1 || k < 0 || B < 0 || b_begin < 0 || b_end > B || !(T > 0.0) ||
+        !(tau > 0.0) || !(tau <= 1.0))
+        return -1;
+    const double log_tau = log(tau);
+    for (int b = b_begin; b < b_end; ++b) {
+        int n = k;
+        double acc = 0.0; /* ln score(i+1) */
+        for (int i = 0; i < k; ++i) {
+            row_t rt = {target, t_dtype, (int64_t)b * t_sb + (int64_t)i * t_sp};
+            int32_t x = tokens[(int64_t)b * k + i];
+            double lp = -INFINITY;
+            if (x >= 0 && x < V) {
+                double m, s;
+                softmax_stats(rt, V, T, &m, &s);
+                lp = log(softmax_prob(rt, x, T, m, s));
+            }
+            acc += lp;
+            if (log_scores) log_scores[(int64_t)b * k + i] = acc;
+            if (!(acc >= log_tau)) {
+                n = i;
+                break;
+            }
+        }
+        if (log_scores)
+            for (int i = n + 1; i < k; ++i) log_scores[(int64_t)b * k + i] = NAN;
+        row_t rn = {target, t_dtype, (int64_t)b * t_sb + (int64_t)n * t_sp};
+        int32_t a_n = row_argmax(rn, V);
         accepted_len[b] = n;
         for (int i = 0; i <= k; ++i) {
             int32_t v = -1;

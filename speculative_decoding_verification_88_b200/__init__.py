@@ -30,7 +30,7 @@ EXPORTS = (
     "spec_verify_workspace_size", "spec_verify_status_string", "spec_verify_workspace_init",
     "spec_verify_read_device_status", "spec_verify_stochastic", "spec_verify_greedy",
     "spec_verify_multi_candidate", "spec_verify_multi_candidate_rows", "spec_verify_commit",
-    "spec_verify_tree_workspace_size", "spec_verify_tree_greedy",
+    "spec_verify_tree_workspace_size", "spec_verify_tree_greedy", "spec_verify_threshold",
     "spec_verify_philox4x32_10", "spec_verify_greedy_noalloc",
 )
 
@@ -86,6 +86,8 @@ def load_library():
         lib.spec_verify_tree_workspace_size.restype = SZ
         lib.spec_verify_tree_greedy.argtypes = [P, I, I64, I64, P, P, I, I, I, P, P, P, P, SZ, P]
         lib.spec_verify_tree_greedy.restype = I
+        lib.spec_verify_threshold.argtypes = [P, I, I64, I64, P, I, I, I, F, F, P, P, P, SZ, P]
+        lib.spec_verify_threshold.restype = I
         lib.spec_verify_philox4x32_10.argtypes = [P, I64, U64, P, P]
         lib.spec_verify_philox4x32_10.restype = I
         lib.spec_verify_greedy_noalloc.argtypes = [P, I, I64, I64, P, I, I, I, P, P, P]
@@ -315,6 +317,32 @@ def multi_candidate_rows(rows: torch.Tensor, row_of: torch.Tensor, cand_tokens: 
             res["best_candidate"].data_ptr(), res["accepted_len"].data_ptr(),
             res["out_tokens"].data_ptr(), ws.buf.data_ptr(), ws.nbytes, _stream_ptr(stream, dev))
     _check(code, "spec_verify_multi_candidate_rows")
+    _count()
+    return res
+
+
+def threshold(target: torch.Tensor, draft_tokens: torch.Tensor, temperature: float,
+              threshold: float, *, out: dict | None = None, workspace: Workspace | None = None,
+              stream=None) -> dict:
+    """Threshold acceptance: target [B,k+1,V], draft_tokens [B,k]; accept the
+    longest prefix whose probability under softmax(target/T) is at least
+    `threshold`, then the argmax of the next row."""
+    lib = load_library()
+    tc, (tsb, tsp, _) = _logits(target, 3, "target")
+    B, kp1, V = target.shape
+    k = kp1 - 1
+    dev = target.device
+    tok = _tokens(draft_tokens, (B, k), dev, "draft_tokens")
+    res = {"accepted_len": _out(out, "accepted_len", (B,), torch.int32, dev),
+           "out_tokens": _out(out, "out_tokens", (B, k + 1), torch.int32, dev)}
+    ws = workspace or default_workspace(dev)
+    ws.ensure(workspace_size(B, 1, k, V), stream)
+    with torch.cuda.device(dev):
+        code = lib.spec_verify_threshold(
+            target.data_ptr(), tc, tsb, tsp, tok.data_ptr(), B, k, V, float(temperature),
+            float(threshold), res["accepted_len"].data_ptr(), res["out_tokens"].data_ptr(),
+            ws.buf.data_ptr(), ws.nbytes, _stream_ptr(stream, dev))
+    _check(code, "spec_verify_threshold")
     _count()
     return res
 

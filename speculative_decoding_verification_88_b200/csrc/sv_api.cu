@@ -74,6 +74,21 @@ size_t stochastic_part_bytes(int B, int k, int V, int bpe, int es_min) {
   return stochastic_layout(B, k, pl.nch).bytes;
 }
 
+// Threshold acceptance: the argmax layout followed by chunk statistics
+// [B][k+1][nch] and row statistics [B][k+1] (8 bytes each).
+struct ThreshLayout {
+  ArgLayout a;
+  size_t sslots, rstats, bytes;
+};
+ThreshLayout threshold_layout(long long rows, int nch) {
+  ThreshLayout l;
+  l.a = argmax_layout(rows, nch);
+  l.sslots = l.a.bytes;
+  l.rstats = l.sslots + static_cast<size_t>(rows) * nch * 8;
+  l.bytes = l.rstats + static_cast<size_t>(rows) * 8;
+  return l;
+}
+
 size_t argmax_key_bytes(int B, int G, int k, int V, int es) {
   const long long rows = static_cast<long long>(B) * G * (k + 1);
   return argmax_layout(rows, plan_chunks(rows, V, es, es, kArgmaxChunkBytes).nch).bytes;
@@ -119,6 +134,12 @@ extern "C" size_t spec_verify_workspace_size(int B, int G, int k, int V) {
     if (a > tail) tail = a;
   }
   if (G == 1) {
+    for (int es : {2, 4}) {  // threshold acceptance
+      const long long rows = static_cast<long long>(B) * (k + 1);
+      const size_t t =
+          threshold_layout(rows, plan_chunks(rows, V, es, es, kArgmaxChunkBytes).nch).bytes;
+      if (t > tail) tail = t;
+    }
     // (bytes per entry, narrowest element) of bf16/bf16, bf16/fp32 (either
     // way round) and fp32/fp32 pairs
     static const int kPairs[3][2] = {{4, 2}, {6, 2}, {8, 4}};
@@ -262,7 +283,8 @@ static int argmax_call(const void* target_logits, int t_dtype, int64_t sb, int64
                        const int32_t* row_of, const int32_t* parent, int32_t* path,
                        int32_t* best_g, int32_t* accepted_len, int32_t* out_tokens,
                        void* workspace, size_t workspace_bytes, void* stream,
-                       size_t need_bytes) {
+                       size_t need_bytes, float temperature = 0.0f, float threshold = 0.0f) {
+  const bool thresh = threshold > 0.0f;
   if (!sizes_ok(B, G, k, V)) return SV_ERR_INVALID_ARG;
   const long long full_rows = static_cast<long long>(G) * (k + 1);
   if (R < 0 || R > full_rows || (R > 0) != (row_of != nullptr || parent != nullptr) ||
@@ -315,6 +337,14 @@ static int argmax_call(const void* target_logits, int t_dtype, int64_t sb, int64
   p.total = static_cast<unsigned int>(total);
   p.ctrl = ws.ctrl;
   p.seq = ws.seq;
+  p.t_dtype = t_dtype;
+  const ThreshLayout tl = threshold_layout(rows, pl.nch);
+  if (thresh) {
+    p.c2 = 1.4426950408889634f / temperature;
+    p.log2_tau = std::log2(threshold);
+    p.sslots = reinterpret_cast<unsigned long long*>(static_cast<unsigned char*>(ws.tail) + tl.sslots);
+    p.rstats = reinterpret_cast<unsigned long long*>(static_cast<unsigned char*>(ws.tail) + tl.rstats);
+  }
   const ArgLayout lay = argmax_layout(rows, pl.nch);
   unsigned char* tail = static_cast<unsigned char*>(ws.tail);
   p.slots = reinterpret_cast<unsigned long long*>(tail + lay.slots);
@@ -362,6 +392,21 @@ extern "C" int spec_verify_multi_candidate_rows(const void* row_logits, int t_dt
                      B > 0 ? R : 0, B > 0 ? row_of : nullptr, nullptr, nullptr, best_candidate,
                      accepted_len, out_tokens, workspace, workspace_bytes, stream,
                      spec_verify_workspace_size(B, G, k, V));
+}
+
+extern "C" int spec_verify_threshold(const void* target_logits, int t_dtype, int64_t t_stride_b,
+                                     int64_t t_stride_pos, const int32_t* draft_tokens, int B,
+                                     int k, int V, float temperature, float threshold,
+                                     int32_t* accepted_len, int32_t* out_tokens, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+  if (!(temperature > 0.0f) || !std::isfinite(temperature) ||
+      !std::isfinite(1.4426950408889634f / temperature))
+    return SV_ERR_INVALID_ARG;
+  if (!(threshold > 0.0f) || !(threshold <= 1.0f)) return SV_ERR_INVALID_ARG;
+  return argmax_call(target_logits, t_dtype, t_stride_b, 0, t_stride_pos, draft_tokens, B, 1, k,
+                     V, 0, nullptr, nullptr, nullptr, nullptr, accepted_len, out_tokens,
+                     workspace, workspace_bytes, stream, spec_verify_workspace_size(B, 1, k, V),
+                     temperature, threshold);
 }
 
 extern "C" size_t spec_verify_tree_workspace_size(int B, int N, int V) {

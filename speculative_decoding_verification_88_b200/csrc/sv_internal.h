@@ -118,6 +118,12 @@ struct ArgmaxParams {
   const int* parent;     // tree form: [B, R] parent of each node (tokens and out_tokens
                          // are then [B, R]; G and k only bound R)
   int* path;             // tree form: [B, R] accepted path out
+  // threshold acceptance (sslots != nullptr): row softmax statistics as well
+  int t_dtype;                  // SV_F32 / SV_BF16 (the finalize reads draft-token logits)
+  float c2;                     // log2(e) / T
+  float log2_tau;               // lg2 of the acceptance threshold
+  unsigned long long* sslots;   // [B][R][nch] chunk (max, sum) statistics
+  unsigned long long* rstats;   // [B][R] row statistics
   int* best_g;  // nullable
   int* accepted_len;
   int* out_tokens;

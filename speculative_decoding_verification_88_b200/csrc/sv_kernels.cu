@@ -515,6 +515,53 @@ __device__ __forceinline__ void chunk_argmax_regs(const unsigned char* smem, con
   bi = idx;
 }
 
+// Argmax and softmax statistics of one chunk from the same registers
+// (threshold acceptance): returns (max value, its index as float bits,
+// m = max * c2, s = sum 2^(x c2 - m)), merged over the warp.
+template <typename T>
+__device__ __forceinline__ float4 chunk_argmax_stats_regs(const unsigned char* smem, const Hdr& h,
+                                                          const void* g, float c2, int tid,
+                                                          Shared& sh, int s, int lane) {
+  constexpr int EPV = Elem<T>::kPerVec;
+  constexpr int N = max_vecs<T, 0, kArgmaxChunkBytes>();
+  uint4 v[N];
+  load_vecs<T>(smem, h.nvec_t, tid, v);
+  float best = -INFINITY;
+  int bj = -1;
+  uint4 bvec = v[0];
+  const bool full = h.nvec_t == N * kComputeThreads;
+#pragma unroll
+  for (int j = 0; j < N; ++j) {
+    const float m = vec_max<T>(v[j]);
+    const bool take = (full || tid + j * kComputeThreads < h.nvec_t) && (bj < 0 || m > best);
+    best = take ? m : best;
+    bj = take ? j : bj;
+    bvec = take ? v[j] : bvec;
+  }
+  int idx = INT_MAX;
+  if (bj >= 0) {
+    float f[EPV];
+    unpack(bvec, f);
+    const int x = h.x0 + (tid + bj * kComputeThreads) * EPV;
+#pragma unroll
+    for (int q = EPV - 1; q >= 0; --q)
+      if (f[q] == best) idx = x + q;
+  }
+  const int e = h.nvec_t * EPV + tid;  // the ragged end is shorter than one vector
+  if (e < h.len) {
+    const float t = load_elem<T>(g, h.toff + e);
+    if (better(t, h.x0 + e, best, idx)) {
+      best = t;
+      idx = h.x0 + e;
+    }
+  }
+  float m, sum;
+  thread_stats<T>(v, g, h.toff, h.nvec_t * EPV, h.len, c2, tid, m, sum);
+  warp_argmax(best, idx);
+  const float4 st = warp_stats2(make_float4(m, sum, -INFINITY, 0.0f));
+  return make_float4(best, __int_as_float(idx), st.x, st.y);
+}
+
 // Eight consecutive entries (group j of the chunk) from shared memory.
 template <typename T>
 __device__ __forceinline__ void load8(const unsigned char* smem, int j, float (&f)[8]);
@@ -1227,14 +1274,78 @@ __device__ void argmax_compute(const ArgmaxParams& p, Shared& sh, unsigned char*
     }
     float bv;
     int bi;
-    if (kTma)
-      chunk_argmax_regs<TT>(stages + static_cast<size_t>(s) * kStageBytes, h, p.tgt, tid, bv, bi);
-    else
-      chunk_argmax<TT>(stages + static_cast<size_t>(s) * kStageBytes, h, p.tgt, tid, bv, bi);
+    float4 r = make_float4(0.0f, 0.0f, -INFINITY, 0.0f);
+    if (p.sslots && h.i < p.k) {  // threshold acceptance: row statistics too
+      if (kTma) {
+        r = chunk_argmax_stats_regs<TT>(stages + static_cast<size_t>(s) * kStageBytes, h, p.tgt,
+                                        p.c2, tid, sh, s, lane);
+      } else {
+        chunk_argmax<TT>(stages + static_cast<size_t>(s) * kStageBytes, h, p.tgt, tid, bv, bi);
+        float m, sm;
+        chunk_stats<TT>(stages + static_cast<size_t>(s) * kStageBytes, h.nvec_t, p.tgt, h.toff,
+                        h.len, p.c2, tid, m, sm);
+        r = make_float4(bv, __int_as_float(bi), m, sm);
+      }
+    } else {
+      if (kTma)
+        chunk_argmax_regs<TT>(stages + static_cast<size_t>(s) * kStageBytes, h, p.tgt, tid, bv,
+                              bi);
+      else
+        chunk_argmax<TT>(stages + static_cast<size_t>(s) * kStageBytes, h, p.tgt, tid, bv, bi);
+      r.x = bv;
+      r.y = __int_as_float(bi);
+    }
     if (lane == 0) {
-      sh.res[s][w] = make_float4(bv, __int_as_float(bi), 0.0f, 0.0f);
+      sh.res[s][w] = r;
       mbar_arrive(&sh.rfull[s]);
     }
+  }
+}
+
+// Threshold acceptance, finalize of sequence b (one warp, lane i = position
+// i): log2 p_i(x_i) = l_i(x_i) c2 - m_i - lg2 s_i from the row statistics; an
+// inclusive prefix sum gives the log2 score of each prefix; n = the first
+// position whose prefix falls below the threshold (or k); the extra token
+// is row n's argmax.
+__device__ void finalize_threshold(const ArgmaxParams& p, int b, int lane) {
+  const int k = p.k, R = p.R, V = p.V;
+  unsigned long long* keys = p.rkey + static_cast<size_t>(b) * R;
+  unsigned long long* stats = p.rstats + static_cast<size_t>(b) * R;
+  const unsigned long long kv = lane <= k ? take(keys + lane, ld_relaxed_u64(keys + lane), p.ctrl)
+                                          : 0ull;
+  const unsigned long long k32 =
+      (k == 32 && lane == 0) ? take(keys + 32, ld_relaxed_u64(keys + 32), p.ctrl) : 0ull;
+  float lp = 0.0f;  // log2 p_i(x_i)
+  if (lane < k) {
+    float m, sm;
+    unpack_stats(take(stats + lane, ld_relaxed_u64(stats + lane), p.ctrl), m, sm);
+    const int x = __ldg(p.tokens + static_cast<size_t>(b) * k + lane);
+    if (x >= 0 && x < V) {
+      const long long off = static_cast<long long>(b) * p.sb + static_cast<long long>(lane) * p.sp + x;
+      const float l = p.t_dtype == 1 ? load_elem<uint16_t>(p.tgt, off) : load_elem<float>(p.tgt, off);
+      lp = fmaf(l, p.c2, -m) - lg2f(sm);
+    } else {
+      lp = -INFINITY;
+    }
+  }
+  float cum = lp;  // inclusive prefix sum over lanes
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const float up = __shfl_up_sync(0xffffffffu, cum, o);
+    if (lane >= o) cum += up;
+  }
+  const bool fail = lane < k && !(cum >= p.log2_tau);
+  const unsigned int mm = __ballot_sync(0xffffffffu, fail);
+  const int n = mm ? __ffs(mm) - 1 : k;
+  const int an = __shfl_sync(0xffffffffu, key_index(kv), n & 31);
+  const int a32 = __shfl_sync(0xffffffffu, key_index(k32), 0);
+  const int next = n == 32 ? a32 : an;
+  int* out = p.out_tokens + static_cast<size_t>(b) * (k + 1);
+  for (int i = lane; i <= k; i += 32)
+    out[i] = i < n ? __ldg(p.tokens + static_cast<size_t>(b) * k + i) : (i == n ? next : -1);
+  if (lane == 0) {
+    p.accepted_len[b] = n;
+    p.seq[b].cnt1 = 0u;
   }
 }
 
@@ -1416,14 +1527,30 @@ __device__ void merge_argmax_row(const ArgmaxParams& p, int b, int r, int lane) 
     key = v > key ? v : key;
   }
   key = warp_max_u64(key);
+  const bool with_stats = p.sslots && r < p.k;
+  float M = -INFINITY, S = 0.0f;
+  if (with_stats) {
+    unsigned long long* ss = p.sslots + (static_cast<size_t>(b) * R + r) * p.nch;
+    for (int c = lane; c < p.nch; c += 32) {
+      float m, sv;
+      unpack_stats(take(ss + c, ld_relaxed_u64(ss + c), p.ctrl), m, sv);
+      merge_stats(M, S, m, sv);
+    }
+    const float4 w = warp_stats2(make_float4(M, S, -INFINITY, 0.0f));
+    M = w.x;
+    S = w.y;
+  }
   unsigned int old = 0u;
   if (lane == 0) {
+    if (with_stats) st_relaxed_u64(p.rstats + static_cast<size_t>(b) * R + r, pack_stats(M, S));
     st_relaxed_u64(p.rkey + static_cast<size_t>(b) * R + r, key);
     p.rc[static_cast<size_t>(b) * R + r] = 0u;
     old = atomicAdd(&p.seq[b].cnt1, 1u);
   }
   if (__shfl_sync(0xffffffffu, old == R - 1u ? 1 : 0, 0)) {
-    if (p.parent)
+    if (p.sslots)
+      finalize_threshold(p, b, lane);
+    else if (p.parent)
       finalize_argmax_tree(p, b, lane);
     else if (p.row_of)
       finalize_argmax_rows(p, b, lane);
@@ -1450,18 +1577,24 @@ __device__ void argmax_epilogue(const ArgmaxParams& p, Shared& sh, int group, in
     if (h.kind == kKindEnd) break;
     float v = -INFINITY;
     int i = INT_MAX;
+    float4 st = make_float4(-INFINITY, 0.0f, -INFINITY, 0.0f);
     if (lane < kGroupWarps) {
       const float4 r = sh.res[s][lane];
       v = r.x;
       i = __float_as_int(r.y);
+      st.x = r.z;
+      st.y = r.w;
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&sh.empty[s]);
     warp_argmax(v, i);
+    const bool with_stats = p.sslots && h.i < p.k;
+    if (with_stats) st = warp_stats2(st);
     unsigned int old = 0u;
     if (lane == 0) {
-      st_relaxed_u64(p.slots + (static_cast<size_t>(h.b) * R + h.i) * p.nch + h.c,
-                     make_key(v, i));
+      const size_t slot = (static_cast<size_t>(h.b) * R + h.i) * p.nch + h.c;
+      st_relaxed_u64(p.slots + slot, make_key(v, i));
+      if (with_stats) st_relaxed_u64(p.sslots + slot, pack_stats(st.x, st.y));
       old = atomicAdd(&p.rc[static_cast<size_t>(h.b) * R + h.i], 1u);
     }
     if (pend_b >= 0 && __shfl_sync(0xffffffffu, pend_old == last ? 1 : 0, 0))

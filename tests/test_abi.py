@@ -141,6 +141,24 @@ def test_multi_rows_validation(lib):
     assert r(wb=64) == WORKSPACE
 
 
+def test_threshold_validation(lib):
+    def t(**kw):
+        a = dict(x=A16, dt=1, sb=40, sp=8, tok=A16, B=2, k=4, V=8, T=1.0, tau=0.1, acc=A16,
+                 out=A16, ws=A16, wb=1 << 20, st=None)
+        a.update(kw)
+        return lib.spec_verify_threshold(*a.values())
+
+    assert t(B=0, x=None) == OK
+    for T in (0.0, -1.0, float("inf"), float("nan"), 1e-40):
+        assert t(T=T) == INVALID, T
+    for tau in (0.0, -0.5, 1.5, float("nan")):
+        assert t(tau=tau) == INVALID, tau
+    assert t(k=33) == INVALID
+    assert t(tok=None) == INVALID
+    assert t(acc=A16 + 1) == MISALIGNED
+    assert t(wb=64) == WORKSPACE
+
+
 def test_tree_validation(lib):
     assert sv.tree_workspace_size(4, 26, 128256) > 0
     assert sv.tree_workspace_size(4, 0, 10) == 0

@@ -259,6 +259,59 @@ def test_multi_rows_invalid_entries_and_limits(dev):
                                 torch.zeros((1, 2, 1), dtype=torch.int32, device=dev))
 
 
+# ------------------------------------------------------ threshold acceptance
+
+TOL_SCORE = 1e-4  # |ln score - ln tau| below which a decision is a near tie
+
+
+def compare_threshold(r, o, tau):
+    """Exact except sequences whose examined prefix score is within TOL_SCORE
+    of the threshold (natural-log units); returns how many were near."""
+    ls = o["log_scores"]
+    lt = np.log(np.float32(tau))
+    near = np.zeros(len(o["accepted_len"]), bool)
+    k = ls.shape[1]
+    for b in range(len(near)):
+        upto = min(int(o["accepted_len"][b]) + 1, k)
+        v = ls[b, :upto]
+        near[b] = bool((np.abs(v[np.isfinite(v)] - lt) < TOL_SCORE).any())
+    acc = r["accepted_len"].cpu().numpy()
+    out = r["out_tokens"].cpu().numpy()
+    ok = ~near
+    np.testing.assert_array_equal(acc[ok], o["accepted_len"][ok])
+    np.testing.assert_array_equal(out[ok], o["out_tokens"][ok])
+    return int(near.sum())
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("B,k,V,T,tau", [(1, 1, 1, 1.0, 0.5), (5, 4, 33, 0.7, 0.01),
+                                         (64, 8, 4097, 1.0, 1e-4), (7, 32, 500, 1.3, 1e-30),
+                                         (16, 4, 128256, 0.7, 1e-3), (40, 0, 100, 1.0, 0.5)])
+def test_threshold_parity(dev, dtype, B, k, V, T, tau):
+    w = workloads.make_greedy(B, k, V, t_dtype=dtype, p_match=0.8, seed=B + k + V)
+    r = sv.threshold(to_dev(w["target"], dtype, dev), torch.from_numpy(w["tokens"]).to(dev),
+                     T, tau)
+    o = oracle.verify_threshold(w["target"], dtype, w["tokens"], T, tau, threads=THREADS)
+    near = compare_threshold(r, o, tau)
+    assert near <= max(1, B // 20)
+
+
+def test_threshold_invalid_tokens_and_workspace(dev):
+    w = workloads.make_greedy(12, 5, 300, p_match=0.9, seed=50)
+    tok = w["tokens"].copy()
+    tok[3, 1] = 300
+    tok[7, 0] = -4
+    ws = sv.Workspace(dev)
+    r = sv.threshold(to_dev(w["target"], "bf16", dev), torch.from_numpy(tok).to(dev), 1.0,
+                     1e-20, workspace=ws)
+    o = oracle.verify_threshold(w["target"], "bf16", tok, 1.0, 1e-20)
+    compare_threshold(r, o, 1e-20)
+    assert int(r["accepted_len"][3]) <= 1 and int(r["accepted_len"][7]) == 0
+    torch.cuda.synchronize()
+    assert int(ws.buf[256:].cpu().count_nonzero()) == 0
+    assert ws.device_status() == 0
+
+
 # ---------------------------------------------------------------- tree verify
 
 def random_tree_case(rng, B, N, V, dtype, dup=0.1):
@@ -484,8 +537,8 @@ def test_one_workspace_across_modes_and_sizes(dev):
     leave it clean for the next."""
     ws = sv.Workspace(dev)
     rng = np.random.default_rng(16)
-    for step in range(12):
-        mode = ("stochastic", "greedy", "multi", "rows", "tree")[step % 5]
+    for step in range(18):
+        mode = ("stochastic", "greedy", "multi", "rows", "tree", "threshold")[step % 6]
         B = int(rng.integers(1, 40))
         k = int(rng.integers(0, 9))
         V = int(rng.integers(2, 3000))
@@ -510,6 +563,12 @@ def test_one_workspace_across_modes_and_sizes(dev):
                                    torch.from_numpy(w["tokens"]).to(dev), workspace=ws)
             o = oracle.verify_multi(w["target"], "bf16", w["tokens"])
             np.testing.assert_array_equal(r["out_tokens"].cpu().numpy(), o["out_tokens"])
+        elif mode == "threshold":
+            w = workloads.make_greedy(B, k, V, seed=step)
+            r = sv.threshold(to_dev(w["target"], "bf16", dev),
+                             torch.from_numpy(w["tokens"]).to(dev), 1.0, 1e-3, workspace=ws)
+            o = oracle.verify_threshold(w["target"], "bf16", w["tokens"], 1.0, 1e-3)
+            compare_threshold(r, o, 1e-3)
         elif mode == "tree":
             w = workloads.make_tree(B, k + 1, V, seed=step)
             r = sv.tree_greedy(to_dev(w["node_logits"], "bf16", dev),
@@ -553,6 +612,13 @@ def test_named_workload_full_size(dev, name):
         o = oracle.verify_multi(w["target"], "bf16", w["tokens"], threads=THREADS)
         for key in ("best_candidate", "accepted_len", "out_tokens"):
             np.testing.assert_array_equal(r[key].cpu().numpy(), o[key], err_msg=key)
+    elif mode == "threshold":
+        r = sv.threshold(to_dev(w["target"], "bf16", dev), torch.from_numpy(w["tokens"]).to(dev),
+                         w["temperature"], w["threshold"])
+        o = oracle.verify_threshold(w["target"], "bf16", w["tokens"], w["temperature"],
+                                    w["threshold"], threads=THREADS)
+        near = compare_threshold(r, o, w["threshold"])
+        print(f"{name}: near ties {near}")
     elif mode == "tree":
         r = sv.tree_greedy(to_dev(w["node_logits"], "bf16", dev),
                            torch.from_numpy(w["parent"]).to(dev),

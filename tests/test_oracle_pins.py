@@ -466,6 +466,45 @@ def test_multi_rows_invalid_entry_hand_case():
     assert r["out_tokens"].tolist() == [[1, -1, -1]]
 
 
+# ------------------------------------------------------ threshold acceptance
+
+def test_threshold_uniform_rows_closed_form():
+    # uniform rows over V: every drafted token has p = 1/V, score(j) = V^-j
+    B, k, V = 3, 6, 4
+    x = np.zeros((B, k + 1, V), np.float32)
+    tokens = np.tile(np.arange(k, dtype=np.int32) % V, (B, 1))
+    for tau, n in ((0.9, 0), (0.2, 1), (0.05, 2), (0.01, 3), (0.003, 4), (1e-30, k)):
+        r = oracle.verify_threshold(x, "f32", tokens, 1.0, tau)
+        assert r["accepted_len"].tolist() == [n] * B, tau
+        assert r["out_tokens"][:, n].tolist() == [0] * B  # argmax of a flat row: first entry
+        assert (r["out_tokens"][:, :n] == tokens[:, :n]).all()
+
+
+def test_threshold_low_temperature_is_greedy():
+    """As T -> 0, p_i(x_i) -> 1 for the row argmax and -> 0 otherwise, so a
+    threshold of 1/2 reproduces greedy verify (rows without tied maxima)."""
+    w = workloads.make_greedy(B=40, k=5, V=200, t_dtype="f32", p_match=0.7, seed=17)
+    srt = np.sort(w["target"], -1)
+    assert (srt[..., -1] - srt[..., -2] > 1e-4).all()  # clear maxima
+    r = oracle.verify_threshold(w["target"], "f32", w["tokens"], 1e-6, 0.5)
+    g = oracle.verify_greedy(w["target"], "f32", w["tokens"])
+    np.testing.assert_array_equal(r["accepted_len"], g["accepted_len"])
+    np.testing.assert_array_equal(r["out_tokens"], g["out_tokens"])
+
+
+def test_threshold_monotone_and_invalid_token():
+    w = workloads.make_greedy(B=30, k=6, V=100, p_match=0.6, seed=18)
+    ns = [oracle.verify_threshold(w["target"], "bf16", w["tokens"], 1.0, tau)["accepted_len"]
+          for tau in (1e-12, 1e-6, 1e-3, 0.1, 0.5, 1.0)]
+    for a, b in zip(ns, ns[1:]):
+        assert (a >= b).all()  # a higher threshold never accepts more
+    tok = w["tokens"].copy()
+    tok[:, 2] = -1  # probability 0 at position 2
+    r = oracle.verify_threshold(w["target"], "bf16", tok, 1.0, 1e-30)
+    assert (r["accepted_len"] <= 2).all()
+    assert (r["accepted_len"] == 2).sum() > 0
+
+
 # ---------------------------------------------------------------- tree verify
 
 def longest_matching_path(parent, tokens, amax):

@@ -49,6 +49,10 @@ WORKLOADS = {
                                   seed=3),
     "multi_b16_g8_k4_v32000": dict(mode="multi", B=16, G=8, k=4, V=32000, t_dtype="bf16",
                                    t_std=3.0, p_match=0.6, p_shared=0.5, seed=4),
+    # threshold acceptance on the greedy workload's rows and drafts
+    "threshold_b64_k4_v128256": dict(mode="threshold", B=64, k=4, V=128256, t_dtype="bf16",
+                                     t_std=3.0, p_match=0.7, seed=2, temperature=1.0,
+                                     threshold=1e-3),
     # an EAGLE-style draft tree per sequence (Top-K children, distinct tokens)
     "tree_b64_n26_v128256": dict(mode="tree", B=64, N=26, V=128256, t_dtype="bf16",
                                  t_std=3.0, p_match=0.7, seed=6),
@@ -330,6 +334,11 @@ def make(name: str, threads: int | None = None, **overrides) -> dict:
         return make_multi_rows(threads=threads, **cfg)
     if mode == "tree":
         return make_tree(threads=threads, **cfg)
+    if mode == "threshold":
+        T, tau = cfg.pop("temperature"), cfg.pop("threshold")
+        w = make_greedy(threads=threads, **cfg)
+        w.update(mode="threshold", temperature=T, threshold=tau)
+        return w
     raise ValueError(mode)
 
 
