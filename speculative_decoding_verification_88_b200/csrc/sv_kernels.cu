@@ -1211,7 +1211,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ================================================================ argmax
 
-template <typename TT, bool kTma>
+// kRowStride: rows or tree form, row h.i of the sequence at stride sg.
+template <typename TT, bool kTma, bool kRowStride>
 __device__ void argmax_producer(const ArgmaxParams& p, Shared& sh, unsigned char* stages) {
   Ctrl* ctrl = p.ctrl;
   const unsigned int per_seq = static_cast<unsigned int>(p.R) * static_cast<unsigned int>(p.nch);
@@ -1231,7 +1232,7 @@ __device__ void argmax_producer(const ArgmaxParams& p, Shared& sh, unsigned char
       h.c = static_cast<int>(rem % p.nch);
       h.x0 = h.c * p.ch;
       h.len = min(p.ch, p.V - h.x0);
-      if (p.row_of || p.parent) {  // rows or tree form: row h.i of the sequence
+      if (kRowStride) {
         h.toff = static_cast<long long>(h.b) * p.sb + static_cast<long long>(h.i) * p.sg + h.x0;
       } else {
         const int g = h.i / (p.k + 1), pos = h.i % (p.k + 1);
@@ -1258,7 +1259,12 @@ __device__ void argmax_producer(const ArgmaxParams& p, Shared& sh, unsigned char
   }
 }
 
-template <typename TT, bool kTma>
+// Argmax kernel modes, one instantiation each so that every kernel carries
+// only its own finalize: plain (greedy and multi-candidate), rows form, tree,
+// threshold acceptance (row softmax statistics as well).
+enum : int { kArgPlain = 0, kArgRows = 1, kArgTree = 2, kArgThreshold = 3 };
+
+template <typename TT, bool kTma, int kMode>
 __device__ void argmax_compute(const ArgmaxParams& p, Shared& sh, unsigned char* stages, int w,
                                int lane) {
   const int group = w / kGroupWarps;
@@ -1275,7 +1281,7 @@ __device__ void argmax_compute(const ArgmaxParams& p, Shared& sh, unsigned char*
     float bv;
     int bi;
     float4 r = make_float4(0.0f, 0.0f, -INFINITY, 0.0f);
-    if (p.sslots && h.i < p.k) {  // threshold acceptance: row statistics too
+    if (kMode == kArgThreshold && h.i < p.k) {  // row statistics too
       if (kTma) {
         r = chunk_argmax_stats_regs<TT>(stages + static_cast<size_t>(s) * kStageBytes, h, p.tgt,
                                         p.c2, tid, sh, s, lane);
@@ -1518,6 +1524,7 @@ __device__ void finalize_argmax(const ArgmaxParams& p, int b, int lane) {
 
 // Row merge (one warp, one lane per chunk): the row's argmax key is the
 // largest chunk key; count the row, and the last row finalizes.
+template <int kMode>
 __device__ void merge_argmax_row(const ArgmaxParams& p, int b, int r, int lane) {
   const unsigned int R = static_cast<unsigned int>(p.R);
   unsigned long long* slot = p.slots + (static_cast<size_t>(b) * R + r) * p.nch;
@@ -1527,7 +1534,7 @@ __device__ void merge_argmax_row(const ArgmaxParams& p, int b, int r, int lane) 
     key = v > key ? v : key;
   }
   key = warp_max_u64(key);
-  const bool with_stats = p.sslots && r < p.k;
+  const bool with_stats = kMode == kArgThreshold && r < p.k;
   float M = -INFINITY, S = 0.0f;
   if (with_stats) {
     unsigned long long* ss = p.sslots + (static_cast<size_t>(b) * R + r) * p.nch;
@@ -1548,17 +1555,18 @@ __device__ void merge_argmax_row(const ArgmaxParams& p, int b, int r, int lane) 
     old = atomicAdd(&p.seq[b].cnt1, 1u);
   }
   if (__shfl_sync(0xffffffffu, old == R - 1u ? 1 : 0, 0)) {
-    if (p.sslots)
+    if constexpr (kMode == kArgThreshold)
       finalize_threshold(p, b, lane);
-    else if (p.parent)
+    else if constexpr (kMode == kArgTree)
       finalize_argmax_tree(p, b, lane);
-    else if (p.row_of)
+    else if constexpr (kMode == kArgRows)
       finalize_argmax_rows(p, b, lane);
     else
       finalize_argmax(p, b, lane);
   }
 }
 
+template <int kMode>
 __device__ void argmax_epilogue(const ArgmaxParams& p, Shared& sh, int group, int lane) {
   const unsigned int R = static_cast<unsigned int>(p.R);
   const unsigned int last = static_cast<unsigned int>(p.nch) - 1u;
@@ -1569,7 +1577,7 @@ __device__ void argmax_epilogue(const ArgmaxParams& p, Shared& sh, int group, in
     const uint32_t parity = (use / kStages) & 1u;
     if (pend_b >= 0 && !mbar_try_wait(&sh.rfull[s], parity)) {
       if (__shfl_sync(0xffffffffu, pend_old == last ? 1 : 0, 0))
-        merge_argmax_row(p, pend_b, pend_r, lane);
+        merge_argmax_row<kMode>(p, pend_b, pend_r, lane);
       pend_b = -1;
     }
     if (!mbar_wait(&sh.rfull[s], parity, p.ctrl)) break;
@@ -1588,7 +1596,7 @@ __device__ void argmax_epilogue(const ArgmaxParams& p, Shared& sh, int group, in
     __syncwarp();
     if (lane == 0) mbar_arrive(&sh.empty[s]);
     warp_argmax(v, i);
-    const bool with_stats = p.sslots && h.i < p.k;
+    const bool with_stats = kMode == kArgThreshold && h.i < p.k;
     if (with_stats) st = warp_stats2(st);
     unsigned int old = 0u;
     if (lane == 0) {
@@ -1598,16 +1606,16 @@ __device__ void argmax_epilogue(const ArgmaxParams& p, Shared& sh, int group, in
       old = atomicAdd(&p.rc[static_cast<size_t>(h.b) * R + h.i], 1u);
     }
     if (pend_b >= 0 && __shfl_sync(0xffffffffu, pend_old == last ? 1 : 0, 0))
-      merge_argmax_row(p, pend_b, pend_r, lane);
+      merge_argmax_row<kMode>(p, pend_b, pend_r, lane);
     pend_b = h.b;
     pend_r = h.i;
     pend_old = old;
   }
   if (pend_b >= 0 && __shfl_sync(0xffffffffu, pend_old == last ? 1 : 0, 0))
-    merge_argmax_row(p, pend_b, pend_r, lane);
+    merge_argmax_row<kMode>(p, pend_b, pend_r, lane);
 }
 
-template <typename TT, bool kTma>
+template <typename TT, bool kTma, int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
     argmax_verify_kernel(const __grid_constant__ ArgmaxParams p) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
@@ -1624,11 +1632,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   __syncthreads();
   if (warp == 0) {
-    if (lane == 0) argmax_producer<TT, kTma>(p, sh, stages);
+    if (lane == 0) argmax_producer<TT, kTma, kMode == kArgRows || kMode == kArgTree>(p, sh, stages);
   } else if (warp <= kComputeWarps) {
-    argmax_compute<TT, kTma>(p, sh, stages, warp - 1, lane);
+    argmax_compute<TT, kTma, kMode>(p, sh, stages, warp - 1, lane);
   } else {
-    argmax_epilogue(p, sh, warp - 1 - kComputeWarps, lane);
+    argmax_epilogue<kMode>(p, sh, warp - 1 - kComputeWarps, lane);
   }
 }
 
@@ -1716,23 +1724,40 @@ cudaError_t launch_stochastic(const StochParams& p, int t_dtype, int d_dtype, bo
   return launch_stoch_tma<float, float>(p, tma, grid, smem, st);
 }
 
-template <typename TT, bool kTma>
+template <typename TT, bool kTma, int kMode>
 static cudaError_t launch_argmax_t(const ArgmaxParams& p, int grid, size_t smem, cudaStream_t st) {
   static bool done[64] = {};
-  auto kernel = argmax_verify_kernel<TT, kTma>;
+  auto kernel = argmax_verify_kernel<TT, kTma, kMode>;
   cudaError_t e = prepare(kernel, smem, done);
   if (e != cudaSuccess) return e;
   kernel<<<grid, kThreads, smem, st>>>(p);
   return cudaGetLastError();
 }
 
+template <typename TT>
+static cudaError_t launch_argmax_mode(const ArgmaxParams& p, int mode, bool tma, int grid,
+                                      size_t smem, cudaStream_t st) {
+  switch (mode) {
+    case kArgRows:
+      return tma ? launch_argmax_t<TT, true, kArgRows>(p, grid, smem, st)
+                 : launch_argmax_t<TT, false, kArgRows>(p, grid, smem, st);
+    case kArgTree:
+      return tma ? launch_argmax_t<TT, true, kArgTree>(p, grid, smem, st)
+                 : launch_argmax_t<TT, false, kArgTree>(p, grid, smem, st);
+    case kArgThreshold:
+      return tma ? launch_argmax_t<TT, true, kArgThreshold>(p, grid, smem, st)
+                 : launch_argmax_t<TT, false, kArgThreshold>(p, grid, smem, st);
+    default:
+      return tma ? launch_argmax_t<TT, true, kArgPlain>(p, grid, smem, st)
+                 : launch_argmax_t<TT, false, kArgPlain>(p, grid, smem, st);
+  }
+}
+
 cudaError_t launch_argmax(const ArgmaxParams& p, int t_dtype, bool tma, int grid, size_t smem,
                           cudaStream_t st) {
-  if (t_dtype == 1)
-    return tma ? launch_argmax_t<uint16_t, true>(p, grid, smem, st)
-               : launch_argmax_t<uint16_t, false>(p, grid, smem, st);
-  return tma ? launch_argmax_t<float, true>(p, grid, smem, st)
-             : launch_argmax_t<float, false>(p, grid, smem, st);
+  const int mode = p.sslots ? kArgThreshold : p.parent ? kArgTree : p.row_of ? kArgRows : kArgPlain;
+  return t_dtype == 1 ? launch_argmax_mode<uint16_t>(p, mode, tma, grid, smem, st)
+                      : launch_argmax_mode<float>(p, mode, tma, grid, smem, st);
 }
 
 cudaError_t launch_commit(const int* accepted_len, const int* out_tokens, int B, int k,
