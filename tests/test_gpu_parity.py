@@ -589,6 +589,37 @@ def test_one_workspace_across_modes_and_sizes(dev):
     assert ws.device_status() == 0
 
 
+# --------------------------------------------- bounded waits (no GPU fault)
+
+def test_device_wait_runs_out_and_the_workspace_recovers(dev):
+    """A sequence record whose row counter can never reach its target makes
+    the sequence's phase-1 finalize never fire, so its phase-2 chunks wait for
+    a ready flag that nothing sets; that wait gives up after its bounded limit
+    (about 2 s), every other wait sees the abort, the kernel returns, the
+    status word reports SV_FLAG_TIMEOUT, and a re-initialised workspace works
+    again."""
+    w = workloads.make_stochastic(4, 3, 5000, "bf16", "f32", seed=3)
+    t, d = to_dev(w["target"], "bf16", dev), to_dev(w["draft"], "f32", dev)
+    tok = torch.from_numpy(w["tokens"]).to(dev)
+    call = lambda ws: sv.stochastic(t, d, tok, w["temperature"], 5, workspace=ws)
+    size = sv.workspace_size(4, 1, 3, 5000)
+    ws = sv.Workspace(dev)
+    ws.ensure(size)
+    # sequence 0's row counter (first word of its 64-byte record after the
+    # 256 control bytes) starts far from any count the kernel can reach
+    ws.buf[256:260] = torch.tensor([0xff, 0xff, 0xff, 0x3f], dtype=torch.uint8, device=dev)
+    call(ws)
+    flags = ws.device_status(clear=True)
+    assert flags & sv.SV_FLAG_TIMEOUT, flags
+    ws.reset()
+    r = call(ws)
+    torch.cuda.synchronize()
+    assert ws.device_status() == 0
+    o = oracle.verify_stochastic(w["target"], "bf16", w["draft"], "f32", w["tokens"],
+                                 w["temperature"], 5)
+    compare_stochastic(r, o, w["k"], "after recovery")
+
+
 # ------------------------------------------------------- named workloads
 
 @pytest.mark.parametrize("name", list(workloads.WORKLOADS))
