@@ -261,6 +261,8 @@ extern "C" int spec_verify_stochastic(const void* target_logits, int t_dtype,
   p.nch = pl.nch;
   p.lag = static_cast<int>(lag);
   p.slot_items = static_cast<unsigned int>(slot_items);
+  p.div_slot = make_udiv(p.slot_items);
+  p.div_nch = make_udiv(static_cast<unsigned int>(pl.nch));
   p.total = static_cast<unsigned int>(total);
   p.ctrl = ws.ctrl;
   p.seq = ws.seq;
@@ -334,6 +336,8 @@ static int argmax_call(const void* target_logits, int t_dtype, int64_t sb, int64
   p.out_tokens = out_tokens;
   p.ch = pl.ch;
   p.nch = pl.nch;
+  p.div_seq = make_udiv(static_cast<unsigned int>(rows_per_seq) * static_cast<unsigned int>(pl.nch));
+  p.div_nch = make_udiv(static_cast<unsigned int>(pl.nch));
   p.total = static_cast<unsigned int>(total);
   p.ctrl = ws.ctrl;
   p.seq = ws.seq;

@@ -82,6 +82,23 @@ Plan plan_chunks(long long rows, int V, int bpe, int es_min, int chunk_bytes);
 constexpr int kStochChunkBytes = kStageBytes;
 constexpr int kArgmaxChunkBytes = 40 * 1024;
 
+// Division of 31-bit values by a divisor fixed per call, as a multiply-high
+// and a shift (Granlund and Montgomery, "Division by invariant integers using
+// multiplication", PLDI 1994): with l = ceil(log2 d) and m = ceil(2^(31+l)/d),
+// floor(n/d) = floor(n m / 2^(31+l)) for 0 <= n < 2^31, and m < 2^32.
+struct UDiv {
+  unsigned int d, m, shift;  // d == 1: m == 0, the quotient is n
+};
+inline UDiv make_udiv(unsigned int d) {
+  UDiv u{d, 0u, 0u};
+  if (d <= 1u) return u;
+  unsigned int l = 0;
+  while ((1ull << l) < d) ++l;
+  u.m = static_cast<unsigned int>(((1ull << (31 + l)) + d - 1) / d);
+  u.shift = l - 1;  // 31 + l - 32
+  return u;
+}
+
 struct StochParams {
   const void* tgt;
   long long t_sb, t_sp;
@@ -96,6 +113,7 @@ struct StochParams {
   float* probs;  // nullable
   int ch, nch, lag;
   unsigned int slot_items;  // (k + 1) * nch tickets per slot
+  UDiv div_slot, div_nch;   // ticket decode: / slot_items, / nch
   unsigned int total;       // tickets
   Ctrl* ctrl;
   SeqRec* seq;
@@ -128,6 +146,7 @@ struct ArgmaxParams {
   int* accepted_len;
   int* out_tokens;
   int ch, nch;
+  UDiv div_seq, div_nch;  // ticket decode: / (R * nch), / nch
   unsigned int total;
   Ctrl* ctrl;
   SeqRec* seq;

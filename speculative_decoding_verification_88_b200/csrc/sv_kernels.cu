@@ -183,6 +183,10 @@ __device__ void drain_stages(Shared& sh, uint32_t uses) {
   }
 }
 
+__device__ __forceinline__ unsigned int udiv(unsigned int n, const UDiv& u) {
+  return u.m ? __umulhi(n, u.m) >> u.shift : n;
+}
+
 __device__ __forceinline__ void leave_grid(Ctrl* ctrl) {
   // The last CTA to take its final ticket rewinds the ticket counter.
   if (atomicAdd(&ctrl->exits, 1u) == gridDim.x - 1) {
@@ -862,10 +866,10 @@ __device__ void stoch_producer(const StochParams& p, Shared& sh, unsigned char* 
     }
     const unsigned int t = base + j;
     if (j == 0u) {
-      slot = t / p.slot_items;
-      o = t % p.slot_items;
-      ci = o < p1_items ? o / nch : 0u;
-      cc = o < p1_items ? o % nch : 0u;
+      slot = udiv(t, p.div_slot);
+      o = t - slot * p.slot_items;
+      ci = o < p1_items ? udiv(o, p.div_nch) : 0u;
+      cc = o < p1_items ? o - ci * nch : 0u;
     } else if (++o == p.slot_items) {
       o = 0u;
       ++slot;
@@ -1226,10 +1230,12 @@ __device__ void argmax_producer(const ArgmaxParams& p, Shared& sh, unsigned char
       if (t >= p.total) break;
       Hdr h;
       h.kind = kKindArgmax;
-      h.b = static_cast<int>(t / per_seq);
-      const unsigned int rem = t % per_seq;
-      h.i = static_cast<int>(rem / p.nch);
-      h.c = static_cast<int>(rem % p.nch);
+      const unsigned int b = udiv(t, p.div_seq);
+      const unsigned int rem = t - b * per_seq;
+      const unsigned int i = udiv(rem, p.div_nch);
+      h.b = static_cast<int>(b);
+      h.i = static_cast<int>(i);
+      h.c = static_cast<int>(rem - i * static_cast<unsigned int>(p.nch));
       h.x0 = h.c * p.ch;
       h.len = min(p.ch, p.V - h.x0);
       if (kRowStride) {
