@@ -220,13 +220,14 @@ extern "C" int spec_verify_stochastic(const void* target_logits, int t_dtype,
   const long long p1 = static_cast<long long>(k) * pl.nch;
   long long lag = 0;
   if (p1 > 0) {
-    // phase-2 chunks of a sequence come about 6 ring-fulls of the whole grid
+    // phase-2 chunks of a sequence come about 12 ring-fulls of the whole grid
     // after its phase-1 chunks: late enough that the sequence is nearly
-    // always finalized (a producer that has to wait for it stalls its whole
-    // CTA), early enough that row n is often still in L2.  Measured on
-    // B = 256, k = 8, V = 128256 (ring-fulls -> us): 1.5 -> 265, 3 -> 253,
-    // 6 -> 244, 12 -> 251, 24 -> 272, all of phase 1 first -> 295.
-    lag = (static_cast<long long>(6 * kStages) * grid + p1 - 1) / p1 + 1;
+    // always finalized (a producer that has to wait for it stalls its compute
+    // group), early enough that row n is often still in L2.  Measured on
+    // B = 256, k = 8, V = 128256 with one producer per compute group
+    // (ring-fulls -> us): 3 -> 205, 6 -> 201, 12 -> 197, 16 -> 199,
+    // 24 -> 204, all of phase 1 first -> 208.
+    lag = (static_cast<long long>(12 * kStages) * grid + p1 - 1) / p1 + 1;
     if (lag > B) lag = B;
   }
   const long long slot_items = static_cast<long long>(k + 1) * pl.nch;

@@ -9,10 +9,11 @@
 namespace sv {
 
 // ---- CTA shape of the persistent verify kernels -------------------------
-// warp 0: producer (one thread: ticket, waits, bulk copies)
-// warps 1..kComputeWarps: compute (reduce one chunk held in shared memory)
+// warps 0..kProducerWarps-1: producers (one thread each: tickets, waits, bulk
+//   copies), one per compute group in the stochastic kernel
+// next kComputeWarps warps: compute (reduce one chunk held in shared memory)
 // last kComputeGroups warps: epilogues, one per compute group (publish chunk
-// partials, merge rows, finalize sequences)
+//   partials, merge rows, finalize sequences)
 #ifndef SV_COMPUTE_WARPS
 #define SV_COMPUTE_WARPS 16
 #endif
@@ -22,7 +23,9 @@ constexpr int kComputeWarps = SV_COMPUTE_WARPS;
 // each group has its own epilogue warp.
 constexpr int kComputeGroups = 2;
 constexpr int kGroupWarps = kComputeWarps / kComputeGroups;
-constexpr int kThreads = 32 * (1 + kComputeWarps + kComputeGroups);
+// One producer warp per compute group (the argmax kernel uses the first).
+constexpr int kProducerWarps = kComputeGroups;
+constexpr int kThreads = 32 * (kProducerWarps + kComputeWarps + kComputeGroups);
 constexpr int kComputeThreads = kGroupWarps * 32;  // threads that share one chunk
 constexpr int kStages = 4;
 constexpr int kStageBytes = 56 * 1024;

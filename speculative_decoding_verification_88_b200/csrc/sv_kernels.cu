@@ -4,14 +4,18 @@
 // chunk of one row (or row pair): the vocabulary of every row is split into
 // `nch` chunks, so each (sequence, position) row is reduced by many CTAs.
 //
-//   warp 0, lane 0   producer: takes tickets (atomicAdd, two at a time, one
-//                    grab ahead) and streams each chunk into a 4-stage shared-
+//   warps 0, 1       producers (lane 0): take tickets (atomicAdd, one grab
+//                    ahead) and stream each chunk into a 4-stage shared-
 //                    memory ring with 1-D bulk copies (TMA, cp.async.bulk)
-//                    that complete on an mbarrier.  A chunk whose sequence is
-//                    not ready yet (phase 2 below) is set aside in a short
-//                    queue and issued once it is, so the ring keeps flowing.
-//   warps 1..16      compute: reduce the chunk held in shared memory (softmax
-//                    statistics, Gumbel-max, or argmax) to one record per warp.
+//                    that complete on an mbarrier.  In the stochastic kernel
+//                    each producer feeds its own compute group's two stages;
+//                    the argmax kernels use warp 0 alone, alternating groups.
+//                    A chunk whose sequence is not ready yet (phase 2 below)
+//                    is set aside in a short queue and issued once it is, so
+//                    the ring keeps flowing.
+//   warps 2..17      compute, two groups of 8: reduce the chunk held in shared
+//                    memory (softmax statistics, Gumbel-max, or argmax) to one
+//                    record per warp.
 //   last 2 warps     epilogues, one per compute group: merge the warp records, publish the
 //                    chunk's partial with one 64-bit store and counts it with
 //                    a relaxed atomicAdd on its row's counter.  A published
@@ -187,9 +191,9 @@ __device__ __forceinline__ unsigned int udiv(unsigned int n, const UDiv& u) {
   return u.m ? __umulhi(n, u.m) >> u.shift : n;
 }
 
-__device__ __forceinline__ void leave_grid(Ctrl* ctrl) {
-  // The last CTA to take its final ticket rewinds the ticket counter.
-  if (atomicAdd(&ctrl->exits, 1u) == gridDim.x - 1) {
+__device__ __forceinline__ void leave_grid(Ctrl* ctrl, unsigned int producers_per_cta) {
+  // The last producer to take its final ticket rewinds the ticket counter.
+  if (atomicAdd(&ctrl->exits, 1u) == gridDim.x * producers_per_cta - 1) {
     atomicExch(&ctrl->ticket, 0u);
     atomicExch(&ctrl->exits, 0u);
   }
@@ -222,11 +226,10 @@ __device__ __forceinline__ void issue_chunk(Shared& sh, unsigned char* stage, in
 }
 
 // --- per-group rings (stochastic kernel) -----------------------------------
-// Compute group g owns stages g and g + 2; its j-th use is stage
-// g + 2 (j % 2), phase (j / 2) & 1 -- the order in which its compute warps and
-// its epilogue warp walk them.  The producer keeps one use counter per group
-// and gives each chunk to whichever group frees a stage first, so a group
-// busy with a long chunk does not hold the other back.
+// Compute group g owns stages g and g + 2 and has its own producer; its j-th
+// use is stage g + 2 (j % 2), phase (j / 2) & 1 -- the order in which its
+// producer, compute warps and epilogue warp walk them.  Each group is its own
+// pipeline, so a group busy with a long chunk does not hold the other back.
 constexpr int kGroupStages = kStages / kComputeGroups;
 static_assert(kGroupStages * kComputeGroups == kStages, "stages split evenly over groups");
 
@@ -235,48 +238,22 @@ __device__ __forceinline__ int group_stage(int g, uint32_t j) {
 }
 __device__ __forceinline__ uint32_t group_phase(uint32_t j) { return (j / kGroupStages) & 1u; }
 
-// Waits (bounded) until some group's next stage is free; returns that group,
-// trying `pref` first, or -1 on abort or timeout.
-__device__ int take_group_stage(Shared& sh, const uint32_t (&used)[kComputeGroups], int pref,
-                                Ctrl* ctrl) {
-  const unsigned long long t0 = global_ns();
-  for (unsigned int spin = 0;; ++spin) {
-#pragma unroll
-    for (int q = 0; q < kComputeGroups; ++q) {
-      const int g = (pref + q) % kComputeGroups;
-      if (mbar_test_wait(&sh.empty[group_stage(g, used[g])], group_phase(used[g]) ^ 1u)) return g;
-    }
-    if ((spin & 255u) == 255u) {
-      if (aborted(ctrl)) return -1;
-      if (global_ns() - t0 > kWaitLimitNs) {
-        atomicOr(&ctrl->flags, kFlagTimeout);
-        return -1;
-      }
-    }
-  }
+// One end marker into group g's next stage.
+__device__ __forceinline__ void push_group_end(Shared& sh, int g, uint32_t used, Ctrl* ctrl) {
+  const int s = group_stage(g, used);
+  if (!mbar_wait(&sh.empty[s], group_phase(used) ^ 1u, ctrl)) return;
+  sh.hdr[s].kind = kKindEnd;
+  mbar_arrive(&sh.full[s]);
 }
 
-// One end marker into each group's next stage.
-__device__ __forceinline__ void push_group_ends(Shared& sh, const uint32_t (&used)[kComputeGroups],
-                                                Ctrl* ctrl) {
-  for (int g = 0; g < kComputeGroups; ++g) {
-    const int s = group_stage(g, used[g]);
-    if (!mbar_wait(&sh.empty[s], group_phase(used[g]) ^ 1u, ctrl)) return;
-    sh.hdr[s].kind = kKindEnd;
-    mbar_arrive(&sh.full[s]);
-  }
-}
-
-// After an abort: wait (bounded) until the last bulk copy issued into each
-// group's stages has landed.
-__device__ void drain_group_stages(Shared& sh, const uint32_t (&used)[kComputeGroups]) {
-  for (int g = 0; g < kComputeGroups; ++g) {
-    for (uint32_t r = 0; r < static_cast<uint32_t>(kGroupStages) && r < used[g]; ++r) {
-      const uint32_t last = r + ((used[g] - 1 - r) / kGroupStages) * kGroupStages;
-      const unsigned long long t0 = global_ns();
-      while (!mbar_try_wait(&sh.full[group_stage(g, r)], group_phase(last))) {
-        if (global_ns() - t0 > 100000000ull) break;
-      }
+// After an abort: wait (bounded) until the last bulk copy issued into each of
+// group g's stages has landed.
+__device__ void drain_group_stages(Shared& sh, int g, uint32_t used) {
+  for (uint32_t r = 0; r < static_cast<uint32_t>(kGroupStages) && r < used; ++r) {
+    const uint32_t last = r + ((used - 1 - r) / kGroupStages) * kGroupStages;
+    const unsigned long long t0 = global_ns();
+    while (!mbar_try_wait(&sh.full[group_stage(g, r)], group_phase(last))) {
+      if (global_ns() - t0 > 100000000ull) break;
     }
   }
 }
@@ -761,20 +738,17 @@ __device__ __forceinline__ void chunk_argmax(const unsigned char* smem, const Hd
 // Place a chunk in the next ring stage (waits for the stage to be free).
 template <typename TT, typename TD, bool kTma>
 __device__ __forceinline__ bool stoch_issue(const StochParams& p, Shared& sh,
-                                            unsigned char* stages,
-                                            uint32_t (&used)[kComputeGroups], int& pref, Hdr& h,
-                                            const float4* stat) {
+                                            unsigned char* stages, int g, uint32_t& used,
+                                            Hdr& h, const float4* stat) {
   h.x0 = h.c * p.ch;
   h.len = min(p.ch, p.V - h.x0);
   h.toff = static_cast<long long>(h.b) * p.t_sb + static_cast<long long>(h.i) * p.t_sp + h.x0;
   h.doff = static_cast<long long>(h.b) * p.d_sb + static_cast<long long>(h.i) * p.d_sp + h.x0;
-  const int g = take_group_stage(sh, used, pref, p.ctrl);
-  if (g < 0) return false;
-  const int s = group_stage(g, used[g]);
+  const int s = group_stage(g, used);
+  if (!mbar_wait(&sh.empty[s], group_phase(used) ^ 1u, p.ctrl)) return false;
   issue_chunk<TT, TD, kTma>(sh, stages + static_cast<size_t>(s) * kStageBytes, s, h, p.tgt,
                             p.drf, p.ch, h.kind != kKindBonus, stat);
-  ++used[g];
-  pref = (g + 1) % kComputeGroups;  // alternate while both have room
+  ++used;
   return true;
 }
 
@@ -783,9 +757,9 @@ __device__ __forceinline__ bool stoch_issue(const StochParams& p, Shared& sh,
 // statistics travel with the chunk as a 16-byte bulk copy.
 template <typename TT, typename TD, bool kTma>
 __device__ __forceinline__ bool stoch_issue_phase2(const StochParams& p, Shared& sh,
-                                                   unsigned char* stages,
-                                                   uint32_t (&used)[kComputeGroups], int& pref,
-                                                   int b, int c, unsigned int ready) {
+                                                   unsigned char* stages, int g,
+                                                   uint32_t& used, int b, int c,
+                                                   unsigned int ready) {
   Hdr h;
   h.b = b;
   h.c = c;
@@ -800,24 +774,24 @@ __device__ __forceinline__ bool stoch_issue_phase2(const StochParams& p, Shared&
   } else {
     h.kind = kKindBonus;
   }
-  return stoch_issue<TT, TD, kTma>(p, sh, stages, used, pref, h, stat);
+  return stoch_issue<TT, TD, kTma>(p, sh, stages, g, used, h, stat);
 }
 
-// The producer takes tickets kGrabStoch at a time (the next grab's atomic in
-// flight meanwhile) and decodes them incrementally: ticket t is slot
+// Producer of compute group g.  It takes tickets kGrabStoch at a time (the
+// next grab's atomic in flight meanwhile) and decodes them incrementally:
+// ticket t is slot
 // t / slot_items, offset o = t % slot_items; offsets below k * nch are
 // phase-1 chunks (i, c) = (o / nch, o % nch) of sequence `slot`, the rest
 // phase-2 chunks of sequence slot - lag.  A phase-2 chunk whose sequence is
 // not ready yet is set aside (at most kDefer); set-aside chunks are polled
 // together with relaxed loads and issued once ready.
 template <typename TT, typename TD, bool kTma>
-__device__ void stoch_producer(const StochParams& p, Shared& sh, unsigned char* stages) {
+__device__ void stoch_producer(const StochParams& p, Shared& sh, unsigned char* stages, int g) {
   constexpr int kDefer = 4;
   Ctrl* ctrl = p.ctrl;
   const unsigned int nch = static_cast<unsigned int>(p.nch);
   const unsigned int p1_items = static_cast<unsigned int>(p.k) * nch;
-  uint32_t used[kComputeGroups] = {};  // uses issued per group
-  int pref = 0;
+  uint32_t used = 0;  // uses of group g's stages issued
   bool ok = true;
   int db[kDefer], dc[kDefer];  // set-aside phase-2 chunks, oldest first
   int nd = 0;
@@ -840,7 +814,7 @@ __device__ void stoch_producer(const StochParams& p, Shared& sh, unsigned char* 
         for (int d = 0; d < kDefer; ++d) {
           if (d < nd) {
             if (ok && rd[d]) {
-              ok = stoch_issue_phase2<TT, TD, kTma>(p, sh, stages, used, pref, db[d], dc[d], rd[d]);
+              ok = stoch_issue_phase2<TT, TD, kTma>(p, sh, stages, g, used, db[d], dc[d], rd[d]);
             } else {
               db[keep] = db[d];
               dc[keep] = dc[d];
@@ -892,7 +866,7 @@ __device__ void stoch_producer(const StochParams& p, Shared& sh, unsigned char* 
       h.b = static_cast<int>(slot);
       h.i = static_cast<int>(ci);
       h.c = static_cast<int>(cc);
-      ok = stoch_issue<TT, TD, kTma>(p, sh, stages, used, pref, h, nullptr);
+      ok = stoch_issue<TT, TD, kTma>(p, sh, stages, g, used, h, nullptr);
     } else {
       const int b = static_cast<int>(slot) - p.lag;
       if (b < 0 || b >= p.B) continue;
@@ -900,7 +874,7 @@ __device__ void stoch_producer(const StochParams& p, Shared& sh, unsigned char* 
       const unsigned int rd = p.k == 0 ? 1u : ld_relaxed_u32(&p.seq[b].ready);
       if (rd) {
         if (p.k > 0) fence_acq_rel_gpu();
-        ok = stoch_issue_phase2<TT, TD, kTma>(p, sh, stages, used, pref, b, c, rd);
+        ok = stoch_issue_phase2<TT, TD, kTma>(p, sh, stages, g, used, b, c, rd);
       } else {
         if (nd == kDefer) {  // queue full: the oldest must go first
           const unsigned int r0 = wait_flag(&p.seq[db[0]].ready, ctrl);
@@ -908,7 +882,7 @@ __device__ void stoch_producer(const StochParams& p, Shared& sh, unsigned char* 
             ok = false;
             break;
           }
-          ok = stoch_issue_phase2<TT, TD, kTma>(p, sh, stages, used, pref, db[0], dc[0], r0);
+          ok = stoch_issue_phase2<TT, TD, kTma>(p, sh, stages, g, used, db[0], dc[0], r0);
 #pragma unroll
           for (int d = 1; d < kDefer; ++d) {
             db[d - 1] = db[d];
@@ -923,10 +897,10 @@ __device__ void stoch_producer(const StochParams& p, Shared& sh, unsigned char* 
     }
   }
   if (ok) {
-    push_group_ends(sh, used, ctrl);
-    leave_grid(ctrl);
+    push_group_end(sh, g, used, ctrl);
+    leave_grid(ctrl, kProducerWarps);
   } else if (kTma) {
-    drain_group_stages(sh, used);
+    drain_group_stages(sh, g, used);
   }
 }
 
@@ -1204,12 +1178,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_fence_init();
   }
   __syncthreads();
-  if (warp == 0) {
-    if (lane == 0) stoch_producer<TT, TD, kTma>(p, sh, stages);
-  } else if (warp <= kComputeWarps) {
-    stoch_compute<TT, TD, kTma>(p, sh, stages, warp - 1, lane);
+  if (warp < kProducerWarps) {
+    if (lane == 0) stoch_producer<TT, TD, kTma>(p, sh, stages, warp);
+  } else if (warp < kProducerWarps + kComputeWarps) {
+    stoch_compute<TT, TD, kTma>(p, sh, stages, warp - kProducerWarps, lane);
   } else {
-    stoch_epilogue<TT, TD>(p, sh, warp - 1 - kComputeWarps, lane);
+    stoch_epilogue<TT, TD>(p, sh, warp - kProducerWarps - kComputeWarps, lane);
   }
 }
 
@@ -1259,7 +1233,7 @@ __device__ void argmax_producer(const ArgmaxParams& p, Shared& sh, unsigned char
   }
   if (ok) {
     push_end(sh, use, ctrl);
-    leave_grid(ctrl);
+    leave_grid(ctrl, 1u);
   } else if (kTma) {
     drain_stages(sh, use);
   }
@@ -1637,12 +1611,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_fence_init();
   }
   __syncthreads();
-  if (warp == 0) {
-    if (lane == 0) argmax_producer<TT, kTma, kMode == kArgRows || kMode == kArgTree>(p, sh, stages);
-  } else if (warp <= kComputeWarps) {
-    argmax_compute<TT, kTma, kMode>(p, sh, stages, warp - 1, lane);
+  if (warp < kProducerWarps) {  // one producer: it alternates the groups' stages
+    if (warp == 0 && lane == 0)
+      argmax_producer<TT, kTma, kMode == kArgRows || kMode == kArgTree>(p, sh, stages);
+  } else if (warp < kProducerWarps + kComputeWarps) {
+    argmax_compute<TT, kTma, kMode>(p, sh, stages, warp - kProducerWarps, lane);
   } else {
-    argmax_epilogue<kMode>(p, sh, warp - 1 - kComputeWarps, lane);
+    argmax_epilogue<kMode>(p, sh, warp - kProducerWarps - kComputeWarps, lane);
   }
 }
 
