@@ -220,18 +220,17 @@ extern "C" int spec_verify_stochastic(const void* target_logits, int t_dtype,
   const long long p1 = static_cast<long long>(k) * pl.nch;
   long long lag = 0;
   if (p1 > 0) {
-    // phase-2 chunks of a sequence come about 12 ring-fulls of the whole grid
+    // phase-2 chunks of a sequence come about 24 ring-fulls of the whole grid
     // after its phase-1 chunks: late enough that the sequence is nearly
     // always finalized (a producer that has to wait for it stalls its compute
-    // group), early enough that row n is often still in L2.  Measured on
-    // B = 256, k = 8, V = 128256 with one producer per compute group
-    // (ring-fulls -> us): 3 -> 205, 6 -> 201, 12 -> 197, 16 -> 199,
-    // 24 -> 204, all of phase 1 first -> 208.
-    lag = (static_cast<long long>(12 * kStages) * grid + p1 - 1) / p1 + 1;
+    // group).  Measured on B = 256, k = 8, V = 128256 (ring-fulls -> us):
+    // 6 -> 199.4, 12 -> 194.8, 24 -> 192.4, all of phase 1 first -> 193.3;
+    // at B = 64 every choice is within 1 %.
+    lag = (static_cast<long long>(24 * kStages) * grid + p1 - 1) / p1 + 1;
     if (lag > B) lag = B;
   }
   const long long slot_items = static_cast<long long>(k + 1) * pl.nch;
-  const long long total = (static_cast<long long>(B) + lag) * slot_items;
+  const long long total = static_cast<long long>(B) * slot_items;
   if (total >= (1ll << 31)) return SV_ERR_INVALID_ARG;
 
   const bool tma = aligned(target_logits, 16) && stride16(t_stride_b, st) &&
@@ -261,10 +260,14 @@ extern "C" int spec_verify_stochastic(const void* target_logits, int t_dtype,
   p.ch = pl.ch;
   p.nch = pl.nch;
   p.lag = static_cast<int>(lag);
+  p.p1_items = static_cast<unsigned int>(p1);
   p.slot_items = static_cast<unsigned int>(slot_items);
+  p.a_end = static_cast<unsigned int>(lag * p1);
+  p.b_end = p.a_end + static_cast<unsigned int>((B - lag) * slot_items);
+  p.total = static_cast<unsigned int>(total);
+  p.div_p1 = make_udiv(p1 > 0 ? p.p1_items : 1u);
   p.div_slot = make_udiv(p.slot_items);
   p.div_nch = make_udiv(static_cast<unsigned int>(pl.nch));
-  p.total = static_cast<unsigned int>(total);
   p.ctrl = ws.ctrl;
   p.seq = ws.seq;
   const StochLayout lay = stochastic_layout(B, k, pl.nch);

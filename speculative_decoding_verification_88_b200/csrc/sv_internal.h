@@ -115,9 +115,15 @@ struct StochParams {
   int* out_tokens;
   float* probs;  // nullable
   int ch, nch, lag;
-  unsigned int slot_items;  // (k + 1) * nch tickets per slot
-  UDiv div_slot, div_nch;   // ticket decode: / slot_items, / nch
-  unsigned int total;       // tickets
+  // Ticket map, three runs with no unused ticket: [0, a_end) phase-1 chunks
+  // of sequences 0..lag-1 (k * nch each); [a_end, b_end) slots of
+  // slot_items = (k + 1) * nch tickets, slot s >= lag holding the phase-1
+  // chunks of sequence s and then the phase-2 chunks of sequence s - lag;
+  // [b_end, total) phase-2 chunks of sequences B-lag..B-1 (nch each).
+  unsigned int p1_items;    // k * nch
+  unsigned int slot_items;  // (k + 1) * nch
+  unsigned int a_end, b_end, total;
+  UDiv div_p1, div_slot, div_nch;  // ticket decode: / p1_items, / slot_items, / nch
   Ctrl* ctrl;
   SeqRec* seq;
   // Partials, published with one 64-bit store each and never zero once

@@ -778,26 +778,23 @@ __device__ __forceinline__ bool stoch_issue_phase2(const StochParams& p, Shared&
 }
 
 // Producer of compute group g.  It takes tickets kGrabStoch at a time (the
-// next grab's atomic in flight meanwhile) and decodes them incrementally:
-// ticket t is slot
-// t / slot_items, offset o = t % slot_items; offsets below k * nch are
-// phase-1 chunks (i, c) = (o / nch, o % nch) of sequence `slot`, the rest
-// phase-2 chunks of sequence slot - lag.  A phase-2 chunk whose sequence is
-// not ready yet is set aside (at most kDefer); set-aside chunks are polled
-// together with relaxed loads and issued once ready.
+// next grab's atomic in flight meanwhile) and decodes each by multiply-high
+// divisions along the three runs of the ticket map (StochParams): phase-1
+// chunk (i, c) of a sequence, or phase-2 chunk c of a sequence `lag` slots
+// back.  A phase-2 chunk whose sequence is not ready yet is set aside (at most
+// kDefer); set-aside chunks are polled together with relaxed loads and issued
+// once ready.
 template <typename TT, typename TD, bool kTma>
 __device__ void stoch_producer(const StochParams& p, Shared& sh, unsigned char* stages, int g) {
   constexpr int kDefer = 4;
   Ctrl* ctrl = p.ctrl;
   const unsigned int nch = static_cast<unsigned int>(p.nch);
-  const unsigned int p1_items = static_cast<unsigned int>(p.k) * nch;
   uint32_t used = 0;  // uses of group g's stages issued
   bool ok = true;
   int db[kDefer], dc[kDefer];  // set-aside phase-2 chunks, oldest first
   int nd = 0;
   unsigned int base = atomicAdd(&ctrl->ticket, kGrabStoch), next = 0u, j = 0u;
   bool prefetched = false;
-  unsigned int slot = 0u, o = 0u, ci = 0u, cc = 0u;  // decoded ticket base + j
   while (ok) {
     if (nd > 0) {
       unsigned int rd[kDefer];
@@ -839,38 +836,40 @@ __device__ void stoch_producer(const StochParams& p, Shared& sh, unsigned char* 
       prefetched = true;
     }
     const unsigned int t = base + j;
-    if (j == 0u) {
-      slot = udiv(t, p.div_slot);
-      o = t - slot * p.slot_items;
-      ci = o < p1_items ? udiv(o, p.div_nch) : 0u;
-      cc = o < p1_items ? o - ci * nch : 0u;
-    } else if (++o == p.slot_items) {
-      o = 0u;
-      ++slot;
-      ci = 0u;
-      cc = 0u;
-    } else if (o < p1_items && ++cc == nch) {
-      cc = 0u;
-      ++ci;
-    }
     if (++j == kGrabStoch) {
       j = 0u;
       base = next;
       prefetched = false;
     }
     if (t >= p.total) continue;
-    if (o < p1_items) {
-      if (static_cast<int>(slot) >= p.B) continue;
+    // Decode: sequence sq and offset o within its phase-1 chunks
+    // (o < p1_items), or phase-2 chunk o - p1_items of sequence sq.
+    unsigned int sq, o;
+    if (t < p.a_end) {
+      sq = udiv(t, p.div_p1);
+      o = t - sq * p.p1_items;
+    } else if (t < p.b_end) {
+      const unsigned int u = t - p.a_end;
+      const unsigned int q = udiv(u, p.div_slot);
+      o = u - q * p.slot_items;
+      sq = static_cast<unsigned int>(p.lag) + q - (o < p.p1_items ? 0u : static_cast<unsigned int>(p.lag));
+    } else {
+      const unsigned int u = t - p.b_end;
+      const unsigned int q = udiv(u, p.div_nch);
+      sq = static_cast<unsigned int>(p.B - p.lag) + q;
+      o = p.p1_items + (u - q * nch);
+    }
+    if (o < p.p1_items) {
+      const unsigned int ci = udiv(o, p.div_nch);
       Hdr h;
       h.kind = kKindStats;
-      h.b = static_cast<int>(slot);
+      h.b = static_cast<int>(sq);
       h.i = static_cast<int>(ci);
-      h.c = static_cast<int>(cc);
+      h.c = static_cast<int>(o - ci * nch);
       ok = stoch_issue<TT, TD, kTma>(p, sh, stages, g, used, h, nullptr);
     } else {
-      const int b = static_cast<int>(slot) - p.lag;
-      if (b < 0 || b >= p.B) continue;
-      const int c = static_cast<int>(o - p1_items);
+      const int b = static_cast<int>(sq);
+      const int c = static_cast<int>(o - p.p1_items);
       const unsigned int rd = p.k == 0 ? 1u : ld_relaxed_u32(&p.seq[b].ready);
       if (rd) {
         if (p.k > 0) fence_acq_rel_gpu();
