@@ -70,6 +70,9 @@ def _load():
             lib.oracle_verify_threshold.argtypes = [
                 P, i32, i64, i64, P, i32, i32, i32, dbl, dbl, i32, i32, P, P, P]
             lib.oracle_verify_threshold.restype = i32
+            lib.oracle_verify_tree_stochastic.argtypes = [
+                P, i32, i64, i64, P, P, i32, i32, i32, dbl, u64, u32, i32, i32, P, P, P, P, P, P]
+            lib.oracle_verify_tree_stochastic.restype = i32
             _lib = lib
     return _lib
 
@@ -317,6 +320,43 @@ def verify_tree_greedy(node_logits: np.ndarray, t_dtype: str, parent: np.ndarray
             out["path"][b, n] = u
         out["out_tokens"][b, n] = amax[b, u]
         out["accepted_len"][b] = n
+    return out
+
+
+def verify_tree_stochastic(node_logits: np.ndarray, t_dtype: str, parent: np.ndarray,
+                           tokens: np.ndarray, temperature: float, seed: int,
+                           seq_offset: int = 0, threads: int = 1) -> dict:
+    """Stochastic verify of a draft token tree [B,N,V] with parent/tokens
+    [B,N] (node 0 the root; Top-K siblings tried in node order, each accepted
+    with probability p(x)/R of the target's distribution left after the
+    rejected siblings; the final token drawn from p outside the rejected
+    tokens).  ``temperature`` is rounded to float32 first.  Returns
+    accepted_len [B], path [B,N], out_tokens [B,N], margins [B,N], gaps [B],
+    flags [B] and invalid_tree."""
+    lib = _load()
+    tc, (sb, sn) = _logits(node_logits, t_dtype, 3)
+    B, N, V = node_logits.shape
+    par = np.ascontiguousarray(parent, dtype=np.int32).reshape(B, N)
+    tok = np.ascontiguousarray(tokens, dtype=np.int32).reshape(B, N)
+    T = float(np.float32(temperature))
+    out = {
+        "accepted_len": np.zeros(B, np.int32),
+        "path": np.full((B, N), -1, np.int32),
+        "out_tokens": np.full((B, N), -1, np.int32),
+        "margins": np.full((B, N), np.nan, np.float64),
+        "gaps": np.zeros(B, np.float64),
+        "flags": np.zeros(B, np.int32),
+    }
+
+    def fn(b0, b1):
+        return lib.oracle_verify_tree_stochastic(
+            _ptr(node_logits), tc, sb, sn, _ptr(par), _ptr(tok), B, N, V, T,
+            int(seed) & (2**64 - 1), int(seq_offset) & 0xFFFFFFFF, b0, b1,
+            _ptr(out["accepted_len"]), _ptr(out["path"]), _ptr(out["out_tokens"]),
+            _ptr(out["margins"]), _ptr(out["gaps"]), _ptr(out["flags"]))
+
+    _run_parallel(fn, B, threads)
+    out["invalid_tree"] = bool((out["flags"] & 32).any())
     return out
 
 

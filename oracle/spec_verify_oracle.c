@@ -27,6 +27,24 @@
  *      n < k : y ~ normalize(max(0, p_n - q_n))   (Gumbel-max)
  *      n = k : y ~ p_k                            (Gumbel-max)
  *
+ *  Stochastic tree verify.  Same page, section "EAGLE": at every node of
+ *  the draft tree the Top-K candidates are explored, and the longest
+ *  acceptable path is kept with one more token from the target.  Reading
+ *  (the page writes no rule down): Top-K siblings are fixed, not sampled, so
+ *  the draft distribution behind each child is a point mass on its token,
+ *  and the rejection rule above applied to the siblings one after another
+ *  (multi-draft recursive rejection, as in SpecInfer and Sequoia) becomes:
+ *      at node u, p = softmax(row u / T), R = 1, E = {};
+ *      for each child c of u in node order, with token x_c:
+ *          accept  <=>  x_c valid, x_c not in E, and u_c * R < p(x_c)
+ *          else     E += {x_c},  R -= p(x_c)        (when x_c valid, new)
+ *      an accepted child becomes u; otherwise y ~ p restricted to V \ E
+ *      (Gumbel-max over l/T), which keeps the output distributed as p.
+ *  Draws: u_c is the acceptance draw of position c - 1; the final draw uses
+ *  position u with tag CORRECTION when u has children, BONUS when it is a
+ *  leaf.  On a chain tree this is exactly stochastic verify with one-hot
+ *  draft distributions.
+ *
  *  Greedy verify.  Same page, section "Speculative decoding": the longest
  *  prefix that the target accepts, plus the target's own next token.  In
  *  greedy mode "accepts" means "equals the target argmax" (first maximum).
@@ -317,6 +335,117 @@ int oracle_verify_stochastic(const void *target, int t_dtype, int64_t t_sb, int6
             else if (i == n) v = y;
             out_tokens[(int64_t)b * (k + 1) + i] = v;
         }
+        if (gaps) gaps[b] = scan_gap(&sc);
+        if (flags) flags[b] = flag;
+    }
+    return 0;
+}
+
+/* ------------------------------------------------- stochastic tree verify */
+
+/*
+ * Sequences b in [b_begin, b_end) of a batch of B trees of N nodes.
+ * Layouts (element strides, vocabulary contiguous):
+ *   logits[b][j][x] at b*sb + j*sn + x: the target's distribution after the
+ *                   path root..j (node 0 is the root, the last committed
+ *                   token)
+ *   parent[b][j], tokens[b][j] at b*N + j (entries of node 0 unused); a node
+ *                   j >= 1 with parent outside [0, j) is never entered
+ * Outputs: accepted_len[b] = n; path[b][0..n] = accepted nodes from the
+ * root, out_tokens[b][0..n] = their tokens then the drawn token (both -1
+ * after); margins[b][j] = |u_j - p(x_j)/R| for every examined child j
+ * (inf when it could not be accepted: invalid or repeated token; NaN when
+ * not examined); gaps[b] = best minus second-best score of the final draw;
+ * flags[b] (bit 0: invalid token, bit 1: no candidate left outside E, bit 5:
+ * invalid parent).  margins, gaps and flags may be NULL.
+ * Returns 0, or -1 on bad arguments.
+ */
+int oracle_verify_tree_stochastic(const void *logits, int dtype, int64_t sb, int64_t sn,
+                                  const int32_t *parent, const int32_t *tokens, int B, int N,
+                                  int V, double T, uint64_t seed, uint32_t seq_offset,
+                                  int b_begin, int b_end, int32_t *accepted_len, int32_t *path,
+                                  int32_t *out_tokens, double *margins, double *gaps,
+                                  int32_t *flags)
+{
+    if (!(T > 0.0) || V < 1 || N < 1 || N > 64 || B < 0 || b_begin < 0 || b_end > B)
+        return -1;
+    for (int b = b_begin; b < b_end; ++b) {
+        const int32_t *par = parent + (int64_t)b * N;
+        const int32_t *tok = tokens + (int64_t)b * N;
+        uint32_t seq = (uint32_t)b + seq_offset;
+        int32_t flag = 0;
+        for (int j = 1; j < N; ++j)
+            if (par[j] < 0 || par[j] >= j) flag |= 32;
+        for (int j = 0; j < N; ++j) {
+            if (margins) margins[(int64_t)b * N + j] = NAN;
+            path[(int64_t)b * N + j] = -1;
+            out_tokens[(int64_t)b * N + j] = -1;
+        }
+
+        int u = 0, n = 0;
+        int32_t excl[64];
+        int nexcl = 0, has_child = 0;
+        path[(int64_t)b * N] = 0;
+        for (;;) {
+            row_t r = {logits, dtype, (int64_t)b * sb + (int64_t)u * sn};
+            double m, s;
+            softmax_stats(r, V, T, &m, &s);
+            double R = 1.0;
+            int next = -1;
+            nexcl = 0;
+            has_child = 0;
+            for (int j = u + 1; j < N; ++j) {
+                if (par[j] != u) continue;
+                has_child = 1;
+                int32_t x = tok[j];
+                int valid = (x >= 0 && x < V);
+                if (!valid) flag |= 1;
+                int repeated = 0;
+                for (int e = 0; e < nexcl; ++e)
+                    if (excl[e] == x) repeated = 1;
+                double uj = accept_uniform(draw_word(seed, 0u, (uint32_t)(j - 1), seq, TAG_ACCEPT, 0));
+                double p = (valid && !repeated) ? softmax_prob(r, x, T, m, s) : 0.0;
+                int open = valid && !repeated;
+                if (margins)
+                    margins[(int64_t)b * N + j] = (open && R > 0.0) ? fabs(uj - p / R) : INFINITY;
+                if (open && uj * R < p) {
+                    next = j;
+                    break;
+                }
+                if (open) {
+                    excl[nexcl++] = x;
+                    R -= p;
+                }
+            }
+            if (next < 0) break;
+            u = next;
+            out_tokens[(int64_t)b * N + n] = tok[u];
+            ++n;
+            path[(int64_t)b * N + n] = u;
+        }
+
+        /* the final draw: y ~ p_u outside E */
+        row_t r = {logits, dtype, (int64_t)b * sb + (int64_t)u * sn};
+        uint32_t tag = has_child ? TAG_CORRECTION : TAG_BONUS;
+        scan_t sc;
+        scan_init(&sc);
+        for (int64_t x = 0; x < V; ++x) {
+            double l = row_at(r, x);
+            if (l == -INFINITY) continue;
+            int in_e = 0;
+            for (int e = 0; e < nexcl; ++e)
+                if (excl[e] == x) in_e = 1;
+            if (in_e) continue;
+            scan_push(&sc, l / T + vocab_gumbel(seed, x, (uint32_t)u, seq, tag), x);
+        }
+        if (sc.arg < 0) {
+            /* nothing left outside E (possible only through rounding) */
+            flag |= 2;
+            for (int64_t x = 0; x < V; ++x)
+                scan_push(&sc, row_at(r, x) / T + vocab_gumbel(seed, x, (uint32_t)u, seq, tag), x);
+        }
+        out_tokens[(int64_t)b * N + n] = (int32_t)sc.arg;
+        accepted_len[b] = n;
         if (gaps) gaps[b] = scan_gap(&sc);
         if (flags) flags[b] = flag;
     }

@@ -584,6 +584,161 @@ def test_tree_duplicate_siblings_and_invalid_parent_hand_cases():
     assert r["out_tokens"].tolist() == [[2, 2, 2, -1]]
 
 
+# ------------------------------------------------------ stochastic tree verify
+
+def chain_tree(B, k):
+    parent = np.tile(np.arange(-1, k, dtype=np.int32), (B, 1))
+    return parent
+
+
+def one_hot_draft(tokens, V):
+    B, k = tokens.shape
+    d = np.full((B, k, V), -np.inf, np.float32)
+    for b in range(B):
+        d[b, np.arange(k), tokens[b]] = 0.0
+    return d
+
+
+@pytest.mark.parametrize("dtype,T", [("f32", 1.0), ("bf16", 0.7)])
+def test_tree_stochastic_chain_is_stochastic_verify_with_one_hot_drafts(dtype, T):
+    """A chain tree is linear drafting with a point-mass draft at every
+    position: the rejection rule, draws and committed tokens must coincide."""
+    rng = np.random.default_rng(61)
+    B, k, V = 300, 5, 50
+    x = (rng.standard_normal((B, k + 1, V)) * 2.0).astype(np.float32)
+    p = softmax64(x, T)
+    drafts = np.zeros((B, k), np.int32)
+    for b in range(B):
+        for i in range(k):  # mostly likely tokens, so that long prefixes occur
+            drafts[b, i] = int(np.argmax(p[b, i])) if rng.random() < 0.6 else int(rng.integers(V))
+    arr = workloads.f32_to_bf16_bits(x) if dtype == "bf16" else x
+    tokens = np.concatenate([np.zeros((B, 1), np.int32), drafts], axis=1)
+    r = oracle.verify_tree_stochastic(arr, dtype, chain_tree(B, k), tokens, T, seed=5)
+    lin = oracle.verify_stochastic(arr, dtype, one_hot_draft(drafts, V), "f32", drafts, T, seed=5)
+    ok = lin["gaps"] > 1e-9
+    assert ok.sum() > B - 3
+    np.testing.assert_array_equal(r["accepted_len"][ok], lin["accepted_len"][ok])
+    np.testing.assert_array_equal(r["out_tokens"][ok], lin["out_tokens"][ok])
+    for b in np.nonzero(ok)[0]:
+        n = int(r["accepted_len"][b])
+        assert r["path"][b, : n + 1].tolist() == list(range(n + 1))
+        seen = ~np.isnan(r["margins"][b, 1:])  # children examined on the walk
+        assert seen.sum() == min(n + 1, k)
+        np.testing.assert_allclose(r["margins"][b, 1:][seen], lin["margins"][b][seen], atol=1e-12)
+    assert 0 < r["accepted_len"].mean() < k
+
+
+def test_tree_stochastic_root_only_is_the_bonus_draw():
+    rng = np.random.default_rng(62)
+    B, V, T = 200, 70, 0.9
+    x = (rng.standard_normal((B, 1, V)) * 1.5).astype(np.float32)
+    r = oracle.verify_tree_stochastic(x, "f32", np.full((B, 1), -1, np.int32),
+                                      np.zeros((B, 1), np.int32), T, seed=8)
+    lin = oracle.verify_stochastic(x, "f32", np.zeros((B, 0, V), np.float32), "f32",
+                                   np.zeros((B, 0), np.int32), T, seed=8)
+    assert np.all(r["accepted_len"] == 0)
+    np.testing.assert_array_equal(r["out_tokens"][:, 0], lin["out_tokens"][:, 0])
+    np.testing.assert_array_equal(r["path"], np.zeros((B, 1), np.int32))
+
+
+@pytest.fixture(scope="module")
+def tree_law_case():
+    """One 8-node tree shared by 400k sequences (stride-0 batch): root with
+    children 1, 2, 3 (node 3 repeats node 2's token), node 1 with children 4
+    and 5, node 2 with child 6, node 4 with child 7."""
+    rng = np.random.default_rng(63)
+    V, T, trials = 6, 0.8, 400_000
+    parent = np.array([-1, 0, 0, 0, 1, 1, 2, 4], np.int32)
+    tokens = np.array([0, 1, 4, 4, 2, 0, 5, 3], np.int32)
+    rows = (rng.standard_normal((8, V)) * 1.2).astype(np.float32)
+    r = oracle.verify_tree_stochastic(np.broadcast_to(rows, (trials, 8, V)), "f32",
+                                      np.broadcast_to(parent, (trials, 8)),
+                                      np.broadcast_to(tokens, (trials, 8)), T, seed=21,
+                                      threads=THREADS)
+    return dict(V=V, p=softmax64(rows, T), parent=parent, tokens=tokens, r=r, trials=trials)
+
+
+def test_tree_stochastic_first_token_follows_the_root_row(tree_law_case):
+    c = tree_law_case
+    counts = np.bincount(c["r"]["out_tokens"][:, 0], minlength=c["V"])
+    assert chi2_pvalue(counts, c["p"][0]) > P_MIN
+
+
+def test_tree_stochastic_each_child_is_taken_with_its_target_probability(tree_law_case):
+    c = tree_law_case
+    first = c["r"]["path"][:, 1]
+    for j in (1, 2):
+        hits = int((first == j).sum())
+        assert scipy.stats.binomtest(hits, c["trials"], c["p"][0, c["tokens"][j]]).pvalue > P_MIN
+    assert not (first == 3).any()  # a repeated sibling token is never taken
+
+
+def test_tree_stochastic_after_an_accepted_node_its_row_takes_over(tree_law_case):
+    c = tree_law_case
+    r = c["r"]
+    for u in (1, 2, 4):
+        sel = (r["path"] == u).any(axis=1)
+        depth = {1: 1, 2: 1, 4: 2}[u]
+        counts = np.bincount(r["out_tokens"][sel, depth], minlength=c["V"])
+        assert sel.sum() > 1000
+        assert chi2_pvalue(counts, c["p"][u]) > P_MIN
+
+
+def test_tree_stochastic_final_draw_skips_rejected_siblings(tree_law_case):
+    c = tree_law_case
+    r = c["r"]
+    stop0 = r["accepted_len"] == 0  # every root child was rejected
+    drawn = r["out_tokens"][stop0, 0]
+    assert not np.isin(drawn, [1, 4]).any()
+    law = c["p"][0].copy()
+    law[[1, 4]] = 0.0
+    counts = np.bincount(drawn, minlength=c["V"])
+    assert chi2_pvalue(counts, law / law.sum()) > P_MIN
+    # node 1 accepted, both its children rejected: the draw avoids 2 and 0
+    stop1 = (r["accepted_len"] == 1) & (r["path"][:, 1] == 1)
+    assert not np.isin(r["out_tokens"][stop1, 1], [2, 0]).any()
+    # leaf reached (node 6 under node 2): the bonus draw is unrestricted
+    leaf = r["path"][:, 2] == 6
+    counts = np.bincount(r["out_tokens"][leaf, 2], minlength=c["V"])
+    assert chi2_pvalue(counts, c["p"][6]) > P_MIN
+
+
+def test_tree_stochastic_sure_and_impossible_children():
+    V = 5
+    rows = np.zeros((1, 3, V), np.float32)
+    rows[0, 0] = [-np.inf, 0.0, -np.inf, -np.inf, -np.inf]  # root puts all mass on 1
+    parent = np.array([[-1, 0, 0]], np.int32)
+    r = oracle.verify_tree_stochastic(rows, "f32", parent, np.array([[0, 3, 1]], np.int32),
+                                      1.0, seed=1)
+    # node 1 (token 3, p = 0) is rejected, node 2 (token 1, p / R = 1) accepted
+    assert r["path"].tolist() == [[0, 2, -1]]
+    assert r["out_tokens"][0, 0] == 1
+    assert np.isfinite(r["margins"][0, 1]) and np.isfinite(r["margins"][0, 2])
+    # invalid token and a forward parent
+    r = oracle.verify_tree_stochastic(rows, "f32", np.array([[-1, 0, 5]], np.int32),
+                                      np.array([[0, V, 1]], np.int32), 1.0, seed=1)
+    assert r["flags"].tolist() == [1 | 32]
+    assert r["invalid_tree"]
+    assert r["accepted_len"].tolist() == [0]
+    assert r["out_tokens"][0, 0] == 1  # the root's only token with mass
+    assert np.isinf(r["margins"][0, 1]) and np.isnan(r["margins"][0, 2])
+
+
+def test_tree_stochastic_sequence_offset_selects_the_stream():
+    rng = np.random.default_rng(64)
+    B, N, V = 12, 9, 30
+    x = (rng.standard_normal((1, N, V)) * 2).astype(np.float32)
+    par = workloads.tree_parents(N, rng)[None, :]
+    tok = rng.integers(0, V, (1, N)).astype(np.int32)
+    xb = np.broadcast_to(x, (B, N, V))
+    full = oracle.verify_tree_stochastic(xb, "f32", np.broadcast_to(par, (B, N)),
+                                         np.broadcast_to(tok, (B, N)), 1.0, seed=3)
+    for s in (0, 5, 11):
+        one = oracle.verify_tree_stochastic(x, "f32", par, tok, 1.0, seed=3, seq_offset=s)
+        np.testing.assert_array_equal(one["out_tokens"][0], full["out_tokens"][s])
+        np.testing.assert_array_equal(one["path"][0], full["path"][s])
+
+
 # ------------------------------------------------------------ device commit
 
 def test_commit_hand_case():
