@@ -46,12 +46,13 @@ STEP = ["greedy_b64_k4_v128256", "stoch_b64_k4_v128256", "stoch_b256_k8_v128256"
 DOMINANT = "stoch_b256_k8_v128256"
 HBM_FALLBACK_GBS = 6650.0
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic_stochastic_verify_b256_k8.json")
+TREE_MODES = ("tree", "tree_stochastic")
 
 
 # ------------------------------------------------------------------ helpers
 
 def positions(w: dict) -> int:
-    if w["mode"] == "tree":  # every drafted node is a verified position
+    if w["mode"] in TREE_MODES:  # every drafted node is a verified position
         return w["B"] * w["N"]
     return w["B"] * w.get("G", 1) * (w["k"] + 1)
 
@@ -66,7 +67,7 @@ def algorithmic_bytes(w: dict, accepted_len: np.ndarray | None) -> int:
     from workloads import ELEM_BYTES
 
     st = ELEM_BYTES[w["t_dtype"]]
-    if w["mode"] == "tree":  # every node row, parents and tokens, path and tokens out
+    if w["mode"] in TREE_MODES:  # every node row, parents and tokens, path and tokens out
         B, N, V = w["B"], w["N"], w["V"]
         return B * N * V * st + 8 * B * N + 4 * B + 8 * B * N
     B, k, V = w["B"], w["k"], w["V"]
@@ -93,20 +94,31 @@ def measured_hbm_peak() -> tuple[float, str]:
         return HBM_FALLBACK_GBS, "fallback"
 
 
+# The sources that build the dominant kernel and set its launch (chunking,
+# ticket map, lag); a traffic record is valid only for these exact bytes.
+DOMINANT_SOURCES = ("sv_api.cu", "sv_device.cuh", "sv_internal.h", "sv_kernels.cu")
+KERNEL_OF_MODE = {"stochastic": "stochastic_verify_kernel", "greedy": "argmax_verify_kernel",
+                  "multi": "argmax_verify_kernel", "multi_rows": "argmax_verify_kernel",
+                  "tree": "argmax_verify_kernel", "threshold": "argmax_verify_kernel",
+                  "tree_stochastic": "tree_stats_kernel + tree_walk_kernel + tree_sample_kernel"}
+
+
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "speculative_decoding_verification_88_b200", "csrc")
-    for p in sorted(glob.glob(os.path.join(csrc, "*"))) + [os.path.join(ROOT, "include",
-                                                                         "spec_verify.h")]:
-        with open(p, "rb") as f:
-            h.update(os.path.basename(p).encode())
+    for name in DOMINANT_SOURCES:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
             h.update(f.read())
     return h.hexdigest()
 
 
-def recorded_traffic() -> float | None:
+def recorded_traffic(workload: str, batch_override: bool) -> float | None:
     """DRAM bytes per launch of the dominant kernel from an ncu capture of the
-    current kernel sources, or None if the sources changed since."""
+    current kernel sources, or None if the sources changed since or the run
+    times another workload or batch than the one the record covers."""
+    if workload != "stoch_b256_k8_v128256" or batch_override:
+        return None
     try:
         with open(TRAFFIC_FILE) as f:
             rec = json.load(f)
@@ -204,6 +216,10 @@ def run_reference(args, rank: int) -> None:
         elif w["mode"] == "tree":
             oracle.verify_tree_greedy(w["node_logits"][b:b + 1], w["t_dtype"],
                                       w["parent"][b:b + 1], w["tokens"][b:b + 1])
+        elif w["mode"] == "tree_stochastic":
+            oracle.verify_tree_stochastic(w["node_logits"][b:b + 1], w["t_dtype"],
+                                          w["parent"][b:b + 1], w["tokens"][b:b + 1],
+                                          w["temperature"], w["seed"], seq_offset=b)
         elif w["mode"] == "threshold":
             oracle.verify_threshold(w["target"][b:b + 1], w["t_dtype"], w["tokens"][b:b + 1],
                                     w["temperature"], w["threshold"])
@@ -266,6 +282,10 @@ def oracle_baseline(ws: dict) -> dict:
             elif w["mode"] == "tree":
                 oracle.verify_tree_greedy(w["node_logits"], w["t_dtype"], w["parent"],
                                           w["tokens"], threads=cores)
+            elif w["mode"] == "tree_stochastic":
+                oracle.verify_tree_stochastic(w["node_logits"], w["t_dtype"], w["parent"],
+                                              w["tokens"], w["temperature"], w["seed"],
+                                              threads=cores)
             elif w["mode"] == "threshold":
                 oracle.verify_threshold(w["target"], w["t_dtype"], w["tokens"],
                                         w["temperature"], w["threshold"], threads=cores)
@@ -310,10 +330,10 @@ def run_ours(args, rank: int, world: int, dist) -> None:
         d_d = d_h.to(dev) if d_h is not None else None
         wsp = sv.Workspace(dev)
         B = w["B"]
-        width = w["N"] if w["mode"] == "tree" else w["k"] + 1
+        width = w["N"] if w["mode"] in TREE_MODES else w["k"] + 1
         if w["mode"] in ("multi", "multi_rows"):
             out = {"best_candidate": torch.empty(B, dtype=torch.int32, device=dev)}
-        elif w["mode"] == "tree":
+        elif w["mode"] in TREE_MODES:
             out = {"path": torch.empty((B, width), dtype=torch.int32, device=dev)}
         else:
             out = {}
@@ -332,6 +352,12 @@ def run_ours(args, rank: int, world: int, dist) -> None:
             par = torch.from_numpy(w["parent"]).to(dev)
             fn = (lambda t=t_d, pa=par, tok=tok_d, o=out, wsp=wsp:
                   sv.tree_greedy(t, pa, tok, out=o, workspace=wsp))
+        elif w["mode"] == "tree_stochastic":
+            par = torch.from_numpy(w["parent"]).to(dev)
+            off = rank * B
+            fn = (lambda w=w, t=t_d, pa=par, tok=tok_d, o=out, wsp=wsp, off=off:
+                  sv.tree_stochastic(t, pa, tok, w["temperature"], w["seed"], off, out=o,
+                                     workspace=wsp))
         elif w["mode"] == "multi_rows":
             rmap = torch.from_numpy(w["row_of"]).to(dev)
             fn = (lambda t=t_d, rm=rmap, tok=tok_d, o=out, wsp=wsp:
@@ -425,8 +451,9 @@ def run_ours(args, rank: int, world: int, dist) -> None:
         per[name]["frac_of_hbm_peak"] = per[name]["alg_gbs"] / peak
     d = per[DOMINANT]
     roofline = {"bound": "hbm", "achieved": d["alg_gbs"], "peak": peak, "unit": "GB/s",
-                "frac": d["alg_gbs"] / peak, "traffic": recorded_traffic(),
-                "kernel": "stochastic_verify_kernel (" + DOMINANT + ")",
+                "frac": d["alg_gbs"] / peak,
+                "traffic": recorded_traffic(DOMINANT, bool(args.batch)),
+                "kernel": KERNEL_OF_MODE[ws[DOMINANT]["mode"]] + " (" + DOMINANT + ")",
                 "peak_source": peak_kind + " (MEASURED_PEAKS.json hbm_gbs)"
                 if peak_kind == "measured" else "fallback 6.65 TB/s"}
 

@@ -255,6 +255,46 @@ int spec_verify_tree_greedy(const void *node_logits, int t_dtype, int64_t stride
                             void *stream);
 
 /*
+ * Stochastic verify of a draft token tree (EAGLE-style tree drafting).
+ *
+ * "Accelerating Sonar through speculation", section "EAGLE": the tree holds
+ * the Top-K candidates of every node; the longest acceptable path is kept
+ * and the target adds one token.  The siblings are fixed candidates, so the
+ * draft distribution behind each child is a point mass on its token, and
+ * speculative rejection over the siblings in node order reads: at node u,
+ * with p = softmax(row u / T), the residual mass R = 1 and the rejected set
+ * E empty, child c (token x) is accepted iff x is in [0, V), x is not in E
+ * and u_c * R < p(x); a rejected child puts x in E and takes p(x) off R.
+ * The walk enters the accepted child; when none is accepted, the last token
+ * is drawn from p restricted to the vocabulary outside E (Gumbel-max over
+ * l/T).  The committed tokens follow the target's distribution at every
+ * depth.  Draws (Philox4x32-10, key = seed, counter (c0, position,
+ * seq_offset + b, tag)): u_c is the acceptance draw of position c - 1; the
+ * final draw uses position u, tag CORRECTION when u has children and BONUS
+ * at a leaf -- so a chain tree gives exactly spec_verify_stochastic with
+ * one-hot draft distributions.
+ *
+ * node_logits, parent, tokens and the outputs are laid out as for
+ * spec_verify_tree_greedy (out_tokens [B, N]: the n accepted tokens, the
+ * drawn token, then -1).  temperature > 0 (normal, finite).  An invalid or
+ * repeated sibling token is never accepted (SV_FLAG_INVALID_TOKEN for an
+ * invalid one); a node with an invalid parent is never entered
+ * (SV_FLAG_INVALID_TREE); if rounding leaves nothing outside E the draw
+ * uses the whole row (SV_FLAG_RESIDUAL_FALLBACK).  1 <= N <= 64.
+ * Workspace: spec_verify_tree_stochastic_workspace_size(B, N, V) bytes,
+ * zeroed once as for the other calls (the call leaves it zeroed).  Three
+ * kernel launches on `stream`.
+ */
+size_t spec_verify_tree_stochastic_workspace_size(int B, int N, int V);
+
+int spec_verify_tree_stochastic(const void *node_logits, int t_dtype, int64_t stride_b,
+                                int64_t stride_node, const int32_t *parent,
+                                const int32_t *tokens, int B, int N, int V, float temperature,
+                                uint64_t seed, uint32_t seq_offset, int32_t *accepted_len,
+                                int32_t *path, int32_t *out_tokens, void *workspace,
+                                size_t workspace_bytes, void *stream);
+
+/*
  * Device-side commit: the step after verify, with no host synchronisation.
  *
  * "Accelerating Sonar through speculation", section "Single-token MTP

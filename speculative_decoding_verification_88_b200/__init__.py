@@ -32,6 +32,7 @@ EXPORTS = (
     "spec_verify_multi_candidate", "spec_verify_multi_candidate_rows", "spec_verify_commit",
     "spec_verify_tree_workspace_size", "spec_verify_tree_greedy", "spec_verify_threshold",
     "spec_verify_philox4x32_10", "spec_verify_greedy_noalloc",
+    "spec_verify_tree_stochastic_workspace_size", "spec_verify_tree_stochastic",
 )
 
 _lib = None
@@ -88,6 +89,11 @@ def load_library():
         lib.spec_verify_tree_greedy.restype = I
         lib.spec_verify_threshold.argtypes = [P, I, I64, I64, P, I, I, I, F, F, P, P, P, SZ, P]
         lib.spec_verify_threshold.restype = I
+        lib.spec_verify_tree_stochastic_workspace_size.argtypes = [I, I, I]
+        lib.spec_verify_tree_stochastic_workspace_size.restype = SZ
+        lib.spec_verify_tree_stochastic.argtypes = [
+            P, I, I64, I64, P, P, I, I, I, F, U64, U32, P, P, P, P, SZ, P]
+        lib.spec_verify_tree_stochastic.restype = I
         lib.spec_verify_philox4x32_10.argtypes = [P, I64, U64, P, P]
         lib.spec_verify_philox4x32_10.restype = I
         lib.spec_verify_greedy_noalloc.argtypes = [P, I, I64, I64, P, I, I, I, P, P, P]
@@ -110,9 +116,9 @@ def launch_count() -> int:
     return _launches
 
 
-def _count():
+def _count(n: int = 1):
     global _launches
-    _launches += 1
+    _launches += n
 
 
 def workspace_size(B: int, G: int, k: int, V: int) -> int:
@@ -375,6 +381,40 @@ def tree_greedy(node_logits: torch.Tensor, parent: torch.Tensor, tokens: torch.T
             ws.buf.data_ptr(), ws.nbytes, _stream_ptr(stream, dev))
     _check(code, "spec_verify_tree_greedy")
     _count()
+    return res
+
+
+def tree_stochastic_workspace_size(B: int, N: int, V: int) -> int:
+    return int(load_library().spec_verify_tree_stochastic_workspace_size(B, N, V))
+
+
+def tree_stochastic(node_logits: torch.Tensor, parent: torch.Tensor, tokens: torch.Tensor,
+                    temperature: float, seed: int, seq_offset: int = 0, *,
+                    out: dict | None = None, workspace: Workspace | None = None,
+                    stream=None) -> dict:
+    """Stochastic verify of a draft token tree whose siblings are Top-K
+    candidates: node_logits [B,N,V], parent [B,N] and tokens [B,N] int32 as
+    for tree_greedy.  Returns accepted_len [B], path [B,N] and out_tokens
+    [B,N] (the accepted tokens, the drawn token, then -1)."""
+    lib = load_library()
+    tc, (tsb, tsn, _) = _logits(node_logits, 3, "node_logits")
+    B, N, V = node_logits.shape
+    dev = node_logits.device
+    par = _tokens(parent, (B, N), dev, "parent")
+    tok = _tokens(tokens, (B, N), dev, "tokens")
+    res = {"accepted_len": _out(out, "accepted_len", (B,), torch.int32, dev),
+           "path": _out(out, "path", (B, N), torch.int32, dev),
+           "out_tokens": _out(out, "out_tokens", (B, N), torch.int32, dev)}
+    ws = workspace or default_workspace(dev)
+    ws.ensure(tree_stochastic_workspace_size(B, N, V), stream)
+    with torch.cuda.device(dev):
+        code = lib.spec_verify_tree_stochastic(
+            node_logits.data_ptr(), tc, tsb, tsn, par.data_ptr(), tok.data_ptr(), B, N, V,
+            float(temperature), int(seed) & (2**64 - 1), int(seq_offset) & 0xFFFFFFFF,
+            res["accepted_len"].data_ptr(), res["path"].data_ptr(), res["out_tokens"].data_ptr(),
+            ws.buf.data_ptr(), ws.nbytes, _stream_ptr(stream, dev))
+    _check(code, "spec_verify_tree_stochastic")
+    _count(3)
     return res
 
 

@@ -19,7 +19,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB_DIR = os.path.join(PKG, "_lib")
 LIB_PATH = os.path.join(LIB_DIR, "libspecverify.so")
 
-SOURCES = ["sv_api.cu", "sv_kernels.cu", "sv_noalloc.cu"]
+SOURCES = ["sv_api.cu", "sv_kernels.cu", "sv_noalloc.cu", "sv_tree_stoch.cu"]
 HEADERS = [os.path.join(CSRC, h) for h in ("sv_internal.h", "sv_device.cuh")] + [
     os.path.join(INCLUDE, "spec_verify.h")]
 

@@ -183,6 +183,39 @@ def test_tree_validation(lib):
     assert t(wb=64) == WORKSPACE
 
 
+def test_tree_stochastic_validation(lib):
+    assert sv.tree_stochastic_workspace_size(64, 26, 128256) > 0
+    assert sv.tree_stochastic_workspace_size(4, 0, 10) == 0
+    assert sv.tree_stochastic_workspace_size(4, 65, 10) == 0
+    assert sv.tree_stochastic_workspace_size(-1, 4, 10) == 0
+    assert sv.tree_stochastic_workspace_size(8, 26, 128256) >= \
+        sv.tree_stochastic_workspace_size(4, 26, 128256)
+
+    def t(**kw):
+        a = dict(x=A16, dt=1, sb=80, sn=8, par=A16, tok=A16, B=2, N=10, V=8, T=1.0, seed=3,
+                 off=0, acc=A16, path=A16, out=A16, ws=A16, wb=1 << 20, st=None)
+        a.update(kw)
+        return lib.spec_verify_tree_stochastic(*a.values())
+
+    assert t(B=0, x=None, par=None, tok=None) == OK
+    for T in (0.0, -1.0, float("inf"), float("nan"), 1e-40):
+        assert t(T=T) == INVALID, T
+    assert t(N=0) == INVALID
+    assert t(N=65) == INVALID
+    assert t(B=-1) == INVALID
+    assert t(sn=-8) == INVALID
+    assert t(par=None) == INVALID
+    assert t(tok=None) == INVALID
+    assert t(path=None) == INVALID
+    assert t(ws=None) == INVALID
+    assert t(dt=3) == INVALID
+    assert t(x=A16 + 1) == MISALIGNED
+    assert t(par=A16 + 2) == MISALIGNED
+    assert t(out=A16 + 1) == MISALIGNED
+    assert t(ws=A16 + 8) == MISALIGNED
+    assert t(wb=64) == WORKSPACE
+
+
 def test_commit_validation(lib):
     def c(**kw):
         a = dict(acc=A16, out=A16, B=2, k=4, lens=A16, buf=A16, stride=16, cap=16, nxt=A16,

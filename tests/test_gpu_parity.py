@@ -372,6 +372,145 @@ def test_tree_invalid_parent_flag(dev):
     assert int(ws.buf[256:].cpu().count_nonzero()) == 0
 
 
+# ---------------------------------------------------- stochastic tree verify
+
+def stoch_tree_case(rng, B, N, V, dtype, sigma=4.0):
+    """Random node rows; children carry their parent row's argmax with
+    probability 0.6 (so paths are accepted and sibling tokens repeat), else a
+    uniform token."""
+    x = (rng.standard_normal((B, N, V)) * sigma).astype(np.float32)
+    arr = workloads.f32_to_bf16_bits(x) if dtype == "bf16" else x
+    am = np.argmax(workloads.to_f32(arr, dtype), -1)
+    parent = np.zeros((B, N), np.int32)
+    tokens = rng.integers(0, V, (B, N)).astype(np.int32)
+    for b in range(B):
+        parent[b] = workloads.tree_parents(N, rng)
+        for j in range(1, N):
+            if rng.random() < 0.6:
+                tokens[b, j] = am[b, parent[b, j]]
+    return arr, parent, tokens
+
+
+def compare_tree_stochastic(r, o, what=""):
+    """Exact except sequences with a near-tie decision in the oracle (an
+    examined child with |u - p/R| < TOL_MARGIN, or a final-draw gap below
+    TOL_GAP); returns (near ties, near ties that differ)."""
+    m = np.where(np.isnan(o["margins"]), np.inf, o["margins"])
+    near = (m < TOL_MARGIN).any(axis=1) | (o["gaps"] < TOL_GAP)
+    acc = r["accepted_len"].cpu().numpy()
+    path = r["path"].cpu().numpy()
+    tok = r["out_tokens"].cpu().numpy()
+    mism = (acc != o["accepted_len"]) | (path != o["path"]).any(1) | \
+        (tok != o["out_tokens"]).any(1)
+    bad = np.nonzero(mism & ~near)[0]
+    assert bad.size == 0, (
+        f"{what}: {bad.size} mismatches outside near ties, first b={bad[0]}: gpu n={acc[bad[0]]} "
+        f"path={path[bad[0]]} tok={tok[bad[0]]} oracle n={o['accepted_len'][bad[0]]} "
+        f"path={o['path'][bad[0]]} tok={o['out_tokens'][bad[0]]}")
+    return int(near.sum()), int((mism & near).sum())
+
+
+def run_tree_stochastic(arr, dtype, parent, tokens, T, seed, dev, seq_offset=0, t=None,
+                        workspace=None):
+    t = to_dev(arr, dtype, dev) if t is None else t
+    r = sv.tree_stochastic(t, torch.from_numpy(parent).to(dev), torch.from_numpy(tokens).to(dev),
+                           T, seed, seq_offset, workspace=workspace)
+    o = oracle.verify_tree_stochastic(arr, dtype, parent, tokens, T, seed, seq_offset,
+                                      threads=THREADS)
+    torch.cuda.synchronize()
+    return r, o
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("B,N,V,T", [(1, 1, 10, 1.0), (3, 5, 17, 0.7), (16, 26, 3001, 1.0),
+                                     (4, 64, 40, 1.3), (2, 33, 2 * 16384 + 9, 1.0),
+                                     (70, 12, 300, 0.8), (5, 8, 3 * 8192, 1.0)])
+def test_tree_stochastic_parity_shapes(dev, dtype, B, N, V, T):
+    rng = np.random.default_rng(B * 11 + N * 5 + V)
+    arr, parent, tokens = stoch_tree_case(rng, B, N, V, dtype)
+    r, o = run_tree_stochastic(arr, dtype, parent, tokens, T, 17, dev)
+    compare_tree_stochastic(r, o, f"{dtype} B={B} N={N} V={V}")
+    if N > 1:
+        assert o["accepted_len"].max() >= 1 or B < 4
+
+
+def test_tree_stochastic_strided_unaligned_and_broadcast(dev):
+    rng = np.random.default_rng(71)
+    B, N, V = 6, 9, 2500
+    arr, parent, tokens = stoch_tree_case(rng, B, N, V, "bf16")
+    big = np.zeros((B, N + 1, V + 5), np.uint16)
+    big[:, 1:, 3:3 + V] = arr
+    t = to_dev(big, "bf16", dev)[:, 1:, 3:3 + V]  # rows 6 bytes off alignment
+    r, o = run_tree_stochastic(arr, "bf16", parent, tokens, 1.0, 4, dev, t=t)
+    compare_tree_stochastic(r, o, "unaligned")
+    # one tree's rows shared by every sequence (stride 0): independent draws
+    trials = 4000
+    one = arr[:1]
+    t = to_dev(one, "bf16", dev).expand(trials, N, V)
+    par = np.broadcast_to(parent[:1], (trials, N)).copy()
+    tok = np.broadcast_to(tokens[:1], (trials, N)).copy()
+    r, o = run_tree_stochastic(np.broadcast_to(one, (trials, N, V)), "bf16", par, tok, 1.0, 4,
+                               dev, t=t)
+    near, flipped = compare_tree_stochastic(r, o, "broadcast")
+    assert flipped <= 2
+
+
+def test_tree_stochastic_chain_equals_stochastic_on_gpu(dev):
+    """A chain tree against stochastic verify with one-hot draft rows."""
+    rng = np.random.default_rng(72)
+    B, k, V = 40, 6, 5000
+    x = (rng.standard_normal((B, k + 1, V)) * 4).astype(np.float32)
+    am = np.argmax(x, -1)
+    drafts = np.where(rng.random((B, k)) < 0.7, am[:, :k],
+                      rng.integers(0, V, (B, k))).astype(np.int32)
+    tokens = np.concatenate([np.zeros((B, 1), np.int32), drafts], 1)
+    parent = np.tile(np.arange(-1, k, dtype=np.int32), (B, 1))
+    r, o = run_tree_stochastic(x, "f32", parent, tokens, 1.0, 9, dev)
+    compare_tree_stochastic(r, o, "chain")
+    d = np.full((B, k, V), -np.inf, np.float32)
+    for b in range(B):
+        d[b, np.arange(k), drafts[b]] = 0.0
+    s = sv.stochastic(to_dev(x, "f32", dev), to_dev(d, "f32", dev),
+                      torch.from_numpy(drafts).to(dev), 1.0, 9)
+    m = np.where(np.isnan(o["margins"]), np.inf, o["margins"])
+    clear = ~((m < TOL_MARGIN).any(1) | (o["gaps"] < TOL_GAP))
+    np.testing.assert_array_equal(s["accepted_len"].cpu().numpy()[clear],
+                                  r["accepted_len"].cpu().numpy()[clear])
+    np.testing.assert_array_equal(s["out_tokens"].cpu().numpy()[clear],
+                                  r["out_tokens"].cpu().numpy()[clear])
+
+
+def test_tree_stochastic_flags_and_clean_workspace(dev):
+    rng = np.random.default_rng(73)
+    arr, parent, tokens = stoch_tree_case(rng, 8, 12, 400, "f32")
+    parent[2, 5] = 11   # forward pointer
+    parent[6, 3] = -2   # negative
+    tokens[:, 1] = np.where(np.arange(8) % 2 == 0, 400, -1)  # invalid tokens
+    parent[:, 1] = 0    # ... under the root, so the walk examines them
+    ws = sv.Workspace(dev)
+    r, o = run_tree_stochastic(arr, "f32", parent, tokens, 1.0, 2, dev, workspace=ws)
+    compare_tree_stochastic(r, o, "flags")
+    assert o["invalid_tree"]
+    want = sv.SV_FLAG_INVALID_TREE | sv.SV_FLAG_INVALID_TOKEN
+    assert int(np.bitwise_or.reduce(o["flags"])) & want == want
+    assert ws.device_status(clear=True) == int(np.bitwise_or.reduce(o["flags"]))
+    assert int(ws.buf[256:].cpu().count_nonzero()) == 0
+    # the clean workspace serves the other modes next
+    w = workloads.make_stochastic(5, 3, 3000, "bf16", "f32", seed=19)
+    r2 = sv.stochastic(to_dev(w["target"], "bf16", dev), to_dev(w["draft"], "f32", dev),
+                       torch.from_numpy(w["tokens"]).to(dev), w["temperature"], w["seed"],
+                       probs=True, workspace=ws)
+    o2 = oracle.verify_stochastic(w["target"], "bf16", w["draft"], "f32", w["tokens"],
+                                  w["temperature"], w["seed"])
+    compare_stochastic(r2, o2, 3, "after tree")
+    r3, o3 = run_tree_stochastic(arr, "f32", parent, tokens, 0.9, 5, dev, seq_offset=77,
+                                 workspace=ws)
+    compare_tree_stochastic(r3, o3, "again")
+    torch.cuda.synchronize()
+    ws.device_status(clear=True)
+    assert int(ws.buf[256:].cpu().count_nonzero()) == 0
+
+
 # ------------------------------------------------------------ device commit
 
 @pytest.mark.parametrize("B,k,cap", [(1, 0, 4), (7, 1, 9), (300, 8, 40), (33, 32, 100),
@@ -650,6 +789,12 @@ def test_named_workload_full_size(dev, name):
                                     w["threshold"], threads=THREADS)
         near = compare_threshold(r, o, w["threshold"])
         print(f"{name}: near ties {near}")
+    elif mode == "tree_stochastic":
+        r, o = run_tree_stochastic(w["node_logits"], "bf16", w["parent"], w["tokens"],
+                                   w["temperature"], w["seed"], dev)
+        near, flipped = compare_tree_stochastic(r, o, name)
+        print(f"{name}: near ties {near}, of which differing {flipped}; "
+              f"mean accepted {o['accepted_len'].mean():.2f}")
     elif mode == "tree":
         r = sv.tree_greedy(to_dev(w["node_logits"], "bf16", dev),
                            torch.from_numpy(w["parent"]).to(dev),

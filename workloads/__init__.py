@@ -10,8 +10,8 @@ greedy and lookahead workloads).
 Logit arrays are numpy arrays: float32 for "f32", uint16 bf16 bit patterns
 for "bf16".  ``as_torch`` turns one into a torch tensor of the right dtype.
 
-The five named workloads (sizes, distributions, temperatures and seeds of the
-verify step they stand for):
+The named workloads (sizes, distributions, temperatures and seeds of the
+verify step they stand for; the first five, plus the profiling cases below):
 
   stoch_b1_k4_v32000_f32   stochastic, B=1 k=4 V=32000, target fp32 ~ N(0, 2^2),
                            draft fp32 = target + N(0, 1), T=1.0, seed 0
@@ -25,6 +25,10 @@ verify step they stand for):
                            half the sequences share a random-length (1..3) prefix
                            of candidate 0 across branches; each other token is the
                            row argmax w.p. 0.6 else uniform, seed 4
+  threshold_b64_k4_v128256, multi_rows_b16_g8_k4_v32000, tree_b64_n26_v128256 and
+  tree_stoch_b64_n26_v128256 (26-node trees of depth <= 3, node rows bf16 ~
+  N(0, 10^2), first child = the row argmax w.p. 0.9, T=1.0, seed 7): see
+  WORKLOADS.
 """
 from __future__ import annotations
 
@@ -56,6 +60,12 @@ WORKLOADS = {
     # an EAGLE-style draft tree per sequence (Top-K children, distinct tokens)
     "tree_b64_n26_v128256": dict(mode="tree", B=64, N=26, V=128256, t_dtype="bf16",
                                  t_std=3.0, p_match=0.7, seed=6),
+    # the same tree shape under stochastic acceptance; sharper rows (sigma 10:
+    # the row maximum holds about 2/3 of the mass) stand for a confident target,
+    # and the first child carries it with probability 0.9
+    "tree_stoch_b64_n26_v128256": dict(mode="tree_stochastic", B=64, N=26, V=128256,
+                                       t_dtype="bf16", t_std=10.0, p_match=0.9,
+                                       temperature=1.0, seed=7),
     # the same lookahead step with each distinct candidate prefix's row once
     "multi_rows_b16_g8_k4_v32000": dict(mode="multi_rows", B=16, G=8, k=4, V=32000,
                                         t_dtype="bf16", t_std=3.0, p_match=0.6,
@@ -334,6 +344,11 @@ def make(name: str, threads: int | None = None, **overrides) -> dict:
         return make_multi_rows(threads=threads, **cfg)
     if mode == "tree":
         return make_tree(threads=threads, **cfg)
+    if mode == "tree_stochastic":
+        T = cfg.pop("temperature")
+        w = make_tree(threads=threads, **cfg)
+        w.update(mode="tree_stochastic", temperature=T)
+        return w
     if mode == "threshold":
         T, tau = cfg.pop("temperature"), cfg.pop("threshold")
         w = make_greedy(threads=threads, **cfg)
