@@ -48,10 +48,20 @@ def _worker(rank, world, port, result_dir):
                                      w["tokens"][b0:b1], w["temperature"], 99, seq_offset=b0)
         acc = gather_rows(torch.from_numpy(r["accepted_len"]), w["B"])
         tok = gather_rows(torch.from_numpy(r["out_tokens"]), w["B"])
+        # a tree batch shards the same way
+        tr = workloads.make_tree(B=5, N=9, V=400, seed=8, threads=1)
+        t0, t1 = shard(tr["B"], rank, world)
+        rt = oracle.verify_tree_stochastic(tr["node_logits"][t0:t1], "bf16",
+                                           tr["parent"][t0:t1], tr["tokens"][t0:t1], 0.8, 41,
+                                           seq_offset=t0)
+        tree_tok = gather_rows(torch.from_numpy(rt["out_tokens"]), tr["B"])
+        tree_path = gather_rows(torch.from_numpy(rt["path"]), tr["B"])
         slowest = max_over_ranks(10.0 + rank)
         if rank == 0:
             np.save(os.path.join(result_dir, "acc.npy"), acc.numpy())
             np.save(os.path.join(result_dir, "tok.npy"), tok.numpy())
+            np.save(os.path.join(result_dir, "tree_tok.npy"), tree_tok.numpy())
+            np.save(os.path.join(result_dir, "tree_path.npy"), tree_path.numpy())
             np.save(os.path.join(result_dir, "slowest.npy"), np.array([slowest]))
     finally:
         dist.destroy_process_group()
@@ -68,4 +78,9 @@ def test_sharded_batch_reproduces_unsharded_result(tmp_path):
                                     w["temperature"], 99)
     np.testing.assert_array_equal(np.load(tmp_path / "acc.npy"), full["accepted_len"])
     np.testing.assert_array_equal(np.load(tmp_path / "tok.npy"), full["out_tokens"])
+    tr = workloads.make_tree(B=5, N=9, V=400, seed=8, threads=1)
+    ft = oracle.verify_tree_stochastic(tr["node_logits"], "bf16", tr["parent"], tr["tokens"],
+                                       0.8, 41)
+    np.testing.assert_array_equal(np.load(tmp_path / "tree_tok.npy"), ft["out_tokens"])
+    np.testing.assert_array_equal(np.load(tmp_path / "tree_path.npy"), ft["path"])
     assert float(np.load(tmp_path / "slowest.npy")[0]) == 11.0
