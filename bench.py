@@ -241,7 +241,8 @@ def run_reference(args, rank: int) -> None:
     dt = time.perf_counter() - t0
     pos = sum(positions(ws[n]) // ws[n]["B"] for n in STEP)  # one sequence of each
     value = pos * args.steps / dt
-    sample = "one sequence of each of the four step workloads per step, in parallel threads"
+    sample = (f"one sequence of each of the {len(STEP)} step workload(s) per step "
+              f"({', '.join(STEP)}), in parallel threads")
     print(json.dumps({
         "impl": "reference", "metric": "verified positions/s", "value": value,
         "unit": "positions/s", "n_gpus": args.gpus, "steps": args.steps,
@@ -295,7 +296,7 @@ def oracle_baseline(ws: dict) -> dict:
         reps += 1
     pos = sum(positions(ws[n]) for n in STEP) * reps
     return {"value": pos / t_total, "unit": "positions/s", "cores": cores, "kind": "oracle",
-            "sample": f"{reps} full step(s): every sequence of the four workloads "
+            "sample": f"{reps} full step(s): every sequence of the {len(STEP)} workload(s) "
                       f"({pos // reps} positions per step), {t_total:.1f} s"}
 
 
