@@ -1,0 +1,128 @@
+"""Host logic of bench.py on CPU: the per-mode position and byte counts, the
+traffic record's gating, the clock-sample parser, the workload selection,
+and the JSON line of the CPU-only reference arm."""
+import datetime
+import json
+import os
+import subprocess
+import sys
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+def test_positions_per_mode():
+    assert bench.positions(dict(mode="stochastic", B=3, k=4)) == 15
+    assert bench.positions(dict(mode="greedy", B=2, k=0)) == 2
+    assert bench.positions(dict(mode="multi", B=2, G=8, k=4)) == 80
+    assert bench.positions(dict(mode="tree", B=5, N=26)) == 130
+    assert bench.positions(dict(mode="tree_stochastic", B=5, N=26)) == 130
+
+
+def test_algorithmic_bytes_per_mode():
+    B, k, V = 2, 3, 10
+    g = dict(mode="greedy", B=B, k=k, V=V, t_dtype="bf16")
+    assert bench.algorithmic_bytes(g, None) == B * (k + 1) * V * 2 + 4 * B * k + 4 * B * (k + 2)
+    m = dict(mode="multi", B=B, G=3, k=k, V=V, t_dtype="f32")
+    assert bench.algorithmic_bytes(m, None) == \
+        B * 3 * (k + 1) * V * 4 + 4 * B * 3 * k + 4 * B * (k + 3)
+    s = dict(mode="stochastic", B=B, k=k, V=V, t_dtype="bf16", d_dtype="f32")
+    acc = np.array([k, 1])  # one sequence accepts everything: its row k is read
+    assert bench.algorithmic_bytes(s, acc) == \
+        B * k * V * (2 + 4) + 1 * V * 2 + 4 * B * k + 4 * B * (k + 2)
+    for mode in ("tree", "tree_stochastic"):
+        t = dict(mode=mode, B=B, N=7, V=V, t_dtype="bf16")
+        assert bench.algorithmic_bytes(t, None) == B * 7 * V * 2 + 8 * B * 7 + 4 * B + 8 * B * 7
+    # rows form: each distinct row once
+    row_of = np.array([[[0, 1], [0, 2]], [[0, 1], [0, 1]]], np.int32)  # B=2, G=2, k+1=2
+    r = dict(mode="multi_rows", B=2, G=2, k=1, V=V, t_dtype="bf16", row_of=row_of)
+    assert bench.algorithmic_bytes(r, None) == \
+        (3 + 2) * V * 2 + 4 * 2 * 2 * 2 + 4 * 2 * 2 * 1 + 4 * 2 * (1 + 3)
+
+
+def test_traffic_record_applies_only_to_its_kernel_sources_and_workload(tmp_path, monkeypatch):
+    rec = {"kernel_source_sha256": bench.kernel_source_hash(), "dram_bytes_per_launch": 123.0}
+    f = tmp_path / "traffic.json"
+    f.write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(f))
+    assert bench.recorded_traffic("stoch_b256_k8_v128256", False) == 123.0
+    assert bench.recorded_traffic("stoch_b256_k8_v128256", True) is None
+    assert bench.recorded_traffic("stoch_b64_k4_v128256", False) is None
+    rec["kernel_source_sha256"] = "0" * 64
+    f.write_text(json.dumps(rec))
+    assert bench.recorded_traffic("stoch_b256_k8_v128256", False) is None
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(tmp_path / "missing.json"))
+    assert bench.recorded_traffic("stoch_b256_k8_v128256", False) is None
+
+
+def test_committed_traffic_record_matches_the_sources():
+    with open(bench.TRAFFIC_FILE) as f:
+        rec = json.load(f)
+    assert rec["kernel_source_sha256"] == bench.kernel_source_hash()
+    assert rec["kernel_sources"] == list(bench.DOMINANT_SOURCES)
+
+
+class _Done:
+    def terminate(self):
+        pass
+
+    def wait(self, timeout=None):
+        return 0
+
+    def kill(self):
+        pass
+
+    def join(self, timeout=None):
+        pass
+
+
+def test_clock_sampler_keeps_samples_inside_the_window():
+    cs = object.__new__(bench.ClockSampler)
+    cs.proc, cs.thread = _Done(), _Done()
+    t0 = datetime.datetime(2026, 1, 2, 3, 4, 5)
+
+    def line(dt, mhz, reasons):
+        ts = (t0 + datetime.timedelta(seconds=dt)).strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+        flags = ["Active" if r in reasons else "Not Active" for r in bench.ClockSampler.REASONS]
+        return ", ".join([ts, str(mhz), "1965", "700.0", "0x0"] + flags)
+
+    cs.lines = [line(-1.0, 1000, {"hw_slowdown"}),  # before the window: ignored
+                line(0.2, 1965, set()), line(0.4, 1950, {"sw_power_cap"}),
+                line(0.6, 1965, set()), "garbage", line(5.0, 500, {"hw_thermal_slowdown"})]
+    out = cs.stop(t0.timestamp(), t0.timestamp() + 1.0)
+    assert out == {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"],
+                   "samples": 3}
+
+
+def test_select_workloads(monkeypatch):
+    monkeypatch.setattr(bench, "STEP", list(bench.STEP))
+    monkeypatch.setattr(bench, "DOMINANT", bench.DOMINANT)
+    with pytest.raises(SystemExit):
+        bench.select_workloads("no_such_workload")
+    bench.select_workloads("tree_stoch_b64_n26_v128256")
+    assert bench.STEP == ["tree_stoch_b64_n26_v128256"]
+    assert bench.DOMINANT == "tree_stoch_b64_n26_v128256"
+
+
+def test_reference_arm_prints_one_json_line():
+    p = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--only", "stoch_b1_k4_v32000_f32", "--steps", "2", "--warmup", "3"],
+                       capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert p.returncode == 0, p.stderr[-2000:]
+    lines = [ln for ln in p.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["steps"] == 2 and d["warmup"] == 3
+    assert d["value"] > 0 and d["higher_is_better"] is True
+    assert d["config"]["workload"].endswith("stoch_b1_k4_v32000_f32")
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
