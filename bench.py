@@ -321,6 +321,7 @@ def run_ours(args, rank: int, world: int, dist) -> None:
     over = {"B": args.batch} if args.batch else {}
     ws = {n: workloads.make(n, threads=threads, **over) for n in STEP}
     calls, host, devbuf = {}, {}, {}
+    extra = {n: [] for n in STEP}  # further inputs: (pinned host, device) pairs
     for name in STEP:
         w = ws[name]
         key = "rows" if "rows" in w else ("node_logits" if "node_logits" in w else "target")
@@ -350,17 +351,23 @@ def run_ours(args, rank: int, world: int, dist) -> None:
             fn = (lambda w=w, t=t_d, tok=tok_d, o=out, wsp=wsp:
                   sv.threshold(t, tok, w["temperature"], w["threshold"], out=o, workspace=wsp))
         elif w["mode"] == "tree":
-            par = torch.from_numpy(w["parent"]).to(dev)
+            par_h = torch.from_numpy(w["parent"]).pin_memory()
+            par = par_h.to(dev)
+            extra[name].append((par_h, par))
             fn = (lambda t=t_d, pa=par, tok=tok_d, o=out, wsp=wsp:
                   sv.tree_greedy(t, pa, tok, out=o, workspace=wsp))
         elif w["mode"] == "tree_stochastic":
-            par = torch.from_numpy(w["parent"]).to(dev)
+            par_h = torch.from_numpy(w["parent"]).pin_memory()
+            par = par_h.to(dev)
+            extra[name].append((par_h, par))
             off = rank * B
             fn = (lambda w=w, t=t_d, pa=par, tok=tok_d, o=out, wsp=wsp, off=off:
                   sv.tree_stochastic(t, pa, tok, w["temperature"], w["seed"], off, out=o,
                                      workspace=wsp))
         elif w["mode"] == "multi_rows":
-            rmap = torch.from_numpy(w["row_of"]).to(dev)
+            rmap_h = torch.from_numpy(w["row_of"]).pin_memory()
+            rmap = rmap_h.to(dev)
+            extra[name].append((rmap_h, rmap))
             fn = (lambda t=t_d, rm=rmap, tok=tok_d, o=out, wsp=wsp:
                   sv.multi_candidate_rows(t, rm, tok, out=o, workspace=wsp))
         else:
@@ -466,6 +473,7 @@ def run_ours(args, rank: int, world: int, dist) -> None:
             t_h, d_h, tok_h, out_h = host[name]
             h2d += t_h.numel() * t_h.element_size() + tok_h.numel() * 4
             h2d += d_h.numel() * d_h.element_size() if d_h is not None else 0
+            h2d += sum(h.numel() * h.element_size() for h, _ in extra[name])
             d2h += sum(v.numel() * 4 for v in out_h.values())
 
         def e2e_step():
@@ -476,6 +484,8 @@ def run_ours(args, rank: int, world: int, dist) -> None:
                 tok_d.copy_(tok_h, non_blocking=True)
                 if d_h is not None:
                     d_d.copy_(d_h, non_blocking=True)
+                for h, dv in extra[name]:
+                    dv.copy_(h, non_blocking=True)
                 calls[name]()
                 for kk, v in out.items():
                     out_h[kk].copy_(v, non_blocking=True)
