@@ -16,6 +16,7 @@ import torch
 import oracle
 import speculative_decoding_verification_88_b200 as sv
 import workloads
+from tree_checks import valid_tree_outcome
 
 pytestmark = pytest.mark.gpu
 
@@ -407,6 +408,11 @@ def compare_tree_stochastic(r, o, what=""):
         f"{what}: {bad.size} mismatches outside near ties, first b={bad[0]}: gpu n={acc[bad[0]]} "
         f"path={path[bad[0]]} tok={tok[bad[0]]} oracle n={o['accepted_len'][bad[0]]} "
         f"path={o['path'][bad[0]]} tok={o['out_tokens'][bad[0]]}")
+    # where a near tie went the other way, the GPU's outcome must still be a
+    # possible one
+    for b in np.nonzero(mism & near)[0]:
+        assert valid_tree_outcome(o["inputs"][0][b], o["inputs"][1][b], o["inputs"][2], acc[b],
+                                  path[b], tok[b], not (o["flags"][b] & 2)), (what, b)
     return int(near.sum()), int((mism & near).sum())
 
 
@@ -417,6 +423,7 @@ def run_tree_stochastic(arr, dtype, parent, tokens, T, seed, dev, seq_offset=0, 
                            T, seed, seq_offset, workspace=workspace)
     o = oracle.verify_tree_stochastic(arr, dtype, parent, tokens, T, seed, seq_offset,
                                       threads=THREADS)
+    o["inputs"] = (parent, tokens, arr.shape[-1])
     torch.cuda.synchronize()
     return r, o
 

@@ -724,6 +724,52 @@ def test_tree_stochastic_sure_and_impossible_children():
     assert np.isinf(r["margins"][0, 1]) and np.isnan(r["margins"][0, 2])
 
 
+@pytest.mark.parametrize("T", [0.5, 1.0, 2.0])
+def test_tree_stochastic_outcomes_are_valid_walks(T):
+    """Random trees with repeated and invalid sibling tokens and a few bad
+    parents: every outcome is a root path of accepted children, their tokens,
+    and a drawn token outside the final node's children's tokens; and the
+    invariant checker itself rejects corrupted outcomes."""
+    from tree_checks import valid_tree_outcome
+
+    rng = np.random.default_rng(65)
+    B, N, V = 300, 20, 12
+    x = (rng.standard_normal((B, N, V)) * 2.5).astype(np.float32)
+    am = np.argmax(x, -1)
+    parent = np.zeros((B, N), np.int32)
+    tokens = rng.integers(0, V, (B, N)).astype(np.int32)
+    for b in range(B):
+        parent[b] = workloads.tree_parents(N, rng)
+        for j in range(1, N):
+            if rng.random() < 0.5:
+                tokens[b, j] = am[b, parent[b, j]]
+            if rng.random() < 0.03:
+                tokens[b, j] = V + 2
+        if rng.random() < 0.05:
+            parent[b, N - 1] = N + 3
+    r = oracle.verify_tree_stochastic(x, "f32", parent, tokens, T, seed=13)
+    assert r["accepted_len"].max() >= 2
+    for b in range(B):
+        if r["flags"][b] & 2:
+            continue
+        assert valid_tree_outcome(parent[b], tokens[b], V, r["accepted_len"][b], r["path"][b],
+                                  r["out_tokens"][b]), b
+    b = int(np.argmax(r["accepted_len"]))
+    n, path, out = int(r["accepted_len"][b]), r["path"][b].copy(), r["out_tokens"][b].copy()
+    bad = out.copy()
+    bad[0] = (bad[0] + 1) % V  # a committed token that is not the node's
+    assert not valid_tree_outcome(parent[b], tokens[b], V, n, path, bad)
+    bad = path.copy()
+    bad[n], bad[1] = bad[1], bad[n]  # not a parent chain
+    assert not valid_tree_outcome(parent[b], tokens[b], V, n, bad, out)
+    u = int(path[n])
+    kids = [j for j in range(u + 1, N) if parent[b, j] == u and 0 <= tokens[b, j] < V]
+    if kids:
+        bad = out.copy()
+        bad[n] = tokens[b, kids[0]]  # a rejected child's token drawn
+        assert not valid_tree_outcome(parent[b], tokens[b], V, n, path, bad)
+
+
 def test_tree_stochastic_sequence_offset_selects_the_stream():
     rng = np.random.default_rng(64)
     B, N, V = 12, 9, 30
