@@ -62,6 +62,12 @@ def compare_stochastic(r, o, k, what=""):
         f"{what}: {bad.size} mismatches outside near ties, first b={bad[0]}: gpu n={acc[bad[0]]} "
         f"tok={tok[bad[0]]} oracle n={o['accepted_len'][bad[0]]} tok={o['out_tokens'][bad[0]]} "
         f"margins={o['margins'][bad[0]]} gap={o['gaps'][bad[0]]}")
+    if "inputs" in o:  # a near tie that went the other way still gives a valid commit
+        drafts, V = o["inputs"]
+        for b in np.nonzero(mism & near)[0]:
+            n = int(acc[b])
+            assert 0 <= n <= k and (tok[b, :n] == drafts[b, :n]).all(), (what, b)
+            assert 0 <= tok[b, n] < V and (tok[b, n + 1:] == -1).all(), (what, b)
     return int(near.sum()), int((mism & near).sum())
 
 
@@ -75,6 +81,7 @@ def run_stochastic(w, dev, seed=None, seq_offset=0, **views):
     o = oracle.verify_stochastic(views.get("t_np", w["target"]), w["t_dtype"],
                                  views.get("d_np", w["draft"]), w["d_dtype"], w["tokens"], T,
                                  seed, seq_offset, threads=THREADS)
+    o["inputs"] = (w["tokens"], w["target"].shape[-1])
     torch.cuda.synchronize()
     return r, o
 
