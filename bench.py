@@ -143,7 +143,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200", "-i", gpu_id], stdout=subprocess.PIPE,
+                 "-lms", "50", "-i", gpu_id], stdout=subprocess.PIPE,
                 stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
@@ -163,7 +163,14 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
         self.thread.join(timeout=2)
-        sm, smax, reasons, n = [], [], set(), 0
+        return self.summarise(t0, t1)
+
+    def summarise(self, t0: float, t1: float, margin: float = 0.25) -> dict:
+        """Median SM clock, max clock and active throttle reasons of the
+        samples taken inside [t0, t1]; a timed region shorter than the
+        sampling period may hold none, and then the samples within `margin`
+        seconds on either side stand in (reported in "window")."""
+        rows = []
         for line in self.lines:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
@@ -172,9 +179,14 @@ class ClockSampler:
                 ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
             except ValueError:
                 continue
-            if not (t0 <= ts <= t1):
-                continue
-            n += 1
+            rows.append((ts, parts))
+        window = "timed region"
+        sel = [parts for ts, parts in rows if t0 <= ts <= t1]
+        if not sel:
+            sel = [parts for ts, parts in rows if t0 - margin <= ts <= t1 + margin]
+            window = f"no sample inside the timed region; samples within {margin} s of it"
+        sm, smax, reasons = [], [], set()
+        for parts in sel:
             try:
                 sm.append(float(parts[1]))
                 smax.append(float(parts[2]))
@@ -185,7 +197,7 @@ class ClockSampler:
                     reasons.add(name)
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": n}
+                "reasons": sorted(reasons), "samples": len(sel), "window": window}
 
 
 # --------------------------------------------------------------- reference

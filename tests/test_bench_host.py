@@ -96,7 +96,11 @@ def test_clock_sampler_keeps_samples_inside_the_window():
                 line(0.6, 1965, set()), "garbage", line(5.0, 500, {"hw_thermal_slowdown"})]
     out = cs.stop(t0.timestamp(), t0.timestamp() + 1.0)
     assert out == {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"],
-                   "samples": 3}
+                   "samples": 3, "window": "timed region"}
+    # a region shorter than the sampling period: the neighbouring samples stand in
+    out = cs.summarise(t0.timestamp() + 0.25, t0.timestamp() + 0.3)
+    assert out["samples"] == 2 and out["sm_mhz"] == 1957.5
+    assert out["window"].startswith("no sample inside")
 
 
 def test_select_workloads(monkeypatch):
