@@ -51,7 +51,10 @@ def _load():
     global _lib
     with _lock:
         if _lib is None:
-            lib = ctypes.CDLL(build())
+            # SV_ORACLE_LIB names another build of this same source with one
+            # planted mistake; the planted-mistake tests run the pins against
+            # it to show that they catch the mistake.
+            lib = ctypes.CDLL(os.environ.get("SV_ORACLE_LIB") or build())
             P = ctypes.c_void_p
             i64, i32, u32, u64, dbl = (ctypes.c_int64, ctypes.c_int, ctypes.c_uint32,
                                        ctypes.c_uint64, ctypes.c_double)

@@ -16,6 +16,8 @@ def pytest_configure(config):
 def pytest_collection_modifyitems(config, items):
     # gpu tests are skipped, not failed, when no GPU is present and the run
     # did not select them explicitly
+    if config.option.markexpr.strip() == "not gpu":
+        return  # deselected anyway: no need to import torch to ask for a GPU
     try:
         import torch
         have_gpu = torch.cuda.is_available()

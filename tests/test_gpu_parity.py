@@ -49,6 +49,14 @@ def near_ties(o, k):
     return near
 
 
+def near_tie_bound(B):
+    """Most sequences a test may excuse as near ties: the oracle flags a
+    sequence with probability about 1e-4 or less on these inputs (a margin or
+    a gap below 1e-5), so more than this means a broken report or an input
+    that does not test what it should."""
+    return max(2, B // 100)
+
+
 def compare_stochastic(r, o, k, what=""):
     acc = r["accepted_len"].cpu().numpy()
     tok = r["out_tokens"].cpu().numpy()
@@ -56,6 +64,7 @@ def compare_stochastic(r, o, k, what=""):
         np.testing.assert_allclose(r["probs"].cpu().numpy(), o["probs"], atol=TOL_PROB, rtol=0,
                                    err_msg=what)
     near = near_ties(o, k)
+    assert near.sum() <= near_tie_bound(len(near)), f"{what}: {near.sum()} near ties"
     mism = (acc != o["accepted_len"]) | (tok != o["out_tokens"]).any(axis=1)
     bad = np.nonzero(mism & ~near)[0]
     assert bad.size == 0, (
@@ -405,6 +414,7 @@ def compare_tree_stochastic(r, o, what=""):
     TOL_GAP); returns (near ties, near ties that differ)."""
     m = np.where(np.isnan(o["margins"]), np.inf, o["margins"])
     near = (m < TOL_MARGIN).any(axis=1) | (o["gaps"] < TOL_GAP)
+    assert near.sum() <= near_tie_bound(len(near)), f"{what}: {near.sum()} near ties"
     acc = r["accepted_len"].cpu().numpy()
     path = r["path"].cpu().numpy()
     tok = r["out_tokens"].cpu().numpy()
