@@ -11,7 +11,9 @@ multi-candidate):
   multi_b16_g8_k4_v32000   multi-candidate, bf16 [16,8,5,32000]
 
 Metric: verified positions per second (positions = B (k+1), or B G (k+1)),
-whole job over all GPUs.  Inputs are resident in HBM and 1.45 GB are
+whole job over all GPUs.  The latency-bound single-sequence workload
+stoch_b1_k4_v32000_f32 (fp32 [1,5,32000] + [1,4,32000]) is timed on its own,
+outside the step, and reported in per_workload as microseconds per call.  Inputs are resident in HBM and 1.45 GB are
 streamed per step, more than L2 (126 MB), so no buffer is re-read from L2
 across steps.  Usage:
 
@@ -43,8 +45,11 @@ import numpy as np  # noqa: E402
 
 STEP = ["greedy_b64_k4_v128256", "stoch_b64_k4_v128256", "stoch_b256_k8_v128256",
         "multi_b16_g8_k4_v32000"]
+LATENCY = ["stoch_b1_k4_v32000_f32"]  # timed alone, outside the step
 DOMINANT = "stoch_b256_k8_v128256"
 HBM_FALLBACK_GBS = 6650.0
+HBM_NOMINAL_GBS = 8000.0  # the ~8 TB/s the metric quotes
+NEAR_TIE = 1e-5
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic_stochastic_verify_b256_k8.json")
 TREE_MODES = ("tree", "tree_stochastic")
 
@@ -57,13 +62,10 @@ def positions(w: dict) -> int:
     return w["B"] * w.get("G", 1) * (w["k"] + 1)
 
 
-def algorithmic_bytes(w: dict, accepted_len: np.ndarray | None) -> int:
-    """Bytes the method must move for one call (logits + tokens + outputs).
-
-    Stochastic: rows 0..k-1 of target and draft always; target row k only for
-    sequences that accept all k drafts (it feeds nothing else).  The re-read
-    of the rejected pair for the correction is not counted.
-    """
+def full_bytes(w: dict) -> int:
+    """Bytes of one call when every logit row is read once, rows past the
+    first rejection included (the per-call count of the measurement plan),
+    plus tokens in and results out."""
     from workloads import ELEM_BYTES
 
     st = ELEM_BYTES[w["t_dtype"]]
@@ -81,8 +83,39 @@ def algorithmic_bytes(w: dict, accepted_len: np.ndarray | None) -> int:
         distinct = sum(len(np.unique(w["row_of"][b])) for b in range(B))
         return distinct * V * st + 4 * B * G * (k + 1) + 4 * B * G * k + 4 * B * (k + 3)
     sd = ELEM_BYTES[w["d_dtype"]]
-    n_full = int((accepted_len == k).sum()) if accepted_len is not None else B
-    return B * k * V * (st + sd) + n_full * V * st + 4 * B * k + 4 * B * (k + 2)
+    return B * (k + 1) * V * st + B * k * V * sd + 4 * B * k + 4 * B * (k + 2)
+
+
+def needed_bytes(w: dict, outcome: dict | None) -> int | None:
+    """Bytes the method must read for the outcome the ORACLE computed: rows
+    past the first rejection (or a branch's first mismatch) decide nothing.
+
+    stochastic: row pairs 0..n_b (the rejected pair once), and target row k
+                alone when n_b = k;
+    greedy:     target rows 0..n_b;
+    multi:      rows 0..n_{b,g} of every branch g;
+    other modes: the full count.  None without an oracle outcome.
+    """
+    from workloads import ELEM_BYTES
+
+    if outcome is None:
+        return None
+    if w["mode"] not in ("stochastic", "greedy", "multi"):
+        return full_bytes(w)
+    st = ELEM_BYTES[w["t_dtype"]]
+    B, k, V = w["B"], w["k"], w["V"]
+    if w["mode"] == "greedy":
+        rows = int((np.asarray(outcome["accepted_len"]) + 1).sum())
+        return rows * V * st + 4 * B * k + 4 * B * (k + 2)
+    if w["mode"] == "multi":
+        G = w["G"]
+        rows = int((np.asarray(outcome["branch_len"]) + 1).sum())
+        return rows * V * st + 4 * B * G * k + 4 * B * (k + 3)
+    sd = ELEM_BYTES[w["d_dtype"]]
+    n = np.asarray(outcome["accepted_len"])
+    pairs = int(np.minimum(n + 1, k).sum())
+    n_full = int((n == k).sum())
+    return pairs * V * (st + sd) + n_full * V * st + 4 * B * k + 4 * B * (k + 2)
 
 
 def measured_hbm_peak() -> tuple[float, str]:
@@ -271,45 +304,91 @@ def run_reference(args, rank: int) -> None:
 
 # --------------------------------------------------------------------- ours
 
-def oracle_baseline(ws: dict) -> dict:
-    """The CPU oracle on one full step (all sequences of the four workloads),
-    all host cores; repeated while under 5 s of wall time (at most 3 times)."""
+def oracle_call(w: dict, threads: int) -> dict:
+    """The CPU oracle on every sequence of one workload."""
+    import oracle
+
+    if w["mode"] == "stochastic":
+        return oracle.verify_stochastic(w["target"], w["t_dtype"], w["draft"], w["d_dtype"],
+                                        w["tokens"], w["temperature"], w["seed"],
+                                        threads=threads)
+    if w["mode"] == "greedy":
+        return oracle.verify_greedy(w["target"], w["t_dtype"], w["tokens"], threads=threads)
+    if w["mode"] == "multi_rows":
+        return oracle.verify_multi_rows(w["rows"], w["t_dtype"], w["row_of"], w["tokens"],
+                                        threads=threads)
+    if w["mode"] == "tree":
+        return oracle.verify_tree_greedy(w["node_logits"], w["t_dtype"], w["parent"],
+                                         w["tokens"], threads=threads)
+    if w["mode"] == "tree_stochastic":
+        return oracle.verify_tree_stochastic(w["node_logits"], w["t_dtype"], w["parent"],
+                                             w["tokens"], w["temperature"], w["seed"],
+                                             threads=threads)
+    if w["mode"] == "threshold":
+        return oracle.verify_threshold(w["target"], w["t_dtype"], w["tokens"], w["temperature"],
+                                       w["threshold"], threads=threads)
+    return oracle.verify_multi(w["target"], w["t_dtype"], w["tokens"], threads=threads)
+
+
+def oracle_baseline(ws: dict) -> tuple[dict, dict]:
+    """The CPU oracle on one full step (all sequences of the step workloads),
+    all host cores; repeated while under 5 s of wall time (at most 3 times).
+    Returns the cpu_baseline record and the oracle's outcome per workload
+    (first repetition)."""
     import oracle
 
     oracle.build()
     cores = os.cpu_count() or 1
-    reps, t_total = 0, 0.0
+    reps, t_total, outcome = 0, 0.0, {}
     while reps < 3 and t_total < 5.0:
         t0 = time.perf_counter()
         for name in STEP:
-            w = ws[name]
-            if w["mode"] == "stochastic":
-                oracle.verify_stochastic(w["target"], w["t_dtype"], w["draft"], w["d_dtype"],
-                                         w["tokens"], w["temperature"], w["seed"],
-                                         threads=cores)
-            elif w["mode"] == "greedy":
-                oracle.verify_greedy(w["target"], w["t_dtype"], w["tokens"], threads=cores)
-            elif w["mode"] == "multi_rows":
-                oracle.verify_multi_rows(w["rows"], w["t_dtype"], w["row_of"], w["tokens"],
-                                         threads=cores)
-            elif w["mode"] == "tree":
-                oracle.verify_tree_greedy(w["node_logits"], w["t_dtype"], w["parent"],
-                                          w["tokens"], threads=cores)
-            elif w["mode"] == "tree_stochastic":
-                oracle.verify_tree_stochastic(w["node_logits"], w["t_dtype"], w["parent"],
-                                              w["tokens"], w["temperature"], w["seed"],
-                                              threads=cores)
-            elif w["mode"] == "threshold":
-                oracle.verify_threshold(w["target"], w["t_dtype"], w["tokens"],
-                                        w["temperature"], w["threshold"], threads=cores)
-            else:
-                oracle.verify_multi(w["target"], w["t_dtype"], w["tokens"], threads=cores)
+            o = oracle_call(ws[name], cores)
+            outcome.setdefault(name, o)
         t_total += time.perf_counter() - t0
         reps += 1
     pos = sum(positions(ws[n]) for n in STEP) * reps
-    return {"value": pos / t_total, "unit": "positions/s", "cores": cores, "kind": "oracle",
-            "sample": f"{reps} full step(s): every sequence of the {len(STEP)} workload(s) "
-                      f"({pos // reps} positions per step), {t_total:.1f} s"}
+    return ({"value": pos / t_total, "unit": "positions/s", "cores": cores, "kind": "oracle",
+             "sample": f"{reps} full step(s): every sequence of the {len(STEP)} workload(s) "
+                       f"({pos // reps} positions per step), {t_total:.1f} s"}, outcome)
+
+
+def branch_lengths(w: dict) -> np.ndarray:
+    """Accepted length of every branch of a multi-candidate workload, from the
+    oracle's greedy verify of each branch on its own rows."""
+    import oracle
+
+    B, G, k = w["B"], w["G"], w["k"]
+    o = oracle.verify_greedy(w["target"].reshape(B * G, k + 1, w["V"]), w["t_dtype"],
+                             w["tokens"].reshape(B * G, k), threads=os.cpu_count() or 1)
+    return o["accepted_len"].reshape(B, G)
+
+
+def parity_record(w: dict, gpu: dict, o: dict) -> dict:
+    """The GPU's outputs of the timed launch configuration against the oracle:
+    exact for greedy and multi-candidate; for stochastic verify exact except
+    sequences where an oracle decision was a near tie (an acceptance margin
+    |u - p/q| at an examined position, or the top-2 Gumbel-max score gap,
+    below 1e-5), which are counted."""
+    keys = [k for k in ("best_candidate", "accepted_len", "out_tokens", "path") if k in gpu]
+    mism = np.zeros(w["B"], bool)
+    for key in keys:
+        g, want = gpu[key], o[key]
+        mism |= (g != want) if g.ndim == 1 else (g != want).any(axis=1)
+    rec = {"sequences": int(w["B"]), "mismatches": int(mism.sum())}
+    if w["mode"] == "stochastic":
+        k, n = w["k"], o["accepted_len"]
+        near = o["gaps"] < NEAR_TIE
+        for b in range(w["B"]):
+            if k > 0:
+                near[b] |= bool((o["margins"][b, : min(int(n[b]), k - 1) + 1] < NEAR_TIE).any())
+        rec.update(near_ties=int(near.sum()),
+                   mismatches_outside_near_ties=int((mism & ~near).sum()),
+                   min_gap=float(o["gaps"].min()),
+                   rule="exact except near ties (oracle margin or gap < 1e-5)")
+    else:
+        rec["rule"] = "bit-exact"
+    return rec
 
 
 def run_ours(args, rank: int, world: int, dist) -> None:
@@ -331,10 +410,11 @@ def run_ours(args, rank: int, world: int, dist) -> None:
     # inputs (seeded, synthetic; each rank its own batch through seq_offset)
     threads = max(1, (os.cpu_count() or 1) // max(1, world))
     over = {"B": args.batch} if args.batch else {}
-    ws = {n: workloads.make(n, threads=threads, **over) for n in STEP}
+    lat = [n for n in LATENCY if n not in STEP] if not args.only else []
+    ws = {n: workloads.make(n, threads=threads, **over) for n in STEP + lat}
     calls, host, devbuf = {}, {}, {}
-    extra = {n: [] for n in STEP}  # further inputs: (pinned host, device) pairs
-    for name in STEP:
+    extra = {n: [] for n in STEP + lat}  # further inputs: (pinned host, device) pairs
+    for name in STEP + lat:
         w = ws[name]
         key = "rows" if "rows" in w else ("node_logits" if "node_logits" in w else "target")
         t_h = workloads.as_torch(w[key], w["t_dtype"]).pin_memory()
@@ -390,13 +470,13 @@ def run_ours(args, rank: int, world: int, dist) -> None:
                                         for kk, v in out.items()})
         devbuf[name] = (t_d, d_d, tok_d, out)
 
-    # warm-up, then the accepted lengths that fix the stochastic byte counts
+    # warm-up; the outputs of these calls (the launch configuration timed
+    # below) are kept for the parity record
     for _ in range(max(1, args.warmup)):
-        for name in STEP:
+        for name in STEP + lat:
             calls[name]()
     torch.cuda.synchronize()
-    alg = {n: algorithmic_bytes(ws[n], devbuf[n][3]["accepted_len"].cpu().numpy())
-           for n in STEP}
+    gpu_out = {n: {kk: v.cpu().numpy() for kk, v in devbuf[n][3].items()} for n in STEP + lat}
 
     # One step as a CUDA graph, the way a serving loop issues it: the four
     # verify launches back to back with no host work between them.  External
@@ -459,20 +539,67 @@ def run_ours(args, rank: int, world: int, dist) -> None:
         for name in STEP:
             a, b = ev[name]
             samples[name].append(a.elapsed_time(b))
-    per = {}
-    for name in STEP:
-        us = statistics.fmean(samples[name]) * 1e3
-        per[name] = {"us_per_call": round(us, 2),
-                     "positions_per_s": positions(ws[name]) / (us * 1e-6),
-                     "algorithmic_bytes": alg[name],
-                     "alg_gbs": alg[name] / (us * 1e-6) / 1e9}
+    us_call = {n: statistics.fmean(samples[n]) * 1e3 for n in STEP}
+
+    # latency-bound workloads: one call per graph, replayed back to back
+    for name in lat:
+        g1 = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(gstream):
+            calls[name]()
+        gstream.synchronize()
+        with torch.cuda.graph(g1, stream=gstream):
+            calls[name]()
+        for _ in range(5):
+            g1.replay()
+        reps = 500
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record(stream)
+        for _ in range(reps):
+            g1.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        us_call[name] = a.elapsed_time(b) * 1e3 / reps
+
+    # the oracle on the host cores: the CPU baseline, the outcomes that fix
+    # the bytes each call must read, and the parity of the GPU's outputs
+    cpu, outcome = None, None
+    if rank == 0 and world == 1 and not args.skip_cpu_baseline:
+        cpu, outcome = oracle_baseline(ws)
+        for name in lat:
+            outcome[name] = oracle_call(ws[name], os.cpu_count() or 1)
+        for name in STEP + lat:
+            if ws[name]["mode"] == "multi":
+                outcome[name]["branch_len"] = branch_lengths(ws[name])
+
     peak, peak_kind = measured_hbm_peak()
-    for name in STEP:
-        per[name]["frac_of_hbm_peak"] = per[name]["alg_gbs"] / peak
+    per = {}
+    for name in STEP + lat:
+        us = us_call[name]
+        full = full_bytes(ws[name])
+        need = needed_bytes(ws[name], outcome[name] if outcome else None)
+        rec = {"us_per_call": round(us, 2), "positions_per_s": positions(ws[name]) / (us * 1e-6),
+               "in_step": name in STEP, "full_read_bytes": full,
+               "full_read_gbs": full / (us * 1e-6) / 1e9}
+        rec["frac_full_read"] = rec["full_read_gbs"] / peak
+        if need is not None:
+            rec["needed_bytes"] = need
+            rec["needed_gbs"] = need / (us * 1e-6) / 1e9
+            rec["frac_needed"] = rec["needed_gbs"] / peak
+            rec["frac_needed_of_nominal"] = rec["needed_gbs"] / HBM_NOMINAL_GBS
+            rec["parity"] = parity_record(ws[name], gpu_out[name], outcome[name])
+        per[name] = rec
     d = per[DOMINANT]
-    roofline = {"bound": "hbm", "achieved": d["alg_gbs"], "peak": peak, "unit": "GB/s",
-                "frac": d["alg_gbs"] / peak,
+    counted = "needed_gbs" if "needed_gbs" in d else "full_read_gbs"
+    roofline = {"bound": "hbm", "achieved": d[counted], "peak": peak, "unit": "GB/s",
+                "frac": d[counted] / peak,
                 "traffic": recorded_traffic(DOMINANT, bool(args.batch)),
+                "bytes_counted": ("needed: the rows the oracle's outcome requires (pairs "
+                                  "0..n, target row k only when n = k)"
+                                  if counted == "needed_gbs" else
+                                  "full read: every logit row once"),
+                "achieved_full_read": d["full_read_gbs"],
+                "frac_of_nominal_8tbs": d[counted] / HBM_NOMINAL_GBS,
                 "kernel": KERNEL_OF_MODE[ws[DOMINANT]["mode"]] + " (" + DOMINANT + ")",
                 "peak_source": peak_kind + " (MEASURED_PEAKS.json hbm_gbs)"
                 if peak_kind == "measured" else "fallback 6.65 TB/s"}
@@ -521,12 +648,8 @@ def run_ours(args, rank: int, world: int, dist) -> None:
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": e_ms}
 
-    cpu = None
-    if rank == 0 and world == 1 and not args.skip_cpu_baseline:
-        cpu = oracle_baseline(ws)
-
     if rank == 0:
-        total_bytes = sum(alg.values())
+        total_bytes = sum(per[n].get("needed_bytes", per[n]["full_read_bytes"]) for n in STEP)
         print(json.dumps({
             "metric": "verified positions/s", "value": value, "unit": "positions/s",
             "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": ms_step,
@@ -536,8 +659,11 @@ def run_ours(args, rank: int, world: int, dist) -> None:
             "config": {"workload": "spec_verify step: " + " + ".join(STEP),
                        "global_batch": sum(ws[n]["B"] for n in STEP) * world,
                        "positions_per_step": pos_step * world,
-                       "algorithmic_bytes_per_step": total_bytes,
-                       "step_alg_gbs": total_bytes / (ms_step * 1e-3) / 1e9,
+                       "bytes_per_step": total_bytes,
+                       "step_gbs": total_bytes / (ms_step * 1e-3) / 1e9,
+                       "latency_workloads": lat,
+                       "latency_note": "timed alone, one call per replayed graph; not in the "
+                                       "step or its positions/s",
                        "l2": "inputs larger than L2: 1.45 GB streamed per step, no buffer "
                              "re-read across steps from L2",
                        "parallelism": f"weak: {world} GPU(s), each its own batch, no collective",
