@@ -65,6 +65,9 @@ typedef enum {
 #define SV_FLAG_INVALID_ROW 8u       /* a row map entry was outside [0, R); see the rows form */
 #define SV_FLAG_CAPACITY 16u         /* spec_verify_commit: a token buffer was full */
 #define SV_FLAG_INVALID_TREE 32u     /* a tree node's parent was outside [0, node) */
+#define SV_FLAG_BOUNDS 64u           /* bounds-checked builds (SV_DEBUG_BOUNDS) only: a
+                                        kernel formed an index outside its buffer; the
+                                        access was skipped and the outputs are invalid */
 
 /*
  * Bytes of workspace that calls with these sizes need (any mode, any dtype).
@@ -117,7 +120,14 @@ int spec_verify_read_device_status(void *workspace, uint32_t *flags_host, int cl
  * accepted_len   [B] out: n in [0, k]
  * out_tokens     [B, k+1] out: drafts 0..n-1, the sampled token at n, -1 after
  * probs_out      [B, k, 2] out, may be NULL: p_i(x_i), q_i(x_i) (0 for an
- *                invalid token)
+ *                invalid token) for every position up to the first
+ *                rejection; a later position holds either its values or
+ *                (-1, -1), when its rows were retired without being read
+ *
+ * Rows past a known rejection decide nothing, so the kernel does not read
+ * them: positions are scheduled position by position over the batch, and a
+ * chunk of row pair i of a sequence that already has a rejection before i is
+ * retired unread.  The results are the same bits either way.
  */
 int spec_verify_stochastic(const void *target_logits, int t_dtype, int64_t t_stride_b,
                            int64_t t_stride_pos, const void *draft_logits, int d_dtype,
@@ -137,7 +147,8 @@ int spec_verify_stochastic(const void *target_logits, int t_dtype, int64_t t_str
  *
  * target_logits [B, k+1, V] (strides as above), draft_tokens [B, k];
  * accepted_len [B] out; out_tokens [B, k+1] out: drafts 0..n-1, the argmax
- * of row n at n, -1 after.
+ * of row n at n, -1 after.  A draft token outside [0, V) never matches and
+ * raises SV_FLAG_INVALID_TOKEN (as it does in spec_verify_multi_candidate).
  */
 int spec_verify_greedy(const void *target_logits, int t_dtype, int64_t t_stride_b,
                        int64_t t_stride_pos, const int32_t *draft_tokens, int B, int k, int V,
@@ -340,23 +351,36 @@ int spec_verify_philox4x32_10(const uint32_t *counters, int64_t n, uint64_t seed
  * workspace: the library uses a fixed device array of
  * SV_NOALLOC_SCRATCH_BYTES that it carries in its image (every GPU that loads
  * the library holds it until the process exits).  Each call clears the part
- * it needs with cudaMemsetAsync on `stream`, then runs greedy verify on it;
- * nothing is allocated or freed.
+ * it needs with cudaMemsetAsync on `stream` (all but the sticky status word),
+ * then runs greedy verify on it; nothing is allocated or freed.
  *  - Returns SV_ERR_WORKSPACE when spec_verify_workspace_size(B, 1, k, V)
- *    exceeds SV_NOALLOC_SCRATCH_BYTES (about B <= 512 at k = 8, V = 128256),
- *    SV_ERR_INVALID_ARG for sizes outside the limits, and otherwise what
- *    spec_verify_greedy returns.
- *  - The first call on each device looks up the array's address
- *    (cudaGetSymbolAddress with that device current); make it before any
+ *    exceeds SV_NOALLOC_SCRATCH_BYTES (at V = 128256: B <= 782 at k = 8,
+ *    B <= 1448 at k = 4, B <= 208 at k = 32), SV_ERR_INVALID_ARG for sizes
+ *    outside the limits, and otherwise what spec_verify_greedy returns.
+ *  - Every call looks up the array's device address (cudaGetSymbolAddress,
+ *    host-side, with the caller's device current); the first call on a device
+ *    also loads the library's device code there, so make it before any
  *    stream capture.
  *  - All calls share the array: calls whose kernels may overlap on the GPU
  *    (unordered streams) race.  Order them on one stream.
+ *  - Errors seen on the device (SV_FLAG_* bits: a draft token outside [0, V),
+ *    a device wait that timed out) accumulate in the array's status word;
+ *    read them with spec_verify_greedy_noalloc_read_device_status.
  */
 #define SV_NOALLOC_SCRATCH_BYTES ((size_t)2 << 20)
 
 int spec_verify_greedy_noalloc(const void *target_logits, int t_dtype, int64_t t_stride_b,
                                int64_t t_stride_pos, const int32_t *draft_tokens, int B, int k,
                                int V, int32_t *accepted_len, int32_t *out_tokens, void *stream);
+
+/*
+ * The sticky device status word (SV_FLAG_* bits) of spec_verify_greedy_noalloc
+ * on the current device: copied into *flags_host (a host pointer) and, if
+ * `clear` is nonzero, reset.  SYNCHRONISES `stream`; allocates nothing.  No
+ * counterpart on the pages.
+ */
+int spec_verify_greedy_noalloc_read_device_status(uint32_t *flags_host, int clear,
+                                                  void *stream);
 
 #ifdef __cplusplus
 }

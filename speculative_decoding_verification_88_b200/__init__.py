@@ -24,6 +24,7 @@ from .build import LIB_PATH
 SV_F32, SV_BF16 = 0, 1
 SV_FLAG_INVALID_TOKEN, SV_FLAG_RESIDUAL_FALLBACK, SV_FLAG_TIMEOUT = 1, 2, 4
 SV_FLAG_INVALID_ROW, SV_FLAG_CAPACITY, SV_FLAG_INVALID_TREE = 8, 16, 32
+SV_FLAG_BOUNDS = 64  # raised by the bounds-checked build only
 
 # Entry points declared in include/spec_verify.h.
 EXPORTS = (
@@ -32,6 +33,7 @@ EXPORTS = (
     "spec_verify_multi_candidate", "spec_verify_multi_candidate_rows", "spec_verify_commit",
     "spec_verify_tree_workspace_size", "spec_verify_tree_greedy", "spec_verify_threshold",
     "spec_verify_philox4x32_10", "spec_verify_greedy_noalloc",
+    "spec_verify_greedy_noalloc_read_device_status",
     "spec_verify_tree_stochastic_workspace_size", "spec_verify_tree_stochastic",
 )
 
@@ -48,17 +50,20 @@ def library_path() -> str:
     return LIB_PATH
 
 
-def load_library():
-    """Load libspecverify.so (raises if it has not been built)."""
+def load_library(path: str | None = None):
+    """Load libspecverify.so (raises if it has not been built).  `path` loads
+    another build of the same library (the bounds-checked one) and returns it
+    without making it the default."""
     global _lib
     with _lock:
-        if _lib is not None:
+        if path is None and _lib is not None:
             return _lib
-        if not os.path.exists(LIB_PATH):
+        target = path or LIB_PATH
+        if not os.path.exists(target):
             raise SpecVerifyError(
-                f"{LIB_PATH} is missing: build it with "
+                f"{target} is missing: build it with "
                 "`python -m speculative_decoding_verification_88_b200.build`")
-        lib = ctypes.CDLL(LIB_PATH)
+        lib = ctypes.CDLL(target)
         P, I, I64, U32, U64, SZ, F = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64,
                                       ctypes.c_uint32, ctypes.c_uint64, ctypes.c_size_t,
                                       ctypes.c_float)
@@ -98,7 +103,10 @@ def load_library():
         lib.spec_verify_philox4x32_10.restype = I
         lib.spec_verify_greedy_noalloc.argtypes = [P, I, I64, I64, P, I, I, I, P, P, P]
         lib.spec_verify_greedy_noalloc.restype = I
-        _lib = lib
+        lib.spec_verify_greedy_noalloc_read_device_status.argtypes = [ctypes.POINTER(U32), I, P]
+        lib.spec_verify_greedy_noalloc_read_device_status.restype = I
+        if path is None:
+            _lib = lib
         return lib
 
 
@@ -483,6 +491,19 @@ def greedy_noalloc(target: torch.Tensor, draft_tokens: torch.Tensor, *,
     _check(code, "spec_verify_greedy_noalloc")
     _count()
     return res
+
+
+def greedy_noalloc_device_status(clear: bool = True, device=None, stream=None) -> int:
+    """Sticky SV_FLAG_* bits raised on the device by greedy_noalloc calls on
+    `device` (synchronises the stream; allocates nothing)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else \
+        torch.device(device)
+    v = ctypes.c_uint32(0)
+    with torch.cuda.device(dev):
+        _check(load_library().spec_verify_greedy_noalloc_read_device_status(
+            ctypes.byref(v), int(clear), _stream_ptr(stream, dev)),
+            "spec_verify_greedy_noalloc_read_device_status")
+    return int(v.value)
 
 
 def philox4x32_10(counters: torch.Tensor, seed: int, stream=None) -> torch.Tensor:

@@ -18,6 +18,10 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_DIR = os.path.join(PKG, "_lib")
 LIB_PATH = os.path.join(LIB_DIR, "libspecverify.so")
+# The same sources built with every global index checked against its buffer
+# (SV_DEBUG_BOUNDS): a violation raises SV_FLAG_BOUNDS instead of an access.
+# For tests, in place of a memory checker; never the default library.
+BOUNDS_LIB_PATH = os.path.join(LIB_DIR, "libspecverify_bounds.so")
 
 SOURCES = ["sv_api.cu", "sv_kernels.cu", "sv_noalloc.cu", "sv_tree_stoch.cu"]
 HEADERS = [os.path.join(CSRC, h) for h in ("sv_internal.h", "sv_device.cuh")] + [
@@ -38,27 +42,31 @@ def nvcc_path() -> str:
     raise RuntimeError("nvcc not found; set NVCC or add the CUDA toolkit to PATH")
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB_PATH):
+def _stale(path: str = LIB_PATH) -> bool:
+    if not os.path.exists(path):
         return True
-    t = os.path.getmtime(LIB_PATH)
+    t = os.path.getmtime(path)
     deps = [os.path.join(CSRC, s) for s in SOURCES] + HEADERS + [os.path.abspath(__file__)]
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False, extra_flags: list[str] | None = None) -> str:
-    """Compile the library if a source is newer than it (or `force`)."""
-    if not force and not _stale():
-        return LIB_PATH
+def build(force: bool = False, verbose: bool = False, extra_flags: list[str] | None = None,
+          bounds: bool = False) -> str:
+    """Compile the library if a source is newer than it (or `force`);
+    `bounds` builds the bounds-checked variant instead."""
+    path = BOUNDS_LIB_PATH if bounds else LIB_PATH
+    if not force and not _stale(path):
+        return path
     os.makedirs(LIB_DIR, exist_ok=True)
-    tmp = LIB_PATH + f".tmp{os.getpid()}"
-    cmd = [nvcc_path(), *NVCC_FLAGS, *(extra_flags or []), f"-I{INCLUDE}", f"-I{CSRC}",
+    tmp = path + f".tmp{os.getpid()}"
+    flags = [*(extra_flags or []), *(["-DSV_DEBUG_BOUNDS"] if bounds else [])]
+    cmd = [nvcc_path(), *NVCC_FLAGS, *flags, f"-I{INCLUDE}", f"-I{CSRC}",
            "-o", tmp, *[os.path.join(CSRC, s) for s in SOURCES]]
     if verbose:
         print(" ".join(cmd))
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB_PATH)
-    return LIB_PATH
+    os.replace(tmp, path)
+    return path
 
 
 if __name__ == "__main__":

@@ -4,6 +4,8 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <initializer_list>
+#include <utility>
 
 #include "spec_verify.h"
 #include "sv_internal.h"
@@ -41,11 +43,20 @@ bool stride16(long long stride, int es) { return ((stride * es) % 16) == 0; }
 
 size_t seq_bytes(int B) { return static_cast<size_t>(B) * sizeof(SeqRec); }
 
+// Elements a strided view spans: one past its last element.
+long long span(std::initializer_list<std::pair<long long, long long>> dims, int V) {
+  long long last = V - 1;
+  for (const auto& d : dims) last += (d.first - 1) * d.second;  // (extent, stride)
+  return last + 1;
+}
+
 // Partial slots (8 bytes each) and row counters (4 bytes each):
-//   stochastic: chunk [B][k][nch][2], row [B][k][2], phase-2 [B][nch], rc [B][k]
-//   argmax:     chunk [B][R][nch], row [B][R], rc [B][R]   (R = G (k+1))
+//   stochastic: chunk [B][k][nch][2], row [B][k][2], phase-2 [B][nch],
+//               ready list [B], rc [B][k]
+//   argmax:     chunk [B][R][nch], row [B][R], rc [B][R], branch state [rows]
+//               (R = G (k+1))
 struct StochLayout {
-  size_t p1, r1, p2, rc, bytes;  // offsets from the tail, in bytes
+  size_t p1, r1, p2, list, rc, bytes;  // offsets from the tail, in bytes
 };
 StochLayout stochastic_layout(int B, int k, int nch) {
   StochLayout l;
@@ -53,19 +64,23 @@ StochLayout stochastic_layout(int B, int k, int nch) {
   l.p1 = 0;
   l.r1 = l.p1 + bk * nch * 2 * 8;
   l.p2 = l.r1 + bk * 2 * 8;
-  l.rc = l.p2 + static_cast<size_t>(B) * nch * 8;
+  l.list = l.p2 + static_cast<size_t>(B) * nch * 8;
+  l.rc = l.list + static_cast<size_t>(B) * 8;
   l.bytes = l.rc + (bk * 4 + 15) / 16 * 16;
   return l;
 }
 struct ArgLayout {
-  size_t slots, rkey, rc, bytes;
+  size_t slots, rkey, rc, dead, bytes;
 };
+// dead holds one word per (sequence, branch); `rows` words bound it in
+// every mode.
 ArgLayout argmax_layout(long long rows, int nch) {
   ArgLayout l;
   l.slots = 0;
   l.rkey = static_cast<size_t>(rows) * nch * 8;
   l.rc = l.rkey + static_cast<size_t>(rows) * 8;
-  l.bytes = l.rc + (static_cast<size_t>(rows) * 4 + 15) / 16 * 16;
+  l.dead = l.rc + (static_cast<size_t>(rows) * 4 + 15) / 16 * 16;
+  l.bytes = l.dead + (static_cast<size_t>(rows) * 4 + 15) / 16 * 16;
   return l;
 }
 
@@ -217,21 +232,9 @@ extern "C" int spec_verify_stochastic(const void* target_logits, int t_dtype,
   const int grid = sm_count();
   if (grid <= 0) return SV_ERR_CUDA;
   const Plan pl = plan_chunks(static_cast<long long>(B) * k, V, st + sd, st < sd ? st : sd, kStochChunkBytes);
-  const long long p1 = static_cast<long long>(k) * pl.nch;
-  long long lag = 0;
-  if (p1 > 0) {
-    // phase-2 chunks of a sequence come about 24 ring-fulls of the whole grid
-    // after its phase-1 chunks: late enough that the sequence is nearly
-    // always finalized (a producer that has to wait for it stalls its compute
-    // group).  Measured on B = 256, k = 8, V = 128256 (ring-fulls -> us):
-    // 6 -> 199.4, 12 -> 194.8, 24 -> 192.4, all of phase 1 first -> 193.3;
-    // at B = 64 every choice is within 1 %.
-    lag = (static_cast<long long>(24 * kStages) * grid + p1 - 1) / p1 + 1;
-    if (lag > B) lag = B;
-  }
-  const long long slot_items = static_cast<long long>(k + 1) * pl.nch;
-  const long long total = static_cast<long long>(B) * slot_items;
-  if (total >= (1ll << 31)) return SV_ERR_INVALID_ARG;
+  const long long total1 = static_cast<long long>(k) * B * pl.nch;
+  const long long total2 = static_cast<long long>(B) * pl.nch;
+  if (total1 + total2 >= (1ll << 31)) return SV_ERR_INVALID_ARG;
 
   const bool tma = aligned(target_logits, 16) && stride16(t_stride_b, st) &&
                    stride16(t_stride_pos, st) &&
@@ -246,6 +249,8 @@ extern "C" int spec_verify_stochastic(const void* target_logits, int t_dtype,
   p.drf = draft_logits;
   p.d_sb = d_stride_b;
   p.d_sp = d_stride_pos;
+  p.t_elems = span({{B, t_stride_b}, {k + 1, t_stride_pos}}, V);
+  p.d_elems = k > 0 ? span({{B, d_stride_b}, {k, d_stride_pos}}, V) : 0;
   p.tokens = draft_tokens;
   p.B = B;
   p.k = k;
@@ -259,15 +264,10 @@ extern "C" int spec_verify_stochastic(const void* target_logits, int t_dtype,
   p.probs = probs_out;
   p.ch = pl.ch;
   p.nch = pl.nch;
-  p.lag = static_cast<int>(lag);
-  p.p1_items = static_cast<unsigned int>(p1);
-  p.slot_items = static_cast<unsigned int>(slot_items);
-  p.a_end = static_cast<unsigned int>(lag * p1);
-  p.b_end = p.a_end + static_cast<unsigned int>((B - lag) * slot_items);
-  p.total = static_cast<unsigned int>(total);
-  p.div_p1 = make_udiv(p1 > 0 ? p.p1_items : 1u);
-  p.div_slot = make_udiv(p.slot_items);
+  p.total1 = static_cast<unsigned int>(total1);
+  p.total2 = static_cast<unsigned int>(total2);
   p.div_nch = make_udiv(static_cast<unsigned int>(pl.nch));
+  p.div_B = make_udiv(static_cast<unsigned int>(B));
   p.ctrl = ws.ctrl;
   p.seq = ws.seq;
   const StochLayout lay = stochastic_layout(B, k, pl.nch);
@@ -276,6 +276,7 @@ extern "C" int spec_verify_stochastic(const void* target_logits, int t_dtype,
   p.r1 = reinterpret_cast<unsigned long long*>(tail + lay.r1);
   p.p2 = reinterpret_cast<unsigned long long*>(tail + lay.p2);
   p.rc = reinterpret_cast<unsigned int*>(tail + lay.rc);
+  p.list = reinterpret_cast<unsigned long long*>(tail + lay.list);
   const cudaError_t e = launch_stochastic(p, t_dtype, d_dtype, tma, grid, kernel_smem_bytes(),
                                           static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? SV_OK : SV_ERR_CUDA;
@@ -326,6 +327,7 @@ static int argmax_call(const void* target_logits, int t_dtype, int64_t sb, int64
   p.sb = sb;
   p.sg = sg;
   p.sp = sp;
+  p.t_elems = R > 0 ? span({{B, sb}, {R, sg}}, V) : span({{B, sb}, {G, sg}, {k + 1, sp}}, V);
   p.tokens = tokens;
   p.B = B;
   p.G = G;
@@ -342,6 +344,8 @@ static int argmax_call(const void* target_logits, int t_dtype, int64_t sb, int64
   p.nch = pl.nch;
   p.div_seq = make_udiv(static_cast<unsigned int>(rows_per_seq) * static_cast<unsigned int>(pl.nch));
   p.div_nch = make_udiv(static_cast<unsigned int>(pl.nch));
+  p.div_bg = make_udiv(static_cast<unsigned int>(B) * static_cast<unsigned int>(G));
+  p.div_g = make_udiv(static_cast<unsigned int>(G));
   p.total = static_cast<unsigned int>(total);
   p.ctrl = ws.ctrl;
   p.seq = ws.seq;
@@ -358,6 +362,7 @@ static int argmax_call(const void* target_logits, int t_dtype, int64_t sb, int64
   p.slots = reinterpret_cast<unsigned long long*>(tail + lay.slots);
   p.rkey = reinterpret_cast<unsigned long long*>(tail + lay.rkey);
   p.rc = reinterpret_cast<unsigned int*>(tail + lay.rc);
+  p.dead = reinterpret_cast<unsigned int*>(tail + lay.dead);
   const cudaError_t e = launch_argmax(p, t_dtype, tma, grid, kernel_smem_bytes(),
                                       static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? SV_OK : SV_ERR_CUDA;

@@ -16,12 +16,41 @@ constexpr unsigned int kFlagTimeout = 4u;
 constexpr unsigned int kFlagInvalidRow = 8u;
 constexpr unsigned int kFlagCapacity = 16u;
 constexpr unsigned int kFlagInvalidTree = 32u;
+constexpr unsigned int kFlagBounds = 64u;  // bounds-checked builds only
 
 // A device wait gives up after this long (ns) and raises kFlagTimeout.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
 constexpr float kLn2 = 0.693147180559945309f;
 constexpr float kLog2e = 1.442695040888963407f;
+
+// ------------------------------------------------------------ bounds checks
+// A build with SV_DEBUG_BOUNDS defined checks every global index the kernels
+// form (logit offsets of each chunk and gather, workspace slots, tokens,
+// outputs) against the extent of its buffer.  A violation raises
+// kFlagBounds in the status word, records the first offending source line in
+// the control block's first spare word, and the access is skipped, so that an
+// index error shows up as a status bit rather than a fault.  Release builds
+// compile every check to `true`.
+#ifdef SV_DEBUG_BOUNDS
+static __device__ __noinline__ void bounds_fail(Ctrl* ctrl, int line) {
+  atomicOr(&ctrl->flags, kFlagBounds);
+  atomicCAS(&ctrl->pad[0], 0u, static_cast<unsigned int>(line));
+}
+#define SV_IN(ctrl, idx, n)                                                      \
+  ((static_cast<long long>(idx) >= 0 && static_cast<long long>(idx) < static_cast<long long>(n)) \
+       ? true                                                                    \
+       : (::sv::bounds_fail((ctrl), __LINE__), false))
+// [lo, lo + len) inside [0, n)
+#define SV_IN_RANGE(ctrl, lo, len, n)                                            \
+  ((static_cast<long long>(lo) >= 0 &&                                           \
+    static_cast<long long>(lo) + static_cast<long long>(len) <= static_cast<long long>(n)) \
+       ? true                                                                    \
+       : (::sv::bounds_fail((ctrl), __LINE__), false))
+#else
+#define SV_IN(ctrl, idx, n) true
+#define SV_IN_RANGE(ctrl, lo, len, n) true
+#endif
 
 // ------------------------------------------------------------ PTX helpers
 
@@ -122,19 +151,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return done != 0;
 }
 
-// Non-blocking test of phase `parity`.
-__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t done;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(done)
-      : "r"(smem_addr(bar)), "r"(parity)
-      : "memory");
-  return done != 0;
-}
-
 __device__ __forceinline__ unsigned int ld_acquire_u32(const unsigned int* p) {
   unsigned int v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -143,6 +159,10 @@ __device__ __forceinline__ unsigned int ld_acquire_u32(const unsigned int* p) {
 
 __device__ __forceinline__ void st_release_u32(unsigned int* p, unsigned int v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void st_release_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
 __device__ __forceinline__ unsigned int ld_relaxed_u32(const unsigned int* p) {
@@ -235,8 +255,8 @@ __device__ __forceinline__ float accept_uniform(uint32_t w) {
 // 1), because small E are the ones that win.  So:
 //   v <  1/8 (w >= 0xE0000000):  lg2(1 - v) = -v g(v), g(v) = -ln(1 - v) / (v ln 2),
 //              with g the degree-4 polynomial that interpolates it at the five
-//              Chebyshev nodes of [0, 1/8] (relative error 1.4e-8, 8e-8 with
-//              fp32 rounding);
+//              Chebyshev nodes of [0, 1/8] (relative error 1.4e-8; 1.37e-7,
+//              about 2 ulp, after the fp32 Horner steps);
 //   v >= 1/8:  the hardware lg2 of u', whose absolute error (about 2^-22.6)
 //              is below 1e-6 relative here, since |lg2 u'| >= 0.19.
 constexpr float kOneMinusHalfUlp = 1.0f - 0x1p-24f;

@@ -43,22 +43,24 @@ __host__ __device__ constexpr int full_chunk_entries(int bytes, int bpe, int es_
 
 // Device-wide control words at the start of the workspace (256 bytes).
 struct Ctrl {
-  unsigned int ticket;  // next work ticket (reset by the last CTA to leave)
-  unsigned int exits;   // CTAs that took their last ticket
-  unsigned int flags;   // sticky SV_FLAG_* bits
-  unsigned int pad[61];
+  unsigned int ticket;    // next work ticket (phase 1 of stochastic verify)
+  unsigned int exits;     // producers that took their last ticket
+  unsigned int flags;     // sticky SV_FLAG_* bits
+  unsigned int ticket2;   // stochastic: next phase-2 ticket
+  unsigned int resolved;  // stochastic: sequences whose accepted length is known
+  unsigned int pad[59];   // (all counters are reset by the last producer to leave)
 };
 static_assert(sizeof(Ctrl) == 256, "Ctrl must be 256 bytes");
 
 // Per-sequence record (64 bytes), zero between calls: the kernel that sets
 // a field also clears it.
 struct SeqRec {
-  unsigned int cnt1;       // rows merged (phase 1, or all rows for argmax)
-  unsigned int cnt2;       // phase-2 chunks published
-  unsigned int ready;      // phase 1 finalized (accepted length known)
-  int n;                   // accepted length
-  float mt, ist, md, isd;  // row n: max (log2 units) and 1/sum of p and q
-  unsigned int pad[8];
+  unsigned int cnt1;         // argmax: rows merged
+  unsigned int cnt2;         // stochastic: phase-2 chunks published
+  unsigned long long state;  // stochastic: rows decided (bits 0..31), rows rejected (32..63)
+  float mt, ist, md, isd;    // stochastic: row n max (log2 units) and 1/sum, of p and of q
+  int n;                     // stochastic: accepted length
+  unsigned int pad[7];
 };
 static_assert(sizeof(SeqRec) == 64, "SeqRec must be 64 bytes");
 
@@ -107,6 +109,7 @@ struct StochParams {
   long long t_sb, t_sp;
   const void* drf;
   long long d_sb, d_sp;
+  long long t_elems, d_elems;  // elements the target / draft views span (bounds checks)
   const int* tokens;  // [B, k]
   int B, k, V;
   float c2;    // log2(e) / T: logit -> log2-domain scale
@@ -114,29 +117,33 @@ struct StochParams {
   int* accepted_len;
   int* out_tokens;
   float* probs;  // nullable
-  int ch, nch, lag;
-  // Ticket map, three runs with no unused ticket: [0, a_end) phase-1 chunks
-  // of sequences 0..lag-1 (k * nch each); [a_end, b_end) slots of
-  // slot_items = (k + 1) * nch tickets, slot s >= lag holding the phase-1
-  // chunks of sequence s and then the phase-2 chunks of sequence s - lag;
-  // [b_end, total) phase-2 chunks of sequences B-lag..B-1 (nch each).
-  unsigned int p1_items;    // k * nch
-  unsigned int slot_items;  // (k + 1) * nch
-  unsigned int a_end, b_end, total;
-  UDiv div_p1, div_slot, div_nch;  // ticket decode: / p1_items, / slot_items, / nch
+  int ch, nch;
+  // Tickets.  Phase 1 (counter ticket): chunk t % nch of row pair t / nch,
+  // position-major -- position i = row / B of sequence b = row % B -- so that
+  // every sequence's pair i comes a whole position block (B nch tickets)
+  // after its pair i - 1, late enough for a rejection before it to be known
+  // and the pair to be retired unread.  Phase 2 (counter ticket2): chunk
+  // t % nch of the sequence in ready-list entry t / nch, the list filled in
+  // the order the sequences' accepted lengths become known.
+  unsigned int total1;   // k B nch
+  unsigned int total2;   // B nch
+  UDiv div_nch, div_B;   // / nch, / B
   Ctrl* ctrl;
   SeqRec* seq;
   // Partials, published with one 64-bit store each and never zero once
   // written (so the value is its own "ready" flag):
   unsigned long long* p1;  // [B][k][nch][2]: chunk (max, sum) of target, of draft
-  unsigned long long* r1;  // [B][k][2]: row (max, sum) of target, of draft
+  unsigned long long* r1;  // [B][k][2]: row (max, sum) of target, of draft; written for
+                           // rejected rows only, for the sequence's resolution
   unsigned long long* p2;  // [B][nch]: chunk Gumbel-max key, 1 = no candidate
   unsigned int* rc;        // [B][k]: chunks of a row published
+  unsigned long long* list;  // [B] ready list: (b + 1) | n << 32, in resolution order
 };
 
 struct ArgmaxParams {
   const void* tgt;
   long long sb, sg, sp;  // rows form: sg is the row stride, sp unused
+  long long t_elems;     // elements the logits view spans (bounds checks)
   const int* tokens;     // [B, G, k]
   int B, G, k, V;
   int R;                 // rows per sequence: G * (k + 1), the distinct rows of the rows
@@ -155,13 +162,22 @@ struct ArgmaxParams {
   int* accepted_len;
   int* out_tokens;
   int ch, nch;
-  UDiv div_seq, div_nch;  // ticket decode: / (R * nch), / nch
+  // Ticket decode.  Plain mode (greedy, multi-candidate) is position-major:
+  // ticket t is chunk t % nch of row t / nch, taken as (position, sequence,
+  // branch) with the branch fastest, so that every branch's row i comes a
+  // whole position block (B G nch tickets) after its row i - 1.  The other
+  // modes go sequence by sequence: / (R * nch), then / nch.
+  UDiv div_seq, div_nch, div_bg, div_g;  // / (R * nch), / nch, / (B * G), / G
   unsigned int total;
   Ctrl* ctrl;
   SeqRec* seq;
   unsigned long long* slots;  // [B][R][nch] chunk argmax keys
   unsigned long long* rkey;   // [B][R] row argmax keys
   unsigned int* rc;           // [B][R] chunks of a row published
+  // Plain mode: per (sequence, branch), 64 - the smallest position found so
+  // far whose draft differs from the row argmax (0: none yet).  Rows past it
+  // decide nothing, and their chunks are retired without being read.
+  unsigned int* dead;         // [B][G]
 };
 
 // dtype codes follow sv_dtype (0 = f32, 1 = bf16).  Return cudaError_t.

@@ -65,16 +65,34 @@
 
 namespace sv {
 
-enum : int { kKindEnd = 0, kKindStats = 1, kKindCorrection = 2, kKindBonus = 3, kKindArgmax = 4 };
+enum : int {
+  kKindEnd = 0,
+  kKindStats = 1,
+  kKindCorrection = 2,
+  kKindBonus = 3,
+  kKindArgmax = 4,
+  kKindRowDone = 5  // no data: the producer retired the last chunks of row (b, i) unread
+};
 
-// Tickets per atomicAdd (the next grab's atomic is always in flight).
-// Argmax chunks are uniform work, so larger grabs save atomics; stochastic
-// tickets are taken one at a time, which balances the uneven phase-1 and
-// phase-2 chunks best (grabs of 2 and 3 measured 3% and 19% slower on
-// B = 256, k = 8, V = 128256).
-constexpr unsigned int kGrabStoch = 1;
-constexpr unsigned int kGrabArgmax = 8;
+// Argmax tickets per atomicAdd (the next grab's atomic is always in
+// flight): argmax chunks are uniform work, so larger grabs save atomics.
+// Stochastic tickets are taken one at a time, which balances the uneven
+// phase-1 and phase-2 chunks best.
+#ifndef SV_GRAB_ARGMAX
+#define SV_GRAB_ARGMAX 8
+#endif
+constexpr unsigned int kGrabArgmax = SV_GRAB_ARGMAX;
+// Producers of the argmax kernels: 1 (warp 0 alternates the two groups'
+// stages) or 2 (one per compute group, each filling its own two stages).
+#ifndef SV_ARGMAX_PRODUCERS
+#define SV_ARGMAX_PRODUCERS 1
+#endif
+constexpr int kArgmaxProducers = SV_ARGMAX_PRODUCERS;
+static_assert(kArgmaxProducers == 1 || kArgmaxProducers == kComputeGroups, "1 or one per group");
 constexpr unsigned long long kNoCandidate = 1ull;  // phase-2 key: no positive residual
+// Argmax chunk key of a chunk retired unread: below every real key (whose
+// high word is at least orderable(-inf) > 0), and never zero.
+constexpr unsigned long long kSkippedKey = 1ull;
 
 struct Hdr {
   int kind;
@@ -87,6 +105,7 @@ struct Hdr {
   int nvec_d;  // full 16-byte draft vectors in shared memory
   long long toff;          // element offset of entry x0 in the target
   long long doff;          // element offset of entry x0 in the draft
+  int slot;                // phase 2: the sequence's ready-list entry
 };
 
 struct Shared {
@@ -356,7 +375,10 @@ __device__ __forceinline__ void load_vecs(const unsigned char* smem, int nvec, i
 // One pair in kPolyEvery of the register-resident exponentials runs on the FMA
 // pipe (ex2_poly_x2) instead of the special-function unit, which the
 // statistics otherwise saturate.
-constexpr int kPolyEvery = 8;
+#ifndef SV_POLY_EVERY
+#define SV_POLY_EVERY 8
+#endif
+constexpr int kPolyEvery = SV_POLY_EVERY;
 
 // Warp merge of per-thread (m, s) pairs of two tensors: the maxima first,
 // then one rescale per thread and a plain sum.
@@ -735,7 +757,30 @@ __device__ __forceinline__ void chunk_argmax(const unsigned char* smem, const Hd
 
 // ============================================================ stochastic
 
-// Place a chunk in the next ring stage (waits for the stage to be free).
+// Chunk statistics of a chunk retired unread (a NaN maximum, which no real
+// chunk has): never zero, and it marks its row as not reduced in full.
+constexpr unsigned long long kSkippedStats = 0x7fc00000ull;
+
+// Rows decided / rejected, packed in the sequence state word.
+__device__ __forceinline__ unsigned int decided_bits(unsigned long long st) {
+  return static_cast<unsigned int>(st);
+}
+__device__ __forceinline__ unsigned int rejected_bits(unsigned long long st) {
+  return static_cast<unsigned int>(st >> 32);
+}
+__device__ __forceinline__ unsigned int low_mask(int n) {  // bits 0..n-1, n <= 32
+  return n >= 32 ? 0xffffffffu : (1u << n) - 1u;
+}
+// First rejection n (k when none is known), and whether every row 0..n is
+// decided -- then n is the accepted length.
+__device__ __forceinline__ bool resolved(unsigned long long st, int k, int& n) {
+  const unsigned int rej = rejected_bits(st);
+  n = rej ? __ffs(rej) - 1 : k;
+  const unsigned int need = low_mask(n < k ? n + 1 : k);
+  return (decided_bits(st) & need) == need;
+}
+
+// Place a chunk in the next stage of group g's ring (waits for the stage).
 template <typename TT, typename TD, bool kTma>
 __device__ __forceinline__ bool stoch_issue(const StochParams& p, Shared& sh,
                                             unsigned char* stages, int g, uint32_t& used,
@@ -744,6 +789,10 @@ __device__ __forceinline__ bool stoch_issue(const StochParams& p, Shared& sh,
   h.len = min(p.ch, p.V - h.x0);
   h.toff = static_cast<long long>(h.b) * p.t_sb + static_cast<long long>(h.i) * p.t_sp + h.x0;
   h.doff = static_cast<long long>(h.b) * p.d_sb + static_cast<long long>(h.i) * p.d_sp + h.x0;
+  if (!SV_IN(p.ctrl, h.b, p.B) || !SV_IN(p.ctrl, h.i, p.k + 1) || !SV_IN(p.ctrl, h.c, p.nch) ||
+      !SV_IN_RANGE(p.ctrl, h.toff, h.len, p.t_elems))
+    h.toff = 0;  // (bounds-checked builds: a bad chunk reads the first row instead)
+  if (h.kind != kKindBonus && !SV_IN_RANGE(p.ctrl, h.doff, h.len, p.d_elems)) h.doff = 0;
   const int s = group_stage(g, used);
   if (!mbar_wait(&sh.empty[s], group_phase(used) ^ 1u, p.ctrl)) return false;
   issue_chunk<TT, TD, kTma>(sh, stages + static_cast<size_t>(s) * kStageBytes, s, h, p.tgt,
@@ -752,22 +801,35 @@ __device__ __forceinline__ bool stoch_issue(const StochParams& p, Shared& sh,
   return true;
 }
 
-// Phase-2 chunk c of sequence b.  `ready` is the sequence's published flag,
-// n + 1, already acquired (load + fence) by the caller.  The correction's row
+// A data-free item into group g's next stage: row (b, i) is complete (its
+// last chunks were retired unread) and its epilogue merges it.
+__device__ __forceinline__ bool stoch_push_row_done(Shared& sh, int g, uint32_t& used, int b,
+                                                    int i, Ctrl* ctrl) {
+  const int s = group_stage(g, used);
+  if (!mbar_wait(&sh.empty[s], group_phase(used) ^ 1u, ctrl)) return false;
+  sh.hdr[s].kind = kKindRowDone;
+  sh.hdr[s].b = b;
+  sh.hdr[s].i = i;
+  mbar_arrive(&sh.full[s]);
+  ++used;
+  return true;
+}
+
+// Phase-2 chunk c of sequence b, whose accepted length n is known (the
+// ready-list entry was acquired by the caller).  The correction's row
 // statistics travel with the chunk as a 16-byte bulk copy.
 template <typename TT, typename TD, bool kTma>
 __device__ __forceinline__ bool stoch_issue_phase2(const StochParams& p, Shared& sh,
                                                    unsigned char* stages, int g,
-                                                   uint32_t& used, int b, int c,
-                                                   unsigned int ready) {
+                                                   uint32_t& used, int b, int n, int c,
+                                                   int slot) {
   Hdr h;
   h.b = b;
   h.c = c;
-  // clamped so that no workspace content can steer a read outside the tensors
-  const int n = p.k > 0 ? min(max(static_cast<int>(ready) - 1, 0), p.k) : 0;
-  h.i = n;
+  h.slot = slot;
+  h.i = min(max(n, 0), p.k);  // clamped: no workspace content steers a read out of bounds
   const float4* stat = nullptr;
-  if (n < p.k) {
+  if (h.i < p.k) {
     h.kind = kKindCorrection;
     stat = reinterpret_cast<const float4*>(&p.seq[b].mt);
     if (kTma) fence_proxy_async_global();
@@ -777,127 +839,183 @@ __device__ __forceinline__ bool stoch_issue_phase2(const StochParams& p, Shared&
   return stoch_issue<TT, TD, kTma>(p, sh, stages, g, used, h, stat);
 }
 
-// Producer of compute group g.  It takes tickets kGrabStoch at a time (the
-// next grab's atomic in flight meanwhile) and decodes each by multiply-high
-// divisions along the three runs of the ticket map (StochParams): phase-1
-// chunk (i, c) of a sequence, or phase-2 chunk c of a sequence `lag` slots
-// back.  A phase-2 chunk whose sequence is not ready yet is set aside (at most
-// kDefer); set-aside chunks are polled together with relaxed loads and issued
-// once ready.
+// Producer of compute group g: phase-1 chunks in position-major ticket order,
+// phase-2 chunks from the ready list, the latter first whenever one is ready.
+//  - Phase-1 tickets are taken one at a time, two ahead, and the state word
+//    of each ticket's sequence is loaded one ticket ahead: a chunk of pair i
+//    whose sequence already has a rejection before i is retired unread (its
+//    two slots get kSkippedStats and it is counted on its row; if that
+//    completes the row, a data-free item hands the row to the epilogue).
+//  - Up to kDefer phase-2 tickets are held; their ready-list entries are
+//    polled with relaxed loads (issued before the current chunk's stage wait,
+//    read at the next iteration) and a chunk is issued once its entry is
+//    visible.  When no phase-1 ticket is left, the producer waits (bounded)
+//    for the oldest held entry.
 template <typename TT, typename TD, bool kTma>
 __device__ void stoch_producer(const StochParams& p, Shared& sh, unsigned char* stages, int g) {
   constexpr int kDefer = 4;
+  constexpr unsigned int kNone = 0xffffffffu;
   Ctrl* ctrl = p.ctrl;
   const unsigned int nch = static_cast<unsigned int>(p.nch);
+  const unsigned int B = static_cast<unsigned int>(p.B);
   uint32_t used = 0;  // uses of group g's stages issued
   bool ok = true;
-  int db[kDefer], dc[kDefer];  // set-aside phase-2 chunks, oldest first
+  // the state word of the sequence of a phase-1 ticket past position 0
+  auto state_of = [&](unsigned int t) -> unsigned long long {
+    if (t >= p.total1) return 0ull;
+    const unsigned int row = udiv(t, p.div_nch);
+    const unsigned int i = udiv(row, p.div_B);
+    return i > 0u ? ld_relaxed_u64(&p.seq[row - i * B].state) : 0ull;
+  };
+  // The first three phase-1 tickets of every producer are fixed by its index
+  // (no atomic round trip before the first load); the counter hands out the
+  // tickets after them.
+  const unsigned int fixed = gridDim.x * kProducerWarps * 3u;
+  const unsigned int first = (blockIdx.x * kProducerWarps + static_cast<unsigned int>(g)) * 3u;
+  unsigned int t1 = first;
+  unsigned int t1n = first + 1u;
+  unsigned int t1nn = first + 2u;
+  unsigned long long s1 = state_of(t1);
+  unsigned long long s1n = state_of(t1n);
+  unsigned int dt[kDefer];         // held phase-2 tickets, oldest first
+  unsigned long long dv[kDefer];   // their ready-list entries as last polled
   int nd = 0;
-  unsigned int base = atomicAdd(&ctrl->ticket, kGrabStoch), next = 0u, j = 0u;
-  bool prefetched = false;
+  unsigned int t2p = kNone;        // a phase-2 grab in flight
+  bool t2_done = p.total2 == 0u;
+  int sk_b = -1, sk_i = 0;         // a retired chunk whose count is checked later
+  unsigned int sk_old = 0u;
   while (ok) {
-    if (nd > 0) {
-      unsigned int rd[kDefer];
-      bool any = false;
+    // the retired chunk of the previous iteration: did it complete its row?
+    if (sk_b >= 0) {
+      if (sk_old == nch - 1u) ok = stoch_push_row_done(sh, g, used, sk_b, sk_i, ctrl);
+      sk_b = -1;
+      if (!ok) break;
+    }
+    // (the held arrays are indexed with constants only, so they stay in
+    // registers and a poll's load is not waited for until it is read)
+    if (t2p != kNone) {  // the phase-2 grab of the previous iteration joins the queue
+      if (t2p < p.total2) {
+        const unsigned long long v0 =
+            p.k == 0 ? (static_cast<unsigned long long>(udiv(t2p, p.div_nch)) + 1ull) : 0ull;
 #pragma unroll
-      for (int d = 0; d < kDefer; ++d) {
-        rd[d] = d < nd ? ld_relaxed_u32(&p.seq[db[d]].ready) : 0u;
-        any |= rd[d] != 0u;
+        for (int d = 0; d < kDefer; ++d)
+          if (d == nd) {
+            dt[d] = t2p;
+            dv[d] = v0;
+          }
+        ++nd;
+      } else {
+        t2_done = true;
       }
-      if (any) {
-        fence_acq_rel_gpu();
-        int keep = 0;
+      t2p = kNone;
+    }
+    // a held phase-2 chunk whose sequence is ready goes first
+    int rd = -1;
 #pragma unroll
-        for (int d = 0; d < kDefer; ++d) {
-          if (d < nd) {
-            if (ok && rd[d]) {
-              ok = stoch_issue_phase2<TT, TD, kTma>(p, sh, stages, g, used, db[d], dc[d], rd[d]);
-            } else {
-              db[keep] = db[d];
-              dc[keep] = dc[d];
-              ++keep;
-            }
+    for (int d = kDefer - 1; d >= 0; --d)
+      if (d < nd && dv[d] != 0ull) rd = d;
+    if (rd < 0 && t1 >= p.total1 && nd > 0) {
+      // nothing else to do: wait (bounded) for the oldest held entry
+      const unsigned long long* e = p.list + udiv(dt[0], p.div_nch);
+      unsigned long long v = ld_relaxed_u64(e);
+      const unsigned long long w0 = global_ns();
+      for (unsigned int spin = 1; v == 0ull; ++spin) {
+        __nanosleep(64);
+        v = ld_relaxed_u64(e);
+        if ((spin & 63u) == 0u) {
+          if (aborted(ctrl)) break;
+          if (global_ns() - w0 > kWaitLimitNs) {
+            atomicOr(&ctrl->flags, kFlagTimeout);
+            break;
           }
         }
-        nd = keep;
-        if (!ok) break;
       }
-    }
-    if (base >= p.total) {  // no fresh tickets left: wait for the oldest set-aside chunk
-      if (nd == 0) break;
-      if (!wait_flag(&p.seq[db[0]].ready, ctrl)) {
+      if (v == 0ull) {
         ok = false;
         break;
       }
+      dv[0] = v;
+      rd = 0;
+    }
+    // keep up to kDefer phase-2 tickets in hand (the atomic's result is used
+    // at the next iteration)
+    if (!t2_done && nd < kDefer) t2p = atomicAdd(&ctrl->ticket2, 1u);
+    if (rd >= 0) {
+      unsigned long long v = 0ull;
+      unsigned int tsel = 0u;
+#pragma unroll
+      for (int d = 0; d < kDefer; ++d)
+        if (d == rd) {
+          v = dv[d];
+          tsel = dt[d];
+        }
+      const unsigned int slot = udiv(tsel, p.div_nch);
+      const unsigned int c = tsel - slot * nch;
+      if (!SV_IN(ctrl, slot, p.B)) continue;
+#pragma unroll
+      for (int d = 0; d < kDefer - 1; ++d)
+        if (d >= rd && d + 1 < nd) {
+          dt[d] = dt[d + 1];
+          dv[d] = dv[d + 1];
+        }
+      --nd;
+      // poll the rest now; the stage wait below overlaps the round trip
+#pragma unroll
+      for (int d = 0; d < kDefer; ++d)
+        if (d < nd && dv[d] == 0ull) dv[d] = ld_relaxed_u64(p.list + udiv(dt[d], p.div_nch));
+      if (p.k > 0) fence_acq_rel_gpu();  // acquire: the resolver's record is visible
+      // (clamped so that no workspace content can steer a read outside the
+      // tensors)
+      const int b = static_cast<int>(min(static_cast<unsigned int>(v) - 1u, B - 1u));
+      const int n = static_cast<int>(v >> 32);
+      ok = stoch_issue_phase2<TT, TD, kTma>(p, sh, stages, g, used, b, n, static_cast<int>(c),
+                                            static_cast<int>(slot));
       continue;
     }
-    if (!prefetched) {
-      next = atomicAdd(&ctrl->ticket, kGrabStoch);  // overlaps the chunks of this grab
-      prefetched = true;
-    }
-    const unsigned int t = base + j;
-    if (++j == kGrabStoch) {
-      j = 0u;
-      base = next;
-      prefetched = false;
-    }
-    if (t >= p.total) continue;
-    // Decode: sequence sq and offset o within its phase-1 chunks
-    // (o < p1_items), or phase-2 chunk o - p1_items of sequence sq.
-    unsigned int sq, o;
-    if (t < p.a_end) {
-      sq = udiv(t, p.div_p1);
-      o = t - sq * p.p1_items;
-    } else if (t < p.b_end) {
-      const unsigned int u = t - p.a_end;
-      const unsigned int q = udiv(u, p.div_slot);
-      o = u - q * p.slot_items;
-      sq = static_cast<unsigned int>(p.lag) + q - (o < p.p1_items ? 0u : static_cast<unsigned int>(p.lag));
-    } else {
-      const unsigned int u = t - p.b_end;
-      const unsigned int q = udiv(u, p.div_nch);
-      sq = static_cast<unsigned int>(p.B - p.lag) + q;
-      o = p.p1_items + (u - q * nch);
-    }
-    if (o < p.p1_items) {
-      const unsigned int ci = udiv(o, p.div_nch);
+#pragma unroll
+    for (int d = 0; d < kDefer; ++d)
+      if (d < nd && dv[d] == 0ull) dv[d] = ld_relaxed_u64(p.list + udiv(dt[d], p.div_nch));
+    if (t1 < p.total1) {
+      const unsigned int row = udiv(t1, p.div_nch);
+      const unsigned int i = udiv(row, p.div_B);
       Hdr h;
       h.kind = kKindStats;
-      h.b = static_cast<int>(sq);
-      h.i = static_cast<int>(ci);
-      h.c = static_cast<int>(o - ci * nch);
-      ok = stoch_issue<TT, TD, kTma>(p, sh, stages, g, used, h, nullptr);
-    } else {
-      const int b = static_cast<int>(sq);
-      const int c = static_cast<int>(o - p.p1_items);
-      const unsigned int rd = p.k == 0 ? 1u : ld_relaxed_u32(&p.seq[b].ready);
-      if (rd) {
-        if (p.k > 0) fence_acq_rel_gpu();
-        ok = stoch_issue_phase2<TT, TD, kTma>(p, sh, stages, g, used, b, c, rd);
-      } else {
-        if (nd == kDefer) {  // queue full: the oldest must go first
-          const unsigned int r0 = wait_flag(&p.seq[db[0]].ready, ctrl);
-          if (!r0) {
-            ok = false;
-            break;
-          }
-          ok = stoch_issue_phase2<TT, TD, kTma>(p, sh, stages, g, used, db[0], dc[0], r0);
-#pragma unroll
-          for (int d = 1; d < kDefer; ++d) {
-            db[d - 1] = db[d];
-            dc[d - 1] = dc[d];
-          }
-          --nd;
-        }
-        db[nd] = b;
-        dc[nd] = c;
-        ++nd;
+      h.b = static_cast<int>(row - i * B);
+      h.i = static_cast<int>(i);
+      h.c = static_cast<int>(t1 - row * nch);
+      const unsigned int rej = rejected_bits(s1);
+      // advance the ticket pipeline before this chunk's stage wait
+      t1 = t1n;
+      s1 = s1n;
+      t1n = t1nn;
+      s1n = state_of(t1n);
+      t1nn = fixed + atomicAdd(&ctrl->ticket, 1u);
+      if (rej & low_mask(h.i)) {  // a pair before this one was rejected: retire unread
+        if (!SV_IN(ctrl, h.b, p.B) || !SV_IN(ctrl, h.i, p.k) || !SV_IN(ctrl, h.c, p.nch)) continue;
+        unsigned long long* slot =
+            p.p1 + ((static_cast<size_t>(h.b) * p.k + h.i) * nch + h.c) * 2;
+        st_relaxed_u64(slot, kSkippedStats);
+        st_relaxed_u64(slot + 1, kSkippedStats);
+        sk_old = atomicAdd(&p.rc[static_cast<size_t>(h.b) * p.k + h.i], 1u);
+        sk_b = h.b;
+        sk_i = h.i;
+        continue;
       }
+      ok = stoch_issue<TT, TD, kTma>(p, sh, stages, g, used, h, nullptr);
+      continue;
     }
+    if (nd == 0 && t2_done && t2p == kNone) break;  // no work left
+    if (nd == 0 && t2p != kNone) continue;           // a grab in flight
   }
   if (ok) {
     push_group_end(sh, g, used, ctrl);
-    leave_grid(ctrl, kProducerWarps);
+    // the last producer to leave rewinds every counter
+    if (atomicAdd(&ctrl->exits, 1u) == gridDim.x * kProducerWarps - 1) {
+      atomicExch(&ctrl->ticket, 0u);
+      atomicExch(&ctrl->ticket2, 0u);
+      atomicExch(&ctrl->resolved, 0u);
+      atomicExch(&ctrl->exits, 0u);
+    }
   } else if (kTma) {
     drain_group_stages(sh, g, used);
   }
@@ -913,9 +1031,10 @@ __device__ void stoch_compute(const StochParams& p, Shared& sh, unsigned char* s
     const int s = use % kStages;
     if (!mbar_wait(&sh.full[s], (use / kStages) & 1u, p.ctrl)) break;
     const Hdr h = sh.hdr[s];
-    if (h.kind == kKindEnd) {
+    if (h.kind == kKindEnd || h.kind == kKindRowDone) {
       if (lane == 0) mbar_arrive(&sh.rfull[s]);
-      break;
+      if (h.kind == kKindEnd) break;
+      continue;
     }
     const unsigned char* ts = stages + static_cast<size_t>(s) * kStageBytes;
     const unsigned char* ds = ts + static_cast<size_t>(p.ch) * Elem<TT>::kBytes;
@@ -958,48 +1077,24 @@ __device__ __forceinline__ unsigned long long take(unsigned long long* slot, uns
   return v;
 }
 
-// Phase-1 finalize of sequence b (one warp): row statistics of every
-// position, p_i(x_i), q_i(x_i), accept while u_i q < p, publish n.
-template <typename TT, typename TD>
-__device__ void finalize_accept(const StochParams& p, int b, int lane) {
+// Resolution of sequence b (one warp), once its accepted length n is known:
+// the committed drafts and the -1 padding, the row-n statistics for the
+// phase-2 draw (consumed from the rejected row's record), and an entry in the
+// ready list that releases its phase-2 chunks.
+__device__ void resolve_sequence(const StochParams& p, int b, int n, int lane) {
   const int k = p.k;
-  float MT = -INFINITY, ST = 0.0f, MD = -INFINITY, SD = 0.0f;
-  bool acc = true;
-  if (lane < k) {
-    unsigned long long* row = p.r1 + (static_cast<size_t>(b) * k + lane) * 2;
-    const unsigned long long vt0 = ld_relaxed_u64(row), vd0 = ld_relaxed_u64(row + 1);
-    const int x = __ldg(p.tokens + static_cast<size_t>(b) * k + lane);
-    unpack_stats(take(row, vt0, p.ctrl), MT, ST);
-    unpack_stats(take(row + 1, vd0, p.ctrl), MD, SD);
-    const bool valid = x >= 0 && x < p.V;
-    float pt = 0.0f, qd = 0.0f;
-    if (valid) {
-      const float lt = load_elem<TT>(
-          p.tgt, static_cast<long long>(b) * p.t_sb + static_cast<long long>(lane) * p.t_sp + x);
-      const float ld = load_elem<TD>(
-          p.drf, static_cast<long long>(b) * p.d_sb + static_cast<long long>(lane) * p.d_sp + x);
-      pt = ex2f(fmaf(lt, p.c2, -MT)) / ST;
-      qd = ex2f(fmaf(ld, p.c2, -MD)) / SD;
-    } else {
-      atomicOr(&p.ctrl->flags, kFlagInvalidToken);
-    }
-    const uint4 w = philox10(
-        make_uint4(0u, static_cast<uint32_t>(lane), static_cast<uint32_t>(b) + p.seq_offset,
-                   kTagAccept),
-        p.key0, p.key1);
-    acc = valid && (accept_uniform(w.x) * qd < pt);
-    if (p.probs) {
-      float* pr = p.probs + (static_cast<size_t>(b) * k + lane) * 2;
-      pr[0] = pt;
-      pr[1] = qd;
-    }
+  if (!SV_IN(p.ctrl, b, p.B) || !SV_IN(p.ctrl, n, k + 1)) return;
+  float4 st = make_float4(0.0f, 1.0f, 0.0f, 1.0f);
+  if (n < k) {
+    unsigned long long* row = p.r1 + (static_cast<size_t>(b) * k + n) * 2;
+    float m, sm;
+    unpack_stats(take(row, ld_relaxed_u64(row), p.ctrl), m, sm);
+    st.x = m;
+    st.y = sm;
+    unpack_stats(take(row + 1, ld_relaxed_u64(row + 1), p.ctrl), m, sm);
+    st.z = m;
+    st.w = sm;
   }
-  const unsigned int rej = __ballot_sync(0xffffffffu, !acc);
-  const int n = rej ? __ffs(rej) - 1 : k;
-  const float smt = __shfl_sync(0xffffffffu, MT, n & 31);
-  const float sst = __shfl_sync(0xffffffffu, ST, n & 31);
-  const float smd = __shfl_sync(0xffffffffu, MD, n & 31);
-  const float ssd = __shfl_sync(0xffffffffu, SD, n & 31);
   int* out = p.out_tokens + static_cast<size_t>(b) * (k + 1);
   for (int i = lane; i <= k; i += 32)
     if (i != n) out[i] = i < n ? __ldg(p.tokens + static_cast<size_t>(b) * k + i) : -1;
@@ -1007,55 +1102,127 @@ __device__ void finalize_accept(const StochParams& p, int b, int lane) {
     p.accepted_len[b] = n;
     SeqRec* r = p.seq + b;
     r->n = n;
-    r->mt = smt;
-    r->ist = 1.0f / sst;
-    r->md = smd;
-    r->isd = 1.0f / ssd;
-    r->cnt1 = 0u;
+    r->mt = st.x;
+    r->ist = 1.0f / st.y;
+    r->md = st.z;
+    r->isd = 1.0f / st.w;
+    const unsigned int slot = atomicAdd(&p.ctrl->resolved, 1u);
     __threadfence();
-    fence_proxy_async_global();
-    st_release_u32(&r->ready, static_cast<unsigned int>(n) + 1u);
+    fence_proxy_async_global();  // the statistics are bulk-copied by the producer
+    if (slot < static_cast<unsigned int>(p.B))  // (each sequence resolves once: always true)
+      st_release_u64(p.list + slot, (static_cast<unsigned long long>(n) << 32) |
+                                        (static_cast<unsigned int>(b) + 1u));
   }
 }
 
-// Row merge of position i of sequence b (one warp, one lane per chunk):
-// publish the row statistics and count the row; the last row finalizes.
+// Row merge of pair i of sequence b (one warp, one lane per chunk): the row
+// statistics, then the row's own acceptance decision -- p_i(x_i), q_i(x_i),
+// u_i, accept while u_i q < p -- published in the sequence state word with one
+// atomicOr.  The merge whose update makes rows 0..n decided (n the first
+// rejection, or k) resolves the sequence; the merge that decides the last row
+// clears what the resolution left (statistics of later rejected rows) and the
+// state word.  A row with a chunk retired unread lies past a known rejection:
+// it is marked decided without a decision.
 template <typename TT, typename TD>
 __device__ void merge_row(const StochParams& p, int b, int i, int lane) {
-  unsigned long long* slot = p.p1 + (static_cast<size_t>(b) * p.k + i) * p.nch * 2;
+  const int k = p.k;
+  if (!SV_IN(p.ctrl, b, p.B) || !SV_IN(p.ctrl, i, k)) return;
+  unsigned long long* slot = p.p1 + (static_cast<size_t>(b) * k + i) * p.nch * 2;
   float MT = -INFINITY, ST = 0.0f, MD = -INFINITY, SD = 0.0f;
+  bool skipped = false;
   for (int c = lane; c < p.nch; c += 32) {
     const unsigned long long vt0 = ld_relaxed_u64(slot + 2 * c);
     const unsigned long long vd0 = ld_relaxed_u64(slot + 2 * c + 1);
+    const unsigned long long vt = take(slot + 2 * c, vt0, p.ctrl);
+    const unsigned long long vd = take(slot + 2 * c + 1, vd0, p.ctrl);
+    if (vt == kSkippedStats) {
+      skipped = true;
+      continue;
+    }
     float m, s;
-    unpack_stats(take(slot + 2 * c, vt0, p.ctrl), m, s);
+    unpack_stats(vt, m, s);
     merge_stats(MT, ST, m, s);
-    unpack_stats(take(slot + 2 * c + 1, vd0, p.ctrl), m, s);
+    unpack_stats(vd, m, s);
     merge_stats(MD, SD, m, s);
   }
+  skipped = __any_sync(0xffffffffu, skipped);
   const float4 w = warp_stats2(make_float4(MT, ST, MD, SD));
-  MT = w.x;
-  ST = w.y;
-  MD = w.z;
-  SD = w.w;
-  unsigned int old = 0u;
+  bool rejected = false;
   if (lane == 0) {
-    unsigned long long* row = p.r1 + (static_cast<size_t>(b) * p.k + i) * 2;
-    st_relaxed_u64(row, pack_stats(MT, ST));
-    st_relaxed_u64(row + 1, pack_stats(MD, SD));
-    p.rc[static_cast<size_t>(b) * p.k + i] = 0u;
-    old = atomicAdd(&p.seq[b].cnt1, 1u);
+    const int x = __ldg(p.tokens + static_cast<size_t>(b) * k + i);
+    const bool valid = x >= 0 && x < p.V;
+    if (!valid) atomicOr(&p.ctrl->flags, kFlagInvalidToken);
+    float pt = -1.0f, qd = -1.0f;  // -1: not read in full (past a rejection)
+    if (!skipped) {
+      pt = 0.0f;
+      qd = 0.0f;
+      if (valid &&
+          SV_IN(p.ctrl, static_cast<long long>(b) * p.t_sb + static_cast<long long>(i) * p.t_sp + x,
+                p.t_elems) &&
+          SV_IN(p.ctrl, static_cast<long long>(b) * p.d_sb + static_cast<long long>(i) * p.d_sp + x,
+                p.d_elems)) {
+        const float lt = load_elem<TT>(
+            p.tgt, static_cast<long long>(b) * p.t_sb + static_cast<long long>(i) * p.t_sp + x);
+        const float ld = load_elem<TD>(
+            p.drf, static_cast<long long>(b) * p.d_sb + static_cast<long long>(i) * p.d_sp + x);
+        pt = ex2f(fmaf(lt, p.c2, -w.x)) / w.y;
+        qd = ex2f(fmaf(ld, p.c2, -w.z)) / w.w;
+      }
+      const uint4 u = philox10(
+          make_uint4(0u, static_cast<uint32_t>(i), static_cast<uint32_t>(b) + p.seq_offset,
+                     kTagAccept),
+          p.key0, p.key1);
+      rejected = !(valid && (accept_uniform(u.x) * qd < pt));
+      if (rejected) {  // the statistics a resolution at this row reads
+        unsigned long long* row = p.r1 + (static_cast<size_t>(b) * k + i) * 2;
+        st_relaxed_u64(row, pack_stats(w.x, w.y));
+        st_relaxed_u64(row + 1, pack_stats(w.z, w.w));
+      }
+    }
+    if (p.probs) {
+      float* pr = p.probs + (static_cast<size_t>(b) * k + i) * 2;
+      pr[0] = pt;
+      pr[1] = qd;
+    }
   }
-  if (__shfl_sync(0xffffffffu, old == static_cast<unsigned int>(p.k) - 1u ? 1 : 0, 0))
-    finalize_accept<TT, TD>(p, b, lane);
+  unsigned long long old = 0ull, bits = 0ull;
+  if (lane == 0) {
+    p.rc[static_cast<size_t>(b) * k + i] = 0u;
+    bits = (1ull << i) | (rejected ? (1ull << (32 + i)) : 0ull);
+    fence_acq_rel_gpu();  // release: the row record before the state update
+    old = atomicOr(&p.seq[b].state, bits);
+    fence_acq_rel_gpu();  // acquire: other rows' records after it
+  }
+  old = __shfl_sync(0xffffffffu, old, 0);
+  bits = __shfl_sync(0xffffffffu, bits, 0);
+  rejected = __shfl_sync(0xffffffffu, rejected ? 1 : 0, 0) != 0;
+  const unsigned long long now = old | bits;
+  int n_old, n_now;
+  const bool was = resolved(old, k, n_old);
+  if (!was && resolved(now, k, n_now)) resolve_sequence(p, b, n_now, lane);
+  if (decided_bits(old) != low_mask(k) && decided_bits(now) == low_mask(k)) {
+    // the last row of the sequence: clear the records of rejected rows past
+    // n (rows retired unread are never marked rejected and wrote none)
+    resolved(now, k, n_now);
+    const unsigned int later = rejected_bits(now) & ~low_mask(n_now + 1) & low_mask(k);
+    for (unsigned int m = later; m;) {
+      const int j = __ffs(m) - 1;
+      m &= m - 1u;
+      unsigned long long* row = p.r1 + (static_cast<size_t>(b) * k + j) * 2;
+      if (lane < 2) take(row + lane, ld_relaxed_u64(row + lane), p.ctrl);
+    }
+    if (lane == 0) p.seq[b].state = 0ull;
+  }
 }
 
 // Phase-2 finalize of sequence b (one warp): the largest chunk key gives the
 // token at position n.  With no positive residual mass the token is drawn
-// from p_n with the same CORRECTION stream (slow path, one warp).
+// from p_n with the same CORRECTION stream (slow path, one warp).  Clears the
+// sequence's record and its ready-list entry.
 template <typename TT>
-__device__ void finalize_sample(const StochParams& p, int b, int n, int lane) {
+__device__ void finalize_sample(const StochParams& p, int b, int n, int entry, int lane) {
   const int k = p.k;
+  if (!SV_IN(p.ctrl, b, p.B) || !SV_IN(p.ctrl, n, k + 1) || !SV_IN(p.ctrl, entry, p.B)) return;
   unsigned long long key = 0ull;
   unsigned long long* slot = p.p2 + static_cast<size_t>(b) * p.nch;
   for (int c = lane; c < p.nch; c += 32) {
@@ -1071,7 +1238,8 @@ __device__ void finalize_sample(const StochParams& p, int b, int n, int lane) {
     const long long off = static_cast<long long>(b) * p.t_sb + static_cast<long long>(n) * p.t_sp;
     float bv = -INFINITY;
     int bi = INT_MAX;
-    for (int x = lane; x < p.V; x += 32) {
+    const int V = SV_IN_RANGE(p.ctrl, off, p.V, p.t_elems) ? p.V : 0;
+    for (int x = lane; x < V; x += 32) {
       const float sc = fmaf(load_elem<TT>(p.tgt, off + x), p.c2,
                             gumbel_log2(neg_exp1_log2(
                                 word_of(vocab_words(d, static_cast<uint32_t>(x) >> 2), x & 3))));
@@ -1089,10 +1257,10 @@ __device__ void finalize_sample(const StochParams& p, int b, int n, int lane) {
     p.out_tokens[static_cast<size_t>(b) * (k + 1) + n] = tok;
     p.accepted_len[b] = n;
     SeqRec* r = p.seq + b;
+    if (k > 0) p.list[entry] = 0ull;
     r->n = 0;
     r->mt = r->ist = r->md = r->isd = 0.0f;
     r->cnt2 = 0u;
-    r->ready = 0u;
   }
 }
 
@@ -1100,6 +1268,7 @@ __device__ void finalize_sample(const StochParams& p, int b, int n, int lane) {
 struct Pending {
   int kind;           // 0: none, kKindStats (row counter) or kKindCorrection (cnt2)
   int b, i;           // sequence; position (phase-1 row, or phase-2 row n)
+  int slot;           // phase 2: the sequence's ready-list entry
   unsigned int old;   // counter value before this arrival (lane 0)
 };
 
@@ -1111,14 +1280,14 @@ __device__ __forceinline__ void resolve(const StochParams& p, Pending& pd, int l
     if (pd.kind == kKindStats)
       merge_row<TT, TD>(p, pd.b, pd.i, lane);
     else
-      finalize_sample<TT>(p, pd.b, pd.i, lane);
+      finalize_sample<TT>(p, pd.b, pd.i, pd.slot, lane);
   }
   pd.kind = 0;
 }
 
 template <typename TT, typename TD>
 __device__ void stoch_epilogue(const StochParams& p, Shared& sh, int group, int lane) {
-  Pending pd{0, 0, 0, 0u};
+  Pending pd{0, 0, 0, 0, 0u};
   for (uint32_t use = group;; use += kComputeGroups) {
     const int s = use % kStages;
     const uint32_t parity = (use / kStages) & 1u;
@@ -1127,10 +1296,20 @@ __device__ void stoch_epilogue(const StochParams& p, Shared& sh, int group, int 
     if (!mbar_wait(&sh.rfull[s], parity, p.ctrl)) break;
     const Hdr h = sh.hdr[s];
     if (h.kind == kKindEnd) break;
+    if (h.kind == kKindRowDone) {  // every chunk of the row is counted: merge it
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.empty[s]);
+      resolve<TT, TD>(p, pd, lane);
+      merge_row<TT, TD>(p, h.b, h.i, lane);
+      continue;
+    }
     float4 r = lane < kGroupWarps ? sh.res[s][lane]
                                   : make_float4(-INFINITY, __int_as_float(INT_MAX), 0.f, 0.f);
     __syncwarp();
     if (lane == 0) mbar_arrive(&sh.empty[s]);
+    if (!SV_IN(p.ctrl, h.b, p.B) || !SV_IN(p.ctrl, h.c, p.nch) ||
+        !SV_IN(p.ctrl, h.i, h.kind == kKindStats ? p.k : p.k + 1))
+      continue;
     unsigned int old = 0u;
     Pending next;
     if (h.kind == kKindStats) {
@@ -1143,7 +1322,7 @@ __device__ void stoch_epilogue(const StochParams& p, Shared& sh, int group, int 
         st_relaxed_u64(slot + 1, pack_stats(r.z, r.w));
         old = atomicAdd(&p.rc[static_cast<size_t>(h.b) * p.k + h.i], 1u);
       }
-      next = Pending{kKindStats, h.b, h.i, old};
+      next = Pending{kKindStats, h.b, h.i, 0, old};
     } else {
       float v = r.x;
       int i = __float_as_int(r.y);
@@ -1153,7 +1332,7 @@ __device__ void stoch_epilogue(const StochParams& p, Shared& sh, int group, int 
                        i == INT_MAX ? kNoCandidate : make_key(v, i));
         old = atomicAdd(&p.seq[h.b].cnt2, 1u);
       }
-      next = Pending{kKindCorrection, h.b, h.i, old};
+      next = Pending{kKindCorrection, h.b, h.i, h.slot, old};
     }
     resolve<TT, TD>(p, pd, lane);
     pd = next;
@@ -1188,39 +1367,114 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ================================================================ argmax
 
+// Hand row (b, r), whose last chunk this producer just retired unread, to
+// the epilogue of the group that takes the next stage: a data-free item.
+__device__ __forceinline__ bool push_row_done(Shared& sh, uint32_t& use, int b, int r,
+                                              Ctrl* ctrl, int g) {
+  const int s = g < 0 ? static_cast<int>(use % kStages) : group_stage(g, use);
+  const uint32_t ph = g < 0 ? (use / kStages) & 1u : group_phase(use);
+  if (!mbar_wait(&sh.empty[s], ph ^ 1u, ctrl)) return false;
+  sh.hdr[s].kind = kKindRowDone;
+  sh.hdr[s].b = b;
+  sh.hdr[s].i = r;
+  mbar_arrive(&sh.full[s]);
+  ++use;
+  return true;
+}
+
 // kRowStride: rows or tree form, row h.i of the sequence at stride sg.
-template <typename TT, bool kTma, bool kRowStride>
-__device__ void argmax_producer(const ArgmaxParams& p, Shared& sh, unsigned char* stages) {
+// kEarly (plain mode): tickets are position-major, and a chunk of a row past
+// its branch's first known mismatch is retired without being read: its slot
+// gets kSkippedKey and it is counted on the row like a reduced chunk.  Rows up
+// to the branch's first mismatch are never retired (a mismatch is only known
+// once its row has been reduced in full), so the row argmaxes the finalize
+// uses are exact.
+// g < 0: the one producer of the CTA, alternating the groups' stages; g >= 0:
+// the producer of compute group g, filling that group's stages only.
+template <typename TT, bool kTma, bool kRowStride, bool kEarly>
+__device__ void argmax_producer(const ArgmaxParams& p, Shared& sh, unsigned char* stages, int g) {
   Ctrl* ctrl = p.ctrl;
   const unsigned int per_seq = static_cast<unsigned int>(p.R) * static_cast<unsigned int>(p.nch);
+  const unsigned int nch = static_cast<unsigned int>(p.nch);
+  const unsigned int BG = static_cast<unsigned int>(p.B) * static_cast<unsigned int>(p.G);
   uint32_t use = 0;
   bool ok = true;
-  unsigned int base = atomicAdd(&ctrl->ticket, kGrabArgmax);
+  // plain mode: the branch state of a position >= 1 ticket, loaded one
+  // ticket ahead so that its round trip overlaps the current ticket's work
+  auto branch_state = [&](unsigned int t) -> unsigned int {
+    if (!kEarly || t >= p.total) return 0u;
+    const unsigned int row = udiv(t, p.div_nch);
+    const unsigned int pos = udiv(row, p.div_bg);
+    return pos > 0u && SV_IN(ctrl, row - pos * BG, BG) ? ld_relaxed_u32(p.dead + (row - pos * BG))
+                                                        : 0u;
+  };
+  // The first grab of every CTA is fixed by its index (no atomic round trip
+  // before the first load); the counter hands out the tickets after them.
+  const unsigned int fixed = gridDim.x * kArgmaxProducers * kGrabArgmax;
+  unsigned int base = (blockIdx.x * kArgmaxProducers + static_cast<unsigned int>(g < 0 ? 0 : g)) *
+                      kGrabArgmax;
+  unsigned int dv_next = branch_state(base);
   while (ok && base < p.total) {
-    const unsigned int next = atomicAdd(&ctrl->ticket, kGrabArgmax);
+    const unsigned int next = fixed + atomicAdd(&ctrl->ticket, kGrabArgmax);
+    // retired chunks of the current row, counted with one atomic per run
+    int sk_b = -1, sk_r = 0;
+    unsigned int sk_n = 0u;
+#pragma unroll 1
     for (unsigned int j = 0; j < kGrabArgmax; ++j) {
       const unsigned int t = base + j;
       if (t >= p.total) break;
+      const unsigned int dv = dv_next;
+      dv_next = branch_state(j + 1 < kGrabArgmax ? t + 1 : next);
       Hdr h;
       h.kind = kKindArgmax;
-      const unsigned int b = udiv(t, p.div_seq);
-      const unsigned int rem = t - b * per_seq;
-      const unsigned int i = udiv(rem, p.div_nch);
-      h.b = static_cast<int>(b);
-      h.i = static_cast<int>(i);
-      h.c = static_cast<int>(rem - i * static_cast<unsigned int>(p.nch));
+      int pos = 0;
+      if (kEarly) {
+        const unsigned int row = udiv(t, p.div_nch);
+        const unsigned int ps = udiv(row, p.div_bg);
+        const unsigned int bg = row - ps * BG;
+        const unsigned int b = udiv(bg, p.div_g);
+        const unsigned int g = bg - b * static_cast<unsigned int>(p.G);
+        pos = static_cast<int>(ps);
+        h.b = static_cast<int>(b);
+        h.i = static_cast<int>(g) * (p.k + 1) + pos;
+        h.c = static_cast<int>(t - row * nch);
+      } else {
+        const unsigned int b = udiv(t, p.div_seq);
+        const unsigned int rem = t - b * per_seq;
+        const unsigned int i = udiv(rem, p.div_nch);
+        h.b = static_cast<int>(b);
+        h.i = static_cast<int>(i);
+        h.c = static_cast<int>(rem - i * nch);
+      }
+      if (kEarly && sk_b >= 0 && (h.b != sk_b || h.i != sk_r)) {  // a run of retired chunks ends
+        const unsigned int old = atomicAdd(&p.rc[static_cast<size_t>(sk_b) * p.R + sk_r], sk_n);
+        if (old + sk_n == nch) ok = push_row_done(sh, use, sk_b, sk_r, ctrl, g);
+        sk_b = -1;
+        sk_n = 0u;
+        if (!ok) break;
+      }
+      if (!SV_IN(ctrl, h.b, p.B) || !SV_IN(ctrl, h.i, p.R) || !SV_IN(ctrl, h.c, p.nch)) continue;
+      if (kEarly && dv != 0u && 64 - static_cast<int>(dv) < pos) {
+        st_relaxed_u64(p.slots + (static_cast<size_t>(h.b) * p.R + h.i) * nch + h.c, kSkippedKey);
+        sk_b = h.b;
+        sk_r = h.i;
+        ++sk_n;
+        continue;
+      }
       h.x0 = h.c * p.ch;
       h.len = min(p.ch, p.V - h.x0);
       if (kRowStride) {
         h.toff = static_cast<long long>(h.b) * p.sb + static_cast<long long>(h.i) * p.sg + h.x0;
       } else {
-        const int g = h.i / (p.k + 1), pos = h.i % (p.k + 1);
+        const int g = h.i / (p.k + 1), ps = h.i - g * (p.k + 1);
         h.toff = static_cast<long long>(h.b) * p.sb + static_cast<long long>(g) * p.sg +
-                 static_cast<long long>(pos) * p.sp + h.x0;
+                 static_cast<long long>(ps) * p.sp + h.x0;
       }
       h.doff = 0;
-      const int s = use % kStages;
-      if (!mbar_wait(&sh.empty[s], ((use / kStages) & 1u) ^ 1u, ctrl)) {
+      if (!SV_IN_RANGE(ctrl, h.toff, h.len, p.t_elems)) h.toff = 0;
+      const int s = g < 0 ? static_cast<int>(use % kStages) : group_stage(g, use);
+      const uint32_t ph = g < 0 ? (use / kStages) & 1u : group_phase(use);
+      if (!mbar_wait(&sh.empty[s], ph ^ 1u, ctrl)) {
         ok = false;
         break;
       }
@@ -1228,13 +1482,23 @@ __device__ void argmax_producer(const ArgmaxParams& p, Shared& sh, unsigned char
                                 nullptr, p.ch, false, nullptr);
       ++use;
     }
+    if (kEarly && ok && sk_b >= 0) {
+      const unsigned int old = atomicAdd(&p.rc[static_cast<size_t>(sk_b) * p.R + sk_r], sk_n);
+      if (old + sk_n == nch) ok = push_row_done(sh, use, sk_b, sk_r, ctrl, g);
+    }
     base = next;
   }
   if (ok) {
-    push_end(sh, use, ctrl);
-    leave_grid(ctrl, 1u);
+    if (g < 0)
+      push_end(sh, use, ctrl);
+    else
+      push_group_end(sh, g, use, ctrl);
+    leave_grid(ctrl, static_cast<unsigned int>(kArgmaxProducers));
   } else if (kTma) {
-    drain_stages(sh, use);
+    if (g < 0)
+      drain_stages(sh, use);
+    else
+      drain_group_stages(sh, g, use);
   }
 }
 
@@ -1253,9 +1517,10 @@ __device__ void argmax_compute(const ArgmaxParams& p, Shared& sh, unsigned char*
     const int s = use % kStages;
     if (!mbar_wait(&sh.full[s], (use / kStages) & 1u, p.ctrl)) break;
     const Hdr h = sh.hdr[s];
-    if (h.kind == kKindEnd) {
+    if (h.kind == kKindEnd || h.kind == kKindRowDone) {
       if (lane == 0) mbar_arrive(&sh.rfull[s]);
-      break;
+      if (h.kind == kKindEnd) break;
+      continue;
     }
     float bv;
     int bi;
@@ -1305,7 +1570,9 @@ __device__ void finalize_threshold(const ArgmaxParams& p, int b, int lane) {
     float m, sm;
     unpack_stats(take(stats + lane, ld_relaxed_u64(stats + lane), p.ctrl), m, sm);
     const int x = __ldg(p.tokens + static_cast<size_t>(b) * k + lane);
-    if (x >= 0 && x < V) {
+    if (x >= 0 && x < V &&
+        SV_IN(p.ctrl, static_cast<long long>(b) * p.sb + static_cast<long long>(lane) * p.sp + x,
+              p.t_elems)) {
       const long long off = static_cast<long long>(b) * p.sb + static_cast<long long>(lane) * p.sp + x;
       const float l = p.t_dtype == 1 ? load_elem<uint16_t>(p.tgt, off) : load_elem<float>(p.tgt, off);
       lp = fmaf(l, p.c2, -m) - lg2f(sm);
@@ -1461,6 +1728,7 @@ __device__ void finalize_argmax(const ArgmaxParams& p, int b, int lane) {
   const int k = p.k, G = p.G;
   unsigned long long* keys = p.rkey + static_cast<size_t>(b) * G * (k + 1);
   int best_n = -1, best_g = 0, best_next = -1;
+  bool invalid = false;  // a draft token outside [0, V): it never matches
   for (int g0 = 0; g0 < G; g0 += 4) {
     // row keys of up to four branches: loads issued together
     unsigned long long v[4], v32[4];
@@ -1478,7 +1746,9 @@ __device__ void finalize_argmax(const ArgmaxParams& p, int b, int lane) {
       const int a32 =
           (k == 32 && lane == 0) ? key_index(take(keys + g * (k + 1) + 32, v32[q], p.ctrl)) : -1;
       const int* cand = p.tokens + (static_cast<size_t>(b) * G + g) * k;
-      const bool miss = lane < k && __ldg(cand + lane) != a;
+      const int x = lane < k ? __ldg(cand + lane) : 0;
+      invalid |= x < 0 || x >= p.V;
+      const bool miss = lane < k && x != a;
       const unsigned int mm = __ballot_sync(0xffffffffu, miss);
       const int n = mm ? __ffs(mm) - 1 : k;
       const int an = __shfl_sync(0xffffffffu, a, n & 31);
@@ -1489,6 +1759,13 @@ __device__ void finalize_argmax(const ArgmaxParams& p, int b, int lane) {
         best_next = (n == 32) ? a32b : an;
       }
     }
+  }
+  if (__any_sync(0xffffffffu, invalid) && lane == 0) atomicOr(&p.ctrl->flags, kFlagInvalidToken);
+  if (lane == 0) {
+    // acquire (this lane counted the last row): every branch-state update
+    // lands before the clear
+    fence_acq_rel_gpu();
+    for (int g = 0; g < G; ++g) p.dead[static_cast<size_t>(b) * G + g] = 0u;
   }
   const int* cand = p.tokens + (static_cast<size_t>(b) * G + best_g) * k;
   int* out = p.out_tokens + static_cast<size_t>(b) * (k + 1);
@@ -1506,6 +1783,7 @@ __device__ void finalize_argmax(const ArgmaxParams& p, int b, int lane) {
 template <int kMode>
 __device__ void merge_argmax_row(const ArgmaxParams& p, int b, int r, int lane) {
   const unsigned int R = static_cast<unsigned int>(p.R);
+  if (!SV_IN(p.ctrl, b, p.B) || !SV_IN(p.ctrl, r, p.R)) return;
   unsigned long long* slot = p.slots + (static_cast<size_t>(b) * R + r) * p.nch;
   unsigned long long key = 0ull;
   for (int c = lane; c < p.nch; c += 32) {
@@ -1528,6 +1806,18 @@ __device__ void merge_argmax_row(const ArgmaxParams& p, int b, int r, int lane) 
   }
   unsigned int old = 0u;
   if (lane == 0) {
+    if (kMode == kArgPlain) {
+      // a draft that differs from this row's argmax ends its branch here:
+      // later rows of the branch decide nothing
+      const int g = r / (p.k + 1), pos = r - g * (p.k + 1);
+      if (pos < p.k &&
+          __ldg(p.tokens + (static_cast<size_t>(b) * p.G + g) * p.k + pos) != key_index(key)) {
+        atomicMax(p.dead + static_cast<size_t>(b) * p.G + g, 64u - static_cast<unsigned int>(pos));
+        // release: the finalize, which clears the word, sees this update
+        // before the row count below
+        fence_acq_rel_gpu();
+      }
+    }
     if (with_stats) st_relaxed_u64(p.rstats + static_cast<size_t>(b) * R + r, pack_stats(M, S));
     st_relaxed_u64(p.rkey + static_cast<size_t>(b) * R + r, key);
     p.rc[static_cast<size_t>(b) * R + r] = 0u;
@@ -1562,6 +1852,15 @@ __device__ void argmax_epilogue(const ArgmaxParams& p, Shared& sh, int group, in
     if (!mbar_wait(&sh.rfull[s], parity, p.ctrl)) break;
     const Hdr h = sh.hdr[s];
     if (h.kind == kKindEnd) break;
+    if (h.kind == kKindRowDone) {  // every chunk of the row is counted: merge it
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.empty[s]);
+      if (pend_b >= 0 && __shfl_sync(0xffffffffu, pend_old == last ? 1 : 0, 0))
+        merge_argmax_row<kMode>(p, pend_b, pend_r, lane);
+      pend_b = -1;
+      merge_argmax_row<kMode>(p, h.b, h.i, lane);
+      continue;
+    }
     float v = -INFINITY;
     int i = INT_MAX;
     float4 st = make_float4(-INFINITY, 0.0f, -INFINITY, 0.0f);
@@ -1574,6 +1873,8 @@ __device__ void argmax_epilogue(const ArgmaxParams& p, Shared& sh, int group, in
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&sh.empty[s]);
+    if (!SV_IN(p.ctrl, h.b, p.B) || !SV_IN(p.ctrl, h.i, p.R) || !SV_IN(p.ctrl, h.c, p.nch))
+      continue;
     warp_argmax(v, i);
     const bool with_stats = kMode == kArgThreshold && h.i < p.k;
     if (with_stats) st = warp_stats2(st);
@@ -1610,9 +1911,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_fence_init();
   }
   __syncthreads();
-  if (warp < kProducerWarps) {  // one producer: it alternates the groups' stages
-    if (warp == 0 && lane == 0)
-      argmax_producer<TT, kTma, kMode == kArgRows || kMode == kArgTree>(p, sh, stages);
+  if (warp < kProducerWarps) {
+    if (lane == 0 && warp < kArgmaxProducers)
+      argmax_producer<TT, kTma, kMode == kArgRows || kMode == kArgTree, kMode == kArgPlain>(
+          p, sh, stages, kArgmaxProducers == 1 ? -1 : warp);
   } else if (warp < kProducerWarps + kComputeWarps) {
     argmax_compute<TT, kTma, kMode>(p, sh, stages, warp - kProducerWarps, lane);
   } else {

@@ -11,16 +11,26 @@
 // GPU that loads the library holds kStaticScratchBytes of it until the
 // process exits.
 //
-// The first call on each device looks up that array's device address
-// (cudaGetSymbolAddress, with the device current) and keeps it; make that
-// first call before any stream capture.  Every call clears the part of the
-// array it needs (cudaMemsetAsync on the caller's stream) and then runs the
-// ordinary greedy verify on it.  All calls share the one array, so two calls
-// whose kernels may overlap on the GPU (different streams without ordering
-// between them) race and give wrong results: order them on one stream.
-#include <mutex>
+// Host code cannot use the array's name as a device address (on the host it
+// names a stand-in), so every call looks the address up with
+// cudaGetSymbolAddress, with the caller's device current.  The lookup is a
+// host-side query, not stream work; the first call on a device also loads the
+// library's device code there, so make that first call before any stream
+// capture.  Looking the address up on every call (rather than once) keeps it
+// right after the device's primary context has been reset and recreated.
+//
+// Every call clears the part of the array it needs, except the sticky device
+// status word, with cudaMemsetAsync on the caller's stream, and then runs the
+// ordinary greedy verify on it.  Status bits raised on the device (a timed-out
+// wait, an invalid draft token) accumulate until
+// spec_verify_greedy_noalloc_read_device_status reads and clears them.  All
+// calls share the one array, so two calls whose kernels may overlap on the
+// GPU (different streams without ordering between them) race and give wrong
+// results: order them on one stream.
+#include <cstddef>
 
 #include "spec_verify.h"
+#include "sv_internal.h"
 
 namespace {
 
@@ -30,20 +40,16 @@ static_assert(kStaticScratchBytes == SV_NOALLOC_SCRATCH_BYTES,
 
 static __device__ __align__(256) unsigned char g_scratch[kStaticScratchBytes];
 
-std::mutex g_lock;
-void* g_scratch_ptr[64] = {};
+// The control block at the start of every workspace: the sticky status word
+// sits between the words that must start each call at zero.
+constexpr size_t kFlagsOffset = offsetof(sv::Ctrl, flags);
+static_assert(kFlagsOffset + sizeof(unsigned int) <= sizeof(sv::Ctrl), "status word in Ctrl");
 
-// Device address of g_scratch on the current device, looked up once.
-int scratch_address(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return SV_ERR_CUDA;
-  std::lock_guard<std::mutex> guard(g_lock);
-  if (g_scratch_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || p == nullptr) return SV_ERR_CUDA;
-    g_scratch_ptr[dev] = p;
-  }
-  *out = g_scratch_ptr[dev];
+// Device address of g_scratch on the current device.
+int scratch_address(unsigned char** out) {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || p == nullptr) return SV_ERR_CUDA;
+  *out = static_cast<unsigned char*>(p);
   return SV_OK;
 }
 
@@ -58,11 +64,32 @@ extern "C" int spec_verify_greedy_noalloc(const void* target_logits, int t_dtype
   if (need == 0) return SV_ERR_INVALID_ARG;  // B, k or V outside the limits
   if (need > kStaticScratchBytes) return SV_ERR_WORKSPACE;
   if (B == 0) return SV_OK;
-  void* ws = nullptr;
+  unsigned char* ws = nullptr;
   const int rc = scratch_address(&ws);
   if (rc != SV_OK) return rc;
-  if (cudaMemsetAsync(ws, 0, need, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(ws, 0, kFlagsOffset, st) != cudaSuccess ||
+      cudaMemsetAsync(ws + kFlagsOffset + sizeof(unsigned int), 0,
+                      need - kFlagsOffset - sizeof(unsigned int), st) != cudaSuccess)
     return SV_ERR_CUDA;
   return spec_verify_greedy(target_logits, t_dtype, t_stride_b, t_stride_pos, draft_tokens, B, k,
                             V, accepted_len, out_tokens, ws, need, stream);
+}
+
+extern "C" int spec_verify_greedy_noalloc_read_device_status(uint32_t* flags_host, int clear,
+                                                             void* stream) {
+  if (!flags_host) return SV_ERR_INVALID_ARG;
+  unsigned char* ws = nullptr;
+  const int rc = scratch_address(&ws);
+  if (rc != SV_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t v = 0;
+  if (cudaMemcpyAsync(&v, ws + kFlagsOffset, sizeof v, cudaMemcpyDeviceToHost, st) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return SV_ERR_CUDA;
+  *flags_host = v;
+  if (clear && cudaMemsetAsync(ws + kFlagsOffset, 0, sizeof v, st) != cudaSuccess)
+    return SV_ERR_CUDA;
+  return SV_OK;
 }

@@ -20,10 +20,14 @@
 //                       then walks the tree with warp-uniform shuffles and
 //                       ballots.  Writes the path and accepted tokens, and the
 //                       final node and E for the draw.
-//   tree_sample_kernel  one block per (sequence, chunk) of the final node's
-//                       row: Gumbel-max over l c2 outside E (and over the whole
-//                       row as the fallback), merged by 64-bit atomicMax; the
-//                       last block of a sequence writes the token.
+//   tree_sample_kernel  one block per (sequence, 2048-entry piece) of the
+//                       final node's row: Gumbel-max over l c2 outside E (and
+//                       over the whole row as the fallback), merged by 64-bit
+//                       atomicMax; the last block of a sequence writes the
+//                       token.  The draw is issue-bound (a Philox block per
+//                       four entries, two lg2 per entry) on one row per
+//                       sequence, so it runs on many short blocks that fill
+//                       every SM several times over.
 // Every workspace word written here is cleared again by the kernel that
 // consumes it, so the workspace stays zero between calls of any mode.
 #include <climits>
@@ -38,6 +42,7 @@ namespace {
 
 constexpr int kTsThreads = 256;
 constexpr int kTsVecs = 8;  // 16-byte vectors per thread and chunk
+constexpr int kSampleEntries = 2048;  // entries per block of the final draw
 constexpr int kWalkWarps = 4;
 constexpr int kMaxNodes = 64;
 
@@ -56,9 +61,11 @@ static_assert(sizeof(TreeRec) % 16 == 0, "TreeRec keeps 16-byte alignment");
 struct TreeStochParams {
   const void* logits;
   long long sb, sn;  // element strides of sequence and node
+  long long l_elems;  // elements the logits view spans (bounds checks)
   const int* parent;
   const int* tokens;
-  int B, N, V, nch;  // nch chunks per row
+  int B, N, V, nch;  // nch chunks per row (statistics)
+  int nch_s;         // pieces of kSampleEntries per row (final draw)
   bool vec;          // every row starts 16-byte aligned
   float c2;          // log2(e) / T
   unsigned int key0, key1, seq_offset;
@@ -95,8 +102,11 @@ __global__ void __launch_bounds__(kTsThreads) tree_stats_kernel(TreeStochParams 
   const int b = static_cast<int>(row / p.N), j = static_cast<int>(row % p.N);
   const long long off = static_cast<long long>(b) * p.sb + static_cast<long long>(j) * p.sn;
   const int x0 = c * CH;
-  const int len = min(CH, p.V - x0);
+  int len = min(CH, p.V - x0);
   const int tid = threadIdx.x;
+  if (!SV_IN(p.ctrl, row, static_cast<long long>(p.B) * p.N) ||
+      !SV_IN_RANGE(p.ctrl, off + x0, len, p.l_elems))
+    len = 0;  // (bounds-checked builds: a bad block reads nothing)
   float mx = -INFINITY, s = 0.0f;
   if (p.vec) {
     const uint4* src = reinterpret_cast<const uint4*>(static_cast<const T*>(p.logits) + off + x0);
@@ -204,7 +214,9 @@ __global__ void __launch_bounds__(32 * kWalkWarps) tree_walk_kernel(TreeStochPar
         bad_parent = true;
       } else {
         par[h] = q;
-        if (x >= 0 && x < p.V) {
+        if (x >= 0 && x < p.V &&
+            SV_IN(p.ctrl, static_cast<long long>(b) * p.sb + static_cast<long long>(q) * p.sn + x,
+                  p.l_elems)) {
           const float l = load_elem<T>(p.logits, static_cast<long long>(b) * p.sb +
                                                      static_cast<long long>(q) * p.sn + x);
           pr[h] = ex2f(fmaf(l, p.c2, -s_m[w][q])) * s_is[w][q];
@@ -281,14 +293,14 @@ __global__ void __launch_bounds__(32 * kWalkWarps) tree_walk_kernel(TreeStochPar
 template <typename T>
 __global__ void __launch_bounds__(kTsThreads) tree_sample_kernel(TreeStochParams p) {
   constexpr int EPV = Elem<T>::kPerVec;
-  constexpr int CH = tree_chunk<T>();
+  constexpr int CH = kSampleEntries;
   __shared__ int s_ex[kMaxNodes];
   __shared__ unsigned long long s_ke[kTsThreads / 32], s_ka[kTsThreads / 32];
-  const int c = static_cast<int>(blockIdx.x % p.nch);
-  const int b = static_cast<int>(blockIdx.x / p.nch);
+  const int c = static_cast<int>(blockIdx.x % p.nch_s);
+  const int b = static_cast<int>(blockIdx.x / p.nch_s);
   const int tid = threadIdx.x;
   TreeRec& rec = p.rec[b];
-  const int u = rec.u, ne = rec.ne;
+  const int u = rec.u, ne = min(rec.ne, kMaxNodes);
   const uint32_t tag = static_cast<uint32_t>(rec.tag);
   if (tid < ne) s_ex[tid] = rec.excl[tid];
   __syncthreads();
@@ -296,7 +308,10 @@ __global__ void __launch_bounds__(kTsThreads) tree_sample_kernel(TreeStochParams
   const long long off = static_cast<long long>(b) * p.sb + static_cast<long long>(u) * p.sn;
   const uint32_t seq = static_cast<uint32_t>(b) + p.seq_offset;
   const int x0 = c * CH;
-  const int len = min(CH, p.V - x0);
+  int len = min(CH, p.V - x0);
+  if (!SV_IN(p.ctrl, u, p.N) ||
+      !SV_IN_RANGE(p.ctrl, off + x0, len, p.l_elems))
+    len = 0;  // (bounds-checked builds: a bad block reads nothing)
   float bv = -INFINITY, av = -INFINITY;  // best outside E, best of the row
   int bi = INT_MAX, ai = INT_MAX;
   auto take = [&](float l, uint32_t word, int x) {
@@ -362,7 +377,7 @@ __global__ void __launch_bounds__(kTsThreads) tree_sample_kernel(TreeStochParams
     if (ke) atomicMax(&p.keys[2 * b], ke);
     if (ka) atomicMax(&p.keys[2 * b + 1], ka);
     __threadfence();
-    if (atomicAdd(&p.cnt[b], 1u) == static_cast<unsigned int>(p.nch) - 1u) {
+    if (atomicAdd(&p.cnt[b], 1u) == static_cast<unsigned int>(p.nch_s) - 1u) {
       __threadfence();
       ke = atomicExch(&p.keys[2 * b], 0ull);
       ka = atomicExch(&p.keys[2 * b + 1], 0ull);
@@ -420,7 +435,7 @@ cudaError_t launch_tree_stoch(const TreeStochParams& p, cudaStream_t st) {
   tree_walk_kernel<T><<<(p.B + kWalkWarps - 1) / kWalkWarps, 32 * kWalkWarps, 0, st>>>(p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  tree_sample_kernel<T><<<static_cast<unsigned int>(static_cast<long long>(p.B) * p.nch),
+  tree_sample_kernel<T><<<static_cast<unsigned int>(static_cast<long long>(p.B) * p.nch_s),
                           kTsThreads, 0, st>>>(p);
   return cudaGetLastError();
 }
@@ -458,19 +473,24 @@ extern "C" int spec_verify_tree_stochastic(const void* node_logits, int t_dtype,
   const TreeLayout lay = tree_layout(B, N, V);
   if (workspace_bytes < lay.total) return SV_ERR_WORKSPACE;
   const int nch = tree_nch(V, es);
-  if (static_cast<long long>(B) * N * nch >= (1ll << 31)) return SV_ERR_INVALID_ARG;
+  const int nch_s = (V + kSampleEntries - 1) / kSampleEntries;
+  if (static_cast<long long>(B) * N * nch >= (1ll << 31) ||
+      static_cast<long long>(B) * nch_s >= (1ll << 31))
+    return SV_ERR_INVALID_ARG;
 
   unsigned char* ws = static_cast<unsigned char*>(workspace);
   TreeStochParams p{};
   p.logits = node_logits;
   p.sb = stride_b;
   p.sn = stride_node;
+  p.l_elems = (static_cast<long long>(B) - 1) * stride_b + (static_cast<long long>(N) - 1) * stride_node + V;
   p.parent = parent;
   p.tokens = tokens;
   p.B = B;
   p.N = N;
   p.V = V;
   p.nch = nch;
+  p.nch_s = nch_s;
   p.vec = is_aligned(node_logits, 16) && (stride_b * es) % 16 == 0 && (stride_node * es) % 16 == 0;
   p.c2 = 1.4426950408889634f / temperature;
   p.key0 = static_cast<unsigned int>(seed & 0xffffffffull);
