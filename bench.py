@@ -339,18 +339,21 @@ def oracle_baseline(ws: dict) -> tuple[dict, dict]:
 
     oracle.build()
     cores = os.cpu_count() or 1
-    reps, t_total, outcome = 0, 0.0, {}
+    reps, t_total, outcome, per_s = 0, 0.0, {}, {}
     while reps < 3 and t_total < 5.0:
         t0 = time.perf_counter()
         for name in STEP:
+            t1 = time.perf_counter()
             o = oracle_call(ws[name], cores)
+            per_s.setdefault(name, time.perf_counter() - t1)
             outcome.setdefault(name, o)
         t_total += time.perf_counter() - t0
         reps += 1
     pos = sum(positions(ws[n]) for n in STEP) * reps
     return ({"value": pos / t_total, "unit": "positions/s", "cores": cores, "kind": "oracle",
              "sample": f"{reps} full step(s): every sequence of the {len(STEP)} workload(s) "
-                       f"({pos // reps} positions per step), {t_total:.1f} s"}, outcome)
+                       f"({pos // reps} positions per step), {t_total:.1f} s",
+             "seconds_per_call": {n: round(v, 4) for n, v in per_s.items()}}, outcome)
 
 
 def branch_lengths(w: dict) -> np.ndarray:

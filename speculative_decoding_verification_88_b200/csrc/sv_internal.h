@@ -27,8 +27,15 @@ constexpr int kGroupWarps = kComputeWarps / kComputeGroups;
 constexpr int kProducerWarps = kComputeGroups;
 constexpr int kThreads = 32 * (kProducerWarps + kComputeWarps + kComputeGroups);
 constexpr int kComputeThreads = kGroupWarps * 32;  // threads that share one chunk
-constexpr int kStages = 4;
-constexpr int kStageBytes = 56 * 1024;
+#ifndef SV_STAGES
+#define SV_STAGES 4
+#endif
+#ifndef SV_STAGE_BYTES
+#define SV_STAGE_BYTES (56 * 1024)
+#endif
+constexpr int kStages = SV_STAGES;          // ring stages per CTA, split evenly over the groups
+constexpr int kStageBytes = SV_STAGE_BYTES;  // a multiple of 128
+static_assert(kStageBytes % 128 == 0, "stages stay 128-byte aligned");
 
 // Entries of a full chunk: as many as fit `bytes` at `bpe` bytes per entry,
 // rounded down to whole rounds of 16-byte vectors over the kComputeThreads
@@ -85,7 +92,7 @@ Plan plan_chunks(long long rows, int V, int bpe, int es_min, int chunk_bytes);
 // enough that the ramp of the ring dominates (greedy B = 64, k = 4,
 // V = 128256: 40 KB chunks 15.9 us, 48 KB 16.9 us, 54 KB 18.1 us).
 constexpr int kStochChunkBytes = kStageBytes;
-constexpr int kArgmaxChunkBytes = 40 * 1024;
+constexpr int kArgmaxChunkBytes = 40 * 1024 < kStageBytes ? 40 * 1024 : kStageBytes;
 
 // Division of 31-bit values by a divisor fixed per call, as a multiply-high
 // and a shift (Granlund and Montgomery, "Division by invariant integers using
@@ -168,6 +175,9 @@ struct ArgmaxParams {
   // whole position block (B G nch tickets) after its row i - 1.  The other
   // modes go sequence by sequence: / (R * nch), then / nch.
   UDiv div_seq, div_nch, div_bg, div_g;  // / (R * nch), / nch, / (B * G), / G
+  // One-shot form (small plain calls): nch1 chunks of a row per block grid.
+  int nch1;
+  UDiv div_nch1, div_R;  // / nch1, / R
   unsigned int total;
   Ctrl* ctrl;
   SeqRec* seq;
@@ -185,6 +195,11 @@ cudaError_t launch_stochastic(const StochParams& p, int t_dtype, int d_dtype, bo
                               int grid, size_t smem, cudaStream_t stream);
 cudaError_t launch_argmax(const ArgmaxParams& p, int t_dtype, bool tma, int grid, size_t smem,
                           cudaStream_t stream);
+// Plain greedy / multi-candidate verify as one grid of row-chunk blocks (no
+// persistent pipeline): every row is read, all of a block's loads are in
+// flight at once, and the last block of a sequence finalizes it.
+cudaError_t launch_argmax_oneshot(const ArgmaxParams& p, int t_dtype, bool vec, cudaStream_t st);
+int oneshot_chunk_entries(int t_dtype);
 cudaError_t launch_commit(const int* accepted_len, const int* out_tokens, int B, int k,
                           int* seq_len, int* token_buf, long long buf_stride, int capacity,
                           int* next_input, Ctrl* ctrl, cudaStream_t st);

@@ -590,6 +590,26 @@ __device__ __forceinline__ uint4 vocab_words(const Draw& d, uint32_t c0) {
   return philox10(make_uint4(c0, d.pos, d.seq, d.tag), d.key0, d.key1);
 }
 
+
+// Round keys computed once per chunk (SV_PHILOX_ROUND_KEYS) or per draw.
+#ifndef SV_PHILOX_ROUND_KEYS
+#define SV_PHILOX_ROUND_KEYS 0
+#endif
+#if SV_PHILOX_ROUND_KEYS
+struct ChunkDraw {
+  PhiloxKeys k;
+  uint32_t pos, seq, tag;
+};
+__device__ __forceinline__ ChunkDraw chunk_draw(const Draw& d) {
+  return ChunkDraw{philox_keys(d.key0, d.key1), d.pos, d.seq, d.tag};
+}
+__device__ __forceinline__ uint4 vocab_words(const ChunkDraw& d, uint32_t c0) {
+  return philox10(make_uint4(c0, d.pos, d.seq, d.tag), d.k);
+}
+#else
+__device__ __forceinline__ const Draw& chunk_draw(const Draw& d) { return d; }
+#endif
+
 // Residual of the correction race, rescaled by the row's target sum s_t:
 //   r'(x) = 2^(l_t(x) c2 - m_t) - 2^(l_d(x) c2 - m_d + o),   o = lg2(1/s_d) - lg2(1/s_t),
 // which is s_t (p(x) - q(x)).  s_t is one positive constant per row, so the
@@ -638,6 +658,29 @@ __device__ __forceinline__ void race_push(Race& b, float r, float e, int x) {
   b.x = win ? x : b.x;
 }
 
+// Eight consecutive entries (group j of the chunk) of the correction race.
+template <typename TT, typename TD, typename DK>
+__device__ __forceinline__ void residual_group(const unsigned char* ts, const unsigned char* ds,
+                                               int j, const ResidualTerms& rt, const DK& dk,
+                                               int x0, Race& best) {
+  float lt[8], ld[8], r[8];
+  load8<TT>(ts, j, lt);
+  load8<TD>(ds, j, ld);
+  residual8(lt, ld, rt, r);
+  const int xg = x0 + 8 * j;
+  // both Philox words in straight-line code, so their round chains
+  // interleave; candidates are selected without branches
+  const uint4 w0 = vocab_words(dk, static_cast<uint32_t>(xg) >> 2);
+  const uint4 w1 = vocab_words(dk, (static_cast<uint32_t>(xg) >> 2) + 1u);
+  float e[8];
+  neg_exp1_log2_x2(w0.x, w0.y, e[0], e[1]);
+  neg_exp1_log2_x2(w0.z, w0.w, e[2], e[3]);
+  neg_exp1_log2_x2(w1.x, w1.y, e[4], e[5]);
+  neg_exp1_log2_x2(w1.z, w1.w, e[6], e[7]);
+#pragma unroll
+  for (int q = 0; q < 8; ++q) race_push(best, r[q], e[q], xg + q);
+}
+
 // Gumbel-max over the positive residual of one chunk.  Returns the warp's
 // best (score lg2 r' - lg2 E + const, x); x = INT_MAX if the warp saw no
 // positive residual.
@@ -649,24 +692,9 @@ __device__ __forceinline__ void chunk_residual(const unsigned char* ts, const un
   const ResidualTerms rt = residual_terms(c2, st);
   Race best{0.0f, -1.0f, INT_MAX};
   const int ng = kTma ? h.len / 8 : 0;
-  for (int j = tid; j < ng; j += kComputeThreads) {
-    float lt[8], ld[8], r[8];
-    load8<TT>(ts, j, lt);
-    load8<TD>(ds, j, ld);
-    residual8(lt, ld, rt, r);
-    const int xg = h.x0 + 8 * j;
-    // both Philox words in straight-line code, so their round chains
-    // interleave; candidates are selected without branches
-    const uint4 w0 = vocab_words(d, static_cast<uint32_t>(xg) >> 2);
-    const uint4 w1 = vocab_words(d, (static_cast<uint32_t>(xg) >> 2) + 1u);
-    float e[8];
-    neg_exp1_log2_x2(w0.x, w0.y, e[0], e[1]);
-    neg_exp1_log2_x2(w0.z, w0.w, e[2], e[3]);
-    neg_exp1_log2_x2(w1.x, w1.y, e[4], e[5]);
-    neg_exp1_log2_x2(w1.z, w1.w, e[6], e[7]);
-#pragma unroll
-    for (int q = 0; q < 8; ++q) race_push(best, r[q], e[q], xg + q);
-  }
+  const auto dk = chunk_draw(d);
+  for (int j = tid; j < ng; j += kComputeThreads)
+    residual_group<TT, TD>(ts, ds, j, rt, dk, h.x0, best);
   for (int e = 8 * ng + tid; e < h.len; e += kComputeThreads) {
     const int x = h.x0 + e;
     const float r = residual(load_elem<TT>(tgt, h.toff + e), load_elem<TD>(drf, h.doff + e), rt);
@@ -687,12 +715,13 @@ __device__ __forceinline__ void chunk_bonus(const unsigned char* ts, const Hdr& 
   bv = -INFINITY;
   bi = INT_MAX;
   const int ng = kTma ? h.len / 8 : 0;
+  const auto dk = chunk_draw(d);
   for (int j = tid; j < ng; j += kComputeThreads) {
     float lt[8];
     load8<TT>(ts, j, lt);
     const int xg = h.x0 + 8 * j;
-    const uint4 w0 = vocab_words(d, static_cast<uint32_t>(xg) >> 2);
-    const uint4 w1 = vocab_words(d, (static_cast<uint32_t>(xg) >> 2) + 1u);
+    const uint4 w0 = vocab_words(dk, static_cast<uint32_t>(xg) >> 2);
+    const uint4 w1 = vocab_words(dk, (static_cast<uint32_t>(xg) >> 2) + 1u);
     float e[8];
     neg_exp1_log2_x2(w0.x, w0.y, e[0], e[1]);
     neg_exp1_log2_x2(w0.z, w0.w, e[2], e[3]);
@@ -882,15 +911,23 @@ __device__ void stoch_producer(const StochParams& p, Shared& sh, unsigned char* 
   int nd = 0;
   unsigned int t2p = kNone;        // a phase-2 grab in flight
   bool t2_done = p.total2 == 0u;
-  int sk_b = -1, sk_i = 0;         // a retired chunk whose count is checked later
-  unsigned int sk_old = 0u;
+  // Retired chunks whose count is checked later (the counter's old value
+  // arrives while the producer goes on): a count that completes the row
+  // hands the row to the epilogue.  No resolution waits on a retired row (it
+  // lies past a rejection), so the hand-over may lag.
+  constexpr int kSk = 4;
+  int skb[kSk], ski[kSk];
+  unsigned int sko[kSk];
+  int nsk = 0;
+  auto settle_retired = [&]() -> bool {
+#pragma unroll
+    for (int d = 0; d < kSk; ++d)
+      if (d < nsk && sko[d] == nch - 1u && !stoch_push_row_done(sh, g, used, skb[d], ski[d], ctrl))
+        return false;
+    nsk = 0;
+    return true;
+  };
   while (ok) {
-    // the retired chunk of the previous iteration: did it complete its row?
-    if (sk_b >= 0) {
-      if (sk_old == nch - 1u) ok = stoch_push_row_done(sh, g, used, sk_b, sk_i, ctrl);
-      sk_b = -1;
-      if (!ok) break;
-    }
     // (the held arrays are indexed with constants only, so they stay in
     // registers and a poll's load is not waited for until it is read)
     if (t2p != kNone) {  // the phase-2 grab of the previous iteration joins the queue
@@ -915,6 +952,10 @@ __device__ void stoch_producer(const StochParams& p, Shared& sh, unsigned char* 
     for (int d = kDefer - 1; d >= 0; --d)
       if (d < nd && dv[d] != 0ull) rd = d;
     if (rd < 0 && t1 >= p.total1 && nd > 0) {
+      if (!settle_retired()) {
+        ok = false;
+        break;
+      }
       // nothing else to do: wait (bounded) for the oldest held entry
       const unsigned long long* e = p.list + udiv(dt[0], p.div_nch);
       unsigned long long v = ld_relaxed_u64(e);
@@ -970,6 +1011,7 @@ __device__ void stoch_producer(const StochParams& p, Shared& sh, unsigned char* 
       const int n = static_cast<int>(v >> 32);
       ok = stoch_issue_phase2<TT, TD, kTma>(p, sh, stages, g, used, b, n, static_cast<int>(c),
                                             static_cast<int>(slot));
+      if (ok) ok = settle_retired();  // their counts arrived during the stage wait
       continue;
     }
 #pragma unroll
@@ -996,15 +1038,29 @@ __device__ void stoch_producer(const StochParams& p, Shared& sh, unsigned char* 
             p.p1 + ((static_cast<size_t>(h.b) * p.k + h.i) * nch + h.c) * 2;
         st_relaxed_u64(slot, kSkippedStats);
         st_relaxed_u64(slot + 1, kSkippedStats);
-        sk_old = atomicAdd(&p.rc[static_cast<size_t>(h.b) * p.k + h.i], 1u);
-        sk_b = h.b;
-        sk_i = h.i;
+        if (nsk == kSk && !settle_retired()) {
+          ok = false;
+          break;
+        }
+        const unsigned int old = atomicAdd(&p.rc[static_cast<size_t>(h.b) * p.k + h.i], 1u);
+#pragma unroll
+        for (int d = 0; d < kSk; ++d)
+          if (d == nsk) {
+            skb[d] = h.b;
+            ski[d] = h.i;
+            sko[d] = old;
+          }
+        ++nsk;
         continue;
       }
       ok = stoch_issue<TT, TD, kTma>(p, sh, stages, g, used, h, nullptr);
+      if (ok) ok = settle_retired();  // their counts arrived during the stage wait
       continue;
     }
-    if (nd == 0 && t2_done && t2p == kNone) break;  // no work left
+    if (nd == 0 && t2_done && t2p == kNone) {  // no work left
+      ok = settle_retired();
+      break;
+    }
     if (nd == 0 && t2p != kNone) continue;           // a grab in flight
   }
   if (ok) {
@@ -1107,8 +1163,9 @@ __device__ void resolve_sequence(const StochParams& p, int b, int n, int lane) {
     r->md = st.z;
     r->isd = 1.0f / st.w;
     const unsigned int slot = atomicAdd(&p.ctrl->resolved, 1u);
-    __threadfence();
-    fence_proxy_async_global();  // the statistics are bulk-copied by the producer
+    // the release store below orders the record before the entry; the
+    // statistics are bulk-copied by the producer (async proxy)
+    fence_proxy_async_global();
     if (slot < static_cast<unsigned int>(p.B))  // (each sequence resolves once: always true)
       st_release_u64(p.list + slot, (static_cast<unsigned long long>(n) << 32) |
                                         (static_cast<unsigned int>(b) + 1u));
@@ -1156,15 +1213,13 @@ __device__ void merge_row(const StochParams& p, int b, int i, int lane) {
     if (!skipped) {
       pt = 0.0f;
       qd = 0.0f;
-      if (valid &&
-          SV_IN(p.ctrl, static_cast<long long>(b) * p.t_sb + static_cast<long long>(i) * p.t_sp + x,
-                p.t_elems) &&
-          SV_IN(p.ctrl, static_cast<long long>(b) * p.d_sb + static_cast<long long>(i) * p.d_sp + x,
-                p.d_elems)) {
-        const float lt = load_elem<TT>(
-            p.tgt, static_cast<long long>(b) * p.t_sb + static_cast<long long>(i) * p.t_sp + x);
-        const float ld = load_elem<TD>(
-            p.drf, static_cast<long long>(b) * p.d_sb + static_cast<long long>(i) * p.d_sp + x);
+      const long long ot =
+          static_cast<long long>(b) * p.t_sb + static_cast<long long>(i) * p.t_sp + x;
+      const long long od =
+          static_cast<long long>(b) * p.d_sb + static_cast<long long>(i) * p.d_sp + x;
+      if (valid && SV_IN(p.ctrl, ot, p.t_elems) && SV_IN(p.ctrl, od, p.d_elems)) {
+        const float lt = load_elem<TT>(p.tgt, ot);
+        const float ld = load_elem<TD>(p.drf, od);
         pt = ex2f(fmaf(lt, p.c2, -w.x)) / w.y;
         qd = ex2f(fmaf(ld, p.c2, -w.z)) / w.w;
       }
@@ -1189,9 +1244,9 @@ __device__ void merge_row(const StochParams& p, int b, int i, int lane) {
   if (lane == 0) {
     p.rc[static_cast<size_t>(b) * k + i] = 0u;
     bits = (1ull << i) | (rejected ? (1ull << (32 + i)) : 0ull);
-    fence_acq_rel_gpu();  // release: the row record before the state update
-    old = atomicOr(&p.seq[b].state, bits);
-    fence_acq_rel_gpu();  // acquire: other rows' records after it
+    // release: this row's record before the state update; acquire: the
+    // records of the rows whose bits it returns
+    old = atom_or_acq_rel_u64(&p.seq[b].state, bits);
   }
   old = __shfl_sync(0xffffffffu, old, 0);
   bits = __shfl_sync(0xffffffffu, bits, 0);
@@ -1813,8 +1868,9 @@ __device__ void merge_argmax_row(const ArgmaxParams& p, int b, int r, int lane) 
       if (pos < p.k &&
           __ldg(p.tokens + (static_cast<size_t>(b) * p.G + g) * p.k + pos) != key_index(key)) {
         atomicMax(p.dead + static_cast<size_t>(b) * p.G + g, 64u - static_cast<unsigned int>(pos));
-        // release: the finalize, which clears the word, sees this update
-        // before the row count below
+        // the finalize, which clears the word, sees this update before the
+        // row count below (a fence: a release operation would order only
+        // what came before it)
         fence_acq_rel_gpu();
       }
     }
@@ -1920,6 +1976,130 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     argmax_epilogue<kMode>(p, sh, warp - kProducerWarps - kComputeWarps, lane);
   }
+}
+
+// ========================================================= one-shot argmax
+
+// Plain greedy and multi-candidate verify for calls too small for the
+// persistent pipeline to pay off (a few microseconds of ramp and a dependent
+// tail of several L2 round trips after the last chunk, against a call of a
+// few tens of microseconds, and too short for a rejection to be known before
+// the rows after it are read).  One 256-thread block per chunk of one row:
+// every thread loads its (up to) eight 16-byte vectors at once, takes the
+// first maximum, the block merges its warps in shared memory and publishes
+// the chunk's key with one 64-bit atomicMax on the row key (keys order like
+// (value, -index), so the max is the row's first maximum); a fence and a
+// per-sequence counter then tell the last block of the sequence, which runs
+// the same finalize as the persistent kernel.  Blocks go sequence by
+// sequence, so sequences finalize while later ones stream.
+constexpr int kOsThreads = 256;
+constexpr int kOsVecs = 8;
+
+template <typename T>
+__host__ __device__ constexpr int oneshot_chunk() {
+  return kOsThreads * kOsVecs * Elem<T>::kPerVec;  // 16384 bf16 or 8192 f32 entries
+}
+
+int oneshot_chunk_entries(int t_dtype) {
+  return t_dtype == 1 ? oneshot_chunk<uint16_t>() : oneshot_chunk<float>();
+}
+
+template <typename T, bool kVec>
+__global__ void __launch_bounds__(kOsThreads)
+    argmax_oneshot_kernel(const __grid_constant__ ArgmaxParams p) {
+  constexpr int EPV = Elem<T>::kPerVec;
+  constexpr int CH = oneshot_chunk<T>();
+  __shared__ unsigned long long s_key[kOsThreads / 32];
+  __shared__ int s_last;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const unsigned int row = udiv(blockIdx.x, p.div_nch1);  // b * R + r
+  const int c = static_cast<int>(blockIdx.x - row * static_cast<unsigned int>(p.nch1));
+  const unsigned int bu = udiv(row, p.div_R);
+  const int b = static_cast<int>(bu);
+  const int r = static_cast<int>(row - bu * static_cast<unsigned int>(p.R));
+  const int g = r / (p.k + 1), pos = r - g * (p.k + 1);
+  const long long off = static_cast<long long>(b) * p.sb + static_cast<long long>(g) * p.sg +
+                        static_cast<long long>(pos) * p.sp;
+  const int x0 = c * CH;
+  int len = min(CH, p.V - x0);
+  if (!SV_IN(p.ctrl, b, p.B) || !SV_IN_RANGE(p.ctrl, off + x0, len, p.t_elems)) len = 0;
+  float best = -INFINITY;
+  int idx = INT_MAX;
+  if (kVec) {
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const T*>(p.tgt) + off + x0);
+    const int nv = len / EPV;
+    uint4 v[kOsVecs];
+#pragma unroll
+    for (int q = 0; q < kOsVecs; ++q) {
+      const int i = tid + q * kOsThreads;
+      v[q] = i < nv ? __ldcs(src + i) : neg_inf_vec<T>();  // read once: streaming hint
+    }
+    int bj = -1;
+    uint4 bvec = v[0];
+#pragma unroll
+    for (int q = 0; q < kOsVecs; ++q) {  // increasing index: the first maximum is kept
+      const float m = vec_max<T>(v[q]);
+      const bool take = tid + q * kOsThreads < nv && (bj < 0 || m > best);
+      best = take ? m : best;
+      bj = take ? q : bj;
+      bvec = take ? v[q] : bvec;
+    }
+    if (bj >= 0) {
+      float f[EPV];
+      unpack(bvec, f);
+      const int x = x0 + (tid + bj * kOsThreads) * EPV;
+#pragma unroll
+      for (int q = EPV - 1; q >= 0; --q)
+        if (f[q] == best) idx = x + q;
+    }
+    const int e = nv * EPV + tid;  // the ragged end is shorter than one vector
+    if (e < len) {
+      const float t = load_elem<T>(p.tgt, off + x0 + e);
+      if (better(t, x0 + e, best, idx)) {
+        best = t;
+        idx = x0 + e;
+      }
+    }
+  } else {
+    for (int e = tid; e < len; e += kOsThreads) {
+      const float t = load_elem<T>(p.tgt, off + x0 + e);
+      if (better(t, x0 + e, best, idx)) {
+        best = t;
+        idx = x0 + e;
+      }
+    }
+  }
+  warp_argmax(best, idx);
+  if (lane == 0) s_key[tid >> 5] = idx == INT_MAX ? 0ull : make_key(best, idx);
+  __syncthreads();
+  if (tid == 0) {
+    unsigned long long key = 0ull;
+#pragma unroll
+    for (int w = 0; w < kOsThreads / 32; ++w) key = s_key[w] > key ? s_key[w] : key;
+    if (key && SV_IN(p.ctrl, row, static_cast<long long>(p.B) * p.R))
+      atomicMax(p.rkey + row, key);
+    __threadfence();  // the row key before the count
+    const unsigned int done = atomicAdd(&p.seq[b].cnt1, 1u);
+    s_last = done == static_cast<unsigned int>(p.R) * static_cast<unsigned int>(p.nch1) - 1u;
+    if (s_last) __threadfence();  // every block's row keys after the count
+  }
+  __syncthreads();
+  if (s_last && tid < 32) finalize_argmax(p, b, lane);
+}
+
+template <typename T>
+static cudaError_t launch_oneshot_t(const ArgmaxParams& p, bool vec, cudaStream_t st) {
+  const long long blocks = static_cast<long long>(p.B) * p.R * p.nch1;
+  if (blocks <= 0) return cudaSuccess;
+  if (vec)
+    argmax_oneshot_kernel<T, true><<<static_cast<unsigned int>(blocks), kOsThreads, 0, st>>>(p);
+  else
+    argmax_oneshot_kernel<T, false><<<static_cast<unsigned int>(blocks), kOsThreads, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_argmax_oneshot(const ArgmaxParams& p, int t_dtype, bool vec, cudaStream_t st) {
+  return t_dtype == 1 ? launch_oneshot_t<uint16_t>(p, vec, st) : launch_oneshot_t<float>(p, vec, st);
 }
 
 // ================================================================ philox

@@ -294,7 +294,9 @@ template <typename T>
 __global__ void __launch_bounds__(kTsThreads) tree_sample_kernel(TreeStochParams p) {
   constexpr int EPV = Elem<T>::kPerVec;
   constexpr int CH = kSampleEntries;
-  __shared__ int s_ex[kMaxNodes];
+  // E (the rejected tokens at the final node) as a bitmap over this block's
+  // entries: one shared-memory word per 32 entries
+  __shared__ uint32_t s_emask[CH / 32];
   __shared__ unsigned long long s_ke[kTsThreads / 32], s_ka[kTsThreads / 32];
   const int c = static_cast<int>(blockIdx.x % p.nch_s);
   const int b = static_cast<int>(blockIdx.x / p.nch_s);
@@ -302,36 +304,37 @@ __global__ void __launch_bounds__(kTsThreads) tree_sample_kernel(TreeStochParams
   TreeRec& rec = p.rec[b];
   const int u = rec.u, ne = min(rec.ne, kMaxNodes);
   const uint32_t tag = static_cast<uint32_t>(rec.tag);
-  if (tid < ne) s_ex[tid] = rec.excl[tid];
+  const int x0 = c * CH;
+  if (tid < CH / 32) s_emask[tid] = 0u;
+  __syncthreads();
+  if (tid < ne) {
+    const int xe = rec.excl[tid] - x0;
+    if (xe >= 0 && xe < CH) atomicOr(&s_emask[xe >> 5], 1u << (xe & 31));
+  }
   __syncthreads();
 
   const long long off = static_cast<long long>(b) * p.sb + static_cast<long long>(u) * p.sn;
   const uint32_t seq = static_cast<uint32_t>(b) + p.seq_offset;
-  const int x0 = c * CH;
   int len = min(CH, p.V - x0);
   if (!SV_IN(p.ctrl, u, p.N) ||
       !SV_IN_RANGE(p.ctrl, off + x0, len, p.l_elems))
     len = 0;  // (bounds-checked builds: a bad block reads nothing)
   float bv = -INFINITY, av = -INFINITY;  // best outside E, best of the row
   int bi = INT_MAX, ai = INT_MAX;
-  auto take = [&](float l, uint32_t word, int x) {
-    const float sc = fmaf(l, p.c2, gumbel_log2(neg_exp1_log2(word)));
-    if (sc > av) {
-      av = sc;
-      ai = x;
-    }
-    if (sc > bv) {  // entries arrive in increasing x: the first maximum is kept
-      bool in_e = false;
-      for (int e = 0; e < ne; ++e) in_e |= s_ex[e] == x;
-      if (!in_e) {
-        bv = sc;
-        bi = x;
-      }
-    }
+  // entries arrive in increasing x: a strict > keeps the first maximum
+  auto take = [&](float sc, bool in_e, int x) {
+    const bool wa = sc > av, wb = sc > bv && !in_e;
+    av = wa ? sc : av;
+    ai = wa ? x : ai;
+    bv = wb ? sc : bv;
+    bi = wb ? x : bi;
   };
   auto words = [&](int x) {
     return philox10(make_uint4(static_cast<uint32_t>(x) >> 2, static_cast<uint32_t>(u), seq, tag),
                     p.key0, p.key1);
+  };
+  auto score1 = [&](float l, uint32_t word) {
+    return fmaf(l, p.c2, gumbel_log2(neg_exp1_log2(word)));
   };
   if (p.vec) {
     const uint4* src = reinterpret_cast<const uint4*>(static_cast<const T*>(p.logits) + off + x0);
@@ -339,25 +342,31 @@ __global__ void __launch_bounds__(kTsThreads) tree_sample_kernel(TreeStochParams
     for (int i = tid; i < nv; i += kTsThreads) {
       float f[EPV];
       unpack(__ldg(src + i), f);
-      const int xv = x0 + i * EPV;
+      const int e0 = i * EPV;
+      const uint32_t m = s_emask[e0 >> 5] >> (e0 & 31);  // EPV bits, one word (EPV | 32)
 #pragma unroll
       for (int g = 0; g < EPV / 4; ++g) {
-        const uint4 wd = words(xv + 4 * g);
-        take(f[4 * g + 0], wd.x, xv + 4 * g + 0);
-        take(f[4 * g + 1], wd.y, xv + 4 * g + 1);
-        take(f[4 * g + 2], wd.z, xv + 4 * g + 2);
-        take(f[4 * g + 3], wd.w, xv + 4 * g + 3);
+        const uint4 wd = words(x0 + e0 + 4 * g);
+        float ev[4], sc[4];
+        neg_exp1_log2_x2(wd.x, wd.y, ev[0], ev[1]);
+        neg_exp1_log2_x2(wd.z, wd.w, ev[2], ev[3]);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) sc[q] = fmaf(f[4 * g + q], p.c2, gumbel_log2(ev[q]));
+#pragma unroll
+        for (int q = 0; q < 4; ++q) take(sc[q], (m >> (4 * g + q)) & 1u, x0 + e0 + 4 * g + q);
       }
     }
     const int te = nv * EPV + tid;
     if (te < len) {
       const int x = x0 + te;
-      take(load_elem<T>(p.logits, off + x), word_of(words(x), x & 3), x);
+      take(score1(load_elem<T>(p.logits, off + x), word_of(words(x), x & 3)),
+           (s_emask[te >> 5] >> (te & 31)) & 1u, x);
     }
   } else {
     for (int e = tid; e < len; e += kTsThreads) {
       const int x = x0 + e;
-      take(load_elem<T>(p.logits, off + x), word_of(words(x), x & 3), x);
+      take(score1(load_elem<T>(p.logits, off + x), word_of(words(x), x & 3)),
+           (s_emask[e >> 5] >> (e & 31)) & 1u, x);
     }
   }
   warp_argmax(bv, bi);

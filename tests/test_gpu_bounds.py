@@ -21,7 +21,9 @@ import test_gpu_parity as tp
 
 pytestmark = pytest.mark.gpu
 
-CASES = [
+# greedy and multi-candidate cases run on both of their paths (one grid of
+# row-chunk blocks, the persistent pipeline)
+ARGMAX_CASES = [
     (tp.test_greedy_parity_shapes, dict(dtype="bf16", B=129, k=4, V=7)),
     (tp.test_greedy_parity_shapes, dict(dtype="f32", B=3, k=32, V=31)),
     (tp.test_greedy_parity_shapes, dict(dtype="bf16", B=1, k=8, V=4097)),
@@ -35,6 +37,9 @@ CASES = [
     (tp.test_multi_parity_shapes, dict(dtype="f32", B=4, G=5, k=32, V=40)),
     (tp.test_multi_early_exit_is_exact_and_leaves_the_workspace_clean,
      dict(B=64, G=8, k=4, V=32000)),
+]
+CASES = [(fn, dict(kw, argmax_path=path)) for fn, kw in ARGMAX_CASES
+         for path in ("oneshot", "persistent")] + [
     (tp.test_multi_rows_invalid_entries_and_limits, {}),
     (tp.test_threshold_invalid_tokens_and_workspace, {}),
     (tp.test_tree_invalid_parent_flag, {}),
@@ -79,6 +84,9 @@ def test_parity_case_on_the_bounds_checked_build(bounds_lib, monkeypatch, fn, kw
         init(self, *a, **k)
         made.append(self)
 
+    if "argmax_path" in kw:
+        monkeypatch.setenv("SV_ONESHOT_MAX_BYTES",
+                           "0" if kw["argmax_path"] == "persistent" else str(1 << 62))
     monkeypatch.setattr(sv, "_lib", bounds_lib)
     monkeypatch.setattr(sv, "_default_ws", {})
     monkeypatch.setattr(sv.Workspace, "__init__", recording_init)

@@ -26,6 +26,21 @@ TOL_GAP = 1e-5
 THREADS = os.cpu_count() or 1
 
 
+@pytest.fixture
+def argmax_path(request, monkeypatch):
+    """Plain greedy and multi-candidate calls run either as one grid of
+    row-chunk blocks (small calls) or on the persistent pipeline with early
+    exit (large calls); the size limit between them is overridden here so
+    that both paths meet every case."""
+    monkeypatch.setenv("SV_ONESHOT_MAX_BYTES", "0" if request.param == "persistent" else
+                       str(1 << 62))
+    return request.param
+
+
+both_argmax_paths = pytest.mark.parametrize("argmax_path", ["oneshot", "persistent"],
+                                            indirect=True)
+
+
 @pytest.fixture(scope="module")
 def dev():
     from speculative_decoding_verification_88_b200 import build
@@ -131,11 +146,12 @@ def tie_heavy(rng, shape):
     return x
 
 
+@both_argmax_paths
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("B,k,V", [(1, 0, 1), (3, 1, 2), (129, 4, 7), (3, 8, 8), (1, 4, 9),
                                    (3, 32, 31), (129, 2, 33), (3, 4, 4095), (1, 8, 4097),
                                    (5, 3, 32000), (2, 4, 128256)])
-def test_greedy_parity_shapes(dev, dtype, B, k, V):
+def test_greedy_parity_shapes(dev, argmax_path, dtype, B, k, V):
     rng = np.random.default_rng(B * 1000 + k * 10 + V)
     if V <= 64:
         x = tie_heavy(rng, (B, k + 1, V))
@@ -152,7 +168,8 @@ def test_greedy_parity_shapes(dev, dtype, B, k, V):
     np.testing.assert_array_equal(r["out_tokens"].cpu().numpy(), o["out_tokens"])
 
 
-def test_greedy_strided_unaligned_and_broadcast(dev):
+@both_argmax_paths
+def test_greedy_strided_unaligned_and_broadcast(dev, argmax_path):
     rng = np.random.default_rng(3)
     B, k, V = 6, 4, 1001
     big = workloads.f32_to_bf16_bits(rng.standard_normal((B, k + 2, V + 3)).astype(np.float32))
@@ -172,7 +189,8 @@ def test_greedy_strided_unaligned_and_broadcast(dev):
     np.testing.assert_array_equal(r["out_tokens"].cpu().numpy(), o["out_tokens"])
 
 
-def test_greedy_all_accepted_and_none(dev):
+@both_argmax_paths
+def test_greedy_all_accepted_and_none(dev, argmax_path):
     rng = np.random.default_rng(4)
     B, k, V = 40, 6, 5000
     x = workloads.f32_to_bf16_bits(rng.standard_normal((B, k + 1, V)).astype(np.float32))
@@ -187,9 +205,10 @@ def test_greedy_all_accepted_and_none(dev):
     np.testing.assert_array_equal(r["out_tokens"].cpu().numpy()[:, 0], am[:, 0])
 
 
+@both_argmax_paths
 @pytest.mark.parametrize("B,k,V,p_match", [(512, 8, 32000, 0.5), (300, 32, 4000, 0.9),
                                            (1024, 2, 20000, 0.3)])
-def test_greedy_early_exit_is_exact_and_leaves_the_workspace_clean(dev, B, k, V, p_match):
+def test_greedy_early_exit_is_exact_and_leaves_the_workspace_clean(dev, argmax_path, B, k, V, p_match):
     """Batches large enough that rows past a branch's first mismatch are
     retired unread: results stay bit-exact, the flag word stays clear for
     valid drafts, and the workspace (branch states included) is left zero."""
@@ -208,8 +227,9 @@ def test_greedy_early_exit_is_exact_and_leaves_the_workspace_clean(dev, B, k, V,
     assert 0 < o["accepted_len"].mean() < k
 
 
+@both_argmax_paths
 @pytest.mark.parametrize("B,G,k,V", [(64, 8, 4, 32000), (40, 64, 6, 3000)])
-def test_multi_early_exit_is_exact_and_leaves_the_workspace_clean(dev, B, G, k, V):
+def test_multi_early_exit_is_exact_and_leaves_the_workspace_clean(dev, argmax_path, B, G, k, V):
     w = workloads.make_multi(B, G, k, V, p_match=0.5, seed=G + k, threads=THREADS)
     t = to_dev(w["target"], "bf16", dev)
     tok = torch.from_numpy(w["tokens"]).to(dev)
@@ -224,7 +244,8 @@ def test_multi_early_exit_is_exact_and_leaves_the_workspace_clean(dev, B, G, k, 
     assert ws.device_status() == 0
 
 
-def test_greedy_invalid_drafts_raise_the_flag(dev):
+@both_argmax_paths
+def test_greedy_invalid_drafts_raise_the_flag(dev, argmax_path):
     w = workloads.make_greedy(9, 4, 3000, seed=5)
     w["tokens"][4, 2] = -7
     w["tokens"][8, 0] = 3000
@@ -242,10 +263,11 @@ def test_greedy_invalid_drafts_raise_the_flag(dev):
 
 # ---------------------------------------------------------- multi-candidate
 
+@both_argmax_paths
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("B,G,k,V", [(1, 1, 4, 100), (3, 3, 2, 17), (16, 8, 4, 3001),
                                      (2, 64, 3, 50), (4, 5, 32, 40), (2, 2, 0, 10)])
-def test_multi_parity_shapes(dev, dtype, B, G, k, V):
+def test_multi_parity_shapes(dev, argmax_path, dtype, B, G, k, V):
     rng = np.random.default_rng(B + G * 7 + k * 13 + V)
     x = tie_heavy(rng, (B, G, k + 1, V)) if V < 64 else \
         rng.standard_normal((B, G, k + 1, V)).astype(np.float32) * 3

@@ -23,12 +23,26 @@ def lib():
     return sv.load_library()
 
 
+def largest_batch(lib, k, V):
+    """The largest B whose workspace fits the 2 MiB array."""
+    lo, hi = 0, 1 << 16
+    while lo < hi:
+        m = (lo + hi + 1) // 2
+        if lib.spec_verify_workspace_size(m, 1, k, V) <= (2 << 20):
+            lo = m
+        else:
+            hi = m - 1
+    return lo
+
+
 def test_noalloc_rejects_problems_beyond_its_scratch(lib):
-    # Fails on the host before any device work: too large for the 2 MiB array
-    # (spec_verify_workspace_size(783, 1, 8, 128256) is above it).
-    rc = lib.spec_verify_greedy_noalloc(None, 1, 0, 0, None, 783, 8, 128256, None, None, None)
+    # Fails on the host before any device work: one sequence more than the
+    # 2 MiB array holds.
+    top = largest_batch(lib, 8, 128256)
+    assert top >= 700
+    rc = lib.spec_verify_greedy_noalloc(None, 1, 0, 0, None, top + 1, 8, 128256, None, None,
+                                        None)
     assert rc == 3  # SV_ERR_WORKSPACE
-    assert lib.spec_verify_workspace_size(782, 1, 8, 128256) <= (2 << 20)
     rc = lib.spec_verify_greedy_noalloc(None, 1, 0, 0, None, 4, 40, 100, None, None, None)
     assert rc == 1  # SV_ERR_INVALID_ARG (k > 32)
     assert lib.spec_verify_greedy_noalloc(None, 1, 0, 0, None, 0, 4, 100, None, None, None) == 0
@@ -36,7 +50,7 @@ def test_noalloc_rejects_problems_beyond_its_scratch(lib):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("B,k,V", [(64, 4, 128256), (7, 3, 4097), (782, 8, 2000)])
+@pytest.mark.parametrize("B,k,V", [(64, 4, 128256), (7, 3, 4097), (760, 8, 2000)])
 def test_noalloc_matches_oracle_and_workspace_entry_point_twice(lib, B, k, V):
     dev = torch.device("cuda:0")
     w = workloads.make_greedy(B, k, V, p_match=0.7, seed=B + k)
