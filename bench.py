@@ -162,6 +162,61 @@ def recorded_traffic(workload: str, batch_override: bool) -> float | None:
     return float(rec["dram_bytes_per_launch"])
 
 
+class NvmlSampler:
+    """SM clock and throttle reasons of one GPU read through NVML every half
+    millisecond from a background thread, so that a timed region of a few
+    milliseconds holds samples (nvidia-smi samples every 50-100 ms).  Reads
+    only; changes no setting."""
+
+    BITS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+            ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+            ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+            ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
+
+    def __init__(self, gpu_uuid: str):
+        self.samples: list[tuple[float, float, int]] = []
+        self.ok = False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+
+            self.nv = pynvml
+            pynvml.nvmlInit()
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(gpu_uuid)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+            self.mask = {name: getattr(pynvml, attr) for name, attr in self.BITS}
+            self.thread = threading.Thread(target=self._run, daemon=True)
+            self.thread.start()
+            self.ok = True
+        except Exception:
+            self.ok = False
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                sm = float(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                rs = int(nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+            except Exception:
+                break
+            self.samples.append((time.time(), sm, rs))
+            time.sleep(0.0005)
+
+    def stop(self, t0: float, t1: float) -> dict | None:
+        if not self.ok:
+            return None
+        self._stop.set()
+        self.thread.join(timeout=2)
+        sel = [(sm, rs) for ts, sm, rs in self.samples if t0 <= ts <= t1]
+        if not sel:
+            return None
+        reasons = sorted({name for name, bit in self.mask.items()
+                          for _, rs in sel if rs & bit})
+        return {"sm_mhz": statistics.median(sm for sm, _ in sel), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(sel),
+                "window": "timed region (NVML, every 0.5 ms)"}
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle samples of one GPU while it runs."""
 
@@ -510,7 +565,9 @@ def run_ours(args, rank: int, world: int, dist) -> None:
     K = args.steps
     e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     uuid = str(torch.cuda.get_device_properties(dev).uuid)
-    sampler = ClockSampler(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+    gpu_uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+    sampler = ClockSampler(gpu_uuid)
+    fast = NvmlSampler(gpu_uuid)
     time.sleep(1.0 if sampler.proc is not None else 0.0)
     if dist is not None:
         dist.barrier()
@@ -523,7 +580,9 @@ def run_ours(args, rank: int, world: int, dist) -> None:
     torch.cuda.synchronize()
     t1 = time.time()
     launches = K * per_replay
-    clocks = sampler.stop(t0, t1)
+    clocks = fast.stop(t0, t1) or sampler.stop(t0, t1)
+    if sampler.proc is not None and sampler.proc.poll() is None:
+        sampler.stop(t0, t1)
     elapsed_ms = e_start.elapsed_time(e_end)
     if dist is not None:
         t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)

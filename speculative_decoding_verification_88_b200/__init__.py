@@ -35,11 +35,11 @@ EXPORTS = (
     "spec_verify_philox4x32_10", "spec_verify_greedy_noalloc",
     "spec_verify_greedy_noalloc_read_device_status",
     "spec_verify_tree_stochastic_workspace_size", "spec_verify_tree_stochastic",
+    "spec_verify_kernel_launches",
 )
 
 _lib = None
 _lock = threading.Lock()
-_launches = 0
 
 
 class SpecVerifyError(RuntimeError):
@@ -105,6 +105,8 @@ def load_library(path: str | None = None):
         lib.spec_verify_greedy_noalloc.restype = I
         lib.spec_verify_greedy_noalloc_read_device_status.argtypes = [ctypes.POINTER(U32), I, P]
         lib.spec_verify_greedy_noalloc_read_device_status.restype = I
+        lib.spec_verify_kernel_launches.argtypes = []
+        lib.spec_verify_kernel_launches.restype = U64
         if path is None:
             _lib = lib
         return lib
@@ -120,13 +122,9 @@ def _check(code: int, what: str):
 
 
 def launch_count() -> int:
-    """Number of verify/philox calls (one kernel launch each) so far."""
-    return _launches
-
-
-def _count(n: int = 1):
-    global _launches
-    _launches += n
+    """Kernels the library has launched in this process so far (its own
+    count; a launch captured into a CUDA graph counts once, at capture)."""
+    return int(load_library().spec_verify_kernel_launches())
 
 
 def workspace_size(B: int, G: int, k: int, V: int) -> int:
@@ -253,7 +251,6 @@ def stochastic(target: torch.Tensor, draft: torch.Tensor, draft_tokens: torch.Te
             res["probs"].data_ptr() if probs else None, ws.buf.data_ptr(), ws.nbytes,
             _stream_ptr(stream, dev))
     _check(code, "spec_verify_stochastic")
-    _count()
     return res
 
 
@@ -276,7 +273,6 @@ def greedy(target: torch.Tensor, draft_tokens: torch.Tensor, *, out: dict | None
             res["accepted_len"].data_ptr(), res["out_tokens"].data_ptr(), ws.buf.data_ptr(),
             ws.nbytes, _stream_ptr(stream, dev))
     _check(code, "spec_verify_greedy")
-    _count()
     return res
 
 
@@ -300,7 +296,6 @@ def multi_candidate(target: torch.Tensor, cand_tokens: torch.Tensor, *, out: dic
             res["best_candidate"].data_ptr(), res["accepted_len"].data_ptr(),
             res["out_tokens"].data_ptr(), ws.buf.data_ptr(), ws.nbytes, _stream_ptr(stream, dev))
     _check(code, "spec_verify_multi_candidate")
-    _count()
     return res
 
 
@@ -331,7 +326,6 @@ def multi_candidate_rows(rows: torch.Tensor, row_of: torch.Tensor, cand_tokens: 
             res["best_candidate"].data_ptr(), res["accepted_len"].data_ptr(),
             res["out_tokens"].data_ptr(), ws.buf.data_ptr(), ws.nbytes, _stream_ptr(stream, dev))
     _check(code, "spec_verify_multi_candidate_rows")
-    _count()
     return res
 
 
@@ -357,7 +351,6 @@ def threshold(target: torch.Tensor, draft_tokens: torch.Tensor, temperature: flo
             float(threshold), res["accepted_len"].data_ptr(), res["out_tokens"].data_ptr(),
             ws.buf.data_ptr(), ws.nbytes, _stream_ptr(stream, dev))
     _check(code, "spec_verify_threshold")
-    _count()
     return res
 
 
@@ -388,7 +381,6 @@ def tree_greedy(node_logits: torch.Tensor, parent: torch.Tensor, tokens: torch.T
             res["accepted_len"].data_ptr(), res["path"].data_ptr(), res["out_tokens"].data_ptr(),
             ws.buf.data_ptr(), ws.nbytes, _stream_ptr(stream, dev))
     _check(code, "spec_verify_tree_greedy")
-    _count()
     return res
 
 
@@ -422,7 +414,6 @@ def tree_stochastic(node_logits: torch.Tensor, parent: torch.Tensor, tokens: tor
             res["accepted_len"].data_ptr(), res["path"].data_ptr(), res["out_tokens"].data_ptr(),
             ws.buf.data_ptr(), ws.nbytes, _stream_ptr(stream, dev))
     _check(code, "spec_verify_tree_stochastic")
-    _count(3)
     return res
 
 
@@ -461,7 +452,6 @@ def commit(result: dict, seq_len: torch.Tensor, token_buf: torch.Tensor, *,
             workspace.buf.data_ptr() if workspace is not None and workspace.buf is not None
             else None, _stream_ptr(stream, dev))
     _check(code, "spec_verify_commit")
-    _count()
 
 
 def greedy_noalloc(target: torch.Tensor, draft_tokens: torch.Tensor, *,
@@ -489,7 +479,6 @@ def greedy_noalloc(target: torch.Tensor, draft_tokens: torch.Tensor, *,
             target.data_ptr(), tc, tsb, tsp, tok.data_ptr(), B, k, V,
             res["accepted_len"].data_ptr(), res["out_tokens"].data_ptr(), _stream_ptr(stream, dev))
     _check(code, "spec_verify_greedy_noalloc")
-    _count()
     return res
 
 
@@ -517,5 +506,4 @@ def philox4x32_10(counters: torch.Tensor, seed: int, stream=None) -> torch.Tenso
         code = lib.spec_verify_philox4x32_10(c.data_ptr(), c.shape[0], int(seed) & (2**64 - 1),
                                               out.data_ptr(), _stream_ptr(stream, c.device))
     _check(code, "spec_verify_philox4x32_10")
-    _count()
     return out

@@ -1,6 +1,7 @@
 // sv_api.cu -- the C ABI of libspecverify.so (include/spec_verify.h):
 // argument validation, chunk planning, workspace layout and kernel dispatch.
 // Host code only; every step of the verify path runs in sv_kernels.cu.
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstdlib>
@@ -183,6 +184,19 @@ extern "C" size_t spec_verify_workspace_size(int B, int G, int k, int V) {
   const size_t total = kCtrlBytes + seq_bytes(B) + tail;
   return (total + 255) / 256 * 256;
 }
+
+namespace sv {
+namespace {
+std::atomic<unsigned long long> g_launches{0};
+}  // namespace
+cudaError_t counted(cudaError_t e, int n) {
+  if (e == cudaSuccess) g_launches.fetch_add(static_cast<unsigned long long>(n));
+  return e;
+}
+unsigned long long launches_so_far() { return g_launches.load(); }
+}  // namespace sv
+
+extern "C" unsigned long long spec_verify_kernel_launches(void) { return sv::launches_so_far(); }
 
 extern "C" const char* spec_verify_status_string(int status) {
   switch (status) {

@@ -186,6 +186,18 @@ __device__ __forceinline__ void fence_acq_rel_gpu() {
   asm volatile("fence.acq_rel.gpu;" ::: "memory");
 }
 
+// Programmatic dependent launch: a grid lets the next grid on its stream be
+// scheduled (once every block of it has executed this or exited), and the
+// dependent grid waits until its prerequisite grid has completed and that
+// grid's memory operations are visible.  Without a programmatic launch the
+// wait returns at once.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // Orders this thread's generic-proxy accesses to global memory before its
 // later async-proxy (bulk copy) accesses, and the reverse.
 __device__ __forceinline__ void fence_proxy_async_global() {

@@ -196,8 +196,9 @@ cudaError_t launch_stochastic(const StochParams& p, int t_dtype, int d_dtype, bo
 cudaError_t launch_argmax(const ArgmaxParams& p, int t_dtype, bool tma, int grid, size_t smem,
                           cudaStream_t stream);
 // Plain greedy / multi-candidate verify as one grid of row-chunk blocks (no
-// persistent pipeline): every row is read, all of a block's loads are in
-// flight at once, and the last block of a sequence finalizes it.
+// persistent pipeline): every row is read and all of a block's loads are in
+// flight at once; a second grid (a programmatic dependent launch) finalizes
+// every sequence.
 cudaError_t launch_argmax_oneshot(const ArgmaxParams& p, int t_dtype, bool vec, cudaStream_t st);
 int oneshot_chunk_entries(int t_dtype);
 cudaError_t launch_commit(const int* accepted_len, const int* out_tokens, int B, int k,
@@ -206,5 +207,12 @@ cudaError_t launch_commit(const int* accepted_len, const int* out_tokens, int B,
 cudaError_t launch_philox(const uint4* ctr, long long n, unsigned int key0, unsigned int key1,
                           uint4* out, cudaStream_t stream);
 size_t kernel_smem_bytes();
+
+// Kernels of this library launched in this process, counted when a launch
+// returns success (a launch captured into a CUDA graph counts once, at
+// capture).  Returns its argument, so a launcher can end with
+// `return counted(cudaGetLastError(), n)`.
+cudaError_t counted(cudaError_t e, int n);
+unsigned long long launches_so_far();
 
 }  // namespace sv

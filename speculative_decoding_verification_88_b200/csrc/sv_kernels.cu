@@ -869,7 +869,16 @@ __device__ __forceinline__ bool stoch_issue_phase2(const StochParams& p, Shared&
 }
 
 // Producer of compute group g: phase-1 chunks in position-major ticket order,
-// phase-2 chunks from the ready list, the latter first whenever one is ready.
+// then phase-2 chunks from the ready list.
+//  - Phase 1 goes first: the decisions of the last positions, which only
+//    phase-1 chunks advance, are the kernel's critical path, while the
+//    phase-2 chunks of sequences resolved early can wait.  A producer that
+//    served every ready phase-2 chunk before its drawn phase-1 tickets held
+//    those tickets (and the rows they complete) for up to kDefer phase-2
+//    computations.  Graph-timed, same box (us): B = 256, k = 8: 175.8 ->
+//    168.4; B = 64, k = 4: 75.6 -> 73.9; B = 1: 22.6 -> 21.6 (SV_P1_FIRST 0
+//    restores phase 2 first; SV_P2_RUN n > 0 lets n phase-2 chunks pass a
+//    drawn phase-1 ticket, which measured no better than 0).
 //  - Phase-1 tickets are taken one at a time, two ahead, and the state word
 //    of each ticket's sequence is loaded one ticket ahead: a chunk of pair i
 //    whose sequence already has a rejection before i is retired unread (its
@@ -879,10 +888,24 @@ __device__ __forceinline__ bool stoch_issue_phase2(const StochParams& p, Shared&
 //    polled with relaxed loads (issued before the current chunk's stage wait,
 //    read at the next iteration) and a chunk is issued once its entry is
 //    visible.  When no phase-1 ticket is left, the producer waits (bounded)
-//    for the oldest held entry.
+//    for the oldest held entry.  Holding fewer tickets spreads a late
+//    sequence's chunks over more producers.  kDefer 1 / 2 / 3, phase 1
+//    first (us): B = 256: 162.5 / 163.8 / 164.7; B = 64: 70.0 / 70.8 / 72.0;
+//    in another run 4 against 2: 168.0 against 163.9 and 73.7 against 71.1,
+//    and 8 was slower still.
+#ifndef SV_P2_RUN
+#define SV_P2_RUN 0
+#endif
+#ifndef SV_P1_FIRST
+#define SV_P1_FIRST 1
+#endif
+#ifndef SV_DEFER
+#define SV_DEFER 1
+#endif
 template <typename TT, typename TD, bool kTma>
 __device__ void stoch_producer(const StochParams& p, Shared& sh, unsigned char* stages, int g) {
-  constexpr int kDefer = 4;
+  constexpr int kDefer = SV_DEFER;
+  int run = 0;  // phase-2 chunks issued since the last phase-1 ticket was served
   constexpr unsigned int kNone = 0xffffffffu;
   Ctrl* ctrl = p.ctrl;
   const unsigned int nch = static_cast<unsigned int>(p.nch);
@@ -981,7 +1004,10 @@ __device__ void stoch_producer(const StochParams& p, Shared& sh, unsigned char* 
     // keep up to kDefer phase-2 tickets in hand (the atomic's result is used
     // at the next iteration)
     if (!t2_done && nd < kDefer) t2p = atomicAdd(&ctrl->ticket2, 1u);
+    if (rd >= 0 && t1 < p.total1 && (SV_P1_FIRST || (SV_P2_RUN > 0 && run >= SV_P2_RUN)))
+      rd = -1;  // the drawn phase-1 ticket goes first; the ready entry stays held
     if (rd >= 0) {
+      ++run;
       unsigned long long v = 0ull;
       unsigned int tsel = 0u;
 #pragma unroll
@@ -1026,6 +1052,7 @@ __device__ void stoch_producer(const StochParams& p, Shared& sh, unsigned char* 
       h.i = static_cast<int>(i);
       h.c = static_cast<int>(t1 - row * nch);
       const unsigned int rej = rejected_bits(s1);
+      run = 0;
       // advance the ticket pipeline before this chunk's stage wait
       t1 = t1n;
       s1 = s1n;
@@ -1135,21 +1162,31 @@ __device__ __forceinline__ unsigned long long take(unsigned long long* slot, uns
 
 // Resolution of sequence b (one warp), once its accepted length n is known:
 // the committed drafts and the -1 padding, the row-n statistics for the
-// phase-2 draw (consumed from the rejected row's record), and an entry in the
-// ready list that releases its phase-2 chunks.
-__device__ void resolve_sequence(const StochParams& p, int b, int n, int lane) {
+// phase-2 draw (consumed from the rejected row's record; `own`, when not null,
+// holds them already -- the caller merged row n -- and the record is only
+// cleared), and an entry in the ready list that releases its phase-2 chunks.
+__device__ void resolve_sequence(const StochParams& p, int b, int n, int lane,
+                                 const float4* own) {
   const int k = p.k;
   if (!SV_IN(p.ctrl, b, p.B) || !SV_IN(p.ctrl, n, k + 1)) return;
   float4 st = make_float4(0.0f, 1.0f, 0.0f, 1.0f);
   if (n < k) {
     unsigned long long* row = p.r1 + (static_cast<size_t>(b) * k + n) * 2;
-    float m, sm;
-    unpack_stats(take(row, ld_relaxed_u64(row), p.ctrl), m, sm);
-    st.x = m;
-    st.y = sm;
-    unpack_stats(take(row + 1, ld_relaxed_u64(row + 1), p.ctrl), m, sm);
-    st.z = m;
-    st.w = sm;
+    if (own) {
+      st = *own;
+      if (lane == 0) {  // the lane that wrote the record
+        row[0] = 0ull;
+        row[1] = 0ull;
+      }
+    } else {
+      float m, sm;
+      unpack_stats(take(row, ld_relaxed_u64(row), p.ctrl), m, sm);
+      st.x = m;
+      st.y = sm;
+      unpack_stats(take(row + 1, ld_relaxed_u64(row + 1), p.ctrl), m, sm);
+      st.z = m;
+      st.w = sm;
+    }
   }
   int* out = p.out_tokens + static_cast<size_t>(b) * (k + 1);
   for (int i = lane; i <= k; i += 32)
@@ -1254,7 +1291,8 @@ __device__ void merge_row(const StochParams& p, int b, int i, int lane) {
   const unsigned long long now = old | bits;
   int n_old, n_now;
   const bool was = resolved(old, k, n_old);
-  if (!was && resolved(now, k, n_now)) resolve_sequence(p, b, n_now, lane);
+  if (!was && resolved(now, k, n_now))
+    resolve_sequence(p, b, n_now, lane, rejected && n_now == i ? &w : nullptr);
   if (decided_bits(old) != low_mask(k) && decided_bits(now) == low_mask(k)) {
     // the last row of the sequence: clear the records of rejected rows past
     // n (rows retired unread are never marked rejected and wrote none)
@@ -1988,12 +2026,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 // every thread loads its (up to) eight 16-byte vectors at once, takes the
 // first maximum, the block merges its warps in shared memory and publishes
 // the chunk's key with one 64-bit atomicMax on the row key (keys order like
-// (value, -index), so the max is the row's first maximum); a fence and a
-// per-sequence counter then tell the last block of the sequence, which runs
-// the same finalize as the persistent kernel.  Blocks go sequence by
-// sequence, so sequences finalize while later ones stream.
-constexpr int kOsThreads = 256;
-constexpr int kOsVecs = 8;
+// (value, -index), so the max is the row's first maximum), whose result it
+// does not wait for, and exits.  A block that also counted itself and let the
+// last block finalize would hold its slot on the SM for two more L2 round
+// trips (a third of its life), and the slots are what limits the bytes in
+// flight (55 registers a thread: four blocks, 128 KB, an SM).  So a second
+// grid of one warp per sequence runs the same finalize as the persistent
+// kernel; it is launched as a programmatic dependent of the first, so its
+// launch overlaps the streaming and its griddepcontrol.wait returns once the
+// first grid has completed and its atomics are visible.
+#ifndef SV_OS_THREADS
+#define SV_OS_THREADS 256
+#endif
+#ifndef SV_OS_VECS
+#define SV_OS_VECS 8
+#endif
+constexpr int kOsThreads = SV_OS_THREADS;
+constexpr int kOsVecs = SV_OS_VECS;
 
 template <typename T>
 __host__ __device__ constexpr int oneshot_chunk() {
@@ -2010,7 +2059,9 @@ __global__ void __launch_bounds__(kOsThreads)
   constexpr int EPV = Elem<T>::kPerVec;
   constexpr int CH = oneshot_chunk<T>();
   __shared__ unsigned long long s_key[kOsThreads / 32];
-  __shared__ int s_last;
+  // the finalize grid may be scheduled once every block has started; it
+  // still waits for this grid to complete
+  griddep_launch_dependents();
   const int tid = threadIdx.x, lane = tid & 31;
   const unsigned int row = udiv(blockIdx.x, p.div_nch1);  // b * R + r
   const int c = static_cast<int>(blockIdx.x - row * static_cast<unsigned int>(p.nch1));
@@ -2077,14 +2128,17 @@ __global__ void __launch_bounds__(kOsThreads)
 #pragma unroll
     for (int w = 0; w < kOsThreads / 32; ++w) key = s_key[w] > key ? s_key[w] : key;
     if (key && SV_IN(p.ctrl, row, static_cast<long long>(p.B) * p.R))
-      atomicMax(p.rkey + row, key);
-    __threadfence();  // the row key before the count
-    const unsigned int done = atomicAdd(&p.seq[b].cnt1, 1u);
-    s_last = done == static_cast<unsigned int>(p.R) * static_cast<unsigned int>(p.nch1) - 1u;
-    if (s_last) __threadfence();  // every block's row keys after the count
+      atomicMax(p.rkey + row, key);  // result unused: a fire-and-forget reduction
   }
-  __syncthreads();
-  if (s_last && tid < 32) finalize_argmax(p, b, lane);
+}
+
+// One warp per sequence, once every block of the streaming grid has published
+// its key (griddepcontrol.wait: that grid has completed and its atomics are
+// visible).
+__global__ void __launch_bounds__(256) argmax_finalize_kernel(const __grid_constant__ ArgmaxParams p) {
+  griddep_wait();
+  const int b = static_cast<int>(blockIdx.x) * 8 + (static_cast<int>(threadIdx.x) >> 5);
+  if (b < p.B) finalize_argmax(p, b, threadIdx.x & 31);
 }
 
 template <typename T>
@@ -2095,7 +2149,20 @@ static cudaError_t launch_oneshot_t(const ArgmaxParams& p, bool vec, cudaStream_
     argmax_oneshot_kernel<T, true><<<static_cast<unsigned int>(blocks), kOsThreads, 0, st>>>(p);
   else
     argmax_oneshot_kernel<T, false><<<static_cast<unsigned int>(blocks), kOsThreads, 0, st>>>(p);
-  return cudaGetLastError();
+  cudaError_t e = counted(cudaGetLastError(), 1);
+  if (e != cudaSuccess) return e;
+  // launched while the streaming grid runs; its warps wait for that grid
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned int>((p.B + 7) / 8));
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return counted(cudaLaunchKernelEx(&cfg, argmax_finalize_kernel, p), 1);
 }
 
 cudaError_t launch_argmax_oneshot(const ArgmaxParams& p, int t_dtype, bool vec, cudaStream_t st) {
@@ -2168,7 +2235,7 @@ static cudaError_t launch_stoch_t(const StochParams& p, int grid, size_t smem, c
   cudaError_t e = prepare(kernel, smem, done);
   if (e != cudaSuccess) return e;
   kernel<<<grid, kThreads, smem, st>>>(p);
-  return cudaGetLastError();
+  return counted(cudaGetLastError(), 1);
 }
 
 template <typename TT, typename TD>
@@ -2193,7 +2260,7 @@ static cudaError_t launch_argmax_t(const ArgmaxParams& p, int grid, size_t smem,
   cudaError_t e = prepare(kernel, smem, done);
   if (e != cudaSuccess) return e;
   kernel<<<grid, kThreads, smem, st>>>(p);
-  return cudaGetLastError();
+  return counted(cudaGetLastError(), 1);
 }
 
 template <typename TT>
@@ -2229,7 +2296,7 @@ cudaError_t launch_commit(const int* accepted_len, const int* out_tokens, int B,
   constexpr int kWarps = 8;
   commit_kernel<<<(B + kWarps - 1) / kWarps, 32 * kWarps, 0, st>>>(
       accepted_len, out_tokens, B, k, seq_len, token_buf, buf_stride, capacity, next_input, ctrl);
-  return cudaGetLastError();
+  return counted(cudaGetLastError(), 1);
 }
 
 cudaError_t launch_philox(const uint4* ctr, long long n, unsigned int key0, unsigned int key1,
@@ -2238,7 +2305,7 @@ cudaError_t launch_philox(const uint4* ctr, long long n, unsigned int key0, unsi
   const long long blocks = (n + 255) / 256;
   const int grid = static_cast<int>(blocks < 4096 ? blocks : 4096);
   philox_kernel<<<grid, 256, 0, st>>>(ctr, n, key0, key1, out);
-  return cudaGetLastError();
+  return counted(cudaGetLastError(), 1);
 }
 
 }  // namespace sv

@@ -439,14 +439,14 @@ template <typename T>
 cudaError_t launch_tree_stoch(const TreeStochParams& p, cudaStream_t st) {
   const long long rows = static_cast<long long>(p.B) * p.N;
   tree_stats_kernel<T><<<static_cast<unsigned int>(rows * p.nch), kTsThreads, 0, st>>>(p);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = counted(cudaGetLastError(), 1);
   if (e != cudaSuccess) return e;
   tree_walk_kernel<T><<<(p.B + kWalkWarps - 1) / kWalkWarps, 32 * kWalkWarps, 0, st>>>(p);
-  e = cudaGetLastError();
+  e = counted(cudaGetLastError(), 1);
   if (e != cudaSuccess) return e;
   tree_sample_kernel<T><<<static_cast<unsigned int>(static_cast<long long>(p.B) * p.nch_s),
                           kTsThreads, 0, st>>>(p);
-  return cudaGetLastError();
+  return counted(cudaGetLastError(), 1);
 }
 
 }  // namespace

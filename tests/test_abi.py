@@ -40,6 +40,11 @@ def test_library_exports_every_declared_symbol(lib):
         assert hasattr(lib, name), name
 
 
+def test_launch_counter_needs_no_device(lib):
+    n = lib.spec_verify_kernel_launches()
+    assert n >= 0 and lib.spec_verify_kernel_launches() == n  # nothing launched between
+
+
 def test_status_strings(lib):
     for code in range(6):
         assert sv.status_string(code).startswith("SV_")

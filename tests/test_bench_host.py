@@ -2,6 +2,7 @@
 traffic record's gating, the clock-sample parser, the workload selection,
 and the JSON line of the CPU-only reference arm."""
 import datetime
+import time
 import json
 import os
 import subprocess
@@ -140,6 +141,57 @@ def test_clock_sampler_keeps_samples_inside_the_window():
     out = cs.summarise(t0.timestamp() + 0.25, t0.timestamp() + 0.3)
     assert out["samples"] == 2 and out["sm_mhz"] == 1957.5
     assert out["window"].startswith("no sample inside")
+
+
+class _FakeNvml:
+    """The NVML calls the fast sampler makes, answering from a script of
+    (clock, reason bits) readings."""
+    NVML_CLOCK_SM = 1
+    nvmlClocksEventReasonHwSlowdown = 0x8
+    nvmlClocksEventReasonHwThermalSlowdown = 0x40
+    nvmlClocksEventReasonSwThermalSlowdown = 0x20
+    nvmlClocksEventReasonSwPowerCap = 0x4
+
+    def __init__(self, script):
+        self.script = list(script)
+
+    def nvmlInit(self):
+        pass
+
+    def nvmlDeviceGetHandleByUUID(self, uuid):
+        assert uuid.startswith("GPU-")
+        return "h"
+
+    def nvmlDeviceGetMaxClockInfo(self, h, kind):
+        return 1965
+
+    def nvmlDeviceGetClockInfo(self, h, kind):
+        if not self.script:
+            raise RuntimeError("done")  # ends the sampling thread
+        return self.script[0][0]
+
+    def nvmlDeviceGetCurrentClocksEventReasons(self, h):
+        return self.script.pop(0)[1]
+
+
+def test_nvml_sampler_reads_clocks_and_reasons(monkeypatch):
+    fake = _FakeNvml([(1965, 0), (1950, 0x4), (1965, 0x1), (1900, 0x4 | 0x8)])
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    t0 = time.time()
+    s = bench.NvmlSampler("GPU-0000")
+    assert s.ok
+    s.thread.join(timeout=5)
+    out = s.stop(t0 - 1.0, time.time() + 1.0)
+    # bit 0x1 (idle) is not a reason the record keeps
+    assert out["samples"] == 4 and out["sm_mhz"] == 1957.5 and out["sm_max_mhz"] == 1965.0
+    assert out["reasons"] == ["hw_slowdown", "sw_power_cap"]
+    assert s.stop(t0 - 10.0, t0 - 9.0) is None  # no sample inside: the caller falls back
+
+
+def test_nvml_sampler_absent(monkeypatch):
+    monkeypatch.setitem(sys.modules, "pynvml", None)  # import fails
+    s = bench.NvmlSampler("GPU-0000")
+    assert not s.ok and s.stop(0.0, 1.0) is None
 
 
 def test_select_workloads(monkeypatch):

@@ -789,6 +789,45 @@ def test_stochastic_seq_offset_and_repeat(dev):
         np.testing.assert_array_equal(a[both], b[both])
 
 
+@both_argmax_paths
+def test_kernel_launch_counts(dev, argmax_path):
+    """The library counts its own launches: one kernel per stochastic, commit
+    and Philox call, three per stochastic tree call, and per greedy or
+    multi-candidate call two on the one-grid path (the streaming grid, then
+    the finalize grid) and one on the persistent pipeline."""
+    ws = sv.Workspace(dev)
+    g = workloads.make_greedy(B=3, k=2, V=3000, seed=21)
+    t = to_dev(g["target"], "bf16", dev)
+    tok = torch.from_numpy(g["tokens"]).to(dev)
+    per_argmax = 2 if argmax_path == "oneshot" else 1
+    st = workloads.make_stochastic(B=3, k=2, V=3000, t_dtype="bf16", d_dtype="bf16", t_std=2.0,
+                                   d_noise=0.5, temperature=1.0, seed=22)
+    tr = workloads.make_tree(B=2, N=5, V=3000, seed=23)
+    seq = torch.zeros(3, dtype=torch.int32, device=dev)
+    buf = torch.full((3, 8), -1, dtype=torch.int32, device=dev)
+    calls = [
+        (per_argmax, lambda: sv.greedy(t, tok, workspace=ws)),
+        (per_argmax, lambda: sv.multi_candidate(t[:, None], tok[:, None], workspace=ws)),
+        (1, lambda: sv.stochastic(to_dev(st["target"], "bf16", dev), to_dev(st["draft"], "bf16", dev),
+                                  torch.from_numpy(st["tokens"]).to(dev), 1.0, 5, workspace=ws)),
+        (3, lambda: sv.tree_stochastic(to_dev(tr["node_logits"], "bf16", dev),
+                                       torch.from_numpy(tr["parent"]).to(dev),
+                                       torch.from_numpy(tr["tokens"]).to(dev), 1.0, 5)),
+        (1, lambda: sv.tree_greedy(to_dev(tr["node_logits"], "bf16", dev),
+                                   torch.from_numpy(tr["parent"]).to(dev),
+                                   torch.from_numpy(tr["tokens"]).to(dev))),
+        (1, lambda: sv.philox4x32_10(torch.zeros(5, 4, dtype=torch.int32, device=dev), 3)),
+    ]
+    for want, fn in calls:
+        n0 = sv.launch_count()
+        r = fn()
+        assert sv.launch_count() - n0 == want
+    n0 = sv.launch_count()
+    sv.commit(sv.greedy(t, tok, workspace=ws), seq, buf)
+    assert sv.launch_count() - n0 == per_argmax + 1
+    torch.cuda.synchronize()
+
+
 def test_one_workspace_across_modes_and_sizes(dev):
     """Calls of every mode and many sizes share one workspace; each call must
     leave it clean for the next."""
