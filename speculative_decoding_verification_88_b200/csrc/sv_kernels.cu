@@ -1817,6 +1817,9 @@ __device__ void finalize_argmax_rows(const ArgmaxParams& p, int b, int lane) {
 // Finalize of sequence b (one warp): per branch, the accepted length is the
 // first position whose draft differs from the row argmax (ballot); the
 // longest branch (lowest g on a tie) is committed.
+// kOneGrid: called by the finalize grid of the one-grid path, which runs after
+// the streaming grid has completed; no branch state to clear, so no fence.
+template <bool kOneGrid>
 __device__ void finalize_argmax(const ArgmaxParams& p, int b, int lane) {
   const int k = p.k, G = p.G;
   unsigned long long* keys = p.rkey + static_cast<size_t>(b) * G * (k + 1);
@@ -1854,7 +1857,7 @@ __device__ void finalize_argmax(const ArgmaxParams& p, int b, int lane) {
     }
   }
   if (__any_sync(0xffffffffu, invalid) && lane == 0) atomicOr(&p.ctrl->flags, kFlagInvalidToken);
-  if (lane == 0) {
+  if (!kOneGrid && lane == 0) {
     // acquire (this lane counted the last row): every branch-state update
     // lands before the clear
     fence_acq_rel_gpu();
@@ -1925,7 +1928,7 @@ __device__ void merge_argmax_row(const ArgmaxParams& p, int b, int r, int lane) 
     else if constexpr (kMode == kArgRows)
       finalize_argmax_rows(p, b, lane);
     else
-      finalize_argmax(p, b, lane);
+      finalize_argmax<false>(p, b, lane);
   }
 }
 
@@ -2022,49 +2025,50 @@ __global__ void __launch_bounds__(kThreads, 1)
 // persistent pipeline to pay off (a few microseconds of ramp and a dependent
 // tail of several L2 round trips after the last chunk, against a call of a
 // few tens of microseconds, and too short for a rejection to be known before
-// the rows after it are read).  One 256-thread block per chunk of one row:
-// every thread loads its (up to) eight 16-byte vectors at once, takes the
-// first maximum, the block merges its warps in shared memory and publishes
-// the chunk's key with one 64-bit atomicMax on the row key (keys order like
-// (value, -index), so the max is the row's first maximum), whose result it
-// does not wait for, and exits.  A block that also counted itself and let the
-// last block finalize would hold its slot on the SM for two more L2 round
-// trips (a third of its life), and the slots are what limits the bytes in
-// flight (55 registers a thread: four blocks, 128 KB, an SM).  So a second
-// grid of one warp per sequence runs the same finalize as the persistent
-// kernel; it is launched as a programmatic dependent of the first, so its
-// launch overlaps the streaming and its griddepcontrol.wait returns once the
-// first grid has completed and its atomics are visible.
+// the rows after it are read).  One 256-thread block per chunk of one row
+// (16 KB; 8 KB and 32 KB chunks measured slower, 26.0 and 21.9 against
+// 19.8 us at B = 64, k = 4, V = 128256): every thread loads its (up to) four
+// 16-byte vectors at once and takes the first maximum, the block merges its
+// warps in shared memory and publishes the chunk's key with one 64-bit
+// atomicMax on the row key (keys order like (value, -index), so the max is
+// the row's first maximum), whose result it does not wait for, and exits.
+// A block that also counted itself and let the last block of its sequence
+// finalize held its slot on the SM for two more L2 round trips, a third of
+// its life, and the resident blocks are what keeps bytes in flight.  So a
+// second grid of one warp per sequence runs the same finalize as the
+// persistent kernel; it is launched as a programmatic dependent of the
+// first, so its launch overlaps the streaming, and its griddepcontrol.wait
+// returns once the first grid has completed and its atomics are visible.
 #ifndef SV_OS_THREADS
 #define SV_OS_THREADS 256
 #endif
 #ifndef SV_OS_VECS
-#define SV_OS_VECS 8
+#define SV_OS_VECS 4
 #endif
 constexpr int kOsThreads = SV_OS_THREADS;
 constexpr int kOsVecs = SV_OS_VECS;
 
 template <typename T>
 __host__ __device__ constexpr int oneshot_chunk() {
-  return kOsThreads * kOsVecs * Elem<T>::kPerVec;  // 16384 bf16 or 8192 f32 entries
+  return kOsThreads * kOsVecs * Elem<T>::kPerVec;  // 8192 bf16 or 4096 f32 entries
 }
 
 int oneshot_chunk_entries(int t_dtype) {
   return t_dtype == 1 ? oneshot_chunk<uint16_t>() : oneshot_chunk<float>();
 }
 
+// Largest key of chunk `ch` (row b * R + r, column chunk c) over the block;
+// returned in thread 0 (0 for a chunk with no finite-or-infinite entry).
 template <typename T, bool kVec>
-__global__ void __launch_bounds__(kOsThreads)
-    argmax_oneshot_kernel(const __grid_constant__ ArgmaxParams p) {
+__device__ __forceinline__ unsigned long long oneshot_chunk_key(const ArgmaxParams& p,
+                                                                unsigned int ch, int tid,
+                                                                unsigned long long* s_key,
+                                                                unsigned int& row_out) {
   constexpr int EPV = Elem<T>::kPerVec;
   constexpr int CH = oneshot_chunk<T>();
-  __shared__ unsigned long long s_key[kOsThreads / 32];
-  // the finalize grid may be scheduled once every block has started; it
-  // still waits for this grid to complete
-  griddep_launch_dependents();
-  const int tid = threadIdx.x, lane = tid & 31;
-  const unsigned int row = udiv(blockIdx.x, p.div_nch1);  // b * R + r
-  const int c = static_cast<int>(blockIdx.x - row * static_cast<unsigned int>(p.nch1));
+  const int lane = tid & 31;
+  const unsigned int row = udiv(ch, p.div_nch1);  // b * R + r
+  const int c = static_cast<int>(ch - row * static_cast<unsigned int>(p.nch1));
   const unsigned int bu = udiv(row, p.div_R);
   const int b = static_cast<int>(bu);
   const int r = static_cast<int>(row - bu * static_cast<unsigned int>(p.R));
@@ -2123,11 +2127,35 @@ __global__ void __launch_bounds__(kOsThreads)
   warp_argmax(best, idx);
   if (lane == 0) s_key[tid >> 5] = idx == INT_MAX ? 0ull : make_key(best, idx);
   __syncthreads();
+  unsigned long long key = 0ull;
   if (tid == 0) {
-    unsigned long long key = 0ull;
 #pragma unroll
     for (int w = 0; w < kOsThreads / 32; ++w) key = s_key[w] > key ? s_key[w] : key;
-    if (key && SV_IN(p.ctrl, row, static_cast<long long>(p.B) * p.R))
+  }
+  row_out = row;
+  return key;
+}
+
+// Blocks take chunks blockIdx.x, + gridDim.x, ... (one each when the grid
+// covers every chunk).  The warp keys alternate between two shared arrays,
+// so one barrier a chunk suffices: thread 0 has read a chunk's array before
+// it passes the next chunk's barrier, and the array is written again only
+// after that.
+template <typename T, bool kVec>
+__global__ void __launch_bounds__(kOsThreads)
+    argmax_oneshot_kernel(const __grid_constant__ ArgmaxParams p) {
+  __shared__ unsigned long long s_key[2][kOsThreads / 32];
+  // the finalize grid may be scheduled once every block has started; it
+  // still waits for this grid to complete
+  griddep_launch_dependents();
+  const int tid = threadIdx.x;
+  const unsigned int total =
+      static_cast<unsigned int>(p.B) * static_cast<unsigned int>(p.R) * static_cast<unsigned int>(p.nch1);
+  int par = 0;
+  for (unsigned int ch = blockIdx.x; ch < total; ch += gridDim.x, par ^= 1) {
+    unsigned int row;
+    const unsigned long long key = oneshot_chunk_key<T, kVec>(p, ch, tid, s_key[par], row);
+    if (tid == 0 && key && SV_IN(p.ctrl, row, static_cast<long long>(p.B) * p.R))
       atomicMax(p.rkey + row, key);  // result unused: a fire-and-forget reduction
   }
 }
@@ -2136,9 +2164,18 @@ __global__ void __launch_bounds__(kOsThreads)
 // its key (griddepcontrol.wait: that grid has completed and its atomics are
 // visible).
 __global__ void __launch_bounds__(256) argmax_finalize_kernel(const __grid_constant__ ArgmaxParams p) {
-  griddep_wait();
   const int b = static_cast<int>(blockIdx.x) * 8 + (static_cast<int>(threadIdx.x) >> 5);
-  if (b < p.B) finalize_argmax(p, b, threadIdx.x & 31);
+  const int lane = threadIdx.x & 31;
+  // The draft tokens are inputs, complete before the streaming grid began:
+  // bring this sequence's into L2 while that grid still runs.
+  if (b < p.B) {
+    const char* tok = reinterpret_cast<const char*>(p.tokens + static_cast<size_t>(b) * p.G * p.k);
+    const int bytes = p.G * p.k * static_cast<int>(sizeof(int));
+    for (int o = lane * 128; o < bytes; o += 32 * 128)
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(tok + o));
+  }
+  griddep_wait();
+  if (b < p.B) finalize_argmax<true>(p, b, lane);
 }
 
 template <typename T>
