@@ -628,8 +628,10 @@ def run_ours(args, rank: int, world: int, dist) -> None:
     cpu, outcome = None, None
     if rank == 0 and world == 1 and not args.skip_cpu_baseline:
         cpu, outcome = oracle_baseline(ws)
-        for name in lat:
+        for name in lat:  # timed too, though not part of the step's baseline
+            t1 = time.perf_counter()
             outcome[name] = oracle_call(ws[name], os.cpu_count() or 1)
+            cpu["seconds_per_call"][name] = round(time.perf_counter() - t1, 4)
         for name in STEP + lat:
             if ws[name]["mode"] == "multi":
                 outcome[name]["branch_len"] = branch_lengths(ws[name])

@@ -137,10 +137,13 @@ struct WsView {
 // pipeline (the pipeline's ramp and tail, and early exit's need for a
 // rejection to be known a whole position block ahead, only pay off on larger
 // calls).  SV_ONESHOT_MAX_BYTES overrides it (0: never), for tests and tuning.
-// Measured on B200 (greedy, k = 4, V = 128256, one grid vs the pipeline, µs):
-// B = 16 14.4 vs 23.0, 64 25.0 vs 31.7, 128 40.1 vs 46.3, 256 63.9 vs 66.3,
-// 512 117.5 vs 102.2; multi-candidate B = 16, G = 8, V = 32000 21.0 vs 35.1.
-constexpr long long kOneshotMaxBytes = 384ll << 20;
+// Measured on B200 (one grid vs the pipeline, µs per call in a graph of
+// calls on four copies of the logits): greedy, k = 4, V = 128256: B = 16
+// (20.5 MB) 11.6 vs 22.2, 64 19.8 vs 28.1, 128 30.2 vs 40.1, 256 (328 MB)
+// 52.6 vs 58.4, 512 (657 MB) 95.6 vs 92.3, 1024 183.5 vs 168.2;
+// multi-candidate, G = 8, k = 4, V = 32000: B = 16 15.9 vs 33.2, 64 33.6 vs
+// 51.2, 256 (655 MB) 97.7 vs 122.7.
+constexpr long long kOneshotMaxBytes = 512ll << 20;
 
 bool use_oneshot(long long bytes) {
   long long limit = kOneshotMaxBytes;
