@@ -134,6 +134,7 @@ struct StochParams {
   // the order the sequences' accepted lengths become known.
   unsigned int total1;   // k B nch
   unsigned int total2;   // B nch
+  int park;              // 1: producers park phase-1 chunks of undecided pairs
   UDiv div_nch, div_B;   // / nch, / B
   Ctrl* ctrl;
   SeqRec* seq;

@@ -902,6 +902,9 @@ __device__ __forceinline__ bool stoch_issue_phase2(const StochParams& p, Shared&
 #ifndef SV_DEFER
 #define SV_DEFER 1
 #endif
+#ifndef SV_HOLD
+#define SV_HOLD 1
+#endif
 template <typename TT, typename TD, bool kTma>
 __device__ void stoch_producer(const StochParams& p, Shared& sh, unsigned char* stages, int g) {
   constexpr int kDefer = SV_DEFER;
@@ -929,6 +932,37 @@ __device__ void stoch_producer(const StochParams& p, Shared& sh, unsigned char* 
   unsigned int t1nn = first + 2u;
   unsigned long long s1 = state_of(t1);
   unsigned long long s1n = state_of(t1n);
+  // Parked phase-1 tickets (p.park): a chunk of pair i >= 1 whose sequence
+  // has rows before i undecided waits here, oldest first, while the producer
+  // takes later tickets; it leaves once the state word decides it (a
+  // rejection before i: retired unread; rows 0..i-1 all accepted: issued),
+  // or, oldest first, when the queue is full or no new ticket is left.  A
+  // parked chunk thus waits at least one stage wait, and its sequence's
+  // state is read again just before it goes.  Queue of 1 / 2 / 3 / none
+  // (graph-timed, same box, us): B = 256, k = 8: 167.7 / 170.4 / 173.8 /
+  // 175.8; B = 64, k = 4: 61.1 / 63.2 / 65.8 / 68.9; B = 1: 22.0 / 24.1 /
+  // 22.6 / 23.8; a queue of 8 was slower still (195.6 at B = 256).
+  constexpr int kHold = SV_HOLD;
+  unsigned int pt[kHold];
+  unsigned long long ps[kHold];  // their sequences' state words as last polled
+  int np = 0;
+  auto pair_of = [&](unsigned int t) -> unsigned int {  // i of ticket t
+    return udiv(udiv(t, p.div_nch), p.div_B);
+  };
+  auto parkable = [&](unsigned int t, unsigned long long st) -> bool {
+    const unsigned int i = pair_of(t);
+    const unsigned int need = low_mask(static_cast<int>(i));
+    return i > 0u && (rejected_bits(st) & need) == 0u && (decided_bits(st) & need) != need;
+  };
+  // reload the parked tickets' state words (read at the next iteration)
+  auto poll_parked = [&]() {
+#pragma unroll
+    for (int d = 0; d < kHold; ++d)
+      if (d < np) {
+        const unsigned int r = udiv(pt[d], p.div_nch);
+        ps[d] = ld_relaxed_u64(&p.seq[r - udiv(r, p.div_B) * B].state);
+      }
+  };
   unsigned int dt[kDefer];         // held phase-2 tickets, oldest first
   unsigned long long dv[kDefer];   // their ready-list entries as last polled
   int nd = 0;
@@ -974,7 +1008,7 @@ __device__ void stoch_producer(const StochParams& p, Shared& sh, unsigned char* 
 #pragma unroll
     for (int d = kDefer - 1; d >= 0; --d)
       if (d < nd && dv[d] != 0ull) rd = d;
-    if (rd < 0 && t1 >= p.total1 && nd > 0) {
+    if (rd < 0 && t1 >= p.total1 && np == 0 && nd > 0) {
       if (!settle_retired()) {
         ok = false;
         break;
@@ -1004,7 +1038,8 @@ __device__ void stoch_producer(const StochParams& p, Shared& sh, unsigned char* 
     // keep up to kDefer phase-2 tickets in hand (the atomic's result is used
     // at the next iteration)
     if (!t2_done && nd < kDefer) t2p = atomicAdd(&ctrl->ticket2, 1u);
-    if (rd >= 0 && t1 < p.total1 && (SV_P1_FIRST || (SV_P2_RUN > 0 && run >= SV_P2_RUN)))
+    if (rd >= 0 && (t1 < p.total1 || np > 0) &&
+        (SV_P1_FIRST || (SV_P2_RUN > 0 && run >= SV_P2_RUN)))
       rd = -1;  // the drawn phase-1 ticket goes first; the ready entry stays held
     if (rd >= 0) {
       ++run;
@@ -1043,22 +1078,64 @@ __device__ void stoch_producer(const StochParams& p, Shared& sh, unsigned char* 
 #pragma unroll
     for (int d = 0; d < kDefer; ++d)
       if (d < nd && dv[d] == 0ull) dv[d] = ld_relaxed_u64(p.list + udiv(dt[d], p.div_nch));
-    if (t1 < p.total1) {
-      const unsigned int row = udiv(t1, p.div_nch);
+    if (t1 < p.total1 || np > 0) {
+      // a parked ticket that its state decides (oldest first); else, with
+      // the queue full or no new ticket left, the oldest; else a new ticket,
+      // parked if it can be
+      int pr = -1;
+#pragma unroll
+      for (int d = kHold - 1; d >= 0; --d)
+        if (d < np && !parkable(pt[d], ps[d])) pr = d;
+      if (pr < 0 && np > 0 && (t1 >= p.total1 || (np == kHold && parkable(t1, s1)))) pr = 0;
+      unsigned int tk;
+      unsigned long long sk;
+      if (pr >= 0) {
+        tk = 0u;
+        sk = 0ull;
+#pragma unroll
+        for (int d = 0; d < kHold; ++d)
+          if (d == pr) {
+            tk = pt[d];
+            sk = ps[d];
+          }
+#pragma unroll
+        for (int d = 0; d < kHold - 1; ++d)
+          if (d >= pr && d + 1 < np) {
+            pt[d] = pt[d + 1];
+            ps[d] = ps[d + 1];
+          }
+        --np;
+      } else {
+        tk = t1;
+        sk = s1;
+        // advance the ticket pipeline before this chunk's stage wait
+        t1 = t1n;
+        s1 = s1n;
+        t1n = t1nn;
+        s1n = state_of(t1n);
+        t1nn = fixed + atomicAdd(&ctrl->ticket, 1u);
+        if (p.park && np < kHold && parkable(tk, sk)) {
+#pragma unroll
+          for (int d = 0; d < kHold; ++d)
+            if (d == np) {
+              pt[d] = tk;
+              ps[d] = sk;
+            }
+          ++np;
+          poll_parked();
+          continue;
+        }
+      }
+      poll_parked();  // the stage wait below overlaps the round trips
+      const unsigned int row = udiv(tk, p.div_nch);
       const unsigned int i = udiv(row, p.div_B);
       Hdr h;
       h.kind = kKindStats;
       h.b = static_cast<int>(row - i * B);
       h.i = static_cast<int>(i);
-      h.c = static_cast<int>(t1 - row * nch);
-      const unsigned int rej = rejected_bits(s1);
+      h.c = static_cast<int>(tk - row * nch);
+      const unsigned int rej = rejected_bits(sk);
       run = 0;
-      // advance the ticket pipeline before this chunk's stage wait
-      t1 = t1n;
-      s1 = s1n;
-      t1n = t1nn;
-      s1n = state_of(t1n);
-      t1nn = fixed + atomicAdd(&ctrl->ticket, 1u);
       if (rej & low_mask(h.i)) {  // a pair before this one was rejected: retire unread
         if (!SV_IN(ctrl, h.b, p.B) || !SV_IN(ctrl, h.i, p.k) || !SV_IN(ctrl, h.c, p.nch)) continue;
         unsigned long long* slot =

@@ -688,6 +688,32 @@ def test_stochastic_parity_shapes(dev, t_dtype, d_dtype, B, k, V, T):
     compare_stochastic(r, o, k, f"{t_dtype}/{d_dtype} B={B} k={k} V={V}")
 
 
+@pytest.mark.parametrize("parking", ["parked", "unparked"])
+@pytest.mark.parametrize("B,k,V,d_noise", [(1, 4, 32000, 1.0), (64, 4, 32000, 1.5),
+                                           (256, 8, 8000, 1.0), (300, 3, 5000, 0.3)])
+def test_stochastic_parked_and_unparked_tickets(dev, monkeypatch, parking, B, k, V, d_noise):
+    """The producers park chunks of pairs whose earlier rows are undecided
+    (every batch size by default); the size limit is overridden here so that
+    both ways meet the same cases: results equal the oracle's, and the
+    workspace is left zero."""
+    monkeypatch.setenv("SV_PARK_MIN_B", "1" if parking == "parked" else str(1 << 30))
+    w = workloads.make_stochastic(B, k, V, "bf16", "bf16", t_std=3.0, d_noise=d_noise,
+                                  temperature=1.0, seed=B + k + V, threads=THREADS)
+    ws = sv.Workspace(dev)
+    t = to_dev(w["target"], "bf16", dev)
+    d = to_dev(w["draft"], "bf16", dev)
+    tok = torch.from_numpy(w["tokens"]).to(dev)
+    o = oracle.verify_stochastic(w["target"], "bf16", w["draft"], "bf16", w["tokens"], 1.0,
+                                 w["seed"], threads=THREADS)
+    o["inputs"] = (w["tokens"], V)
+    for _ in range(2):
+        r = sv.stochastic(t, d, tok, 1.0, w["seed"], probs=True, workspace=ws)
+        torch.cuda.synchronize()
+        compare_stochastic(r, o, k, f"{parking} B={B} k={k} V={V}")
+        assert int(ws.buf[256:].cpu().count_nonzero()) == 0
+    assert ws.device_status() == 0
+
+
 def test_stochastic_zero_drafts_samples_bonus(dev):
     w = workloads.make_stochastic(50, 0, 3000, "bf16", "bf16", seed=8)
     r, o = run_stochastic(w, dev)
