@@ -1526,6 +1526,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_fence_init();
   }
   __syncthreads();
+  dep_enter();
   if (warp < kProducerWarps) {
     if (lane == 0) stoch_producer<TT, TD, kTma>(p, sh, stages, warp);
   } else if (warp < kProducerWarps + kComputeWarps) {
@@ -2085,6 +2086,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_fence_init();
   }
   __syncthreads();
+  dep_enter();
   if (warp < kProducerWarps) {
     if (lane == 0 && warp < kArgmaxProducers)
       argmax_producer<TT, kTma, kMode == kArgRows || kMode == kArgTree, kMode == kArgPlain>(
@@ -2222,9 +2224,9 @@ template <typename T, bool kVec>
 __global__ void __launch_bounds__(kOsThreads)
     argmax_oneshot_kernel(const __grid_constant__ ArgmaxParams p) {
   __shared__ unsigned long long s_key[2][kOsThreads / 32];
-  // the finalize grid may be scheduled once every block has started; it
-  // still waits for this grid to complete
-  griddep_launch_dependents();
+  // (the finalize grid may then be scheduled once every block has started;
+  // it still waits for this grid to complete)
+  dep_enter();
   const int tid = threadIdx.x;
   const unsigned int total =
       static_cast<unsigned int>(p.B) * static_cast<unsigned int>(p.R) * static_cast<unsigned int>(p.nch1);
@@ -2251,7 +2253,7 @@ __global__ void __launch_bounds__(256) argmax_finalize_kernel(const __grid_const
     for (int o = lane * 128; o < bytes; o += 32 * 128)
       asm volatile("prefetch.global.L2 [%0];" ::"l"(tok + o));
   }
-  griddep_wait();
+  dep_enter();
   if (b < p.B) finalize_argmax<true>(p, b, lane);
 }
 
@@ -2259,24 +2261,17 @@ template <typename T>
 static cudaError_t launch_oneshot_t(const ArgmaxParams& p, bool vec, cudaStream_t st) {
   const long long blocks = static_cast<long long>(p.B) * p.R * p.nch1;
   if (blocks <= 0) return cudaSuccess;
-  if (vec)
-    argmax_oneshot_kernel<T, true><<<static_cast<unsigned int>(blocks), kOsThreads, 0, st>>>(p);
-  else
-    argmax_oneshot_kernel<T, false><<<static_cast<unsigned int>(blocks), kOsThreads, 0, st>>>(p);
-  cudaError_t e = counted(cudaGetLastError(), 1);
+  const dim3 grid(static_cast<unsigned int>(blocks));
+  cudaError_t e = counted(
+      vec ? launch_k(SV_PDL >= 2, argmax_oneshot_kernel<T, true>, grid, dim3(kOsThreads), 0, st, p)
+          : launch_k(SV_PDL >= 2, argmax_oneshot_kernel<T, false>, grid, dim3(kOsThreads), 0, st,
+                     p),
+      1);
   if (e != cudaSuccess) return e;
   // launched while the streaming grid runs; its warps wait for that grid
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(static_cast<unsigned int>((p.B + 7) / 8));
-  cfg.blockDim = dim3(256);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = st;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return counted(cudaLaunchKernelEx(&cfg, argmax_finalize_kernel, p), 1);
+  return counted(launch_k(SV_PDL >= 1, argmax_finalize_kernel,
+                          dim3(static_cast<unsigned int>((p.B + 7) / 8)), dim3(256), 0, st, p),
+                 1);
 }
 
 cudaError_t launch_argmax_oneshot(const ArgmaxParams& p, int t_dtype, bool vec, cudaStream_t st) {
@@ -2287,6 +2282,7 @@ cudaError_t launch_argmax_oneshot(const ArgmaxParams& p, int t_dtype, bool vec, 
 
 __global__ void philox_kernel(const uint4* __restrict__ ctr, long long n, uint32_t k0,
                               uint32_t k1, uint4* __restrict__ out) {
+  dep_enter();
   for (long long j = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; j < n;
        j += static_cast<long long>(gridDim.x) * blockDim.x)
     out[j] = philox10(ctr[j], k0, k1);
@@ -2302,6 +2298,7 @@ __global__ void commit_kernel(const int* __restrict__ accepted_len,
                               int* __restrict__ seq_len, int* __restrict__ token_buf,
                               long long buf_stride, int capacity, int* __restrict__ next_input,
                               Ctrl* ctrl) {
+  dep_enter();
   const int b = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (b >= B) return;
@@ -2348,8 +2345,7 @@ static cudaError_t launch_stoch_t(const StochParams& p, int grid, size_t smem, c
   auto kernel = stochastic_verify_kernel<TT, TD, kTma>;
   cudaError_t e = prepare(kernel, smem, done);
   if (e != cudaSuccess) return e;
-  kernel<<<grid, kThreads, smem, st>>>(p);
-  return counted(cudaGetLastError(), 1);
+  return counted(launch_k(SV_PDL >= 2, kernel, dim3(grid), dim3(kThreads), smem, st, p), 1);
 }
 
 template <typename TT, typename TD>
@@ -2373,8 +2369,7 @@ static cudaError_t launch_argmax_t(const ArgmaxParams& p, int grid, size_t smem,
   auto kernel = argmax_verify_kernel<TT, kTma, kMode>;
   cudaError_t e = prepare(kernel, smem, done);
   if (e != cudaSuccess) return e;
-  kernel<<<grid, kThreads, smem, st>>>(p);
-  return counted(cudaGetLastError(), 1);
+  return counted(launch_k(SV_PDL >= 2, kernel, dim3(grid), dim3(kThreads), smem, st, p), 1);
 }
 
 template <typename TT>
@@ -2408,9 +2403,10 @@ cudaError_t launch_commit(const int* accepted_len, const int* out_tokens, int B,
                           int* next_input, Ctrl* ctrl, cudaStream_t st) {
   if (B <= 0) return cudaSuccess;
   constexpr int kWarps = 8;
-  commit_kernel<<<(B + kWarps - 1) / kWarps, 32 * kWarps, 0, st>>>(
-      accepted_len, out_tokens, B, k, seq_len, token_buf, buf_stride, capacity, next_input, ctrl);
-  return counted(cudaGetLastError(), 1);
+  return counted(launch_k(SV_PDL >= 2, commit_kernel, dim3((B + kWarps - 1) / kWarps),
+                          dim3(32 * kWarps), 0, st, accepted_len, out_tokens, B, k, seq_len,
+                          token_buf, buf_stride, capacity, next_input, ctrl),
+                 1);
 }
 
 cudaError_t launch_philox(const uint4* ctr, long long n, unsigned int key0, unsigned int key1,
@@ -2418,8 +2414,9 @@ cudaError_t launch_philox(const uint4* ctr, long long n, unsigned int key0, unsi
   if (n <= 0) return cudaSuccess;
   const long long blocks = (n + 255) / 256;
   const int grid = static_cast<int>(blocks < 4096 ? blocks : 4096);
-  philox_kernel<<<grid, 256, 0, st>>>(ctr, n, key0, key1, out);
-  return counted(cudaGetLastError(), 1);
+  return counted(
+      launch_k(SV_PDL >= 2, philox_kernel, dim3(grid), dim3(256), 0, st, ctr, n, key0, key1, out),
+      1);
 }
 
 }  // namespace sv

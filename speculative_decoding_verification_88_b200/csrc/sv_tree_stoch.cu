@@ -94,6 +94,7 @@ __device__ __forceinline__ uint4 neg_inf_vec<float>() {
 
 template <typename T>
 __global__ void __launch_bounds__(kTsThreads) tree_stats_kernel(TreeStochParams p) {
+  dep_enter();
   constexpr int EPV = Elem<T>::kPerVec;
   constexpr int CH = tree_chunk<T>();
   const long long blk = blockIdx.x;
@@ -168,6 +169,7 @@ __device__ __forceinline__ V node_value(const V (&v)[2], int c) {
 
 template <typename T>
 __global__ void __launch_bounds__(32 * kWalkWarps) tree_walk_kernel(TreeStochParams p) {
+  dep_enter();
   __shared__ float s_m[kWalkWarps][kMaxNodes], s_is[kWalkWarps][kMaxNodes];
   __shared__ int s_path[kWalkWarps][kMaxNodes];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -292,6 +294,7 @@ __global__ void __launch_bounds__(32 * kWalkWarps) tree_walk_kernel(TreeStochPar
 
 template <typename T>
 __global__ void __launch_bounds__(kTsThreads) tree_sample_kernel(TreeStochParams p) {
+  dep_enter();
   constexpr int EPV = Elem<T>::kPerVec;
   constexpr int CH = kSampleEntries;
   // E (the rejected tokens at the final node) as a bitmap over this block's
@@ -438,15 +441,19 @@ bool is_aligned(const void* p, size_t a) { return reinterpret_cast<uintptr_t>(p)
 template <typename T>
 cudaError_t launch_tree_stoch(const TreeStochParams& p, cudaStream_t st) {
   const long long rows = static_cast<long long>(p.B) * p.N;
-  tree_stats_kernel<T><<<static_cast<unsigned int>(rows * p.nch), kTsThreads, 0, st>>>(p);
-  cudaError_t e = counted(cudaGetLastError(), 1);
+  cudaError_t e = counted(launch_k(SV_PDL >= 2, tree_stats_kernel<T>,
+                                   dim3(static_cast<unsigned int>(rows * p.nch)),
+                                   dim3(kTsThreads), 0, st, p),
+                          1);
   if (e != cudaSuccess) return e;
-  tree_walk_kernel<T><<<(p.B + kWalkWarps - 1) / kWalkWarps, 32 * kWalkWarps, 0, st>>>(p);
-  e = counted(cudaGetLastError(), 1);
+  e = counted(launch_k(SV_PDL >= 2, tree_walk_kernel<T>, dim3((p.B + kWalkWarps - 1) / kWalkWarps),
+                       dim3(32 * kWalkWarps), 0, st, p),
+              1);
   if (e != cudaSuccess) return e;
-  tree_sample_kernel<T><<<static_cast<unsigned int>(static_cast<long long>(p.B) * p.nch_s),
-                          kTsThreads, 0, st>>>(p);
-  return counted(cudaGetLastError(), 1);
+  return counted(launch_k(SV_PDL >= 2, tree_sample_kernel<T>,
+                          dim3(static_cast<unsigned int>(static_cast<long long>(p.B) * p.nch_s)),
+                          dim3(kTsThreads), 0, st, p),
+                 1);
 }
 
 }  // namespace
