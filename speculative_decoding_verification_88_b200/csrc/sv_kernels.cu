@@ -1904,13 +1904,17 @@ __device__ void finalize_argmax(const ArgmaxParams& p, int b, int lane) {
   int best_n = -1, best_g = 0, best_next = -1;
   bool invalid = false;  // a draft token outside [0, V): it never matches
   for (int g0 = 0; g0 < G; g0 += 4) {
-    // row keys of up to four branches: loads issued together
+    // row keys and draft tokens of up to four branches: loads issued
+    // together, the tokens (inputs) before any key is examined
     unsigned long long v[4], v32[4];
+    int xs[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const int g = g0 + q;
       v[q] = (g < G && lane <= k) ? ld_relaxed_u64(keys + g * (k + 1) + lane) : 0ull;
       v32[q] = (g < G && k == 32 && lane == 0) ? ld_relaxed_u64(keys + g * (k + 1) + 32) : 0ull;
+      xs[q] = (g < G && lane < k) ? __ldg(p.tokens + (static_cast<size_t>(b) * G + g) * k + lane)
+                                  : 0;
     }
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -1919,8 +1923,7 @@ __device__ void finalize_argmax(const ArgmaxParams& p, int b, int lane) {
       const int a = lane <= k ? key_index(take(keys + g * (k + 1) + lane, v[q], p.ctrl)) : -1;
       const int a32 =
           (k == 32 && lane == 0) ? key_index(take(keys + g * (k + 1) + 32, v32[q], p.ctrl)) : -1;
-      const int* cand = p.tokens + (static_cast<size_t>(b) * G + g) * k;
-      const int x = lane < k ? __ldg(cand + lane) : 0;
+      const int x = xs[q];
       invalid |= x < 0 || x >= p.V;
       const bool miss = lane < k && x != a;
       const unsigned int mm = __ballot_sync(0xffffffffu, miss);
