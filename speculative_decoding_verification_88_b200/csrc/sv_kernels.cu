@@ -1897,19 +1897,23 @@ __device__ void finalize_argmax_rows(const ArgmaxParams& p, int b, int lane) {
 // longest branch (lowest g on a tie) is committed.
 // kOneGrid: called by the finalize grid of the one-grid path, which runs after
 // the streaming grid has completed; no branch state to clear, so no fence.
+#ifndef SV_FIN_BRANCHES
+#define SV_FIN_BRANCHES 8
+#endif
+constexpr int kFinBranches = SV_FIN_BRANCHES;  // branches whose loads go out together
 template <bool kOneGrid>
 __device__ void finalize_argmax(const ArgmaxParams& p, int b, int lane) {
   const int k = p.k, G = p.G;
   unsigned long long* keys = p.rkey + static_cast<size_t>(b) * G * (k + 1);
   int best_n = -1, best_g = 0, best_next = -1;
   bool invalid = false;  // a draft token outside [0, V): it never matches
-  for (int g0 = 0; g0 < G; g0 += 4) {
-    // row keys and draft tokens of up to four branches: loads issued
+  for (int g0 = 0; g0 < G; g0 += kFinBranches) {
+    // row keys and draft tokens of up to kFinBranches branches: loads issued
     // together, the tokens (inputs) before any key is examined
-    unsigned long long v[4], v32[4];
-    int xs[4];
+    unsigned long long v[kFinBranches], v32[kFinBranches];
+    int xs[kFinBranches];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < kFinBranches; ++q) {
       const int g = g0 + q;
       v[q] = (g < G && lane <= k) ? ld_relaxed_u64(keys + g * (k + 1) + lane) : 0ull;
       v32[q] = (g < G && k == 32 && lane == 0) ? ld_relaxed_u64(keys + g * (k + 1) + 32) : 0ull;
@@ -1917,7 +1921,7 @@ __device__ void finalize_argmax(const ArgmaxParams& p, int b, int lane) {
                                   : 0;
     }
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < kFinBranches; ++q) {
       const int g = g0 + q;
       if (g >= G) break;
       const int a = lane <= k ? key_index(take(keys + g * (k + 1) + lane, v[q], p.ctrl)) : -1;
