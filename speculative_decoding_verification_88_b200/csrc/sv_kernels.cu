@@ -879,11 +879,19 @@ __device__ __forceinline__ bool stoch_issue_phase2(const StochParams& p, Shared&
 //    168.4; B = 64, k = 4: 75.6 -> 73.9; B = 1: 22.6 -> 21.6 (SV_P1_FIRST 0
 //    restores phase 2 first; SV_P2_RUN n > 0 lets n phase-2 chunks pass a
 //    drawn phase-1 ticket, which measured no better than 0).
-//  - Phase-1 tickets are taken one at a time, two ahead, and the state word
-//    of each ticket's sequence is loaded one ticket ahead: a chunk of pair i
-//    whose sequence already has a rejection before i is retired unread (its
-//    two slots get kSkippedStats and it is counted on its row; if that
-//    completes the row, a data-free item hands the row to the epilogue).
+//  - Phase-1 tickets come two ahead of their use, and the state word of each
+//    ticket's sequence is loaded one ticket ahead: a chunk of pair i whose
+//    sequence already has a rejection before i is retired unread (its two
+//    slots get kSkippedStats and it is counted on its row; if that completes
+//    the row, a data-free item hands the row to the epilogue).  A retire
+//    costs the producer about one L2 round trip (the state word it waits
+//    for), and at the later positions nearly every ticket is retired; so
+//    after a retired ticket the producer takes the next SV_BATCH (4)
+//    consecutive tickets in one grab, and a ticket in the same row as the one
+//    before it takes that ticket's state word (which only gains decisions)
+//    instead of loading it again.  Batch 1 / 3 / 4 / 6 / 8, step of the four
+//    bench calls (us): 244.5 / 236.1 / 234.4 / 237.6 / 240.3 (across two
+//    runs; B = 256, k = 8: 170.2, 162.0, 162.9, 162.6, 163.7).
 //  - Up to kDefer phase-2 tickets are held; their ready-list entries are
 //    polled with relaxed loads (issued before the current chunk's stage wait,
 //    read at the next iteration) and a chunk is issued once its entry is
@@ -904,6 +912,9 @@ __device__ __forceinline__ bool stoch_issue_phase2(const StochParams& p, Shared&
 #endif
 #ifndef SV_HOLD
 #define SV_HOLD 1
+#endif
+#ifndef SV_BATCH
+#define SV_BATCH 4
 #endif
 template <typename TT, typename TD, bool kTma>
 __device__ void stoch_producer(const StochParams& p, Shared& sh, unsigned char* stages, int g) {
@@ -929,9 +940,14 @@ __device__ void stoch_producer(const StochParams& p, Shared& sh, unsigned char* 
   const unsigned int first = (blockIdx.x * kProducerWarps + static_cast<unsigned int>(g)) * 3u;
   unsigned int t1 = first;
   unsigned int t1n = first + 1u;
-  unsigned int t1nn = first + 2u;
   unsigned long long s1 = state_of(t1);
   unsigned long long s1n = state_of(t1n);
+  // the tickets after t1n: a batch [bq_base, bq_base + bq_cnt) taken from
+  // the counter in one grab, read one advance after its grab; after a
+  // retired ticket the grab takes SV_BATCH tickets (consecutive chunks,
+  // mostly of one row, whose state word is then read once), else one
+  unsigned int bq_base = first + 2u, bq_pos = 0u, bq_cnt = 1u;
+  bool last_retired = false;
   // Parked phase-1 tickets (p.park): a chunk of pair i >= 1 whose sequence
   // has rows before i undecided waits here, oldest first, while the producer
   // takes later tickets; it leaves once the state word decides it (a
@@ -1108,12 +1124,21 @@ __device__ void stoch_producer(const StochParams& p, Shared& sh, unsigned char* 
       } else {
         tk = t1;
         sk = s1;
-        // advance the ticket pipeline before this chunk's stage wait
+        // advance the ticket pipeline before this chunk's stage wait; the
+        // state of a ticket in the same row as the one before it is that
+        // ticket's (a state word only gains decisions)
         t1 = t1n;
         s1 = s1n;
-        t1n = t1nn;
-        s1n = state_of(t1n);
-        t1nn = fixed + atomicAdd(&ctrl->ticket, 1u);
+        t1n = bq_base + bq_pos;
+        ++bq_pos;
+        s1n = (t1n < p.total1 && t1 < p.total1 && udiv(t1n, p.div_nch) == udiv(t1, p.div_nch))
+                  ? s1
+                  : state_of(t1n);
+        if (bq_pos == bq_cnt) {  // the batch is used up: grab the next one now
+          bq_cnt = (SV_BATCH > 1 && last_retired) ? SV_BATCH : 1u;
+          bq_base = fixed + atomicAdd(&ctrl->ticket, bq_cnt);
+          bq_pos = 0u;
+        }
         if (p.park && np < kHold && parkable(tk, sk)) {
 #pragma unroll
           for (int d = 0; d < kHold; ++d)
@@ -1155,8 +1180,10 @@ __device__ void stoch_producer(const StochParams& p, Shared& sh, unsigned char* 
             sko[d] = old;
           }
         ++nsk;
+        last_retired = true;
         continue;
       }
+      last_retired = false;
       ok = stoch_issue<TT, TD, kTma>(p, sh, stages, g, used, h, nullptr);
       if (ok) ok = settle_retired();  // their counts arrived during the stage wait
       continue;
