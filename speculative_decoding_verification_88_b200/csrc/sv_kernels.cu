@@ -988,7 +988,15 @@ __device__ void stoch_producer(const StochParams& p, Shared& sh, unsigned char* 
   // arrives while the producer goes on): a count that completes the row
   // hands the row to the epilogue.  No resolution waits on a retired row (it
   // lies past a rejection), so the hand-over may lag.
-  constexpr int kSk = 4;
+  // One entry: a retire's count is checked at the next iteration, so a row
+  // that its retires complete reaches the epilogue soonest.  Queue of 1 / 2
+  // / 3 / 4 / 8, step of the four bench calls (us, two runs): 228.3 / 230.1
+  // / 234.7 / 234.1 / 252.9; B = 256, k = 8: 157.3 / 159.8 / 161.6 / 162.5 /
+  // 175.1.
+#ifndef SV_SKQ
+#define SV_SKQ 1
+#endif
+  constexpr int kSk = SV_SKQ;
   int skb[kSk], ski[kSk];
   unsigned int sko[kSk];
   int nsk = 0;
