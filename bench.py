@@ -162,6 +162,22 @@ def recorded_traffic(workload: str, batch_override: bool) -> float | None:
     return float(rec["dram_bytes_per_launch"])
 
 
+def call_spread(samples_ms: list) -> dict:
+    """Median and 10th / 90th percentiles, in microseconds, of per-call
+    times in milliseconds (one event pair per call per graph replay).
+    Percentiles interpolate between order statistics."""
+    xs = sorted(samples_ms)
+    if not xs:
+        return {}
+    def q(f):
+        pos = f * (len(xs) - 1)
+        lo = int(pos)
+        hi = min(lo + 1, len(xs) - 1)
+        return (xs[lo] + (xs[hi] - xs[lo]) * (pos - lo)) * 1e3
+    return {"p10": round(q(0.1), 2), "median": round(q(0.5), 2), "p90": round(q(0.9), 2),
+            "samples": len(xs)}
+
+
 class NvmlSampler:
     """SM clock and throttle reasons of one GPU read through NVML every half
     millisecond from a background thread, so that a timed region of a few
@@ -654,6 +670,8 @@ def run_ours(args, rank: int, world: int, dist) -> None:
         rec = {"us_per_call": round(us, 2), "positions_per_s": positions(ws[name]) / (us * 1e-6),
                "in_step": name in STEP, "full_read_bytes": full,
                "full_read_gbs": full / (us * 1e-6) / 1e9}
+        if name in samples:
+            rec["us_spread"] = call_spread(samples[name])
         rec["frac_full_read"] = rec["full_read_gbs"] / peak
         if need is not None:
             rec["needed_bytes"] = need

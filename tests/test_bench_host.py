@@ -1,5 +1,5 @@
 """Host logic of bench.py on CPU: the per-mode position and byte counts, the
-traffic record's gating, the clock-sample parser, the workload selection,
+traffic record's gating, the per-call percentiles, the clock-sample parser, the workload selection,
 and the JSON line of the CPU-only reference arm."""
 import datetime
 import time
@@ -119,6 +119,23 @@ class _Done:
 
     def join(self, timeout=None):
         pass
+
+
+def test_call_spread_percentiles():
+    # 0.001 .. 0.101 ms: percentiles of an evenly spaced set are known exactly
+    xs = [i * 1e-3 for i in range(1, 102)]
+    np.random.default_rng(0).shuffle(xs)
+    sp = bench.call_spread(xs)
+    assert sp["samples"] == 101
+    assert sp["median"] == pytest.approx(51.0)
+    assert sp["p10"] == pytest.approx(11.0)
+    assert sp["p90"] == pytest.approx(91.0)
+    # agrees with numpy's linear interpolation on an uneven set
+    ys = list(np.random.default_rng(1).gamma(2.0, 0.01, size=200))
+    sp = bench.call_spread(ys)
+    for key, f in (("p10", 10), ("median", 50), ("p90", 90)):
+        assert sp[key] == pytest.approx(round(np.percentile(ys, f) * 1e3, 2), abs=0.006)
+    assert bench.call_spread([]) == {}
 
 
 def test_clock_sampler_keeps_samples_inside_the_window():
