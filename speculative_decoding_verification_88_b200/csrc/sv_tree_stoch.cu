@@ -20,14 +20,14 @@
 //                       then walks the tree with warp-uniform shuffles and
 //                       ballots.  Writes the path and accepted tokens, and the
 //                       final node and E for the draw.
-//   tree_sample_kernel  one block per (sequence, 2048-entry piece) of the
+//   tree_sample_kernel  one block per (sequence, 8192-entry piece) of the
 //                       final node's row: Gumbel-max over l c2 outside E (and
 //                       over the whole row as the fallback), merged by 64-bit
 //                       atomicMax; the last block of a sequence writes the
 //                       token.  The draw is issue-bound (a Philox block per
 //                       four entries, two lg2 per entry) on one row per
-//                       sequence, so it runs on many short blocks that fill
-//                       every SM several times over.
+//                       sequence; each thread loads all its vectors before
+//                       it draws, so a block waits for DRAM once.
 // Every workspace word written here is cleared again by the kernel that
 // consumes it, so the workspace stays zero between calls of any mode.
 #include <climits>
@@ -45,7 +45,12 @@ constexpr int kTsThreads = 256;
 // slower for the stochastic tree call: 120.5 against 109.9 us at B = 64,
 // N = 26, V = 128256)
 constexpr int kTsVecs = 8;
-constexpr int kSampleEntries = 2048;  // entries per block of the final draw
+// Entries per block of the final draw, each thread's loads issued before its
+// draws.  2048 / 4096 / 8192 / 12288 / 16384 entries: 111.9 / 108.2 / 106.9 /
+// 108.1 / 108.7 us per stochastic tree call at B = 64, N = 26, V = 128256
+// (1024 entries: 123.4).  Launching the walk and the draw as programmatic
+// dependents of the grid before them was slower (116.9).
+constexpr int kSampleEntries = 8192;
 constexpr int kWalkWarps = 4;
 constexpr int kMaxNodes = 64;
 
@@ -311,7 +316,7 @@ __global__ void __launch_bounds__(kTsThreads) tree_sample_kernel(TreeStochParams
   const int u = rec.u, ne = min(rec.ne, kMaxNodes);
   const uint32_t tag = static_cast<uint32_t>(rec.tag);
   const int x0 = c * CH;
-  if (tid < CH / 32) s_emask[tid] = 0u;
+  for (int w = tid; w < CH / 32; w += kTsThreads) s_emask[w] = 0u;
   __syncthreads();
   if (tid < ne) {
     const int xe = rec.excl[tid] - x0;
@@ -345,9 +350,20 @@ __global__ void __launch_bounds__(kTsThreads) tree_sample_kernel(TreeStochParams
   if (p.vec) {
     const uint4* src = reinterpret_cast<const uint4*>(static_cast<const T*>(p.logits) + off + x0);
     const int nv = len / EPV;
-    for (int i = tid; i < nv; i += kTsThreads) {
+    // every load of the thread first, then the draws
+    constexpr int NV = (CH / EPV + kTsThreads - 1) / kTsThreads;
+    uint4 raw[NV];
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+      const int i = tid + j * kTsThreads;
+      raw[j] = i < nv ? __ldg(src + i) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+      const int i = tid + j * kTsThreads;
+      if (i >= nv) break;
       float f[EPV];
-      unpack(__ldg(src + i), f);
+      unpack(raw[j], f);
       const int e0 = i * EPV;
       const uint32_t m = s_emask[e0 >> 5] >> (e0 & 31);  // EPV bits, one word (EPV | 32)
 #pragma unroll
