@@ -13,7 +13,8 @@
 // Three launches on the caller's stream:
 //   tree_stats_kernel   one block per (node row, chunk): the chunk's softmax
 //                       statistics (max and sum of 2^(l c2 - max), log2 units)
-//                       from 16-byte vector loads, 8 in flight per thread.
+//                       from 16-byte vector loads, 8 in flight per thread;
+//                       one exponential pair in four on the FMA pipe.
 //   tree_walk_kernel    one warp per sequence: merges each node row's chunk
 //                       statistics, gathers p(x) of every child under its
 //                       parent's row and its acceptance draw (lane-parallel),
@@ -45,6 +46,12 @@ constexpr int kTsThreads = 256;
 // slower for the stochastic tree call: 120.5 against 109.9 us at B = 64,
 // N = 26, V = 128256)
 constexpr int kTsVecs = 8;
+// One pair of exponentials in kTsPolyEvery runs on the FMA pipe
+// (ex2_poly_x2), the rest on the special-function unit, which the statistics
+// pass otherwise saturates.  1 in 8 / 4 / 3 / 2 / every pair (us per
+// stochastic tree call at B = 64, N = 26, V = 128256): 106.9 / 101.7 /
+// 104.3 / 110.5 / 128.4; all on the special-function unit 106.7.
+constexpr int kTsPolyEvery = 4;
 // Entries per block of the final draw, each thread's loads issued before its
 // draws.  2048 / 4096 / 8192 / 12288 / 16384 entries: 111.9 / 108.2 / 106.9 /
 // 108.1 / 108.7 us per stochastic tree call at B = 64, N = 26, V = 128256
@@ -132,14 +139,29 @@ __global__ void __launch_bounds__(kTsThreads) tree_stats_kernel(TreeStochParams 
     for (int q = 0; q < kTsVecs; ++q) mx = fmaxf(mx, vec_max<T>(v[q]));
     mx = fmaxf(mx, tail) * p.c2;
     if (mx != -INFINITY) {
+      // pairs of entries: one f32x2 FMA for the exponents, one f32x2 add;
+      // one pair in kTsPolyEvery on the FMA pipe
+      const unsigned long long cc = pack2(p.c2, p.c2), mm = pack2(-mx, -mx);
+      unsigned long long acc0 = 0ull, acc1 = 0ull;
 #pragma unroll
       for (int q = 0; q < kTsVecs; ++q) {
         float f[EPV];
         unpack(v[q], f);
 #pragma unroll
-        for (int e = 0; e < EPV; ++e) s += ex2f(fmaf(f[e], p.c2, -mx));
+        for (int e = 0; e < EPV; e += 2) {
+          float y0, y1;
+          unpack2(fma2(pack2(f[e], f[e + 1]), cc, mm), y0, y1);
+          const unsigned long long x = ((q * EPV + e) / 2) % kTsPolyEvery == kTsPolyEvery - 1
+                                           ? ex2_poly_x2(y0, y1)
+                                           : pack2(ex2f(y0), ex2f(y1));
+          if ((e & 2) == 0) acc0 = add2(acc0, x);
+          else acc1 = add2(acc1, x);
+        }
       }
-      s += ex2f(fmaf(tail, p.c2, -mx));
+      float a0, a1, b0, b1;
+      unpack2(acc0, a0, a1);
+      unpack2(acc1, b0, b1);
+      s = ((a0 + a1) + (b0 + b1)) + ex2f(fmaf(tail, p.c2, -mx));
     }
   } else {
     for (int e = tid; e < len; e += kTsThreads) mx = fmaxf(mx, load_elem<T>(p.logits, off + x0 + e));
