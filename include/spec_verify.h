@@ -82,10 +82,10 @@ const char *spec_verify_status_string(int status);
  * Number of kernels this library has launched in this process, on any device
  * and stream, counted when the launch call returned success.  A launch made
  * while a stream is captured into a CUDA graph counts once, at capture, not
- * at each replay.  Calls launch: stochastic 1; greedy and multi-candidate 1
- * or 2 (calls of up to 512 MB of target logits stream the rows in one grid
- * and finalize in a second); multi-candidate rows, threshold and tree
- * greedy 1; tree stochastic 3; commit 1; Philox 1.  Thread-safe; never fails.
+ * at each replay.  Calls launch: stochastic 1; greedy, multi-candidate and
+ * multi-candidate rows 1 or 2 (calls of up to 512 MB of target logits stream
+ * the rows in one grid and finalize in a second); threshold and tree greedy
+ * 1; tree stochastic 3; commit 1; Philox 1.  Thread-safe; never fails.
  */
 unsigned long long spec_verify_kernel_launches(void);
 

@@ -412,7 +412,14 @@ static int argmax_call(const void* target_logits, int t_dtype, int64_t sb, int64
   p.rc = reinterpret_cast<unsigned int*>(tail + lay.rc);
   p.dead = reinterpret_cast<unsigned int*>(tail + lay.dead);
   cudaError_t e;
-  if (R == 0 && !thresh && use_oneshot(rows * V * st)) {
+  if ((R == 0 || row_of) && !thresh && use_oneshot(rows * V * st)) {
+    if (row_of) {
+      // rows form: row r of sequence b sits at b sb + r sg.  The streaming
+      // grid addresses row r as branch r / (k + 1), position r % (k + 1), so
+      // a branch stride of (k + 1) sg and a position stride of sg reach it.
+      p.sg = sg * (k + 1);
+      p.sp = sg;
+    }
     const int ch1 = oneshot_chunk_entries(t_dtype);
     p.nch1 = (V + ch1 - 1) / ch1;
     p.div_nch1 = make_udiv(static_cast<unsigned int>(p.nch1));

@@ -150,7 +150,9 @@ struct StochParams {
 
 struct ArgmaxParams {
   const void* tgt;
-  long long sb, sg, sp;  // rows form: sg is the row stride, sp unused
+  long long sb, sg, sp;  // rows form: sg is the row stride, sp unused (one-grid path:
+                         // sg = (k + 1) row strides, sp = one, so that row r = g (k + 1) + i
+                         // sits at g sg + i sp)
   long long t_elems;     // elements the logits view spans (bounds checks)
   const int* tokens;     // [B, G, k]
   int B, G, k, V;

@@ -2296,7 +2296,12 @@ __global__ void __launch_bounds__(256) argmax_finalize_kernel(const __grid_const
       asm volatile("prefetch.global.L2 [%0];" ::"l"(tok + o));
   }
   dep_enter();
-  if (b < p.B) finalize_argmax<true>(p, b, lane);
+  if (b < p.B) {
+    if (p.row_of)
+      finalize_argmax_rows(p, b, lane);
+    else
+      finalize_argmax<true>(p, b, lane);
+  }
 }
 
 template <typename T>

@@ -37,10 +37,11 @@ ARGMAX_CASES = [
     (tp.test_multi_parity_shapes, dict(dtype="f32", B=4, G=5, k=32, V=40)),
     (tp.test_multi_early_exit_is_exact_and_leaves_the_workspace_clean,
      dict(B=64, G=8, k=4, V=32000)),
+    (tp.test_multi_rows_parity_shapes, dict(dtype="bf16", B=3, G=6, k=5, V=20480 + 17)),
+    (tp.test_multi_rows_invalid_entries_and_limits, {}),
 ]
 CASES = [(fn, dict(kw, argmax_path=path)) for fn, kw in ARGMAX_CASES
          for path in ("oneshot", "persistent")] + [
-    (tp.test_multi_rows_invalid_entries_and_limits, {}),
     (tp.test_threshold_invalid_tokens_and_workspace, {}),
     (tp.test_tree_invalid_parent_flag, {}),
     (tp.test_stochastic_parity_shapes, dict(t_dtype="bf16", d_dtype="f32", B=129, k=4, V=7,

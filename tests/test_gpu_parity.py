@@ -316,7 +316,8 @@ def random_rows_case(rng, B, G, k, V, dtype, share=0.6):
 @pytest.mark.parametrize("B,G,k,V", [(1, 1, 4, 100), (3, 3, 2, 17), (16, 8, 4, 3001),
                                      (2, 64, 3, 50), (4, 5, 32, 40), (2, 2, 0, 10),
                                      (3, 6, 5, 20480 + 17)])
-def test_multi_rows_parity_shapes(dev, dtype, B, G, k, V):
+@both_argmax_paths
+def test_multi_rows_parity_shapes(dev, argmax_path, dtype, B, G, k, V):
     rng = np.random.default_rng(B * 3 + G * 5 + k * 11 + V)
     arr, row_of, cand = random_rows_case(rng, B, G, k, V, dtype)
     r = sv.multi_candidate_rows(to_dev(arr, dtype, dev), torch.from_numpy(row_of).to(dev),
@@ -326,7 +327,8 @@ def test_multi_rows_parity_shapes(dev, dtype, B, G, k, V):
         np.testing.assert_array_equal(r[key].cpu().numpy(), o[key], err_msg=key)
 
 
-def test_multi_rows_equals_expanded_multi(dev):
+@both_argmax_paths
+def test_multi_rows_equals_expanded_multi(dev, argmax_path):
     """The rows form and the expanded form give the same results."""
     rng = np.random.default_rng(21)
     arr, row_of, cand = random_rows_case(rng, 9, 7, 6, 2000, "bf16")
@@ -340,7 +342,8 @@ def test_multi_rows_equals_expanded_multi(dev):
         assert torch.equal(r[key], e[key]), key
 
 
-def test_multi_rows_invalid_entries_and_limits(dev):
+@both_argmax_paths
+def test_multi_rows_invalid_entries_and_limits(dev, argmax_path):
     rng = np.random.default_rng(22)
     arr, row_of, cand = random_rows_case(rng, 5, 4, 3, 300, "bf16")
     R = arr.shape[1]
@@ -818,9 +821,10 @@ def test_stochastic_seq_offset_and_repeat(dev):
 @both_argmax_paths
 def test_kernel_launch_counts(dev, argmax_path):
     """The library counts its own launches: one kernel per stochastic, commit
-    and Philox call, three per stochastic tree call, and per greedy or
-    multi-candidate call two on the one-grid path (the streaming grid, then
-    the finalize grid) and one on the persistent pipeline."""
+    and Philox call, three per stochastic tree call, and per greedy,
+    multi-candidate or multi-candidate rows call two on the one-grid path (the
+    streaming grid, then the finalize grid) and one on the persistent
+    pipeline."""
     ws = sv.Workspace(dev)
     g = workloads.make_greedy(B=3, k=2, V=3000, seed=21)
     t = to_dev(g["target"], "bf16", dev)
@@ -829,11 +833,15 @@ def test_kernel_launch_counts(dev, argmax_path):
     st = workloads.make_stochastic(B=3, k=2, V=3000, t_dtype="bf16", d_dtype="bf16", t_std=2.0,
                                    d_noise=0.5, temperature=1.0, seed=22)
     tr = workloads.make_tree(B=2, N=5, V=3000, seed=23)
+    rows, row_of, cand = random_rows_case(np.random.default_rng(24), 3, 2, 2, 3000, "bf16")
     seq = torch.zeros(3, dtype=torch.int32, device=dev)
     buf = torch.full((3, 8), -1, dtype=torch.int32, device=dev)
     calls = [
         (per_argmax, lambda: sv.greedy(t, tok, workspace=ws)),
         (per_argmax, lambda: sv.multi_candidate(t[:, None], tok[:, None], workspace=ws)),
+        (per_argmax, lambda: sv.multi_candidate_rows(to_dev(rows, "bf16", dev),
+                                                     torch.from_numpy(row_of).to(dev),
+                                                     torch.from_numpy(cand).to(dev), workspace=ws)),
         (1, lambda: sv.stochastic(to_dev(st["target"], "bf16", dev), to_dev(st["draft"], "bf16", dev),
                                   torch.from_numpy(st["tokens"]).to(dev), 1.0, 5, workspace=ws)),
         (3, lambda: sv.tree_stochastic(to_dev(tr["node_logits"], "bf16", dev),
